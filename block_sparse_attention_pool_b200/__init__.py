@@ -1,0 +1,300 @@
+"""Python binding of libvsa, the B200 block-sparse video attention library.
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+libvsa.so (built in-tree by ``block_sparse_attention_pool_b200.build``).
+PyTorch supplies device memory and the current CUDA stream.  There is no
+fallback: if the shared library is missing or cannot be loaded, every call
+raises :class:`VsaError`.
+
+Functions mirror the C ABI of ``include/vsa.h`` one to one (same names without
+the ``vsa_`` prefix).  :class:`SparseVideoAttention` strings them together into
+the whole path (pool -> select -> Macro pass -> Micro select -> Micro pass with
+the LSE merge) over caller-visible buffers that it allocates once per shape.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+from typing import Dict, Optional, Sequence
+
+import torch
+
+__all__ = [
+    "VsaError", "Shape", "SelectParams", "MicroParams", "lib", "library_path", "EXPORTED",
+    "pool_qk", "select_blocks", "mask_to_lists", "select_micro", "select_micro_workspace_bytes",
+    "block_sparse_fwd", "lse_merge", "read_device_status", "status_string", "version",
+    "PathConfig", "SparseVideoAttention",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libvsa.so")
+
+EXPORTED = (
+    "vsa_status_string", "vsa_version", "vsa_read_device_status", "vsa_pool_qk", "vsa_select_blocks",
+    "vsa_mask_to_lists", "vsa_select_micro_workspace_bytes", "vsa_select_micro", "vsa_block_sparse_fwd",
+    "vsa_lse_merge",
+)
+
+STATUS = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_UNSUPPORTED", 3: "VSA_ERR_CUDA",
+          4: "VSA_ERR_CAPACITY", 5: "VSA_ERR_BAD_INDEX", 6: "VSA_ERR_TIMEOUT"}
+
+
+class VsaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)}")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("n_valid", ctypes.c_int), ("n_pad", ctypes.c_int),
+                ("d", ctypes.c_int)]
+
+
+class SelectParams(ctypes.Structure):
+    _fields_ = [("k_min", ctypes.c_int), ("cum_mass", ctypes.c_float), ("fixed_k", ctypes.c_int),
+                ("n_anchor", ctypes.c_int), ("anchor_rot", ctypes.c_int)]
+
+
+class MicroParams(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int), ("topk", ctypes.c_int), ("percentile", ctypes.c_double),
+                ("head_enable", ctypes.POINTER(ctypes.c_uint8)), ("row_capacity", ctypes.c_int)]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib():
+    """Load libvsa.so (once).  Raises VsaError if it is absent: no fallback."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise VsaError(3, f"libvsa.so not built at {_LIB_PATH} (run python -m block_sparse_attention_pool_b200.build)")
+    L = ctypes.CDLL(_LIB_PATH)
+    P, I, F, D, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_double, ctypes.c_size_t
+    SP = ctypes.POINTER(Shape)
+    L.vsa_status_string.restype = ctypes.c_char_p
+    L.vsa_status_string.argtypes = [I]
+    L.vsa_version.restype = I
+    L.vsa_version.argtypes = []
+    L.vsa_read_device_status.restype = I
+    L.vsa_read_device_status.argtypes = [P]
+    L.vsa_pool_qk.restype = I
+    L.vsa_pool_qk.argtypes = [P, P, SP, I, I, P, P, P, P, P]
+    L.vsa_select_blocks.restype = I
+    L.vsa_select_blocks.argtypes = [P, P, SP, I, I, F, ctypes.POINTER(SelectParams), P, P, P, P]
+    L.vsa_mask_to_lists.restype = I
+    L.vsa_mask_to_lists.argtypes = [P, SP, I, I, P, P, P]
+    L.vsa_select_micro_workspace_bytes.restype = S
+    L.vsa_select_micro_workspace_bytes.argtypes = [SP, ctypes.POINTER(MicroParams)]
+    L.vsa_select_micro.restype = I
+    L.vsa_select_micro.argtypes = [P, P, P, P, SP, I, I, F, ctypes.POINTER(MicroParams), P, P, P, S, P]
+    L.vsa_block_sparse_fwd.restype = I
+    L.vsa_block_sparse_fwd.argtypes = [P, P, P, SP, I, I, P, P, I, F, P, I, P, P, P, P]
+    L.vsa_lse_merge.restype = I
+    L.vsa_lse_merge.argtypes = [P, P, P, P, SP, P, I, P, P]
+    _lib = L
+    return L
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(code: int, what: str) -> None:
+    if code != 0:
+        raise VsaError(code, what)
+
+
+def _shape(B, H, n_valid, n_pad, d) -> Shape:
+    return Shape(int(B), int(H), int(n_valid), int(n_pad), int(d))
+
+
+def shape_of(q: torch.Tensor, n_valid: int) -> Shape:
+    B, H, n_pad, d = q.shape
+    return _shape(B, H, n_valid, n_pad, d)
+
+
+def status_string(code: int) -> str:
+    return lib().vsa_status_string(int(code)).decode()
+
+
+def version() -> int:
+    return lib().vsa_version()
+
+
+def read_device_status(stream=None) -> int:
+    return lib().vsa_read_device_status(_s(stream))
+
+
+def pool_qk(q, k, shape: Shape, bq, bk, q_pool, k_pool, q_pool64=None, k_pool16=None, stream=None):
+    _check(lib().vsa_pool_qk(_p(q), _p(k), ctypes.byref(shape), bq, bk, _p(q_pool), _p(k_pool), _p(q_pool64),
+                             _p(k_pool16), _s(stream)), "vsa_pool_qk")
+
+
+def select_blocks(q_pool, k_pool, shape: Shape, bq, bk, scale, params: SelectParams, counts, idx, mask=None,
+                  stream=None):
+    _check(lib().vsa_select_blocks(_p(q_pool), _p(k_pool), ctypes.byref(shape), bq, bk, float(scale),
+                                   ctypes.byref(params), _p(counts), _p(idx), _p(mask), _s(stream)),
+           "vsa_select_blocks")
+
+
+def mask_to_lists(mask, shape: Shape, bq, bk, counts, idx, stream=None):
+    _check(lib().vsa_mask_to_lists(_p(mask), ctypes.byref(shape), bq, bk, _p(counts), _p(idx), _s(stream)),
+           "vsa_mask_to_lists")
+
+
+def _micro_params(mode, topk, percentile, head_enable: Optional[Sequence[int]], row_capacity):
+    arr = None
+    if head_enable is not None:
+        arr = (ctypes.c_uint8 * len(head_enable))(*[int(x) for x in head_enable])
+    p = MicroParams(int(mode), int(topk), float(percentile),
+                    ctypes.cast(arr, ctypes.POINTER(ctypes.c_uint8)) if arr is not None else None,
+                    int(row_capacity))
+    return p, arr  # keep arr alive with p
+
+
+def select_micro_workspace_bytes(shape: Shape, mode, topk, percentile, head_enable, row_capacity) -> int:
+    p, keep = _micro_params(mode, topk, percentile, head_enable, row_capacity)
+    n = lib().vsa_select_micro_workspace_bytes(ctypes.byref(shape), ctypes.byref(p))
+    del keep
+    return int(n)
+
+
+def select_micro(q_pool64, k_pool16, counts, idx, shape: Shape, bq, bk, scale, mode, topk, percentile, head_enable,
+                 row_capacity, m_counts, m_idx, workspace, stream=None):
+    p, keep = _micro_params(mode, topk, percentile, head_enable, row_capacity)
+    _check(lib().vsa_select_micro(_p(q_pool64), _p(k_pool16), _p(counts), _p(idx), ctypes.byref(shape), bq, bk,
+                                  float(scale), ctypes.byref(p), _p(m_counts), _p(m_idx), _p(workspace),
+                                  workspace.numel() * workspace.element_size(), _s(stream)), "vsa_select_micro")
+    del keep
+
+
+def block_sparse_fwd(q, k, v, shape: Shape, list_rows, seg_keys, counts, idx, idx_stride, scale, o, lse,
+                     merge_o=None, merge_lse=None, stream=None):
+    o_fp32 = 1 if o.dtype == torch.float32 else 0
+    _check(lib().vsa_block_sparse_fwd(_p(q), _p(k), _p(v), ctypes.byref(shape), int(list_rows), int(seg_keys),
+                                      _p(counts), _p(idx), int(idx_stride), float(scale), _p(o), o_fp32, _p(lse),
+                                      _p(merge_o), _p(merge_lse), _s(stream)), "vsa_block_sparse_fwd")
+
+
+def lse_merge(o_a, lse_a, o_b, lse_b, shape: Shape, o_out, lse_out, stream=None):
+    out_fp32 = 1 if o_out.dtype == torch.float32 else 0
+    _check(lib().vsa_lse_merge(_p(o_a), _p(lse_a), _p(o_b), _p(lse_b), ctypes.byref(shape), _p(o_out), out_fp32,
+                               _p(lse_out), _s(stream)), "vsa_lse_merge")
+
+
+# ---------------------------------------------------------------------------
+# The whole path
+# ---------------------------------------------------------------------------
+
+@dataclass
+class PathConfig:
+    """Sizes and knobs of one attention layer (field names as in vsa.h)."""
+    n_valid: int
+    bq: int = 128
+    bk: int = 128
+    scale: Optional[float] = None
+    k_min: int = 0
+    cum_mass: float = 0.0
+    fixed_k: int = 0
+    n_anchor: int = 0
+    anchor_rot: int = 0
+    micro_mode: int = 0
+    micro_topk: int = 0
+    micro_percentile: float = 0.0
+    micro_heads: Optional[Sequence[int]] = None
+    micro_capacity: int = 0          # 0: every tile of the row fits (no overflow possible)
+
+    @staticmethod
+    def from_workload(w, micro_heads=None) -> "PathConfig":
+        return PathConfig(n_valid=w.n_valid, bq=w.bq, bk=w.bk, scale=w.scale, k_min=w.k_min, cum_mass=w.cum_mass,
+                          fixed_k=w.fixed_k, n_anchor=w.n_anchor, anchor_rot=w.anchor_rot, micro_mode=w.micro_mode,
+                          micro_topk=w.micro_topk, micro_percentile=w.micro_percentile,
+                          micro_heads=None if micro_heads is None else [int(x) for x in micro_heads])
+
+
+class SparseVideoAttention:
+    """Pool -> select -> Macro attention -> Micro select -> Micro attention + LSE merge.
+
+    Buffers are allocated once per input shape (torch, on q's device) and
+    reused; outputs of the last call stay readable in ``self.buf``.
+    """
+
+    def __init__(self, cfg: PathConfig):
+        self.cfg = cfg
+        self.buf: Dict[str, torch.Tensor] = {}
+        self._key = None
+
+    def _alloc(self, q: torch.Tensor):
+        B, H, n_pad, d = q.shape
+        key = (B, H, n_pad, d, q.device)
+        if key == self._key:
+            return
+        c = self.cfg
+        dev = q.device
+        n_q, n_k = n_pad // c.bq, n_pad // c.bk
+        f32, i32 = torch.float32, torch.int32
+        b = {
+            "q_pool": torch.empty(B, H, n_q, d, device=dev, dtype=f32),
+            "k_pool": torch.empty(B, H, n_k, d, device=dev, dtype=f32),
+            "counts": torch.empty(B, H, n_q, device=dev, dtype=i32),
+            "idx": torch.empty(B, H, n_q, n_k, device=dev, dtype=i32),
+            "lse": torch.empty(B, H, n_pad, device=dev, dtype=f32),
+            "o": torch.empty(B, H, n_pad, d, device=dev, dtype=torch.bfloat16),
+        }
+        if c.micro_mode:
+            n_r, n_t = n_pad // 64, n_pad // 16
+            cap = c.micro_capacity or n_t
+            shape = _shape(B, H, c.n_valid, n_pad, d)
+            ws = select_micro_workspace_bytes(shape, c.micro_mode, c.micro_topk, c.micro_percentile, c.micro_heads, cap)
+            b.update({
+                "q_pool64": torch.empty(B, H, n_r, d, device=dev, dtype=f32),
+                "k_pool16": torch.empty(B, H, n_t, d, device=dev, dtype=f32),
+                "o_macro": torch.empty(B, H, n_pad, d, device=dev, dtype=f32),
+                "lse_macro": torch.empty(B, H, n_pad, device=dev, dtype=f32),
+                "m_counts": torch.empty(B, H, n_r, device=dev, dtype=i32),
+                "m_idx": torch.empty(B, H, n_r, cap, device=dev, dtype=i32),
+                "workspace": torch.empty(max(16, ws), device=dev, dtype=torch.uint8),
+            })
+            self.micro_cap = cap
+        self.buf = b
+        self._key = key
+
+    def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None) -> Dict[str, torch.Tensor]:
+        c = self.cfg
+        self._alloc(q)
+        b = self.buf
+        B, H, n_pad, d = q.shape
+        shape = _shape(B, H, c.n_valid, n_pad, d)
+        scale = c.scale if c.scale is not None else 1.0 / math.sqrt(d)
+        n_k = n_pad // c.bk
+        micro = c.micro_mode != 0
+        pool_qk(q, k, shape, c.bq, c.bk, b["q_pool"], b["k_pool"], b.get("q_pool64"), b.get("k_pool16"), stream)
+        select_blocks(b["q_pool"], b["k_pool"], shape, c.bq, c.bk, scale,
+                      SelectParams(c.k_min, c.cum_mass, c.fixed_k, c.n_anchor, c.anchor_rot), b["counts"], b["idx"],
+                      None, stream)
+        if not micro:
+            block_sparse_fwd(q, k, v, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, scale, b["o"], b["lse"],
+                             stream=stream)
+            return b
+        block_sparse_fwd(q, k, v, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, scale, b["o_macro"],
+                         b["lse_macro"], stream=stream)
+        select_micro(b["q_pool64"], b["k_pool16"], b["counts"], b["idx"], shape, c.bq, c.bk, scale, c.micro_mode,
+                     c.micro_topk, c.micro_percentile, c.micro_heads, self.micro_cap, b["m_counts"], b["m_idx"],
+                     b["workspace"], stream)
+        block_sparse_fwd(q, k, v, shape, 64, 16, b["m_counts"], b["m_idx"], self.micro_cap, scale, b["o"], b["lse"],
+                         b["o_macro"], b["lse_macro"], stream)
+        return b

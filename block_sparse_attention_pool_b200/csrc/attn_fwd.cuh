@@ -1,0 +1,515 @@
+// a4 / a6 Block-sparse attention forward on the 5th-generation tensor cores.
+//
+// HyperVAttention section 2 Eq. (4): each query block attends only to its
+// selected key blocks; section 4.3: the selected key blocks of a row are
+// walked as one packed sequence of fixed-size tiles.  HyMoR-Attn (abstract):
+// the fine Micro pass over 16-key tiles inside omitted blocks is merged with
+// the Macro output by exact LSE merging; that merge is this kernel's
+// epilogue when merge inputs are given.
+//
+// One CTA = one 128-row query tile of one (batch, head).  The tile's key
+// segments (list entries of seg_keys keys; the union of two 64-row lists
+// when list_rows = 64, each entry tagged with the halves that use it) are
+// packed into 128-key stages.  Warp roles:
+//   warp 0     TMA producer: Q once, then K and V of each stage into
+//              2 + 2 ring slots (128B-swizzled, one box per segment and
+//              64-column chunk; rows past n_valid arrive as zeros).
+//   warp 1     MMA issuer (one thread): S_s = Q K_s^T into one of two TMEM
+//              S buffers, then O += P_{s-1} V_{s-1}; tcgen05.commit frees
+//              ring slots and signals the softmax.
+//   warps 2-5  softmax: one thread per query row reads its S row from TMEM,
+//              masks, keeps a running max in the log2 domain, rescales the
+//              TMEM O row only when the max grew by more than 2^8 (lazy
+//              rescale), writes P (bf16) to shared memory in the swizzled
+//              K-major operand layout, and finally normalises O, computes
+//              LSE and, if asked, merges with a previous (O, LSE).
+// TMEM: S0 [0,128), S1 [128,256), O [256, 256 + d) fp32 columns.
+#pragma once
+
+#include "common.cuh"
+#include "merge.cuh"
+
+namespace vsa {
+
+constexpr int kAttnThreads = 192;
+constexpr int kTileM = 128;
+constexpr int kStageKeys = 128;
+constexpr int kChunkBytes = 128 * 128;  // one 64-column bf16 chunk of a 128-row tile
+constexpr int kInfoRing = 4;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+struct AttnArgs {
+  int n_pad, n_valid;
+  int list_rows, seg_keys, seg_shift, idx_stride;
+  const int32_t *counts;
+  const int32_t *idx;
+  float scale_log2;  // softmax scale * log2(e)
+  void *o;
+  int o_fp32;
+  float *lse;
+  const float *merge_o;
+  const float *merge_lse;
+  unsigned long long timeout_ns;
+};
+
+struct StageInfo {
+  int start[8];   // first key row of each segment of the stage
+  uint32_t mask;  // bit 2*s + h: segment s is used by query half h
+  int full;       // every column of the stage is used by every row
+};
+
+template <int D>
+struct AttnSmem {
+  static constexpr int kQBytes = kTileM * D * 2;
+  static constexpr int kKVBytes = kStageKeys * D * 2;
+  static constexpr int kPBytes = kTileM * kStageKeys * 2;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffV = kOffK + 2 * kKVBytes;
+  static constexpr int kOffP = kOffV + 2 * kKVBytes;
+  static constexpr int kOffCtl = kOffP + kPBytes;
+  static constexpr int kBytes = kOffCtl + 1024;  // barriers, info ring, misc
+  static constexpr int kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
+};
+
+struct AttnCtl {
+  uint64_t q_full;
+  uint64_t k_full[2], k_empty[2];
+  uint64_t v_full[2], v_empty[2];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full, pv_done, mma_drain;
+  uint64_t info_full[kInfoRing];
+  uint32_t tmem_base;
+  int abort;
+  int n_seg;
+  int pad_;
+  StageInfo info[kInfoRing];
+};
+
+// Cursor over the (union of the) sorted list(s) of a tile, walked by a whole
+// warp in lockstep; lane-parallel windows of 32 entries keep the global reads
+// coalesced.
+struct ListCursor {
+  const int32_t *p[2];
+  int n[2];
+  int pos[2];
+  int base[2];
+  int win[2];  // this lane's window entry of each list
+  int nl;
+
+  __device__ void init(const int32_t *p0, int n0, const int32_t *p1, int n1, int lists, int lane) {
+    p[0] = p0; n[0] = n0; p[1] = p1; n[1] = n1; nl = lists;
+    for (int h = 0; h < 2; ++h) {
+      pos[h] = 0;
+      base[h] = 0;
+      win[h] = (h < nl && lane < n[h]) ? __ldg(p[h] + lane) : 0x7fffffff;
+    }
+  }
+  __device__ int peek(int h, int lane) {
+    if (h >= nl || pos[h] >= n[h]) return 0x7fffffff;
+    if (pos[h] - base[h] >= 32) {
+      base[h] = pos[h];
+      const int e = base[h] + lane;
+      win[h] = e < n[h] ? __ldg(p[h] + e) : 0x7fffffff;
+    }
+    return __shfl_sync(0xffffffffu, win[h], pos[h] - base[h]);
+  }
+  // Next segment of the union, or -1 at the end; *m = halves using it.
+  __device__ int next(uint32_t *m, int lane) {
+    const int a = peek(0, lane);
+    const int b = peek(1, lane);
+    if (a == 0x7fffffff && b == 0x7fffffff) return -1;
+    if (nl == 1) {
+      ++pos[0];
+      *m = 3u;
+      return a;
+    }
+    if (a < b) { ++pos[0]; *m = 1u; return a; }
+    if (b < a) { ++pos[1]; *m = 2u; return b; }
+    ++pos[0]; ++pos[1]; *m = 3u; return a;
+  }
+};
+
+// Warp-cooperative validation of one list (strictly ascending, in range);
+// returns false on a violation.
+__device__ __forceinline__ bool list_valid(const int32_t *p, int n, int n_seg_max, int lane) {
+  bool ok = true;
+  for (int e = lane; e < n; e += 32) {
+    const int v = __ldg(p + e);
+    if (v < 0 || v >= n_seg_max) ok = false;
+    if (e > 0 && __ldg(p + e - 1) >= v) ok = false;
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+
+// |A intersect B| of two validated ascending lists, warp-parallel binary search.
+__device__ __forceinline__ int list_intersection(const int32_t *a, int na, const int32_t *b, int nb, int lane) {
+  int c = 0;
+  for (int e = lane; e < na; e += 32) {
+    const int v = __ldg(a + e);
+    int lo = 0, hi = nb;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(b + mid) < v) lo = mid + 1; else hi = mid;
+    }
+    if (lo < nb && __ldg(b + lo) == v) ++c;
+  }
+  return warp_sum_int(c);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
+  using L = AttnSmem<D>;
+  extern __shared__ uint8_t attn_smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(attn_smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  uint8_t *sQ = smem + L::kOffQ;
+  uint8_t *sK = smem + L::kOffK;
+  uint8_t *sV = smem + L::kOffV;
+  uint8_t *sP = smem + L::kOffP;
+  AttnCtl *ctl = reinterpret_cast<AttnCtl *>(smem + L::kOffCtl);
+  volatile int *abort = &ctl->abort;
+
+  const int tile = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_lists = kTileM / a.list_rows;
+  const int lists_per_bh = a.n_pad / a.list_rows;
+  const int seg_per_stage = kStageKeys / a.seg_keys;
+  const size_t lrow0 = (size_t)bh * lists_per_bh + (size_t)tile * n_lists;
+
+  // ---------------------------------------------------------------- setup
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_init(&ctl->q_full, 1);
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&ctl->k_full[i], 1);
+        mbar_init(&ctl->k_empty[i], 1);
+        mbar_init(&ctl->v_full[i], 1);
+        mbar_init(&ctl->v_empty[i], 1);
+        mbar_init(&ctl->s_full[i], 1);
+        mbar_init(&ctl->s_free[i], 128);
+      }
+      mbar_init(&ctl->p_full, 128);
+      mbar_init(&ctl->pv_done, 1);
+      mbar_init(&ctl->mma_drain, 1);
+      for (int i = 0; i < kInfoRing; ++i) mbar_init(&ctl->info_full[i], 1);
+      ctl->abort = 0;
+      fence_barrier_init();
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+    // segment count of the tile (union of its lists), with list validation
+    const int n_seg_max = a.n_pad / a.seg_keys;
+    int cnt[2] = {0, 0};
+    bool ok = true;
+    for (int h = 0; h < n_lists; ++h) {
+      cnt[h] = __ldg(a.counts + lrow0 + h);
+      if (cnt[h] < 0 || cnt[h] > a.idx_stride) ok = false;
+    }
+    for (int h = 0; h < n_lists && ok; ++h) ok = list_valid(a.idx + (lrow0 + h) * a.idx_stride, cnt[h], n_seg_max, lane);
+    int n_seg = 0;
+    if (!ok) {
+      if (lane == 0) latch_status(VSA_ERR_BAD_INDEX);
+    } else if (n_lists == 1) {
+      n_seg = cnt[0];
+    } else {
+      n_seg = cnt[0] + cnt[1] -
+              list_intersection(a.idx + lrow0 * a.idx_stride, cnt[0], a.idx + (lrow0 + 1) * a.idx_stride, cnt[1], lane);
+    }
+    if (lane == 0) ctl->n_seg = n_seg;
+  } else if (warp == 1) {
+    tmem_alloc(&ctl->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const int n_seg = ctl->n_seg;
+  const int n_stages = (n_seg + seg_per_stage - 1) / seg_per_stage;
+  const uint32_t tmem = ctl->tmem_base;
+  const uint32_t tS[2] = {tmem, tmem + 128u};
+  const uint32_t tO = tmem + 256u;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (n_stages > 0) {
+      ListCursor cur;
+      cur.init(a.idx + lrow0 * a.idx_stride, __ldg(a.counts + lrow0),
+               n_lists > 1 ? a.idx + (lrow0 + 1) * a.idx_stride : nullptr,
+               n_lists > 1 ? __ldg(a.counts + lrow0 + 1) : 0, n_lists, lane);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&ctl->q_full, L::kQBytes);
+        for (int c = 0; c < D / 64; ++c) tma_load_3d(sQ + c * kChunkBytes, &tm_q, &ctl->q_full, c * 64, tile * kTileM, bh);
+      }
+      int issued = 0;
+      for (int s = 0; s < n_stages; ++s) {
+        const int slot = s & 1;
+        const uint32_t use_par = ((s >> 1) - 1) & 1;
+        // gather the stage's segments
+        int start[8];
+        uint32_t mask = 0u;
+        int nseg = 0;
+        for (int i = 0; i < seg_per_stage; ++i) {
+          uint32_t m = 0u;
+          const int sg = (nseg == i) ? cur.next(&m, lane) : -1;
+          if (sg >= 0) {
+            start[i] = sg * a.seg_keys;
+            mask |= m << (2 * i);
+            ++nseg;
+          } else {
+            start[i] = start[0];  // repeat a loaded segment; masked out
+          }
+        }
+        const bool full = (nseg == seg_per_stage) && (mask == (seg_per_stage == 8 ? 0xffffu : ((1u << (2 * seg_per_stage)) - 1u))) &&
+                          (start[seg_per_stage - 1] + a.seg_keys <= a.n_valid);
+        bool ok = true;
+        if (s >= 2) ok = mbar_wait_warp(&ctl->k_empty[slot], use_par, abort, a.timeout_ns, lane);
+        if (!ok) break;
+        if (lane == 0) {
+          StageInfo &inf = ctl->info[s & (kInfoRing - 1)];
+          for (int i = 0; i < 8; ++i) inf.start[i] = i < seg_per_stage ? start[i] : 0;
+          inf.mask = mask;
+          inf.full = full ? 1 : 0;
+          mbar_arrive(&ctl->info_full[s & (kInfoRing - 1)]);
+          mbar_arrive_expect_tx(&ctl->k_full[slot], L::kKVBytes);
+          for (int i = 0; i < seg_per_stage; ++i)
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(sK + slot * L::kKVBytes + c * kChunkBytes + i * a.seg_keys * 128, &tm_k, &ctl->k_full[slot],
+                          c * 64, start[i], bh);
+        }
+        if (s >= 2) ok = mbar_wait_warp(&ctl->v_empty[slot], use_par, abort, a.timeout_ns, lane);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&ctl->v_full[slot], L::kKVBytes);
+          for (int i = 0; i < seg_per_stage; ++i)
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(sV + slot * L::kKVBytes + c * kChunkBytes + i * a.seg_keys * 128, &tm_v, &ctl->v_full[slot],
+                          c * 64, start[i], bh);
+        }
+        issued = s + 1;
+        __syncwarp();
+      }
+      if (*abort && lane == 0) {
+        // let copies still in flight land before the CTA's shared memory goes away
+        mbar_drain(&ctl->q_full, 0, a.timeout_ns);
+        for (int s = max(0, issued - 2); s < issued; ++s) {
+          mbar_drain(&ctl->k_full[s & 1], (s >> 1) & 1, a.timeout_ns);
+          mbar_drain(&ctl->v_full[s & 1], (s >> 1) & 1, a.timeout_ns);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (n_stages > 0 && lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16_f32(kTileM, kStageKeys, false);
+      constexpr uint32_t kIdO = idesc_bf16_f32(kTileM, D, true);
+      const uint32_t q_addr = smem_addr(sQ), k_addr = smem_addr(sK), v_addr = smem_addr(sV), p_addr = smem_addr(sP);
+      bool ok = mbar_wait(&ctl->q_full, 0, abort, a.timeout_ns);
+      auto issue_pv = [&](int t) -> bool {
+        if (!mbar_wait(&ctl->p_full, t & 1, abort, a.timeout_ns)) return false;
+        if (!mbar_wait(&ctl->v_full[t & 1], (t >> 1) & 1, abort, a.timeout_ns)) return false;
+        tc_fence_after();
+        const uint32_t vb = v_addr + (t & 1) * L::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < kStageKeys / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(p_addr + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, kChunkBytes, 1024);
+          umma_bf16_ss(tO, ad, bd, kIdO, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&ctl->v_empty[t & 1]);
+        umma_commit(&ctl->pv_done);
+        return true;
+      };
+      for (int s = 0; ok && s < n_stages; ++s) {
+        const int slot = s & 1;
+        ok = mbar_wait(&ctl->k_full[slot], (s >> 1) & 1, abort, a.timeout_ns);
+        if (ok && s >= 2) ok = mbar_wait(&ctl->s_free[slot], ((s - 2) >> 1) & 1, abort, a.timeout_ns);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kb = k_addr + slot * L::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(q_addr + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(kb + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
+          umma_bf16_ss(tS[slot], ad, bd, kIdS, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&ctl->k_empty[slot]);
+        umma_commit(&ctl->s_full[slot]);
+        if (s >= 1) ok = issue_pv(s - 1);
+      }
+      if (ok) issue_pv(n_stages - 1);
+      // every MMA issued by this thread has completed once mma_drain flips
+      umma_commit(&ctl->mma_drain);
+      mbar_drain(&ctl->mma_drain, 0, a.timeout_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;  // row within the tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const int half = row >> 6;
+    float m2 = -INFINITY;  // running max of scaled logits, log2 units
+    float l = 0.f;
+    bool ok = true;
+    for (int t = 0; t < n_stages; ++t) {
+      const int slot = t & 1;
+      ok = mbar_wait_warp(&ctl->info_full[t & (kInfoRing - 1)], (t >> 2) & 1, abort, a.timeout_ns, lane);
+      if (ok) ok = mbar_wait_warp(&ctl->s_full[slot], (t >> 1) & 1, abort, a.timeout_ns, lane);
+      if (!ok) break;
+      tc_fence_after();
+      const StageInfo &inf = ctl->info[t & (kInfoRing - 1)];
+      const int full = inf.full;
+      const uint32_t mask = inf.mask;
+      int start[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) start[i] = inf.start[i];
+      float x[kStageKeys];
+#pragma unroll
+      for (int c = 0; c < kStageKeys / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tS[slot] + lane_off + c * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[c * 32 + j] = __uint_as_float(r[j]) * a.scale_log2;
+      }
+      tc_fence_before();
+      mbar_arrive(&ctl->s_free[slot]);
+      if (!full) {
+#pragma unroll
+        for (int c = 0; c < kStageKeys; ++c) {
+          const int sg = c >> a.seg_shift;
+          const int key = start[sg] + (c & (a.seg_keys - 1));
+          const bool valid = ((mask >> (2 * sg + half)) & 1u) && key < a.n_valid;
+          if (!valid) x[c] = -INFINITY;
+        }
+      }
+      float rmax = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kStageKeys; ++c) rmax = fmaxf(rmax, x[c]);
+      const float m_new = fmaxf(m2, rmax);
+      const bool need = m_new > m2 + kRescaleThreshold || (m2 == -INFINITY && m_new != -INFINITY);
+      if (t > 0) {
+        ok = mbar_wait_warp(&ctl->pv_done, (t - 1) & 1, abort, a.timeout_ns, lane);
+        if (!ok) break;
+      }
+      if (__any_sync(0xffffffffu, need)) {
+        const float alpha = need ? fast_exp2(m2 - m_new) : 1.f;  // exp2(-inf) = 0
+        if (t > 0) {
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tO + lane_off + c * 32, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
+            tmem_st32(tO + lane_off + c * 32, r);
+          }
+          tmem_st_wait();
+        }
+        if (need) {
+          l *= alpha;
+          m2 = m_new;
+        }
+      }
+      // P = exp2(x - m2) in bf16, swizzled K-major layout of the P.V operand
+      const bool live = m2 != -INFINITY;
+      uint8_t *prow = sP + row * 128;
+      float rs = 0.f;
+#pragma unroll
+      for (int g = 0; g < kStageKeys / 8; ++g) {
+        float p[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          p[j] = live ? fast_exp2(x[g * 8 + j] - m2) : 0.f;
+          rs += p[j];
+        }
+        uint4 pk;
+        pk.x = pack_bf16x2(p[0], p[1]);
+        pk.y = pack_bf16x2(p[2], p[3]);
+        pk.z = pack_bf16x2(p[4], p[5]);
+        pk.w = pack_bf16x2(p[6], p[7]);
+        const int cb = g >> 3, cc = g & 7;
+        *reinterpret_cast<uint4 *>(prow + cb * kChunkBytes + ((cc ^ (row & 7)) << 4)) = pk;
+      }
+      l += rs;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&ctl->p_full);
+    }
+
+    // ---------------------------------------------------------- epilogue
+    const int grow = tile * kTileM + row;
+    const size_t orow = (size_t)bh * a.n_pad + grow;
+    float acc[D];
+    bool have = false;
+    if (ok && n_stages > 0) {
+      ok = mbar_wait_warp(&ctl->pv_done, (n_stages - 1) & 1, abort, a.timeout_ns, lane);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + lane_off + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[c * 32 + j] = __uint_as_float(r[j]);
+        }
+        have = true;
+      }
+    }
+    const bool row_ok = grow < a.n_valid && have && l > 0.f;
+    const float inv_l = row_ok ? 1.f / l : 0.f;
+    float lse = row_ok ? (m2 + log2f(l)) * 0.69314718055994531f : -INFINITY;
+#pragma unroll
+    for (int c = 0; c < D; ++c) acc[c] = row_ok ? acc[c] * inv_l : 0.f;
+    if (a.merge_o != nullptr) {
+      const float lm = grow < a.n_valid ? a.merge_lse[orow] : -INFINITY;
+      const MergeWeights w = lse_merge_weights(lm, lse);
+      const float4 *mo = reinterpret_cast<const float4 *>(a.merge_o + orow * D);
+#pragma unroll
+      for (int c = 0; c < D / 4; ++c) {
+        const float4 v = mo[c];
+        acc[4 * c + 0] = w.wa * v.x + w.wb * acc[4 * c + 0];
+        acc[4 * c + 1] = w.wa * v.y + w.wb * acc[4 * c + 1];
+        acc[4 * c + 2] = w.wa * v.z + w.wb * acc[4 * c + 2];
+        acc[4 * c + 3] = w.wa * v.w + w.wb * acc[4 * c + 3];
+      }
+      lse = w.lse;
+    }
+    if (a.o_fp32) {
+      float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.o) + orow * D);
+#pragma unroll
+      for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
+    } else {
+      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.o) + orow * D);
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        uint4 pk;
+        pk.x = pack_bf16x2(acc[8 * c + 0], acc[8 * c + 1]);
+        pk.y = pack_bf16x2(acc[8 * c + 2], acc[8 * c + 3]);
+        pk.z = pack_bf16x2(acc[8 * c + 4], acc[8 * c + 5]);
+        pk.w = pack_bf16x2(acc[8 * c + 6], acc[8 * c + 7]);
+        dst[c] = pk;
+      }
+    }
+    a.lse[orow] = lse;
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace vsa

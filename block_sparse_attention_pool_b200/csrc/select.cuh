@@ -1,0 +1,273 @@
+// a2 + a3 Pooled scoring and block selection, and the explicit-mask path.
+//
+// HyperVAttention section 2 Eq. (2): S_ij = <mu_i, mu_j> / sqrt(d) and the
+// size-weighted softmax P'_ij = s_j e^{S_ij} / sum_o s_o e^{S_io}; Eq. (3):
+// row-wise Top-p, the smallest prefix of key blocks in descending P' whose
+// mass reaches p; App. A.1 "Min-kc": a floor on the kept count; the LVSA
+// abstract: rotating global anchor columns.
+//
+// One CTA owns 16 query-block rows of one (batch, head).  It stages the 16
+// pooled query rows and 32-key chunks of the pooled keys in shared memory and
+// computes the 16 x n_k logits with fp32 FFMA (no TF32, so the ranking
+// matches an fp64 evaluation wherever two blocks differ by more than fp32
+// rounding).  Each warp then ranks two rows: the n_k log-weights
+// w = S + ln s_j, packed with the key index into 64-bit keys, are bitonic-
+// sorted in registers (32 keys per lane at most, n_k <= 1024), the sorted
+// weights are exponentiated and prefix-summed, and the kept prefix plus the
+// anchors is written out as an ascending index list with ballot compaction.
+#pragma once
+
+#include "common.cuh"
+
+namespace vsa {
+
+constexpr int kSelRows = 16;
+constexpr int kSelThreads = 256;
+constexpr int kSelChunk = 32;
+
+struct SelectArgs {
+  const float *q_pool;  // [BH, n_q, d]
+  const float *k_pool;  // [BH, n_k, d]
+  int n_q, n_k, bq, bk, n_valid;
+  float scale;
+  int k_min, fixed_k, n_anchor, anchor_rot;
+  float cum_mass;
+  int32_t *counts;  // [BH, n_q]
+  int32_t *idx;     // [BH, n_q, n_k]
+  uint8_t *mask;    // [BH, n_q, n_k] or null
+};
+
+// Bitonic sort, descending, of NR * 32 64-bit keys held NR per lane; the key at
+// sorted position e = lane * NR + i ends in register i of that lane.
+template <int NR>
+__device__ __forceinline__ void warp_bitonic_sort_desc(uint64_t (&key)[NR], int lane) {
+  constexpr int N = NR * 32;
+#pragma unroll
+  for (int kk = 2; kk <= N; kk <<= 1) {
+#pragma unroll
+    for (int j = kk >> 1; j > 0; j >>= 1) {
+      if (j >= NR) {
+        // partner in lane ^ (j / NR), same register
+        const int lx = j / NR;
+        const bool lower = (lane & lx) == 0;
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+          const int e = lane * NR + i;
+          const bool desc = (e & kk) == 0;
+          const uint64_t other = __shfl_xor_sync(0xffffffffu, key[i], lx);
+          const uint64_t mx = key[i] > other ? key[i] : other;
+          const uint64_t mn = key[i] > other ? other : key[i];
+          key[i] = (desc == lower) ? mx : mn;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+          if ((i & j) == 0) {
+            const int e = lane * NR + i;
+            const bool desc = (e & kk) == 0;
+            const uint64_t a = key[i], b = key[i | j];
+            const bool swap = desc ? (a < b) : (a > b);
+            key[i] = swap ? b : a;
+            key[i | j] = swap ? a : b;
+          }
+        }
+      }
+    }
+  }
+}
+
+// Emit the ascending index list of the set bits of a per-warp bitmap of n bits
+// (word w covers indices [32w, 32w + 32)); returns the count.
+__device__ __forceinline__ int emit_bitmap_list(const uint32_t *bits, int n, int lane, int32_t *dst,
+                                                uint8_t *mask_row) {
+  int total = 0;
+  for (int w0 = 0; w0 * 32 < n; w0 += 32) {
+    const int w = w0 + lane;
+    const uint32_t word = (w * 32 < n) ? bits[w] : 0u;
+    const int cnt = __popc(word);
+    const int off = warp_exclusive_scan(cnt, lane);
+    uint32_t rest = word;
+    int o = total + off;
+    while (rest) {
+      const int b = __ffs(rest) - 1;
+      rest &= rest - 1;
+      dst[o++] = w * 32 + b;
+    }
+    if (mask_row && w * 32 < n) {
+      const int lim = min(32, n - w * 32);
+      for (int b = 0; b < lim; ++b) mask_row[w * 32 + b] = (word >> b) & 1u;
+    }
+    total += __shfl_sync(0xffffffffu, off + cnt, 31);
+  }
+  return total;
+}
+
+template <int D, int NR>
+__global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a) {
+  constexpr int DP = D + 4;  // padded row stride (floats)
+  extern __shared__ __align__(16) float sel_smem[];
+  float *qs = sel_smem;                       // [kSelRows][DP]
+  float *ks = qs + kSelRows * DP;             // [kSelChunk][DP]
+  const int nkp = NR * 32;
+  float *S = ks + kSelChunk * DP;             // [kSelRows][nkp]
+  uint32_t *bitmap = reinterpret_cast<uint32_t *>(S + kSelRows * nkp);  // [8 warps][32]
+
+  const int bh = blockIdx.y;
+  const int row0 = blockIdx.x * kSelRows;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const float *qp = a.q_pool + (size_t)bh * a.n_q * D;
+  const float *kp = a.k_pool + (size_t)bh * a.n_k * D;
+
+  for (int i = t; i < kSelRows * (D / 4); i += kSelThreads) {
+    const int r = i / (D / 4), c4 = i % (D / 4);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (row0 + r < a.n_q) v = __ldg(reinterpret_cast<const float4 *>(qp + (size_t)(row0 + r) * D) + c4);
+    *reinterpret_cast<float4 *>(qs + r * DP + c4 * 4) = v;
+  }
+
+  // ---- logits: thread -> (row t/16, keys (t%16) and (t%16)+16 of the chunk)
+  const int my_row = t >> 4;
+  const int my_key = t & 15;
+  for (int k0 = 0; k0 < a.n_k; k0 += kSelChunk) {
+    __syncthreads();
+    for (int i = t; i < kSelChunk * (D / 4); i += kSelThreads) {
+      const int r = i / (D / 4), c4 = i % (D / 4);
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (k0 + r < a.n_k) v = __ldg(reinterpret_cast<const float4 *>(kp + (size_t)(k0 + r) * D) + c4);
+      *reinterpret_cast<float4 *>(ks + r * DP + c4 * 4) = v;
+    }
+    __syncthreads();
+    float s0 = 0.f, s1 = 0.f;
+    const float *qrow = qs + my_row * DP;
+    const float *k0row = ks + my_key * DP;
+    const float *k1row = ks + (my_key + 16) * DP;
+#pragma unroll 8
+    for (int c = 0; c < D; c += 4) {
+      const float4 qv = *reinterpret_cast<const float4 *>(qrow + c);
+      const float4 a0 = *reinterpret_cast<const float4 *>(k0row + c);
+      const float4 a1 = *reinterpret_cast<const float4 *>(k1row + c);
+      s0 = fmaf(qv.x, a0.x, s0); s0 = fmaf(qv.y, a0.y, s0); s0 = fmaf(qv.z, a0.z, s0); s0 = fmaf(qv.w, a0.w, s0);
+      s1 = fmaf(qv.x, a1.x, s1); s1 = fmaf(qv.y, a1.y, s1); s1 = fmaf(qv.z, a1.z, s1); s1 = fmaf(qv.w, a1.w, s1);
+    }
+    if (k0 + my_key < nkp) S[my_row * nkp + k0 + my_key] = s0 * a.scale;
+    if (k0 + my_key + 16 < nkp) S[my_row * nkp + k0 + my_key + 16] = s1 * a.scale;
+  }
+  __syncthreads();
+
+  // ---- per-row ranking and selection, two rows per warp
+  const float ln_bk = logf((float)a.bk);
+  uint32_t *bits = bitmap + warp * 32;
+  for (int rr = 0; rr < kSelRows / 8; ++rr) {
+    const int r = warp * (kSelRows / 8) + rr;
+    const int qi = row0 + r;
+    if (qi >= a.n_q) break;
+    const size_t orow = (size_t)bh * a.n_q + qi;
+    int32_t *dst = a.idx + orow * a.n_k;
+    uint8_t *mrow = a.mask ? a.mask + orow * a.n_k : nullptr;
+    const bool q_has_rows = qi * a.bq < a.n_valid;
+
+    // Load: element j = i*32 + lane goes to register i (any start placement
+    // sorts to the same result).
+    uint64_t key[NR];
+#pragma unroll
+    for (int i = 0; i < NR; ++i) {
+      const int j = i * 32 + lane;
+      if (j < a.n_k) {
+        const int sj = min(a.bk, max(0, a.n_valid - j * a.bk));
+        const float w = sj > 0 ? S[r * nkp + j] + (sj == a.bk ? ln_bk : logf((float)sj)) : -INFINITY;
+        key[i] = ((uint64_t)float_key(w) << 32) | (uint64_t)(0xffffffffu - (uint32_t)j);
+      } else {
+        key[i] = 0ull;
+      }
+    }
+    warp_bitonic_sort_desc<NR>(key, lane);
+
+    int m = 0;
+    if (q_has_rows) {
+      if (a.fixed_k > 0) {
+        m = min(a.fixed_k, a.n_k);
+      } else {
+        int m_p = 0;
+        if (a.cum_mass > 0.f) {
+          const float wmax = key_float((uint32_t)(__shfl_sync(0xffffffffu, key[0], 0) >> 32));
+          float p[NR];
+          float lsum = 0.f;
+#pragma unroll
+          for (int i = 0; i < NR; ++i) {
+            const bool real = key[i] != 0ull;
+            const float w = key_float((uint32_t)(key[i] >> 32));
+            p[i] = (real && w != -INFINITY) ? expf(w - wmax) : 0.f;
+            lsum += p[i];
+            p[i] = lsum;  // inclusive lane-local prefix
+          }
+          // exclusive prefix of lane totals
+          float base = lsum;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, base, o);
+            if (lane >= o) base += y;
+          }
+          const float total = __shfl_sync(0xffffffffu, base, 31);
+          base -= lsum;
+          const float target = a.cum_mass * total;
+          int first = 0x7fffffff;
+#pragma unroll
+          for (int i = NR - 1; i >= 0; --i)
+            if (base + p[i] >= target) first = lane * NR + i;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) first = min(first, __shfl_xor_sync(0xffffffffu, first, o));
+          m_p = first == 0x7fffffff ? a.n_k : first + 1;
+        }
+        m = min(a.n_k, max(a.k_min, m_p));
+      }
+    }
+
+    // mark the kept prefix and the anchors
+    bits[lane] = 0u;
+    __syncwarp();
+    if (q_has_rows) {
+#pragma unroll
+      for (int i = 0; i < NR; ++i) {
+        if (lane * NR + i < m) {
+          const int j = (int)(0xffffffffu - (uint32_t)(key[i] & 0xffffffffull));
+          atomicOr(&bits[j >> 5], 1u << (j & 31));
+        }
+      }
+      if (lane == 0 && a.n_anchor > 0) {
+        const int step = a.n_k / a.n_anchor;
+        for (int tt = 0; tt < a.n_anchor; ++tt) {
+          const int j = (int)(((long long)a.anchor_rot + (long long)tt * step) % a.n_k);
+          atomicOr(&bits[j >> 5], 1u << (j & 31));
+        }
+      }
+    }
+    __syncwarp();
+    const int total = emit_bitmap_list(bits, a.n_k, lane, dst, mrow);
+    if (lane == 0) a.counts[orow] = total;
+    __syncwarp();
+  }
+}
+
+// Explicit uint8 block mask -> ascending lists: one warp per row.
+__global__ void mask_to_lists_kernel(const uint8_t *__restrict__ mask, int rows, int n_k,
+                                     int32_t *__restrict__ counts, int32_t *__restrict__ idx) {
+  __shared__ uint32_t bitmap[8][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= rows) return;
+  const uint8_t *m = mask + (size_t)row * n_k;
+  uint32_t *bits = bitmap[warp];
+  for (int w = lane; w < 32; w += 32) {
+    uint32_t word = 0u;
+    for (int b = 0; b < 32; ++b) {
+      const int j = w * 32 + b;
+      if (j < n_k && m[j] != 0) word |= 1u << b;
+    }
+    bits[w] = word;
+  }
+  __syncwarp();
+  const int total = emit_bitmap_list(bits, n_k, lane, idx + (size_t)row * n_k, nullptr);
+  if (lane == 0) counts[row] = total;
+}
+
+}  // namespace vsa

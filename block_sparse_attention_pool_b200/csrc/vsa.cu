@@ -1,0 +1,361 @@
+// libvsa: host side of the C ABI declared in include/vsa.h.
+//
+// Validates arguments, builds TMA tensor maps through the driver entry point
+// (no link-time dependency on libcuda), and launches the kernels of this
+// directory.  It allocates no device memory and never synchronises except in
+// vsa_read_device_status.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/vsa.h"
+#include "attn_fwd.cuh"
+#include "common.cuh"
+#include "merge.cuh"
+#include "micro.cuh"
+#include "pool.cuh"
+#include "select.cuh"
+
+namespace {
+
+using vsa::AttnArgs;
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per pipeline wait
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool shape_ok(const vsa_shape *s) {
+  if (!s) return false;
+  if (s->B < 1 || s->H < 1 || s->n_valid < 1 || s->n_pad < s->n_valid) return false;
+  if (s->d != 64 && s->d != 128) return false;
+  if (s->n_pad % 128 != 0) return false;
+  if ((long long)s->B * s->H > 65535) return false;
+  if ((long long)s->n_pad * s->d * s->B * s->H >= (1ll << 40)) return false;
+  return true;
+}
+
+vsa_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+// ---- tensor maps -----------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [BH][n_pad][d] bf16 viewed as a 3-D tensor (d, n_valid, BH): rows at or
+// past n_valid are outside the tensor and arrive as zeros.  Box = 64 columns
+// (128 bytes, one swizzle row) x box_rows rows x 1.
+bool make_map(CUtensorMap *map, const void *base, const vsa_shape *s, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)s->d, (cuuint64_t)s->n_valid, (cuuint64_t)s->B * s->H};
+  cuuint64_t strides[2] = {(cuuint64_t)s->d * 2, (cuuint64_t)s->n_pad * s->d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D>
+vsa_status launch_attn(const void *q, const void *k, const void *v, const vsa_shape *s, const AttnArgs &a,
+                       cudaStream_t st) {
+  using L = vsa::AttnSmem<D>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(vsa::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  });
+  if (attr_err != cudaSuccess) return VSA_ERR_CUDA;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, s, vsa::kTileM) || !make_map(&mk, k, s, a.seg_keys) || !make_map(&mv, v, s, a.seg_keys))
+    return VSA_ERR_CUDA;
+  dim3 grid(s->n_pad / vsa::kTileM, s->B * s->H);
+  vsa::attn_fwd_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, a);
+  return launch_status();
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct MicroLayout {
+  int n_slots;
+  size_t off_slot, off_bitmap, off_keys, off_hist, off_state, total;
+};
+
+MicroLayout micro_layout(const vsa_shape *s, const vsa_micro_params *p) {
+  MicroLayout L;
+  int enabled = 0;
+  for (int h = 0; h < s->H; ++h) enabled += (p->head_enable == nullptr || p->head_enable[h]) ? 1 : 0;
+  L.n_slots = enabled * s->B;
+  const size_t n_r = (size_t)s->n_pad / vsa::kMicroRows, n_t = (size_t)s->n_pad / vsa::kMicroKeys;
+  const size_t n_qmax = (size_t)s->n_pad / 64;
+  size_t off = 0;
+  L.off_slot = off;
+  off = align256(off + (size_t)s->B * s->H * 4);
+  L.off_bitmap = off;
+  off = align256(off + (size_t)L.n_slots * n_qmax * 32 * 4);
+  L.off_keys = off;
+  off = align256(off + (size_t)L.n_slots * n_r * n_t * 4);
+  L.off_hist = off;
+  off = align256(off + (size_t)L.n_slots * 3 * vsa::kHistBins * 4);
+  L.off_state = off;
+  off = align256(off + (size_t)L.n_slots * 8 * 4);
+  L.total = off;
+  return L;
+}
+
+bool micro_params_ok(const vsa_micro_params *p) {
+  if (!p) return false;
+  if (p->mode == 1) return p->topk >= 1 && p->topk <= 32 && p->row_capacity >= 1;
+  if (p->mode == 2) return p->percentile > 0.0 && p->percentile < 1.0 && p->row_capacity >= 1;
+  return false;
+}
+
+int ilog2(int x) {
+  int r = 0;
+  while ((1 << r) < x) ++r;
+  return r;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *vsa_status_string(vsa_status s) {
+  switch (s) {
+    case VSA_OK: return "ok";
+    case VSA_ERR_INVALID_ARG: return "invalid argument";
+    case VSA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case VSA_ERR_CUDA: return "CUDA error";
+    case VSA_ERR_CAPACITY: return "list capacity exceeded";
+    case VSA_ERR_BAD_INDEX: return "invalid index in a list";
+    case VSA_ERR_TIMEOUT: return "pipeline wait timed out";
+  }
+  return "unknown status";
+}
+
+int vsa_version(void) { return 100; }
+
+vsa_status vsa_read_device_status(void *stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return VSA_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpyFromSymbol(&h, vsa::g_status, sizeof(int)) != cudaSuccess) return VSA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(vsa::g_status, &zero, sizeof(int)) != cudaSuccess) return VSA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(vsa::g_timed_out, &zero, sizeof(int)) != cudaSuccess) return VSA_ERR_CUDA;
+  return static_cast<vsa_status>(h);
+}
+
+vsa_status vsa_pool_qk(const void *q, const void *k, const vsa_shape *shape, int bq, int bk, float *q_pool,
+                       float *k_pool, float *q_pool64, float *k_pool16, void *stream) {
+  if (!shape_ok(shape) || !q || !k || !q_pool || !k_pool) return VSA_ERR_INVALID_ARG;
+  if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_pool) || !aligned16(k_pool)) return VSA_ERR_INVALID_ARG;
+  vsa::PoolOut oq{q_pool, bq, q_pool64, 64};
+  vsa::PoolOut ok{k_pool, bk, k_pool16, 16};
+  dim3 grid(shape->n_pad / vsa::kPoolRows, shape->B * shape->H, 2);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const auto *qb = static_cast<const __nv_bfloat16 *>(q);
+  const auto *kb = static_cast<const __nv_bfloat16 *>(k);
+  if (shape->d == 128)
+    vsa::pool_kernel<128><<<grid, vsa::kPoolThreads, 0, st>>>(qb, kb, shape->n_pad, shape->n_valid, oq, ok);
+  else
+    vsa::pool_kernel<64><<<grid, vsa::kPoolThreads, 0, st>>>(qb, kb, shape->n_pad, shape->n_valid, oq, ok);
+  return launch_status();
+}
+
+vsa_status vsa_select_blocks(const float *q_pool, const float *k_pool, const vsa_shape *shape, int bq, int bk,
+                             float scale, const vsa_select_params *params, int32_t *counts, int32_t *idx,
+                             uint8_t *mask, void *stream) {
+  if (!shape_ok(shape) || !q_pool || !k_pool || !params || !counts || !idx) return VSA_ERR_INVALID_ARG;
+  if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(q_pool) || !aligned16(k_pool)) return VSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return VSA_ERR_INVALID_ARG;
+  if (params->k_min < 0 || params->fixed_k < 0 || params->n_anchor < 0 || params->anchor_rot < 0 ||
+      !std::isfinite(params->cum_mass))
+    return VSA_ERR_INVALID_ARG;
+  const int n_q = shape->n_pad / bq, n_k = shape->n_pad / bk;
+  if (n_k > 1024) return VSA_ERR_UNSUPPORTED;
+  vsa::SelectArgs a{q_pool, k_pool, n_q, n_k, bq, bk, shape->n_valid, scale, params->k_min, params->fixed_k,
+                    params->n_anchor, params->anchor_rot, params->cum_mass, counts, idx, mask};
+  int nkp = 32;
+  while (nkp < n_k) nkp <<= 1;
+  const int dp = shape->d + 4;
+  const size_t smem = (size_t)(vsa::kSelRows + vsa::kSelChunk) * dp * 4 + (size_t)vsa::kSelRows * nkp * 4 + 8 * 32 * 4;
+  dim3 grid((n_q + vsa::kSelRows - 1) / vsa::kSelRows, shape->B * shape->H);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+#define VSA_SEL_CASE(DD, NR)                                                                                  \
+  {                                                                                                           \
+    auto kern = vsa::select_blocks_kernel<DD, NR>;                                                            \
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) \
+      return VSA_ERR_CUDA;                                                                                    \
+    kern<<<grid, vsa::kSelThreads, smem, st>>>(a);                                                            \
+  }
+#define VSA_SEL_NR(DD)                     \
+  switch (nkp / 32) {                      \
+    case 1: VSA_SEL_CASE(DD, 1) break;     \
+    case 2: VSA_SEL_CASE(DD, 2) break;     \
+    case 4: VSA_SEL_CASE(DD, 4) break;     \
+    case 8: VSA_SEL_CASE(DD, 8) break;     \
+    case 16: VSA_SEL_CASE(DD, 16) break;   \
+    default: VSA_SEL_CASE(DD, 32) break;   \
+  }
+  if (shape->d == 128) {
+    VSA_SEL_NR(128)
+  } else {
+    VSA_SEL_NR(64)
+  }
+#undef VSA_SEL_NR
+#undef VSA_SEL_CASE
+  return launch_status();
+}
+
+vsa_status vsa_mask_to_lists(const uint8_t *mask, const vsa_shape *shape, int bq, int bk, int32_t *counts,
+                             int32_t *idx, void *stream) {
+  if (!shape_ok(shape) || !mask || !counts || !idx) return VSA_ERR_INVALID_ARG;
+  if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return VSA_ERR_INVALID_ARG;
+  const int n_q = shape->n_pad / bq, n_k = shape->n_pad / bk;
+  if (n_k > 1024) return VSA_ERR_UNSUPPORTED;
+  const int rows = shape->B * shape->H * n_q;
+  vsa::mask_to_lists_kernel<<<(rows + 7) / 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(mask, rows, n_k, counts,
+                                                                                          idx);
+  return launch_status();
+}
+
+size_t vsa_select_micro_workspace_bytes(const vsa_shape *shape, const vsa_micro_params *params) {
+  if (!shape_ok(shape) || !micro_params_ok(params)) return 0;
+  return micro_layout(shape, params).total;
+}
+
+vsa_status vsa_select_micro(const float *q_pool64, const float *k_pool16, const int32_t *counts, const int32_t *idx,
+                            const vsa_shape *shape, int bq, int bk, float scale, const vsa_micro_params *params,
+                            int32_t *m_counts, int32_t *m_idx, void *workspace, size_t workspace_bytes,
+                            void *stream) {
+  if (!shape_ok(shape) || !q_pool64 || !k_pool16 || !counts || !idx || !m_counts || !m_idx || !workspace)
+    return VSA_ERR_INVALID_ARG;
+  if (!micro_params_ok(params)) return VSA_ERR_INVALID_ARG;
+  if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return VSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(q_pool64) || !aligned16(k_pool16) || !aligned16(workspace)) return VSA_ERR_INVALID_ARG;
+  const MicroLayout L = micro_layout(shape, params);
+  if (workspace_bytes < L.total) return VSA_ERR_INVALID_ARG;
+  const int n_q = shape->n_pad / bq, n_k = shape->n_pad / bk;
+  if (n_k > 1024) return VSA_ERR_UNSUPPORTED;
+  const int BH = shape->B * shape->H;
+  const int n_r = shape->n_pad / vsa::kMicroRows, n_t = shape->n_pad / vsa::kMicroKeys;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t *ws8 = static_cast<uint8_t *>(workspace);
+  vsa::MicroWs ws;
+  ws.slot_of_bh = reinterpret_cast<int32_t *>(ws8 + L.off_slot);
+  ws.bitmap = reinterpret_cast<uint32_t *>(ws8 + L.off_bitmap);
+  ws.keys = reinterpret_cast<uint32_t *>(ws8 + L.off_keys);
+  ws.hist = reinterpret_cast<uint32_t *>(ws8 + L.off_hist);
+  ws.state = reinterpret_cast<uint32_t *>(ws8 + L.off_state);
+  ws.n_slots = L.n_slots;
+
+  std::vector<int32_t> slot((size_t)BH, -1);
+  int next = 0;
+  for (int b = 0; b < shape->B; ++b)
+    for (int h = 0; h < shape->H; ++h)
+      if (params->head_enable == nullptr || params->head_enable[h]) slot[(size_t)b * shape->H + h] = next++;
+  if (cudaMemcpyAsync(ws.slot_of_bh, slot.data(), slot.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return VSA_ERR_CUDA;
+  if (L.n_slots == 0) {
+    if (cudaMemsetAsync(m_counts, 0, (size_t)BH * n_r * 4, st) != cudaSuccess) return VSA_ERR_CUDA;
+    return VSA_OK;
+  }
+  if (cudaMemsetAsync(ws8 + L.off_hist, 0, L.total - L.off_hist, st) != cudaSuccess) return VSA_ERR_CUDA;
+
+  vsa::micro_bitmap_kernel<<<dim3(n_q, BH), 128, 0, st>>>(counts, idx, n_q, n_k, BH, ws);
+  vsa::ScoreArgs sa{q_pool64, k_pool16, n_r, n_t, n_q, bq, bk, shape->n_valid, scale, params->mode == 2 ? 1 : 0};
+  dim3 sg((n_t + vsa::kScoreBN - 1) / vsa::kScoreBN, (n_r + vsa::kScoreBM - 1) / vsa::kScoreBM, BH);
+  if (shape->d == 128)
+    vsa::micro_score_kernel<128><<<sg, vsa::kScoreThreads, 0, st>>>(sa, ws);
+  else
+    vsa::micro_score_kernel<64><<<sg, vsa::kScoreThreads, 0, st>>>(sa, ws);
+  const unsigned rows_blocks = (unsigned)(((size_t)BH * n_r + 7) / 8);
+  if (params->mode == 1) {
+    vsa::micro_topk_kernel<<<rows_blocks, 256, 0, st>>>(ws, n_r, n_t, BH, params->topk, params->row_capacity,
+                                                      m_counts, m_idx);
+  } else {
+    const size_t per_slot = (size_t)n_r * n_t;
+    vsa::micro_find_kernel<<<L.n_slots, 32, 0, st>>>(ws, params->percentile, 0);
+    vsa::micro_hist_kernel<<<dim3(256, L.n_slots), 256, 0, st>>>(ws, per_slot, 1);
+    vsa::micro_find_kernel<<<L.n_slots, 32, 0, st>>>(ws, params->percentile, 1);
+    vsa::micro_hist_kernel<<<dim3(256, L.n_slots), 256, 0, st>>>(ws, per_slot, 2);
+    vsa::micro_find_kernel<<<L.n_slots, 32, 0, st>>>(ws, params->percentile, 2);
+    vsa::micro_compact_kernel<<<rows_blocks, 256, 0, st>>>(ws, n_r, n_t, BH, params->row_capacity, m_counts, m_idx);
+  }
+  return launch_status();
+}
+
+vsa_status vsa_block_sparse_fwd(const void *q, const void *k, const void *v, const vsa_shape *shape, int list_rows,
+                                int seg_keys, const int32_t *counts, const int32_t *idx, int idx_stride, float scale,
+                                void *o, int o_fp32, float *lse, const float *merge_o, const float *merge_lse,
+                                void *stream) {
+  if (!shape_ok(shape) || !q || !k || !v || !counts || !idx || !o || !lse) return VSA_ERR_INVALID_ARG;
+  if (list_rows != 64 && list_rows != 128) return VSA_ERR_INVALID_ARG;
+  if (seg_keys != 16 && seg_keys != 32 && seg_keys != 64 && seg_keys != 128) return VSA_ERR_INVALID_ARG;
+  if (idx_stride < 1 || !(scale > 0.f) || !std::isfinite(scale)) return VSA_ERR_INVALID_ARG;
+  if ((merge_o == nullptr) != (merge_lse == nullptr)) return VSA_ERR_INVALID_ARG;
+  if (merge_o && static_cast<const void *>(merge_o) == o) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (merge_o && !aligned16(merge_o)))
+    return VSA_ERR_INVALID_ARG;
+  AttnArgs a;
+  a.n_pad = shape->n_pad;
+  a.n_valid = shape->n_valid;
+  a.list_rows = list_rows;
+  a.seg_keys = seg_keys;
+  a.seg_shift = ilog2(seg_keys);
+  a.idx_stride = idx_stride;
+  a.counts = counts;
+  a.idx = idx;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.o = o;
+  a.o_fp32 = o_fp32 ? 1 : 0;
+  a.lse = lse;
+  a.merge_o = merge_o;
+  a.merge_lse = merge_lse;
+  a.timeout_ns = kWaitLimitNs;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return shape->d == 128 ? launch_attn<128>(q, k, v, shape, a, st) : launch_attn<64>(q, k, v, shape, a, st);
+}
+
+vsa_status vsa_lse_merge(const float *o_a, const float *lse_a, const float *o_b, const float *lse_b,
+                         const vsa_shape *shape, void *o_out, int o_out_fp32, float *lse_out, void *stream) {
+  if (!shape_ok(shape) || !o_a || !lse_a || !o_b || !lse_b || !o_out || !lse_out) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(o_a) || !aligned16(o_b) || !aligned16(o_out)) return VSA_ERR_INVALID_ARG;
+  const size_t rows = (size_t)shape->B * shape->H * shape->n_pad;
+  const unsigned blocks = (unsigned)((rows + 7) / 8);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (shape->d == 128)
+    vsa::lse_merge_kernel<128><<<blocks, 256, 0, st>>>(o_a, lse_a, o_b, lse_b, rows, o_out, o_out_fp32, lse_out);
+  else
+    vsa::lse_merge_kernel<64><<<blocks, 256, 0, st>>>(o_a, lse_a, o_b, lse_b, rows, o_out, o_out_fp32, lse_out);
+  return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,242 @@
+/*
+ * vsa.h -- C ABI of libvsa, block-sparse self-attention over long video-DiT
+ * token sequences on NVIDIA B200 (sm_100a).
+ *
+ * The path, one call per step:
+ *   vsa_pool_qk          block means of Q and K                     (pooling)
+ *   vsa_select_blocks    per-head block mask from the pooled scores (selection)
+ *   vsa_block_sparse_fwd attention over the kept tiles -> O, LSE    (Macro / Micro pass)
+ *   vsa_select_micro     Micro tiles inside omitted blocks          (Micro selection)
+ *   vsa_block_sparse_fwd again on the Micro lists, merged by LSE    (Micro pass + merge)
+ * plus vsa_mask_to_lists (an explicit block mask instead of selection) and
+ * vsa_lse_merge (the stand-alone exact merge).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout.   Q, K, V, O are contiguous row-major [B, H, n_pad, d]: token rows of
+ *           one (batch, head) are consecutive, d is innermost.  Tokens are in
+ *           the video's frame-first (t, y, x) order; blocks are consecutive
+ *           token ranges of that order.  Rows n_valid <= row < n_pad are
+ *           padding: their Q/K/V content is never read into a result, their
+ *           O is written as 0 and their LSE as -inf.
+ * Pointers. Every tensor pointer is a DEVICE pointer (cudaMalloc'd or
+ *           equivalent) unless stated otherwise; the caller allocates and
+ *           owns every buffer, including workspaces.  The library allocates
+ *           no device memory and never synchronises the stream, except
+ *           vsa_read_device_status.  ``stream`` is a cudaStream_t (NULL =
+ *           legacy default stream).  All work is enqueued asynchronously.
+ * Errors.   Argument errors are detected on the host before anything is
+ *           enqueued and returned synchronously (VSA_ERR_INVALID_ARG /
+ *           VSA_ERR_UNSUPPORTED); a failed launch returns VSA_ERR_CUDA.
+ *           Conditions found on the device (a list longer than its capacity,
+ *           an out-of-range index in a caller-given list, a pipeline wait that
+ *           ran out of its time limit) are latched into a device status word
+ *           that vsa_read_device_status returns and clears.
+ * Numerics. Pooling, pooled scores and selection are fp32 (FFMA; no TF32).
+ *           Attention multiplies bf16 operands on the tensor cores with fp32
+ *           accumulation; P is rounded to bf16 before the P.V product; LSE is
+ *           fp32, natural log, softmax scale included.
+ *
+ * Sources (pages by title, section / equation):
+ *   [HVA]   HyperVAttention: Efficient Sparse Attention with Spatio-Temporal
+ *           Clustering for Video Diffusion (arXiv 2607.03012v1)
+ *   [HyMoR] HyMoR-Attn: Granularity-Matched Repair of Omitted Attention
+ *           Support for Video Diffusion (abstract)
+ *   [RSA]   Rectified SpaAttn: Revisiting Attention Sparsity for Efficient
+ *           Video Generation (abstract)
+ *   [LVSA]  Long Video Sparse Attention (abstract on the "FreqFormer" page)
+ *   [MOD]   MOD-DiT (arXiv 2601.11641), "Block-wise Attention Computation"
+ */
+#ifndef VSA_H_
+#define VSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define VSA_API __attribute__((visibility("default")))
+#else
+#define VSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VSA_OK = 0,
+  VSA_ERR_INVALID_ARG = 1,   /* null pointer, bad size or inconsistent shape      */
+  VSA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d not in {64,128}) */
+  VSA_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed                   */
+  VSA_ERR_CAPACITY = 4,      /* device: a list exceeded its caller-given capacity   */
+  VSA_ERR_BAD_INDEX = 5,     /* device: a caller-given list holds an invalid index  */
+  VSA_ERR_TIMEOUT = 6        /* device: a pipeline wait exceeded its time limit     */
+} vsa_status;
+
+/* Problem shape.  d in {64, 128}; n_valid <= n_pad; n_pad a multiple of 128. */
+typedef struct {
+  int B, H;
+  int n_valid;   /* real tokens per (batch, head)                     */
+  int n_pad;     /* padded row count of every [B, H, n_pad, *] tensor */
+  int d;         /* head dimension                                    */
+} vsa_shape;
+
+/* Block selection knobs ([HVA] section 2 Eq. (3), App. A.1 "Min-kc"; [LVSA]).
+ *   fixed_k > 0 : keep exactly min(fixed_k, n_k) blocks per row, cum_mass ignored.
+ *   otherwise   : keep max(k_min, m_p) blocks, m_p = the smallest m whose top-m
+ *                 size-weighted pooled probabilities sum to at least cum_mass
+ *                 (cum_mass <= 0 disables Top-p, leaving the k_min floor).
+ *   n_anchor    : add the key-block columns (anchor_rot + t*floor(n_k/n_anchor))
+ *                 mod n_k, t = 0..n_anchor-1, to every non-empty row.        */
+typedef struct {
+  int k_min;
+  float cum_mass;
+  int fixed_k;
+  int n_anchor;
+  int anchor_rot;
+} vsa_select_params;
+
+/* Micro selection knobs ([HyMoR] abstract: a fine residual over tiles inside
+ * omitted blocks, chosen online).  Micro rows are 64 query rows, Micro tiles
+ * 16 keys; a tile is a candidate for a Micro row iff it lies in a key block the
+ * row's Macro query block omitted and holds at least one valid key.  Score =
+ * mean(Q rows of the Micro row) . mean(K rows of the tile) * scale.
+ *   mode 1 : per Micro row, the min(topk, #candidates) highest scores
+ *            (ties to the lower tile index); 1 <= topk <= 32.
+ *   mode 2 : per enabled head, every candidate whose score is strictly above
+ *            tau = the ceil(percentile * M)-th smallest of the head's M
+ *            candidate scores (ceil evaluated in IEEE double).
+ *   head_enable : HOST array of H flags (NULL = every head); disabled heads
+ *            select nothing.
+ *   row_capacity : entries per Micro row in m_idx (>= 1).                   */
+typedef struct {
+  int mode;
+  int topk;
+  double percentile;
+  const uint8_t *head_enable;
+  int row_capacity;
+} vsa_micro_params;
+
+/* Human-readable name of a status code (static storage). */
+VSA_API const char *vsa_status_string(vsa_status s);
+
+/* Library version as major*10000 + minor*100 + patch. */
+VSA_API int vsa_version(void);
+
+/* Synchronise ``stream``, then return and clear the device status word (the
+ * first device-side error latched since the last call; VSA_OK if none).   */
+VSA_API vsa_status vsa_read_device_status(void *stream);
+
+/* ---------------------------------------------------------------------------
+ * a1 Pooling  ([RSA]: pooled query-key interactions; [HVA] section 4.1: a
+ * centroid is the mean of its tokens; [MOD]: fixed non-overlapping blocks.)
+ *
+ * q, k      : bf16 [B, H, n_pad, d].
+ * bq, bk    : Macro query / key block rows, each in {64, 128}.
+ * q_pool    : fp32 [B, H, n_pad/bq, d]  mean of the valid Q rows of each block.
+ * k_pool    : fp32 [B, H, n_pad/bk, d]  mean of the valid K rows of each block.
+ * q_pool64  : fp32 [B, H, n_pad/64, d]  Micro-row means (NULL to skip).
+ * k_pool16  : fp32 [B, H, n_pad/16, d]  Micro-tile means (NULL to skip).
+ * A block without a valid row has mean 0.  One pass reads Q and K once.
+ * ------------------------------------------------------------------------- */
+VSA_API vsa_status vsa_pool_qk(const void *q, const void *k, const vsa_shape *shape, int bq, int bk,
+                       float *q_pool, float *k_pool, float *q_pool64, float *k_pool16, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * a2 + a3 Scoring and selection ([HVA] section 2 Eq. (2) and Eq. (3);
+ * App. A.1 "Min-kc"; [LVSA] rotating anchors.)
+ *
+ * Per (b, h, query block i): S_ij = q_pool_i . k_pool_j * scale;
+ * P'_ij = s_j exp(S_ij) / sum_o s_o exp(S_io) with s_j the number of valid keys
+ * of block j; blocks ranked by descending S_ij + ln s_j (ties to the lower j);
+ * kept = the rule of vsa_select_params.  A query block without a valid row
+ * keeps nothing.
+ *
+ * n_k = n_pad/bk must be <= 1024.
+ * counts : int32 [B, H, n_pad/bq]           kept blocks per row.
+ * idx    : int32 [B, H, n_pad/bq, n_k]      kept key-block indices, ascending,
+ *          in the first counts[row] slots of the row (the rest is untouched).
+ * mask   : uint8 [B, H, n_pad/bq, n_k] dense 0/1 block mask, or NULL.
+ * ------------------------------------------------------------------------- */
+VSA_API vsa_status vsa_select_blocks(const float *q_pool, const float *k_pool, const vsa_shape *shape, int bq,
+                             int bk, float scale, const vsa_select_params *params, int32_t *counts,
+                             int32_t *idx, uint8_t *mask, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Explicit block mask -> lists (the mask-passed-in path of the same
+ * attention, [HVA] section 2: m_ij = 1 iff key block j is attended by row i).
+ *
+ * mask   : uint8 [B, H, n_pad/bq, n_pad/bk], nonzero = keep.  n_pad/bk <= 1024.
+ * counts, idx : as vsa_select_blocks (idx row stride n_pad/bk).
+ * ------------------------------------------------------------------------- */
+VSA_API vsa_status vsa_mask_to_lists(const uint8_t *mask, const vsa_shape *shape, int bq, int bk, int32_t *counts,
+                             int32_t *idx, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * a5 Micro selection ([HyMoR] abstract: online selection of the omitted tail
+ * at fine granularity; readings in vsa_micro_params.)
+ *
+ * q_pool64, k_pool16 : from vsa_pool_qk.
+ * counts, idx        : the Macro lists (row = Macro query block of bq rows,
+ *                      idx row stride n_pad/bk).
+ * m_counts : int32 [B, H, n_pad/64]                   tiles per Micro row.
+ * m_idx    : int32 [B, H, n_pad/64, row_capacity]     16-key tile indices,
+ *            ascending.  A row with more selected tiles than row_capacity
+ *            keeps the lowest row_capacity of them and latches
+ *            VSA_ERR_CAPACITY.
+ * workspace: device scratch of vsa_select_micro_workspace_bytes() bytes,
+ *            16-byte aligned; its content on entry is irrelevant.
+ * ------------------------------------------------------------------------- */
+VSA_API size_t vsa_select_micro_workspace_bytes(const vsa_shape *shape, const vsa_micro_params *params);
+
+VSA_API vsa_status vsa_select_micro(const float *q_pool64, const float *k_pool16, const int32_t *counts,
+                            const int32_t *idx, const vsa_shape *shape, int bq, int bk, float scale,
+                            const vsa_micro_params *params, int32_t *m_counts, int32_t *m_idx,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * a4 / a6 Block-sparse attention forward ([HVA] section 2 Eq. (4): attention of
+ * each query block restricted to its selected key blocks; section 4.3: the
+ * selected key blocks of a row are walked as one packed sequence.  [HyMoR]
+ * abstract: Micro pass merged with the Macro output by exact LSE merging.)
+ *
+ * For every list row r (list_rows consecutive query rows) and every entry e of
+ * its list, the keys [idx[r][e]*seg_keys, idx[r][e]*seg_keys + seg_keys) are
+ * attended: O = softmax(Q K^T * scale) V over the union of the row's
+ * segments, keys >= n_valid excluded; LSE = ln sum exp(Q K^T * scale).
+ *   Macro pass : list_rows = bq, seg_keys = bk, lists from vsa_select_blocks.
+ *   Micro pass : list_rows = 64, seg_keys = 16, lists from vsa_select_micro.
+ * list_rows in {64, 128}; seg_keys in {16, 32, 64, 128}; entries of a row
+ * strictly ascending and < n_pad/seg_keys (violations latch
+ * VSA_ERR_BAD_INDEX and the row's output is undefined).
+ *
+ * counts    : int32 [B, H, n_pad/list_rows];  idx : int32 [.., idx_stride].
+ * o         : [B, H, n_pad, d], bf16 (o_fp32 = 0) or fp32 (o_fp32 = 1).
+ * lse       : fp32 [B, H, n_pad].
+ * merge_o, merge_lse : NULL, or an fp32 [B, H, n_pad, d] output and its fp32
+ *             LSE over a key support disjoint from this pass's; then o/lse
+ *             receive the exact merge L = ln(e^{L_1} + e^{L_2}),
+ *             O = e^{L_1-L} O_1 + e^{L_2-L} O_2 (a row with an empty list
+ *             passes merge_o through).  o may not alias merge_o.
+ * A row with an empty list and no merge input gets O = 0, LSE = -inf.
+ * ------------------------------------------------------------------------- */
+VSA_API vsa_status vsa_block_sparse_fwd(const void *q, const void *k, const void *v, const vsa_shape *shape,
+                                int list_rows, int seg_keys, const int32_t *counts, const int32_t *idx,
+                                int idx_stride, float scale, void *o, int o_fp32, float *lse,
+                                const float *merge_o, const float *merge_lse, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Stand-alone exact LSE merge of two attention results over disjoint key
+ * supports ([HyMoR] abstract).  o_a, o_b fp32 [B, H, n_pad, d]; lse_* fp32
+ * [B, H, n_pad]; o_out bf16 or fp32 (o_out_fp32); lse_out fp32.  Rows with
+ * both LSE = -inf give O = 0, LSE = -inf.  Outputs may alias inputs of the
+ * same type.
+ * ------------------------------------------------------------------------- */
+VSA_API vsa_status vsa_lse_merge(const float *o_a, const float *lse_a, const float *o_b, const float *lse_b,
+                         const vsa_shape *shape, void *o_out, int o_out_fp32, float *lse_out, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSA_H_ */

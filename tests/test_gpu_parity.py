@@ -1,0 +1,345 @@
+"""GPU parity of every step of the path against the fp64 CPU oracle.
+
+All calls go through the C ABI (libvsa.so via the ctypes binding).  Inputs
+are the seeded workloads of video_inputs; lists fed to the attention kernel in
+the isolated attention tests come from the oracle, never the other way round.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_pool_b200 as vsa
+import oracle as orc
+from video_inputs import WORKLOADS, make_qkv, micro_heads, round_to_bf16, sweep_points
+
+from gpu_helpers import (GAP, LSE_TOL, O_TOL, assert_close_rows, compare_selection, oracle_select_per_head,
+                         sample_blocks, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from block_sparse_attention_pool_b200 import build
+    build.build()
+    vsa.lib()
+    torch.cuda.init()
+    yield
+    assert vsa.read_device_status() == 0
+
+
+_CACHE = {}
+
+
+def inputs(name, heads=None):
+    key = (name, heads)
+    if key not in _CACHE:
+        w = WORKLOADS[name]
+        _CACHE[key] = make_qkv(w, heads=heads)
+    return _CACHE[key]
+
+
+def shape_for(w, H=None):
+    return vsa.Shape(w.B, w.H if H is None else H, w.n_valid, w.n_pad, w.d)
+
+
+def lists_to_dev(kept, n_k, B, H, n_q):
+    counts = np.zeros((B, H, n_q), dtype=np.int32)
+    idx = np.zeros((B, H, n_q, n_k), dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            for i in range(n_q):
+                row = np.asarray(kept[b][h][i], dtype=np.int32)
+                counts[b, h, i] = row.size
+                idx[b, h, i, :row.size] = row
+    return torch.from_numpy(counts).cuda(), torch.from_numpy(idx).cuda()
+
+
+# ---------------------------------------------------------------------------
+# a1 pooling
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name,heads", [("tiny", None), ("wan13b", (0, 3)), ("hunyuan", (0, 2))])
+def test_pool_matches_oracle(name, heads):
+    w = WORKLOADS[name]
+    q, k, _ = inputs(name, heads)
+    H = q.shape[1]
+    shape = shape_for(w, H)
+    dq, dk = to_dev(q), to_dev(k)
+    f = lambda n: torch.empty(w.B, H, w.n_pad // n, w.d, device="cuda", dtype=torch.float32)
+    qp, kp, q64, k16 = f(w.bq), f(w.bk), f(64), f(16)
+    vsa.pool_qk(dq, dk, shape, w.bq, w.bk, qp, kp, q64, k16)
+    torch.cuda.synchronize()
+    for got, x, blk in ((qp, q, w.bq), (kp, k, w.bk), (q64, q, 64), (k16, k, 16)):
+        want = orc.pool_block_means(x, blk, w.n_valid)
+        err = np.abs(got.cpu().numpy().astype(np.float64) - want).max()
+        assert err < 2e-5, (name, blk, err)
+
+
+# ---------------------------------------------------------------------------
+# a2 + a3 selection
+# ---------------------------------------------------------------------------
+
+def _gpu_select(w, q, k, with_mask=False):
+    H = q.shape[1]
+    shape = shape_for(w, H)
+    dq, dk = to_dev(q), to_dev(k)
+    n_q, n_k = w.n_pad // w.bq, w.n_pad // w.bk
+    qp = torch.empty(w.B, H, n_q, w.d, device="cuda")
+    kp = torch.empty(w.B, H, n_k, w.d, device="cuda")
+    vsa.pool_qk(dq, dk, shape, w.bq, w.bk, qp, kp)
+    counts = torch.empty(w.B, H, n_q, dtype=torch.int32, device="cuda")
+    idx = torch.full((w.B, H, n_q, n_k), -7, dtype=torch.int32, device="cuda")
+    mask = torch.empty(w.B, H, n_q, n_k, dtype=torch.uint8, device="cuda") if with_mask else None
+    vsa.select_blocks(qp, kp, shape, w.bq, w.bk, w.scale,
+                      vsa.SelectParams(w.k_min, w.cum_mass, w.fixed_k, w.n_anchor, w.anchor_rot), counts, idx, mask)
+    torch.cuda.synchronize()
+    return counts.cpu().numpy(), idx.cpu().numpy(), (mask.cpu().numpy() if with_mask else None)
+
+
+@pytest.mark.parametrize("name,heads", [("tiny", None), ("wan13b", None), ("wan14b", (0, 4)), ("hunyuan", (0, 4))])
+def test_select_blocks_bit_exact(name, heads):
+    w = WORKLOADS[name]
+    q, k, _ = inputs(name, heads)
+    counts, idx, mask = _gpu_select(w, q, k, with_mask=True)
+    kept, info, logw, probs, _, _ = oracle_select_per_head(q, k, w)
+    n_exact, n_near, n_1e3 = compare_selection(counts, idx, kept, info, logw, probs, w, gpu_mask=mask)
+    print(f"\n{name}: rows bit-exact {n_exact}, near-tie rows validity-checked {n_near}, gap<1e-3 rows {n_1e3}")
+    assert n_exact >= 0.8 * (n_exact + n_near)
+
+
+@pytest.mark.parametrize("point", [0, 4, 5, 9])
+def test_select_sweep_points(point):
+    frac, w = sweep_points()[point]
+    q, k, _ = inputs("hunyuan", (0, 2))
+    counts, idx, _ = _gpu_select(w, q, k)
+    kept, info, logw, probs, _, _ = oracle_select_per_head(q, k, w)
+    n_exact, n_near, _ = compare_selection(counts, idx, kept, info, logw, probs, w)
+    assert n_exact >= 0.8 * (n_exact + n_near)
+    n_q_valid = (w.n_valid + w.bq - 1) // w.bq
+    assert np.all(counts[:, :, :n_q_valid] == min(w.fixed_k, w.n_k))
+    assert np.all(counts[:, :, n_q_valid:] == 0)            # query blocks without a valid row keep nothing
+
+
+def test_mask_to_lists_bit_exact():
+    rng = np.random.default_rng(5)
+    B, H, n = 1, 3, 700                       # 64-row blocks, n_pad = 44,800
+    m = (rng.random((B, H, n, n)) < 0.3).astype(np.uint8)
+    m[0, 0, 0] = 0
+    m[0, 1, 1] = 1
+    m[0, 2, 2] = 7                            # any nonzero byte means kept
+    shape = vsa.Shape(B, H, n * 64, n * 64, 128)
+    counts = torch.empty(B, H, n, dtype=torch.int32, device="cuda")
+    idx = torch.empty(B, H, n, n, dtype=torch.int32, device="cuda")
+    vsa.mask_to_lists(torch.from_numpy(m).cuda(), shape, 64, 64, counts, idx)
+    c, ix = counts.cpu().numpy(), idx.cpu().numpy()
+    for h in range(H):
+        for i in range(n):
+            want = np.nonzero(m[0, h, i])[0]
+            assert c[0, h, i] == want.size and np.array_equal(ix[0, h, i, :want.size], want)
+
+
+# ---------------------------------------------------------------------------
+# a4 attention over given lists (oracle lists -> GPU)
+# ---------------------------------------------------------------------------
+
+def _attention_case(w, q, k, v, kept, blocks, o_fp32=False):
+    B, H = q.shape[0], q.shape[1]
+    n_q, n_k = w.n_pad // w.bq, w.n_pad // w.bk
+    counts, idx = lists_to_dev(kept, n_k, B, H, n_q)
+    shape = vsa.Shape(B, H, w.n_valid, w.n_pad, w.d)
+    o = torch.empty(B, H, w.n_pad, w.d, device="cuda", dtype=torch.float32 if o_fp32 else torch.bfloat16)
+    lse = torch.empty(B, H, w.n_pad, device="cuda")
+    vsa.block_sparse_fwd(to_dev(q), to_dev(k), to_dev(v), shape, w.bq, w.bk, counts, idx, n_k, w.scale, o, lse)
+    assert vsa.read_device_status() == 0
+    Og = o.float().cpu().numpy()
+    Lg = lse.cpu().numpy()
+    O, L = orc.block_sparse_attention(q, k, v, kept, w.bq, w.bk, w.n_valid, w.scale, rows=blocks)
+    rows = [(b, h, i * w.bq, (i + 1) * w.bq) for b, h, i in blocks]
+    return assert_close_rows(Og, Lg, O, L, rows)
+
+
+def test_attention_tiny_all_rows():
+    w = WORKLOADS["tiny"]
+    q, k, v = inputs("tiny")
+    kept, *_ = oracle_select_per_head(q, k, w)
+    blocks = [(0, h, i) for h in range(w.H) for i in range(w.n_q)]
+    print("\ntiny attention worst |dO|, |dLSE|:", _attention_case(w, q, k, v, kept, blocks))
+
+
+def test_attention_dense_equals_full_attention():
+    w = WORKLOADS["wan13b"]
+    q, k, v = inputs("wan13b", (0, 1))
+    n_q, n_k = w.n_pad // w.bq, w.n_pad // w.bk
+    kept = [[[np.arange(n_k) for _ in range(n_q)]]]
+    blocks = [(0, 0, 0), (0, 0, 100), (0, 0, n_q - 1)]
+    print("\ndense worst:", _attention_case(w, q, k, v, kept, blocks, o_fp32=True))
+
+
+@pytest.mark.parametrize("name", ["wan13b", "wan14b", "hunyuan"])
+def test_attention_sampled_rows(name):
+    w = WORKLOADS[name]
+    q, k, v = inputs(name, (0, 2))
+    kept, *_ = oracle_select_per_head(q, k, w)
+    blocks = sample_blocks(w, 6, seed=1, heads=2)
+    print(f"\n{name} attention worst:", _attention_case(w, q, k, v, kept, blocks))
+
+
+@pytest.mark.parametrize("point", [1, 6, 9])
+def test_attention_sweep_points(point):
+    frac, w = sweep_points()[point]
+    q, k, v = inputs("hunyuan", (0, 1))
+    kept, *_ = oracle_select_per_head(q, k, w)
+    blocks = sample_blocks(w, 4, seed=2, heads=1)
+    print(f"\nsweep {w.name} worst:", _attention_case(w, q, k, v, kept, blocks))
+
+
+def test_attention_ragged_and_empty_rows():
+    """n_valid not a multiple of the block, a row with an empty list, lists of
+    different lengths in one 128-row tile (64-row lists), 32-key segments."""
+    rng = np.random.default_rng(9)
+    B, H, n_pad, d, n_valid = 1, 2, 512, 128, 437
+    q, k, v = (round_to_bf16(rng.standard_normal((B, H, n_pad, d)).astype(np.float32)) for _ in range(3))
+    for x in (q, k, v):
+        x[:, :, n_valid:] = 0
+    for list_rows, seg in ((128, 32), (64, 32), (64, 128), (128, 16)):
+        n_l, n_s = n_pad // list_rows, n_pad // seg
+        kept = [[[np.sort(rng.choice(n_s, size=int(rng.integers(0, n_s // 2 + 1)), replace=False))
+                  for _ in range(n_l)] for _ in range(H)]]
+        kept[0][0][1] = np.zeros(0, dtype=np.int64)
+        counts, idx = lists_to_dev(kept, n_s, B, H, n_l)
+        shape = vsa.Shape(B, H, n_valid, n_pad, d)
+        o = torch.empty(B, H, n_pad, d, device="cuda")
+        lse = torch.empty(B, H, n_pad, device="cuda")
+        scale = 1 / math.sqrt(d)
+        vsa.block_sparse_fwd(to_dev(q), to_dev(k), to_dev(v), shape, list_rows, seg, counts, idx, n_s, scale, o, lse)
+        assert vsa.read_device_status() == 0
+        mask = orc.token_mask(kept, None, n_pad, list_rows, seg, n_valid)
+        O, L = orc.masked_attention_bruteforce(q, k, v, mask, scale)
+        assert_close_rows(o.cpu().numpy(), lse.cpu().numpy(), O, L, [(0, h, 0, n_pad) for h in range(H)])
+
+
+def test_attention_bad_list_latches_status():
+    B, H, n_pad, d = 1, 1, 256, 128
+    q = torch.zeros(B, H, n_pad, d, device="cuda", dtype=torch.bfloat16)
+    counts = torch.tensor([[[2, 1]]], dtype=torch.int32, device="cuda")
+    idx = torch.tensor([[[[1, 0], [5, 0]]]], dtype=torch.int32, device="cuda")   # descending; out of range
+    o = torch.empty(B, H, n_pad, d, device="cuda", dtype=torch.bfloat16)
+    lse = torch.empty(B, H, n_pad, device="cuda")
+    vsa.block_sparse_fwd(q, q, q, vsa.Shape(B, H, n_pad, n_pad, d), 128, 128, counts, idx, 2, 0.1, o, lse)
+    assert vsa.read_device_status() == 5
+    assert torch.all(o == 0) and torch.all(torch.isinf(lse))
+    assert vsa.read_device_status() == 0                      # reading clears it
+
+
+# ---------------------------------------------------------------------------
+# a6 merge
+# ---------------------------------------------------------------------------
+
+def test_lse_merge_kernel():
+    rng = np.random.default_rng(3)
+    B, H, n_pad, d = 1, 2, 256, 64
+    oa, ob = rng.normal(size=(2, B, H, n_pad, d)).astype(np.float32)
+    la, lb = rng.normal(scale=3, size=(2, B, H, n_pad)).astype(np.float32)
+    la[0, 0, :10] = -np.inf
+    lb[0, 0, 5:15] = -np.inf
+    O, L = orc.lse_merge(oa, la, ob, lb)
+    t = lambda x: torch.from_numpy(x).cuda()
+    for out_dtype, tol in ((torch.float32, 1e-5), (torch.bfloat16, 1e-2)):
+        o = torch.empty(B, H, n_pad, d, device="cuda", dtype=out_dtype)
+        lo = torch.empty(B, H, n_pad, device="cuda")
+        vsa.lse_merge(t(oa), t(la), t(ob), t(lb), vsa.Shape(B, H, n_pad, n_pad, d), o, lo)
+        Lg = lo.cpu().numpy()
+        assert np.abs(o.float().cpu().numpy() - O).max() < tol
+        fin = np.isfinite(L)
+        assert np.array_equal(np.isfinite(Lg), fin)
+        assert np.abs(Lg[fin] - L[fin]).max() < 1e-5
+
+
+# ---------------------------------------------------------------------------
+# whole path
+# ---------------------------------------------------------------------------
+
+def test_path_tiny_every_row():
+    w = WORKLOADS["tiny"]
+    q, k, v = inputs("tiny")
+    heads = micro_heads(w)
+    res = orc.forward(q, k, v, w, head_enable=heads)
+    run = vsa.SparseVideoAttention(vsa.PathConfig.from_workload(w, heads))
+    out = run(to_dev(q), to_dev(k), to_dev(v))
+    assert vsa.read_device_status() == 0
+    counts = out["counts"].cpu().numpy()
+    idx = out["idx"].cpu().numpy()
+    for h in range(w.H):
+        for i in range(w.n_q):
+            assert np.array_equal(idx[0, h, i, :counts[0, h, i]], res["kept"][0][h][i])
+    mc = out["m_counts"].cpu().numpy()
+    mi = out["m_idx"].cpu().numpy()
+    for h in range(w.H):
+        for r in range(w.n_pad // 64):
+            assert np.array_equal(mi[0, h, r, :mc[0, h, r]], res["tiles"][0][h][r]), (h, r)
+    worst = assert_close_rows(out["o"].float().cpu().numpy(), out["lse"].cpu().numpy(), res["O"], res["LSE"],
+                              [(0, h, 0, w.n_pad) for h in range(w.H)])
+    print("\ntiny path worst:", worst)
+
+
+def test_path_hunyuan_sampled():
+    """The benchmark's launch configuration: the whole hunyuan path (Macro
+    fixed 20%, Micro percentile in 6 of 24 heads) on all heads; sampled rows
+    compared with the oracle."""
+    w = WORKLOADS["hunyuan"]
+    q, k, v = inputs("hunyuan")
+    heads = micro_heads(w)
+    run = vsa.SparseVideoAttention(vsa.PathConfig.from_workload(w, heads))
+    out = run(to_dev(q), to_dev(k), to_dev(v))
+    assert vsa.read_device_status() == 0
+    counts = out["counts"].cpu().numpy()
+    idx = out["idx"].cpu().numpy()
+    mc = out["m_counts"].cpu().numpy()
+    mi = out["m_idx"].cpu().numpy()
+    Og = out["o"].float().cpu().numpy()
+    Lg = out["lse"].cpu().numpy()
+    kept, info, logw, probs, _, _ = oracle_select_per_head(q, k, w)
+    n_exact, n_near, _ = compare_selection(counts, idx, kept, info, logw, probs, w)
+    assert n_exact >= 0.8 * (n_exact + n_near)
+    # Micro selection per enabled head, tiles decided away from tau compared exactly
+    q64 = np.zeros((1, w.H, w.n_pad // 64, w.d))
+    k16 = np.zeros((1, w.H, w.n_pad // 16, w.d))
+    for h in np.nonzero(heads)[0]:
+        q64[0, h] = orc.pool_block_means(q[:, h:h + 1], 64, w.n_valid)[0, 0]
+        k16[0, h] = orc.pool_block_means(k[:, h:h + 1], 16, w.n_valid)[0, 0]
+    tiles, minfo = orc.select_micro_percentile(q64, k16, kept, w.bq, w.bk, w.n_valid, w.scale,
+                                               w.micro_percentile, heads, with_info=True)
+    for h in range(w.H):
+        if not heads[h]:
+            assert np.all(mc[0, h] == 0)
+            continue
+        inf = minfo[0][h]
+        far = inf["cand"] & (np.abs(inf["S"] - inf["tau"]) >= GAP)
+        sel_o = np.zeros_like(far)
+        for r, t in enumerate(tiles[0][h]):
+            sel_o[r, t] = True
+        sel_g = np.zeros_like(far)
+        for r in range(far.shape[0]):
+            sel_g[r, mi[0, h, r, :mc[0, h, r]]] = True
+        assert np.array_equal(sel_g[far], sel_o[far]), h
+        assert not np.any(sel_g & ~inf["cand"])
+        assert abs(int(sel_g.sum()) - int(sel_o.sum())) <= int((inf["cand"] & ~far).sum())
+    # output rows: blocks whose Macro row and both Micro rows match the oracle exactly
+    blocks = sample_blocks(w, 8, seed=4)
+    rows = []
+    for b, h, i in blocks:
+        if not np.array_equal(idx[b, h, i, :counts[b, h, i]], kept[b][h][i]):
+            continue
+        ok = all(np.array_equal(mi[b, h, r, :mc[b, h, r]], tiles[b][h][r]) for r in (2 * i, 2 * i + 1))
+        if ok:
+            rows.append((b, h, i))
+    assert len(rows) >= 4
+    O_M, L_M = orc.block_sparse_attention(q, k, v, kept, w.bq, w.bk, w.n_valid, w.scale, rows=rows)
+    mrows = [(b, h, r) for b, h, i in rows for r in (2 * i, 2 * i + 1)]
+    O_u, L_u = orc.micro_attention(q, k, v, tiles, w.n_valid, w.scale, rows=mrows)
+    O, L = orc.lse_merge(O_M, L_M, O_u, L_u)
+    worst = assert_close_rows(Og, Lg, O, L, [(b, h, i * 128, i * 128 + 128) for b, h, i in rows])
+    print("\nhunyuan path worst:", worst, "rows", rows)
