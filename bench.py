@@ -1,0 +1,438 @@
+#!/usr/bin/env python
+"""Benchmark of the block-sparse video attention path on B200.
+
+One step = one pass of the whole path over one synthetic layer: pooling ->
+pooled scoring + selection -> Macro block-sparse attention -> Micro selection
+-> Micro attention with the fused exact LSE merge.  Default workload: the
+HunyuanVideo-like 720p layer (B1 H24 N=118,800 padded to 118,912, d128,
+128x128 blocks, 20% kept per row, Micro repair above the 99th percentile in 6
+of 24 heads, heavy-tailed Q/K), bf16 inputs resident in HBM.
+
+Metric: effective TFLOP/s over the kept tiles (4*Bq*Bk*d per kept Macro tile
+plus 4*64*16*d per Micro tile, whole job over all ranks) with ms per step,
+the fraction of the measured bf16 tensor peak, and the speedup over the same
+attention kernel run with every block kept (dense).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own full layer
+(independent problems, no data-path collective; weak scaling); the step time
+is the max over ranks.  --impl reference times the fp64 CPU oracle on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from video_inputs import WORKLOADS, make_qkv, micro_heads  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+METRIC = "block-sparse attn ms & effective TFLOP/s (% bf16 peak), speedup vs dense, 1xB200"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16": d["bf16_tflops"], "bf16_sustained": d["bf16_tflops_sustained"],
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+def workload_label(w):
+    T, Y, X = w.grid
+    s = (f"{w.name}: B{w.B} H{w.H} d{w.d} grid {T}x{Y}x{X} N={w.n_valid} (pad {w.n_pad}) "
+         f"blocks {w.bq}x{w.bk}")
+    if w.fixed_k:
+        s += f" keep k={w.fixed_k}/{w.n_pad // w.bk}"
+    if w.cum_mass > 0:
+        s += f" cum-mass {w.cum_mass} k_min {w.k_min}"
+    if w.n_anchor:
+        s += f" + {w.n_anchor} anchors"
+    if w.micro_mode == 2:
+        s += f" + Micro 64x16 tiles > p{int(w.micro_percentile * 100)} in {int(micro_heads(w).sum())}/{w.H} heads"
+    elif w.micro_mode == 1:
+        s += f" + Micro top-{w.micro_topk} 64x16 tiles"
+    return s
+
+
+# ---------------------------------------------------------------------------
+# clocks sampling during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# FLOP accounting (algorithmic, over kept tiles)
+# ---------------------------------------------------------------------------
+
+def macro_flops(counts: torch.Tensor, w) -> float:
+    """4 * Bq * Bk * d per kept (query block, key block) pair."""
+    return 4.0 * w.bq * w.bk * w.d * float(counts.sum().item())
+
+
+def micro_flops(m_counts: torch.Tensor, w) -> float:
+    return 4.0 * 64 * 16 * w.d * float(m_counts.sum().item())
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_gpu(args, rank, world, local_rank):
+    import block_sparse_attention_pool_b200 as vsa
+    from block_sparse_attention_pool_b200 import build as vsa_build
+
+    if rank == 0 or not os.path.exists(vsa_build.LIB):
+        vsa_build.build()
+    if world > 1:
+        torch.distributed.barrier()
+    vsa.lib()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    heads = micro_heads(w)
+    q, k, v = make_qkv(w)
+    to_dev = lambda x: torch.from_numpy(x).to(dev).to(torch.bfloat16).contiguous()
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    pin = lambda x: torch.from_numpy(x).to(torch.bfloat16).pin_memory()
+    hq, hk, hv = pin(q), pin(k), pin(v)
+    del q, k, v
+    cfg = vsa.PathConfig.from_workload(w, heads if w.micro_mode else None)
+    run = vsa.SparseVideoAttention(cfg)
+    stream = torch.cuda.current_stream(dev)
+
+    # the dominant kernel (Macro attention) is timed by events around its own
+    # launch inside every step, on the launching stream
+    macro_ev = []
+
+    def run_with_events(qq, kk, vv):
+        c = run.cfg
+        run._alloc(qq)
+        b = run.buf
+        B, H, n_pad, d = qq.shape
+        shape = vsa.Shape(B, H, c.n_valid, n_pad, d)
+        n_k = n_pad // c.bk
+        vsa.pool_qk(qq, kk, shape, c.bq, c.bk, b["q_pool"], b["k_pool"], b.get("q_pool64"), b.get("k_pool16"))
+        vsa.select_blocks(b["q_pool"], b["k_pool"], shape, c.bq, c.bk, c.scale,
+                          vsa.SelectParams(c.k_min, c.cum_mass, c.fixed_k, c.n_anchor, c.anchor_rot), b["counts"],
+                          b["idx"])
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        if c.micro_mode:
+            vsa.block_sparse_fwd(qq, kk, vv, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, c.scale, b["o_macro"],
+                                 b["lse_macro"])
+        else:
+            vsa.block_sparse_fwd(qq, kk, vv, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, c.scale, b["o"], b["lse"])
+        e1.record(stream)
+        macro_ev.append((e0, e1))
+        if c.micro_mode:
+            vsa.select_micro(b["q_pool64"], b["k_pool16"], b["counts"], b["idx"], shape, c.bq, c.bk, c.scale,
+                             c.micro_mode, c.micro_topk, c.micro_percentile, c.micro_heads, run.micro_cap,
+                             b["m_counts"], b["m_idx"], b["workspace"])
+            vsa.block_sparse_fwd(qq, kk, vv, shape, 64, 16, b["m_counts"], b["m_idx"], run.micro_cap, c.scale, b["o"],
+                                 b["lse"], b["o_macro"], b["lse_macro"])
+        return b
+
+    # kernels launched per step by this path (pool, select, Macro; Micro:
+    # bitmap, score, 3 rank searches, 2 histograms, compaction, Micro pass)
+    launches_per_step = 3 + (9 if w.micro_mode == 2 else (3 if w.micro_mode == 1 else 0))
+
+    for _ in range(args.warmup):
+        run_with_events(dq, dk, dv)
+    torch.cuda.synchronize(dev)
+    st = vsa.read_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {vsa.status_string(st)}")
+    macro_ev.clear()
+    fl_macro = macro_flops(run.buf["counts"], w)
+    fl_micro = micro_flops(run.buf["m_counts"], w) if w.micro_mode else 0.0
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        run_with_events(dq, dk, dv)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    ms_total = t0.elapsed_time(t1)
+    macro_ms = [a.elapsed_time(b) for a, b in macro_ev]
+    st = vsa.read_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status after timed steps: {vsa.status_string(st)}")
+
+    # end to end through the public API with host buffers: H2D of Q/K/V from
+    # pinned memory, the whole path, D2H of O and LSE, every step
+    ho = torch.empty(run.buf["o"].shape, dtype=torch.bfloat16).pin_memory()
+    hl = torch.empty(run.buf["lse"].shape, dtype=torch.float32).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(e2e_steps):
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        out = run(dq, dk, dv)
+        ho.copy_(out["o"], non_blocking=True)
+        hl.copy_(out["lse"], non_blocking=True)
+    s1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = s0.elapsed_time(s1) / e2e_steps
+    h2d = 3 * hq.numel() * 2
+    d2h = ho.numel() * 2 + hl.numel() * 4
+
+    # dense reference: the same attention kernel with every key block kept
+    n_k = w.n_pad // w.bk
+    dense_cfg = vsa.PathConfig(n_valid=w.n_valid, bq=w.bq, bk=w.bk, scale=w.scale, fixed_k=n_k)
+    dense = vsa.SparseVideoAttention(dense_cfg)
+    dense(dq, dk, dv)
+    torch.cuda.synchronize(dev)
+    dense_ms_list = []
+    for _ in range(2):
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b = dense.buf
+        shape = vsa.Shape(w.B, w.H, w.n_valid, w.n_pad, w.d)
+        d0.record(stream)
+        vsa.block_sparse_fwd(dq, dk, dv, shape, w.bq, w.bk, b["counts"], b["idx"], n_k, w.scale, b["o"], b["lse"])
+        d1.record(stream)
+        torch.cuda.synchronize(dev)
+        dense_ms_list.append(d0.elapsed_time(d1))
+    dense_ms = min(dense_ms_list)
+    dense_flops = 4.0 * w.bq * w.bk * w.d * float(dense.buf["counts"].sum().item())
+    del dense
+
+    # max over ranks
+    times = torch.tensor([ms_total, e2e_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
+    ms_total, e2e_ms = times.tolist()
+    ms_step = ms_total / args.steps
+    flops_step = fl_macro + fl_micro
+    value = world * flops_step / (ms_step * 1e-3) / 1e12
+    e2e_value = world * flops_step / (e2e_ms * 1e-3) / 1e12
+    pk = peaks()
+    macro_avg_ms = statistics.mean(macro_ms)
+    achieved = fl_macro / (macro_avg_ms * 1e-3) / 1e12
+    peak = pk["bf16_sustained"]
+    line = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded video-shaped Q/K/V, no model weights)",
+        "config": {
+            "workload": workload_label(w),
+            "global_batch": w.B * world,
+            "seq_len": w.n_valid,
+            "parallelism": f"independent layer per GPU x{world}",
+            "l2": f"inputs {3 * w.B * w.H * w.n_pad * w.d * 2 / 1e9:.2f} GB > 126 MB L2 (no flush needed)",
+            "kept_fraction_macro": round(float(run.buf["counts"].sum().item()) /
+                                         (w.B * w.H * ((w.n_valid + w.bq - 1) // w.bq) * n_k), 4),
+            "micro_tiles": int(run.buf["m_counts"].sum().item()) if w.micro_mode else 0,
+        },
+        "pct_of_bf16_peak": round(100.0 * flops_step / (ms_step * 1e-3) / 1e12 / peak, 2),
+        "peak_tflops": peak,
+        "peak_source": f"{pk['source']} bf16 sustained",
+        "dense_ms": round(dense_ms, 3),
+        "dense_tflops": round(dense_flops / (dense_ms * 1e-3) / 1e12, 2),
+        "speedup_vs_dense": round(dense_ms / ms_step, 3),
+        "macro_kernel_ms": round(macro_avg_ms, 4),
+        "roofline": {
+            "kernel": "attn_fwd_kernel<128> (Macro pass)",
+            "bound": "tensor",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": None,
+        },
+        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 3),
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    return line
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (the baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(w, budget_blocks: int):
+    """Time the fp64 oracle on a bounded sample of the workload: pooling and
+    selection of one head, then Macro attention (and Micro, if any) of
+    ``budget_blocks`` query blocks of that head.  Returns (flops, seconds,
+    description)."""
+    import oracle as orc
+    q, k, v = make_qkv(w, heads=(0, 1))
+    heads = micro_heads(w)[:1]
+    t0 = time.perf_counter()
+    qbar = orc.pool_block_means(q, w.bq, w.n_valid)
+    kbar = orc.pool_block_means(k, w.bk, w.n_valid)
+    kept = orc.select_blocks(qbar, kbar, w.n_valid, w.bq, w.bk, w.scale, w.k_min, w.cum_mass, w.fixed_k,
+                             w.n_anchor, w.anchor_rot)
+    n_q = w.n_pad // w.bq
+    blocks = [(0, 0, int(i)) for i in np.linspace(0, (w.n_valid - 1) // w.bq, budget_blocks).astype(int)]
+    orc.block_sparse_attention(q, k, v, kept, w.bq, w.bk, w.n_valid, w.scale, rows=blocks)
+    flops = sum(4.0 * w.bq * w.bk * w.d * len(kept[0][0][i]) for _, _, i in blocks)
+    desc = f"1 of {w.H} heads pooled+selected, Macro attention of {len(blocks)} of {n_q} query blocks"
+    if w.micro_mode == 2 and heads[0]:
+        q64 = orc.pool_block_means(q, 64, w.n_valid)
+        k16 = orc.pool_block_means(k, 16, w.n_valid)
+        tiles = orc.select_micro_percentile(q64, k16, kept, w.bq, w.bk, w.n_valid, w.scale, w.micro_percentile,
+                                            heads)
+        mrows = [(0, 0, r) for _, _, i in blocks for r in range(i * w.bq // 64, (i + 1) * w.bq // 64)]
+        orc.micro_attention(q, k, v, tiles, w.n_valid, w.scale, rows=mrows)
+        flops += sum(4.0 * 64 * 16 * w.d * len(tiles[0][0][r]) for _, _, r in mrows)
+        desc += " + Micro selection of the head and Micro attention of their rows"
+    dt = time.perf_counter() - t0
+    return flops, dt, desc
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = WORKLOADS[args.workload]
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm state worth priming; warm-up steps are no-ops
+    tot_f, tot_s, desc = 0.0, 0.0, ""
+    for _ in range(args.steps):
+        f, s, desc = oracle_sample(w, budget_blocks=args.ref_blocks)
+        tot_f += f
+        tot_s += s
+    val = tot_f / tot_s / 1e12
+    return {
+        "metric": METRIC, "impl": "reference", "value": val, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded video-shaped Q/K/V)",
+        "config": {"workload": workload_label(w)},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle", "sample": desc},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="vsa", choices=["vsa", "reference"])
+    ap.add_argument("--workload", default="hunyuan", choices=sorted(WORKLOADS))
+    ap.add_argument("--ref-blocks", type=int, default=6, help="query blocks per oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    line = run_gpu(args, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, s, desc = oracle_sample(WORKLOADS[args.workload], budget_blocks=args.ref_blocks)
+        line["cpu_baseline"] = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                                "sample": desc, "seconds": round(s, 2)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -31,7 +31,8 @@
 
 namespace vsa {
 
-constexpr int kAttnThreads = 192;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kAttnThreads = 64 + 32 * kSoftmaxWarps;
 constexpr int kTileM = 128;
 constexpr int kStageKeys = 128;
 constexpr int kChunkBytes = 128 * 128;  // one 64-column bf16 chunk of a 128-row tile
@@ -63,12 +64,12 @@ template <int D>
 struct AttnSmem {
   static constexpr int kQBytes = kTileM * D * 2;
   static constexpr int kKVBytes = kStageKeys * D * 2;
-  static constexpr int kPBytes = kTileM * kStageKeys * 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + 2 * kKVBytes;
-  static constexpr int kOffP = kOffV + 2 * kKVBytes;
-  static constexpr int kOffCtl = kOffP + kPBytes;
+  static constexpr int kOffOnes = kOffV + 2 * kKVBytes;  // 1 KB of bf16 ones (B of the row-sum MMA)
+  static constexpr int kOffX = kOffOnes + 1024;          // row-max [2 parity][2 halves][128] + row-sum [2][128]
+  static constexpr int kOffCtl = kOffX + 4096;
   static constexpr int kBytes = kOffCtl + 1024;  // barriers, info ring, misc
   static constexpr int kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
 };
@@ -80,6 +81,7 @@ struct AttnCtl {
   uint64_t s_full[2], s_free[2];
   uint64_t p_full, pv_done, mma_drain;
   uint64_t info_full[kInfoRing];
+  uint64_t xbar[4];  // per lane quadrant: the two softmax warps' row-max / row-sum exchange
   uint32_t tmem_base;
   int abort;
   int n_seg;
@@ -158,6 +160,14 @@ __device__ __forceinline__ int list_intersection(const int32_t *a, int na, const
   return warp_sum_int(c);
 }
 
+// No-swizzle K-major descriptor over the 1 KB ones block: every address the
+// N = 16, K = 16 operand touches holds bf16 1.0, whatever the layout.
+__device__ __forceinline__ uint64_t smem_desc_ones(uint32_t saddr) {
+  uint64_t lo = ((saddr >> 4) & 0x3fffu) | ((uint64_t)((128u >> 4) & 0x3fffu) << 16);
+  uint64_t hi = ((256u >> 4) & 0x3fffu) | (1u << 14);  // SBO 256 B, version 1, SWIZZLE_NONE
+  return lo | (hi << 32);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -169,7 +179,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t *sQ = smem + L::kOffQ;
   uint8_t *sK = smem + L::kOffK;
   uint8_t *sV = smem + L::kOffV;
-  uint8_t *sP = smem + L::kOffP;
+  uint32_t *sOnes = reinterpret_cast<uint32_t *>(smem + L::kOffOnes);
+  float *sX = reinterpret_cast<float *>(smem + L::kOffX);  // [2 halves][128 rows] partial max, then sum
   AttnCtl *ctl = reinterpret_cast<AttnCtl *>(smem + L::kOffCtl);
   volatile int *abort = &ctl->abort;
 
@@ -192,12 +203,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_init(&ctl->v_full[i], 1);
         mbar_init(&ctl->v_empty[i], 1);
         mbar_init(&ctl->s_full[i], 1);
-        mbar_init(&ctl->s_free[i], 128);
+        mbar_init(&ctl->s_free[i], 32 * kSoftmaxWarps);
       }
-      mbar_init(&ctl->p_full, 128);
+      mbar_init(&ctl->p_full, 32 * kSoftmaxWarps);
       mbar_init(&ctl->pv_done, 1);
       mbar_init(&ctl->mma_drain, 1);
       for (int i = 0; i < kInfoRing; ++i) mbar_init(&ctl->info_full[i], 1);
+      for (int i = 0; i < 4; ++i) mbar_init(&ctl->xbar[i], 64);
       ctl->abort = 0;
       fence_barrier_init();
       tma_prefetch_desc(&tm_q);
@@ -212,7 +224,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       cnt[h] = __ldg(a.counts + lrow0 + h);
       if (cnt[h] < 0 || cnt[h] > a.idx_stride) ok = false;
     }
-    for (int h = 0; h < n_lists && ok; ++h) ok = list_valid(a.idx + (lrow0 + h) * a.idx_stride, cnt[h], n_seg_max, lane);
+    for (int h = 0; h < n_lists && ok; ++h)
+      ok = list_valid(a.idx + (lrow0 + h) * a.idx_stride, cnt[h], n_seg_max, lane);
     int n_seg = 0;
     if (!ok) {
       if (lane == 0) latch_status(VSA_ERR_BAD_INDEX);
@@ -220,12 +233,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       n_seg = cnt[0];
     } else {
       n_seg = cnt[0] + cnt[1] -
-              list_intersection(a.idx + lrow0 * a.idx_stride, cnt[0], a.idx + (lrow0 + 1) * a.idx_stride, cnt[1], lane);
+              list_intersection(a.idx + lrow0 * a.idx_stride, cnt[0], a.idx + (lrow0 + 1) * a.idx_stride, cnt[1],
+                                lane);
     }
     if (lane == 0) ctl->n_seg = n_seg;
   } else if (warp == 1) {
     tmem_alloc(&ctl->tmem_base, kTmemCols);
     tmem_relinquish();
+  } else {
+    for (int i = threadIdx.x - 64; i < 256; i += 32 * kSoftmaxWarps) sOnes[i] = 0x3f803f80u;  // bf16 1.0 pairs
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -236,6 +253,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem = ctl->tmem_base;
   const uint32_t tS[2] = {tmem, tmem + 128u};
   const uint32_t tO = tmem + 256u;
+  const uint32_t tL = tmem + 384u;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -246,13 +264,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                n_lists > 1 ? __ldg(a.counts + lrow0 + 1) : 0, n_lists, lane);
       if (lane == 0) {
         mbar_arrive_expect_tx(&ctl->q_full, L::kQBytes);
-        for (int c = 0; c < D / 64; ++c) tma_load_3d(sQ + c * kChunkBytes, &tm_q, &ctl->q_full, c * 64, tile * kTileM, bh);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(sQ + c * kChunkBytes, &tm_q, &ctl->q_full, c * 64, tile * kTileM, bh);
       }
       int issued = 0;
       for (int s = 0; s < n_stages; ++s) {
         const int slot = s & 1;
         const uint32_t use_par = ((s >> 1) - 1) & 1;
-        // gather the stage's segments
         int start[8];
         uint32_t mask = 0u;
         int nseg = 0;
@@ -267,7 +285,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             start[i] = start[0];  // repeat a loaded segment; masked out
           }
         }
-        const bool full = (nseg == seg_per_stage) && (mask == (seg_per_stage == 8 ? 0xffffu : ((1u << (2 * seg_per_stage)) - 1u))) &&
+        const uint32_t all = seg_per_stage == 8 ? 0xffffu : ((1u << (2 * seg_per_stage)) - 1u);
+        const bool full = (nseg == seg_per_stage) && (mask == all) &&
                           (start[seg_per_stage - 1] + a.seg_keys <= a.n_valid);
         bool ok = true;
         if (s >= 2) ok = mbar_wait_warp(&ctl->k_empty[slot], use_par, abort, a.timeout_ns, lane);
@@ -281,8 +300,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           mbar_arrive_expect_tx(&ctl->k_full[slot], L::kKVBytes);
           for (int i = 0; i < seg_per_stage; ++i)
             for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(sK + slot * L::kKVBytes + c * kChunkBytes + i * a.seg_keys * 128, &tm_k, &ctl->k_full[slot],
-                          c * 64, start[i], bh);
+              tma_load_3d(sK + slot * L::kKVBytes + c * kChunkBytes + i * a.seg_keys * 128, &tm_k,
+                          &ctl->k_full[slot], c * 64, start[i], bh);
         }
         if (s >= 2) ok = mbar_wait_warp(&ctl->v_empty[slot], use_par, abort, a.timeout_ns, lane);
         if (!ok) break;
@@ -290,8 +309,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           mbar_arrive_expect_tx(&ctl->v_full[slot], L::kKVBytes);
           for (int i = 0; i < seg_per_stage; ++i)
             for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(sV + slot * L::kKVBytes + c * kChunkBytes + i * a.seg_keys * 128, &tm_v, &ctl->v_full[slot],
-                          c * 64, start[i], bh);
+              tma_load_3d(sV + slot * L::kKVBytes + c * kChunkBytes + i * a.seg_keys * 128, &tm_v,
+                          &ctl->v_full[slot], c * 64, start[i], bh);
         }
         issued = s + 1;
         __syncwarp();
@@ -310,7 +329,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (n_stages > 0 && lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(kTileM, kStageKeys, false);
       constexpr uint32_t kIdO = idesc_bf16_f32(kTileM, D, true);
-      const uint32_t q_addr = smem_addr(sQ), k_addr = smem_addr(sK), v_addr = smem_addr(sV), p_addr = smem_addr(sP);
+      constexpr uint32_t kIdL = idesc_bf16_f32(kTileM, 16, false);
+      const uint32_t q_addr = smem_addr(sQ), k_addr = smem_addr(sK), v_addr = smem_addr(sV);
+      const uint64_t ones = smem_desc_ones(smem_addr(sOnes));
       bool ok = mbar_wait(&ctl->q_full, 0, abort, a.timeout_ns);
       auto issue_pv = [&](int t) -> bool {
         if (!mbar_wait(&ctl->p_full, t & 1, abort, a.timeout_ns)) return false;
@@ -319,9 +340,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t vb = v_addr + (t & 1) * L::kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < kStageKeys / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(p_addr + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
+          // P (bf16 pairs) sits in the first 64 columns of the stage's S buffer
           const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, kChunkBytes, 1024);
-          umma_bf16_ss(tO, ad, bd, kIdO, (t > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+          umma_bf16_ts(tO, tS[t & 1] + kk * 8, bd, kIdO, acc);
+          umma_bf16_ts(tL, tS[t & 1] + kk * 8, ones, kIdL, acc);
         }
         umma_commit(&ctl->v_empty[t & 1]);
         umma_commit(&ctl->pv_done);
@@ -352,11 +375,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax
     const int quad = warp & 3;
-    const int row = quad * 32 + lane;  // row within the tile == TMEM lane
+    const int ch = (warp - 2) >> 2;           // column half: keys [64 ch, 64 ch + 64)
+    const int row = quad * 32 + lane;         // row within the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const int half = row >> 6;
-    float m2 = -INFINITY;  // running max of scaled logits, log2 units
-    float l = 0.f;
+    const int half = row >> 6;                // query half for 64-row lists
+    float *xmax = sX;                         // [2 tile parity][2 halves][128 rows]
+    float *xsum = sX + 512;                   // [2 halves][128 rows]
+    float m2 = -INFINITY;  // running reference max of scaled logits, log2 units
+    float l = 0.f;         // this thread's share of the unrounded row sum
     bool ok = true;
     for (int t = 0; t < n_stages; ++t) {
       const int slot = t & 1;
@@ -365,35 +391,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const StageInfo &inf = ctl->info[t & (kInfoRing - 1)];
-      const int full = inf.full;
-      const uint32_t mask = inf.mask;
-      int start[8];
+      // this thread's 64 logits: r[c][j] = S[row][64 ch + 32 c + j]
+      uint32_t r[2][32];
+      tmem_ld32(tS[slot] + lane_off + ch * 64, r[0]);
+      tmem_ld32(tS[slot] + lane_off + ch * 64 + 32, r[1]);
+      tmem_ld_wait();
+      if (!inf.full) {
+        // cold path: valid columns of this thread's 64 as a bit mask, built
+        // per segment (a used segment's valid keys form one prefix of it)
+        uint64_t vm = 0ull;
+        const uint32_t mask = inf.mask;
+        const int nseg = kStageKeys >> a.seg_shift;
+#pragma unroll 1
+        for (int sg = 0; sg < nseg; ++sg) {
+          if (!((mask >> (2 * sg + half)) & 1u)) continue;
+          const int nv = min(a.seg_keys, max(0, a.n_valid - inf.start[sg]));
+          const int lo = max(0, sg * a.seg_keys - ch * 64);
+          const int hi = min(64, sg * a.seg_keys + nv - ch * 64);
+          if (hi <= lo) continue;
+          const uint64_t upto = hi >= 64 ? ~0ull : ((1ull << hi) - 1ull);
+          vm |= upto & ~((1ull << lo) - 1ull);
+        }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) start[i] = inf.start[i];
-      float x[kStageKeys];
-#pragma unroll
-      for (int c = 0; c < kStageKeys / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS[slot] + lane_off + c * 32, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) x[c * 32 + j] = __uint_as_float(r[j]) * a.scale_log2;
-      }
-      tc_fence_before();
-      mbar_arrive(&ctl->s_free[slot]);
-      if (!full) {
-#pragma unroll
-        for (int c = 0; c < kStageKeys; ++c) {
-          const int sg = c >> a.seg_shift;
-          const int key = start[sg] + (c & (a.seg_keys - 1));
-          const bool valid = ((mask >> (2 * sg + half)) & 1u) && key < a.n_valid;
-          if (!valid) x[c] = -INFINITY;
+        for (int j = 0; j < 32; ++j) {
+          if (!((vm >> j) & 1ull)) r[0][j] = __float_as_uint(-INFINITY);
+          if (!((vm >> (32 + j)) & 1ull)) r[1][j] = __float_as_uint(-INFINITY);
         }
       }
       float rmax = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kStageKeys; ++c) rmax = fmaxf(rmax, x[c]);
-      const float m_new = fmaxf(m2, rmax);
+      for (int j = 0; j < 32; ++j) rmax = fmaxf(rmax, fmaxf(__uint_as_float(r[0][j]), __uint_as_float(r[1][j])));
+      // exchange the partial row max with the partner warp (same rows, other half)
+      xmax[(t & 1) * 256 + ch * 128 + row] = rmax;
+      mbar_arrive(&ctl->xbar[quad]);
+      ok = mbar_wait_warp(&ctl->xbar[quad], t & 1, abort, a.timeout_ns, lane);
+      if (!ok) break;
+      rmax = fmaxf(rmax, xmax[(t & 1) * 256 + (ch ^ 1) * 128 + row]);
+      const float m_new = fmaxf(m2, rmax * a.scale_log2);
       const bool need = m_new > m2 + kRescaleThreshold || (m2 == -INFINITY && m_new != -INFINITY);
       if (t > 0) {
         ok = mbar_wait_warp(&ctl->pv_done, (t - 1) & 1, abort, a.timeout_ns, lane);
@@ -402,80 +436,93 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (__any_sync(0xffffffffu, need)) {
         const float alpha = need ? fast_exp2(m2 - m_new) : 1.f;  // exp2(-inf) = 0
         if (t > 0) {
+          // cold path: rescale this thread's half of the O row (and, in
+          // half 0, the rounded-P row sum) by alpha
           tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tO + lane_off + c * 32, r);
+#pragma unroll 1
+          for (int c = 0; c < D / 64 + (ch == 0 ? 1 : 0); ++c) {
+            const uint32_t col = c < D / 64 ? tO + ch * (D / 2) + c * 32 : tL;
+            uint32_t o[32];
+            tmem_ld32(col + lane_off, o);
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
-            tmem_st32(tO + lane_off + c * 32, r);
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+            tmem_st32(col + lane_off, o);
           }
-          tmem_st_wait();
         }
         if (need) {
           l *= alpha;
           m2 = m_new;
         }
       }
-      // P = exp2(x - m2) in bf16, swizzled K-major layout of the P.V operand
+      // P = exp2(s * scale * log2(e) - m2) as bf16 pairs over this thread's S columns
       const bool live = m2 != -INFINITY;
-      uint8_t *prow = sP + row * 128;
+      const float neg_m = live ? -m2 : 0.f;
       float rs = 0.f;
 #pragma unroll
-      for (int g = 0; g < kStageKeys / 8; ++g) {
-        float p[8];
+      for (int c = 0; c < 2; ++c) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          p[j] = live ? fast_exp2(x[g * 8 + j] - m2) : 0.f;
-          rs += p[j];
+        for (int j = 0; j < 16; ++j) {
+          const float p0 = live ? fast_exp2(fmaf(__uint_as_float(r[c][2 * j]), a.scale_log2, neg_m)) : 0.f;
+          const float p1 = live ? fast_exp2(fmaf(__uint_as_float(r[c][2 * j + 1]), a.scale_log2, neg_m)) : 0.f;
+          rs += p0 + p1;
+          r[0][c * 16 + j] = pack_bf16x2(p0, p1);
         }
-        uint4 pk;
-        pk.x = pack_bf16x2(p[0], p[1]);
-        pk.y = pack_bf16x2(p[2], p[3]);
-        pk.z = pack_bf16x2(p[4], p[5]);
-        pk.w = pack_bf16x2(p[6], p[7]);
-        const int cb = g >> 3, cc = g & 7;
-        *reinterpret_cast<uint4 *>(prow + cb * kChunkBytes + ((cc ^ (row & 7)) << 4)) = pk;
       }
       l += rs;
-      fence_proxy_async_smem();
+      tmem_st32(tS[slot] + lane_off + ch * 32, r[0]);
+      tmem_st_wait();
       tc_fence_before();
+      mbar_arrive(&ctl->s_free[slot]);
       mbar_arrive(&ctl->p_full);
     }
 
     // ---------------------------------------------------------- epilogue
+    constexpr int DH = D / 2;  // output columns of this thread
     const int grow = tile * kTileM + row;
     const size_t orow = (size_t)bh * a.n_pad + grow;
-    float acc[D];
+    float acc[DH];
+    float lr = 0.f;  // row sum of the rounded P (tensor core)
     bool have = false;
     if (ok && n_stages > 0) {
       ok = mbar_wait_warp(&ctl->pv_done, (n_stages - 1) & 1, abort, a.timeout_ns, lane);
       if (ok) {
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tO + lane_off + c * 32, r);
+        for (int c = 0; c < DH / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + lane_off + ch * DH + c * 32, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) acc[c * 32 + j] = __uint_as_float(r[j]);
+          for (int j = 0; j < 32; ++j) acc[c * 32 + j] = __uint_as_float(o[j]);
         }
+        uint32_t o[32];
+        tmem_ld32(tL + lane_off, o);
+        tmem_ld_wait();
+        lr = __uint_as_float(o[0]);
         have = true;
       }
     }
-    const bool row_ok = grow < a.n_valid && have && l > 0.f;
-    const float inv_l = row_ok ? 1.f / l : 0.f;
-    float lse = row_ok ? (m2 + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    // full unrounded row sum from the two halves
+    xsum[ch * 128 + row] = l;
+    float lsum = l;
+    if (ok) {
+      mbar_arrive(&ctl->xbar[quad]);
+      ok = mbar_wait_warp(&ctl->xbar[quad], n_stages & 1, abort, a.timeout_ns, lane);
+      if (ok) lsum += xsum[(ch ^ 1) * 128 + row];
+    }
+    have = have && ok;
+    const bool row_ok = grow < a.n_valid && have && lsum > 0.f && lr > 0.f;
+    const float inv_l = row_ok ? 1.f / lr : 0.f;
+    float lse = row_ok ? (m2 + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
 #pragma unroll
-    for (int c = 0; c < D; ++c) acc[c] = row_ok ? acc[c] * inv_l : 0.f;
+    for (int c = 0; c < DH; ++c) acc[c] = row_ok ? acc[c] * inv_l : 0.f;
     if (a.merge_o != nullptr) {
       const float lm = grow < a.n_valid ? a.merge_lse[orow] : -INFINITY;
       const MergeWeights w = lse_merge_weights(lm, lse);
-      const float4 *mo = reinterpret_cast<const float4 *>(a.merge_o + orow * D);
+      const float4 *mo = reinterpret_cast<const float4 *>(a.merge_o + orow * D + ch * DH);
 #pragma unroll
-      for (int c = 0; c < D / 4; ++c) {
+      for (int c = 0; c < DH / 4; ++c) {
         const float4 v = mo[c];
         acc[4 * c + 0] = w.wa * v.x + w.wb * acc[4 * c + 0];
         acc[4 * c + 1] = w.wa * v.y + w.wb * acc[4 * c + 1];
@@ -485,13 +532,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       lse = w.lse;
     }
     if (a.o_fp32) {
-      float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.o) + orow * D);
+      float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.o) + orow * D + ch * DH);
 #pragma unroll
-      for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
+      for (int c = 0; c < DH / 4; ++c) dst[c] = make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
     } else {
-      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.o) + orow * D);
+      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.o) + orow * D + ch * DH);
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c) {
+      for (int c = 0; c < DH / 8; ++c) {
         uint4 pk;
         pk.x = pack_bf16x2(acc[8 * c + 0], acc[8 * c + 1]);
         pk.y = pack_bf16x2(acc[8 * c + 2], acc[8 * c + 3]);
@@ -500,7 +547,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         dst[c] = pk;
       }
     }
-    a.lse[orow] = lse;
+    if (ch == 0) a.lse[orow] = lse;
   }
 
   // ---------------------------------------------------------------- teardown

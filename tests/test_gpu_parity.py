@@ -158,7 +158,7 @@ def _attention_case(w, q, k, v, kept, blocks, o_fp32=False):
     Lg = lse.cpu().numpy()
     O, L = orc.block_sparse_attention(q, k, v, kept, w.bq, w.bk, w.n_valid, w.scale, rows=blocks)
     rows = [(b, h, i * w.bq, (i + 1) * w.bq) for b, h, i in blocks]
-    return assert_close_rows(Og, Lg, O, L, rows)
+    return assert_close_rows(Og, Lg, O, L, rows, bf16_out=not o_fp32)
 
 
 def test_attention_tiny_all_rows():
@@ -184,7 +184,8 @@ def test_attention_sampled_rows(name):
     q, k, v = inputs(name, (0, 2))
     kept, *_ = oracle_select_per_head(q, k, w)
     blocks = sample_blocks(w, 6, seed=1, heads=2)
-    print(f"\n{name} attention worst:", _attention_case(w, q, k, v, kept, blocks))
+    print(f"\n{name} attention worst fp32 O:", _attention_case(w, q, k, v, kept, blocks, o_fp32=True))
+    print(f"{name} attention worst bf16 O (beyond rounding):", _attention_case(w, q, k, v, kept, blocks))
 
 
 @pytest.mark.parametrize("point", [1, 6, 9])
@@ -281,7 +282,7 @@ def test_path_tiny_every_row():
         for r in range(w.n_pad // 64):
             assert np.array_equal(mi[0, h, r, :mc[0, h, r]], res["tiles"][0][h][r]), (h, r)
     worst = assert_close_rows(out["o"].float().cpu().numpy(), out["lse"].cpu().numpy(), res["O"], res["LSE"],
-                              [(0, h, 0, w.n_pad) for h in range(w.H)])
+                              [(0, h, 0, w.n_pad) for h in range(w.H)], bf16_out=True)
     print("\ntiny path worst:", worst)
 
 
@@ -341,5 +342,5 @@ def test_path_hunyuan_sampled():
     mrows = [(b, h, r) for b, h, i in rows for r in (2 * i, 2 * i + 1)]
     O_u, L_u = orc.micro_attention(q, k, v, tiles, w.n_valid, w.scale, rows=mrows)
     O, L = orc.lse_merge(O_M, L_M, O_u, L_u)
-    worst = assert_close_rows(Og, Lg, O, L, [(b, h, i * 128, i * 128 + 128) for b, h, i in rows])
+    worst = assert_close_rows(Og, Lg, O, L, [(b, h, i * 128, i * 128 + 128) for b, h, i in rows], bf16_out=True)
     print("\nhunyuan path worst:", worst, "rows", rows)
