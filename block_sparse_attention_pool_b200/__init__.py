@@ -23,7 +23,7 @@ import torch
 
 __all__ = [
     "VsaError", "Shape", "SelectParams", "MicroParams", "lib", "library_path", "EXPORTED",
-    "pool_qk", "select_blocks", "mask_to_lists", "select_micro", "select_micro_workspace_bytes",
+    "pool_qk", "select_blocks", "mask_to_lists", "select_micro", "select_micro_workspace_bytes", "select_micro_noalloc",
     "block_sparse_fwd", "lse_merge", "read_device_status", "status_string", "version",
     "PathConfig", "SparseVideoAttention",
 ]
@@ -33,12 +33,15 @@ _LIB_PATH = os.path.join(_HERE, "libvsa.so")
 
 EXPORTED = (
     "vsa_status_string", "vsa_version", "vsa_read_device_status", "vsa_pool_qk", "vsa_select_blocks",
-    "vsa_mask_to_lists", "vsa_select_micro_workspace_bytes", "vsa_select_micro", "vsa_block_sparse_fwd",
-    "vsa_lse_merge",
+    "vsa_mask_to_lists", "vsa_select_micro_workspace_bytes", "vsa_select_micro", "vsa_select_micro_noalloc",
+    "vsa_block_sparse_fwd", "vsa_lse_merge",
 )
 
 STATUS = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_UNSUPPORTED", 3: "VSA_ERR_CUDA",
-          4: "VSA_ERR_CAPACITY", 5: "VSA_ERR_BAD_INDEX", 6: "VSA_ERR_TIMEOUT"}
+          4: "VSA_ERR_CAPACITY", 5: "VSA_ERR_BAD_INDEX", 6: "VSA_ERR_TIMEOUT", 7: "VSA_ERR_SCRATCH_LIMIT"}
+
+# Fixed scratch of vsa_select_micro_noalloc (include/vsa.h VSA_MICRO_NOALLOC_MAX_BYTES)
+MICRO_NOALLOC_MAX_BYTES = 16 << 20
 
 
 class VsaError(RuntimeError):
@@ -95,6 +98,8 @@ def lib():
     L.vsa_select_micro_workspace_bytes.argtypes = [SP, ctypes.POINTER(MicroParams)]
     L.vsa_select_micro.restype = I
     L.vsa_select_micro.argtypes = [P, P, P, P, SP, I, I, F, ctypes.POINTER(MicroParams), P, P, P, S, P]
+    L.vsa_select_micro_noalloc.restype = I
+    L.vsa_select_micro_noalloc.argtypes = [P, P, P, P, SP, I, I, F, ctypes.POINTER(MicroParams), P, P, P]
     L.vsa_block_sparse_fwd.restype = I
     L.vsa_block_sparse_fwd.argtypes = [P, P, P, SP, I, I, P, P, I, F, P, I, P, P, P, P]
     L.vsa_lse_merge.restype = I
@@ -179,6 +184,18 @@ def select_micro(q_pool64, k_pool16, counts, idx, shape: Shape, bq, bk, scale, m
     _check(lib().vsa_select_micro(_p(q_pool64), _p(k_pool16), _p(counts), _p(idx), ctypes.byref(shape), bq, bk,
                                   float(scale), ctypes.byref(p), _p(m_counts), _p(m_idx), _p(workspace),
                                   workspace.numel() * workspace.element_size(), _s(stream)), "vsa_select_micro")
+    del keep
+
+
+def select_micro_noalloc(q_pool64, k_pool16, counts, idx, shape: Shape, bq, bk, scale, mode, topk, percentile,
+                         head_enable, row_capacity, m_counts, m_idx, stream=None):
+    """vsa_select_micro without a workspace argument: for callers that may not
+    allocate device memory themselves (its scratch is the library's fixed
+    array of MICRO_NOALLOC_MAX_BYTES per GPU; calls must not overlap on the GPU)."""
+    p, keep = _micro_params(mode, topk, percentile, head_enable, row_capacity)
+    _check(lib().vsa_select_micro_noalloc(_p(q_pool64), _p(k_pool16), _p(counts), _p(idx), ctypes.byref(shape), bq,
+                                          bk, float(scale), ctypes.byref(p), _p(m_counts), _p(m_idx), _s(stream)),
+           "vsa_select_micro_noalloc")
     del keep
 
 

@@ -140,6 +140,46 @@ int ilog2(int x) {
   return r;
 }
 
+// Fixed scratch of vsa_select_micro_noalloc: reserved in every GPU that loads
+// this library, for the life of the process.  In host code its name is only a
+// host-side stand-in; the device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_micro_noalloc_scratch[VSA_MICRO_NOALLOC_MAX_BYTES];
+
+constexpr int kNoallocMaxDevices = 64;
+constexpr int kNoallocMaxBH = 1024;
+
+// Device address of the fixed scratch on the current device, looked up once
+// per device (with that device current) and cached.
+vsa_status noalloc_scratch(void **out) {
+  static std::mutex mu;
+  static void *addr[kNoallocMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) return VSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_micro_noalloc_scratch) != cudaSuccess || p == nullptr) return VSA_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return VSA_OK;
+}
+
+// Per-head slot numbers handed to the device by value (no host-to-device copy).
+struct HeadSlots {
+  int16_t slot[kNoallocMaxBH];  // rank among enabled heads, or -1
+  int n_enabled;
+  int H, BH;
+};
+
+__global__ void noalloc_slot_fill_kernel(HeadSlots hs, int32_t *slot_of_bh) {
+  const int bh = blockIdx.x * blockDim.x + threadIdx.x;
+  if (bh >= hs.BH) return;
+  const int b = bh / hs.H, h = bh % hs.H;
+  const int r = hs.slot[h];
+  slot_of_bh[bh] = r < 0 ? -1 : b * hs.n_enabled + r;
+}
+
 }  // namespace
 
 extern "C" {
@@ -153,6 +193,7 @@ const char *vsa_status_string(vsa_status s) {
     case VSA_ERR_CAPACITY: return "list capacity exceeded";
     case VSA_ERR_BAD_INDEX: return "invalid index in a list";
     case VSA_ERR_TIMEOUT: return "pipeline wait timed out";
+    case VSA_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the allocation-free entry point holds";
   }
   return "unknown status";
 }
@@ -288,6 +329,75 @@ vsa_status vsa_select_micro(const float *q_pool64, const float *k_pool16, const 
     if (cudaMemsetAsync(m_counts, 0, (size_t)BH * n_r * 4, st) != cudaSuccess) return VSA_ERR_CUDA;
     return VSA_OK;
   }
+  if (cudaMemsetAsync(ws8 + L.off_hist, 0, L.total - L.off_hist, st) != cudaSuccess) return VSA_ERR_CUDA;
+
+  vsa::micro_bitmap_kernel<<<dim3(n_q, BH), 128, 0, st>>>(counts, idx, n_q, n_k, BH, ws);
+  vsa::ScoreArgs sa{q_pool64, k_pool16, n_r, n_t, n_q, bq, bk, shape->n_valid, scale, params->mode == 2 ? 1 : 0};
+  dim3 sg((n_t + vsa::kScoreBN - 1) / vsa::kScoreBN, (n_r + vsa::kScoreBM - 1) / vsa::kScoreBM, BH);
+  if (shape->d == 128)
+    vsa::micro_score_kernel<128><<<sg, vsa::kScoreThreads, 0, st>>>(sa, ws);
+  else
+    vsa::micro_score_kernel<64><<<sg, vsa::kScoreThreads, 0, st>>>(sa, ws);
+  const unsigned rows_blocks = (unsigned)(((size_t)BH * n_r + 7) / 8);
+  if (params->mode == 1) {
+    vsa::micro_topk_kernel<<<rows_blocks, 256, 0, st>>>(ws, n_r, n_t, BH, params->topk, params->row_capacity,
+                                                      m_counts, m_idx);
+  } else {
+    const size_t per_slot = (size_t)n_r * n_t;
+    vsa::micro_find_kernel<<<L.n_slots, 32, 0, st>>>(ws, params->percentile, 0);
+    vsa::micro_hist_kernel<<<dim3(256, L.n_slots), 256, 0, st>>>(ws, per_slot, 1);
+    vsa::micro_find_kernel<<<L.n_slots, 32, 0, st>>>(ws, params->percentile, 1);
+    vsa::micro_hist_kernel<<<dim3(256, L.n_slots), 256, 0, st>>>(ws, per_slot, 2);
+    vsa::micro_find_kernel<<<L.n_slots, 32, 0, st>>>(ws, params->percentile, 2);
+    vsa::micro_compact_kernel<<<rows_blocks, 256, 0, st>>>(ws, n_r, n_t, BH, params->row_capacity, m_counts, m_idx);
+  }
+  return launch_status();
+}
+
+vsa_status vsa_select_micro_noalloc(const float *q_pool64, const float *k_pool16, const int32_t *counts,
+                                    const int32_t *idx, const vsa_shape *shape, int bq, int bk, float scale,
+                                    const vsa_micro_params *params, int32_t *m_counts, int32_t *m_idx,
+                                    void *stream) {
+  if (!shape_ok(shape) || !q_pool64 || !k_pool16 || !counts || !idx || !m_counts || !m_idx)
+    return VSA_ERR_INVALID_ARG;
+  if (!micro_params_ok(params)) return VSA_ERR_INVALID_ARG;
+  if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return VSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(q_pool64) || !aligned16(k_pool16)) return VSA_ERR_INVALID_ARG;
+  const int n_q = shape->n_pad / bq, n_k = shape->n_pad / bk;
+  if (n_k > 1024) return VSA_ERR_UNSUPPORTED;
+  const int BH = shape->B * shape->H;
+  if (BH > kNoallocMaxBH) return VSA_ERR_SCRATCH_LIMIT;
+  const MicroLayout L = micro_layout(shape, params);
+  if (L.total > VSA_MICRO_NOALLOC_MAX_BYTES) return VSA_ERR_SCRATCH_LIMIT;
+  void *scratch = nullptr;
+  const vsa_status se = noalloc_scratch(&scratch);
+  if (se != VSA_OK) return se;
+
+  const int n_r = shape->n_pad / vsa::kMicroRows, n_t = shape->n_pad / vsa::kMicroKeys;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t *ws8 = static_cast<uint8_t *>(scratch);
+  vsa::MicroWs ws;
+  ws.slot_of_bh = reinterpret_cast<int32_t *>(ws8 + L.off_slot);
+  ws.bitmap = reinterpret_cast<uint32_t *>(ws8 + L.off_bitmap);
+  ws.keys = reinterpret_cast<uint32_t *>(ws8 + L.off_keys);
+  ws.hist = reinterpret_cast<uint32_t *>(ws8 + L.off_hist);
+  ws.state = reinterpret_cast<uint32_t *>(ws8 + L.off_state);
+  ws.n_slots = L.n_slots;
+
+  HeadSlots hs;
+  int next = 0;
+  for (int h = 0; h < shape->H; ++h)
+    hs.slot[h] = (params->head_enable == nullptr || params->head_enable[h]) ? (int16_t)next++ : (int16_t)-1;
+  hs.n_enabled = next;
+  hs.H = shape->H;
+  hs.BH = BH;
+  noalloc_slot_fill_kernel<<<(BH + 255) / 256, 256, 0, st>>>(hs, ws.slot_of_bh);
+  if (L.n_slots == 0) {
+    if (cudaMemsetAsync(m_counts, 0, (size_t)BH * n_r * 4, st) != cudaSuccess) return VSA_ERR_CUDA;
+    return launch_status();
+  }
+  // histograms and rank-search state must start at zero on every call
   if (cudaMemsetAsync(ws8 + L.off_hist, 0, L.total - L.off_hist, st) != cudaSuccess) return VSA_ERR_CUDA;
 
   vsa::micro_bitmap_kernel<<<dim3(n_q, BH), 128, 0, st>>>(counts, idx, n_q, n_k, BH, ws);

@@ -70,7 +70,9 @@ typedef enum {
   VSA_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed                   */
   VSA_ERR_CAPACITY = 4,      /* device: a list exceeded its caller-given capacity   */
   VSA_ERR_BAD_INDEX = 5,     /* device: a caller-given list holds an invalid index  */
-  VSA_ERR_TIMEOUT = 6        /* device: a pipeline wait exceeded its time limit     */
+  VSA_ERR_TIMEOUT = 6,       /* device: a pipeline wait exceeded its time limit     */
+  VSA_ERR_SCRATCH_LIMIT = 7  /* the problem needs more scratch than the fixed
+                                scratch of vsa_select_micro_noalloc holds         */
 } vsa_status;
 
 /* Problem shape.  d in {64, 128}; n_valid <= n_pad; n_pad a multiple of 128. */
@@ -193,6 +195,39 @@ VSA_API vsa_status vsa_select_micro(const float *q_pool64, const float *k_pool16
                             const int32_t *idx, const vsa_shape *shape, int bq, int bk, float scale,
                             const vsa_micro_params *params, int32_t *m_counts, int32_t *m_idx,
                             void *workspace, size_t workspace_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Allocation-free Micro selection.  The pages have no counterpart of this
+ * entry point: it exists for callers that cannot allocate device memory of
+ * their own -- for example a plugin whose host engine owns every byte of
+ * device memory and hands out no extra workspace, or a service running under
+ * a fixed device-memory budget that another allocator controls (cudaMalloc
+ * can also block the whole device while it runs, which such callers avoid).
+ *
+ * Same arguments, meaning and results as vsa_select_micro, minus the
+ * workspace: its scratch lives in one fixed array of
+ * VSA_MICRO_NOALLOC_MAX_BYTES bytes of device memory that this library
+ * reserves statically in every GPU that loads it, until the process exits.
+ * No call allocates or frees anything (no cudaMalloc, cudaFree or allocating
+ * library routine).
+ *   - A problem whose scratch (vsa_select_micro_workspace_bytes for the same
+ *     shape and params) exceeds VSA_MICRO_NOALLOC_MAX_BYTES is rejected with
+ *     VSA_ERR_SCRATCH_LIMIT before anything is enqueued.  B*H <= 1024.
+ *   - The first call on a device looks up the device address of the fixed
+ *     array (once per device, on the current device) and remembers it; make
+ *     that first call before any stream capture.
+ *   - Every call on a device shares the one array.  Calls whose GPU work
+ *     overlaps in time (different streams, or other threads without
+ *     ordering between them) race on it and give undefined lists; order them
+ *     on one stream or synchronise between them.  The state that must start
+ *     at zero is cleared on the call's stream by every call.
+ * ------------------------------------------------------------------------- */
+#define VSA_MICRO_NOALLOC_MAX_BYTES ((size_t)16 << 20)
+
+VSA_API vsa_status vsa_select_micro_noalloc(const float *q_pool64, const float *k_pool16, const int32_t *counts,
+                                            const int32_t *idx, const vsa_shape *shape, int bq, int bk, float scale,
+                                            const vsa_micro_params *params, int32_t *m_counts, int32_t *m_idx,
+                                            void *stream);
 
 /* ---------------------------------------------------------------------------
  * a4 / a6 Block-sparse attention forward ([HVA] section 2 Eq. (4): attention of
