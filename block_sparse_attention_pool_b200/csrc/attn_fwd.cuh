@@ -14,16 +14,38 @@
 //   warp 0     TMA producer: Q once, then K and V of each stage into
 //              2 + 2 ring slots (128B-swizzled, one box per segment and
 //              64-column chunk; rows past n_valid arrive as zeros).
-//   warp 1     MMA issuer (one thread): S_s = Q K_s^T into one of two TMEM
-//              S buffers, then O += P_{s-1} V_{s-1}; tcgen05.commit frees
-//              ring slots and signals the softmax.
-//   warps 2-5  softmax: one thread per query row reads its S row from TMEM,
-//              masks, keeps a running max in the log2 domain, rescales the
-//              TMEM O row only when the max grew by more than 2^8 (lazy
-//              rescale), writes P (bf16) to shared memory in the swizzled
-//              K-major operand layout, and finally normalises O, computes
-//              LSE and, if asked, merges with a previous (O, LSE).
-// TMEM: S0 [0,128), S1 [128,256), O [256, 256 + d) fp32 columns.
+//   warp 1     MMA issuer (one thread): S_s = Q K_s^T into TMEM buffer S[s&1],
+//              then O[s&1] += P_{s-1} V_{s-1}; tcgen05.commit frees ring slots
+//              and signals the softmax.
+//   warps 2-9  softmax in two groups of four warps (one warp per TMEM lane
+//              quadrant): group g owns the stages s with s & 1 = g, its S
+//              buffer and its own O accumulator, so one group's exponentials
+//              overlap the other group's TMEM loads, maxima and stores.  A
+//              thread owns one query row of its group's stages: it reads the
+//              S row from TMEM, masks, keeps its group's running reference
+//              max in the log2 domain, rescales its O row only when the max
+//              grew by more than 2^8 (lazy rescale), and writes P as bf16
+//              pairs back over the first 64 columns of the S buffer (the A
+//              operand of P.V).  It keeps two row sums: of P in fp32 (for
+//              LSE) and of the bf16-rounded P (to normalise O).
+//              Epilogue: the two groups exchange (max, sums) through shared
+//              memory, merge their partial results exactly, normalise, and
+//              each writes half of the row's columns (and, if asked, merges
+//              with a previous (O, LSE)).
+// TMEM: S_0 [0,128), S_1 [128,256), O_0 [256, 256 + d), O_1 [384, 384 + d).
+//
+// Barrier phases.  A parity wait is only unambiguous when the barrier cannot
+// run two phases ahead of its waiter, so every per-stage barrier is split by
+// stage parity: P of stage t (p_full[t&1]) cannot be signalled again before
+// the MMA issuer consumed it, because stage t+2 needs S_{t+2}, which is issued
+// after that wait.  The commit that signals S_t also covers P.V of stage t-2
+// (issued before S_t), so a group that sees S_t may rescale its O at once.
+// The epilogue waits on mma_drain, committed once after the last MMA.
+//
+// Normalising O by the sum of the same bf16-rounded P that multiplied V makes
+// the output an exact convex combination of the selected V rows: a softmax
+// dominated by one key returns that key's V without the rounding of its
+// weight.  LSE uses the fp32 sum.
 #pragma once
 
 #include "common.cuh"
@@ -67,8 +89,7 @@ struct AttnSmem {
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + 2 * kKVBytes;
-  static constexpr int kOffOnes = kOffV + 2 * kKVBytes;  // 1 KB of bf16 ones (B of the row-sum MMA)
-  static constexpr int kOffX = kOffOnes + 1024;          // row-max [2 parity][2 halves][128] + row-sum [2][128]
+  static constexpr int kOffX = kOffV + 2 * kKVBytes;  // epilogue exchange: [2 groups][3][128] floats
   static constexpr int kOffCtl = kOffX + 4096;
   static constexpr int kBytes = kOffCtl + 1024;  // barriers, info ring, misc
   static constexpr int kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
@@ -79,9 +100,10 @@ struct AttnCtl {
   uint64_t k_full[2], k_empty[2];
   uint64_t v_full[2], v_empty[2];
   uint64_t s_full[2], s_free[2];
-  uint64_t p_full, pv_done, mma_drain;
+  uint64_t p_full[2];               // per S buffer: P of the stage written
+  uint64_t mma_drain;               // every MMA of the CTA has completed (one phase)
   uint64_t info_full[kInfoRing];
-  uint64_t xbar[4];  // per lane quadrant: the two softmax warps' row-max / row-sum exchange
+  uint64_t xbar[4];  // per lane quadrant: the two groups' final (max, sum) exchange
   uint32_t tmem_base;
   int abort;
   int n_seg;
@@ -160,12 +182,13 @@ __device__ __forceinline__ int list_intersection(const int32_t *a, int na, const
   return warp_sum_int(c);
 }
 
-// No-swizzle K-major descriptor over the 1 KB ones block: every address the
-// N = 16, K = 16 operand touches holds bf16 1.0, whatever the layout.
-__device__ __forceinline__ uint64_t smem_desc_ones(uint32_t saddr) {
-  uint64_t lo = ((saddr >> 4) & 0x3fffu) | ((uint64_t)((128u >> 4) & 0x3fffu) << 16);
-  uint64_t hi = ((256u >> 4) & 0x3fffu) | (1u << 14);  // SBO 256 B, version 1, SWIZZLE_NONE
-  return lo | (hi << 32);
+// acc += the two bf16 values packed in pk (fp32 accumulation).
+__device__ __forceinline__ float add_bf16x2_f32(float acc, uint32_t pk) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %0, hi, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(pk));
+  return acc;
 }
 
 template <int D>
@@ -179,8 +202,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t *sQ = smem + L::kOffQ;
   uint8_t *sK = smem + L::kOffK;
   uint8_t *sV = smem + L::kOffV;
-  uint32_t *sOnes = reinterpret_cast<uint32_t *>(smem + L::kOffOnes);
-  float *sX = reinterpret_cast<float *>(smem + L::kOffX);  // [2 halves][128 rows] partial max, then sum
+  float *sX = reinterpret_cast<float *>(smem + L::kOffX);  // [2 groups][max, sum, rounded sum][128 rows]
   AttnCtl *ctl = reinterpret_cast<AttnCtl *>(smem + L::kOffCtl);
   volatile int *abort = &ctl->abort;
 
@@ -203,10 +225,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_init(&ctl->v_full[i], 1);
         mbar_init(&ctl->v_empty[i], 1);
         mbar_init(&ctl->s_full[i], 1);
-        mbar_init(&ctl->s_free[i], 32 * kSoftmaxWarps);
+        mbar_init(&ctl->s_free[i], 128);
+        mbar_init(&ctl->p_full[i], 128);
       }
-      mbar_init(&ctl->p_full, 32 * kSoftmaxWarps);
-      mbar_init(&ctl->pv_done, 1);
       mbar_init(&ctl->mma_drain, 1);
       for (int i = 0; i < kInfoRing; ++i) mbar_init(&ctl->info_full[i], 1);
       for (int i = 0; i < 4; ++i) mbar_init(&ctl->xbar[i], 64);
@@ -240,9 +261,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else if (warp == 1) {
     tmem_alloc(&ctl->tmem_base, kTmemCols);
     tmem_relinquish();
-  } else {
-    for (int i = threadIdx.x - 64; i < 256; i += 32 * kSoftmaxWarps) sOnes[i] = 0x3f803f80u;  // bf16 1.0 pairs
-    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -252,8 +270,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int n_stages = (n_seg + seg_per_stage - 1) / seg_per_stage;
   const uint32_t tmem = ctl->tmem_base;
   const uint32_t tS[2] = {tmem, tmem + 128u};
-  const uint32_t tO = tmem + 256u;
-  const uint32_t tL = tmem + 384u;
+  const uint32_t tO[2] = {tmem + 256u, tmem + 384u};
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -329,12 +346,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (n_stages > 0 && lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(kTileM, kStageKeys, false);
       constexpr uint32_t kIdO = idesc_bf16_f32(kTileM, D, true);
-      constexpr uint32_t kIdL = idesc_bf16_f32(kTileM, 16, false);
       const uint32_t q_addr = smem_addr(sQ), k_addr = smem_addr(sK), v_addr = smem_addr(sV);
-      const uint64_t ones = smem_desc_ones(smem_addr(sOnes));
       bool ok = mbar_wait(&ctl->q_full, 0, abort, a.timeout_ns);
       auto issue_pv = [&](int t) -> bool {
-        if (!mbar_wait(&ctl->p_full, t & 1, abort, a.timeout_ns)) return false;
+        if (!mbar_wait(&ctl->p_full[t & 1], (t >> 1) & 1, abort, a.timeout_ns)) return false;
         if (!mbar_wait(&ctl->v_full[t & 1], (t >> 1) & 1, abort, a.timeout_ns)) return false;
         tc_fence_after();
         const uint32_t vb = v_addr + (t & 1) * L::kKVBytes;
@@ -342,12 +357,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int kk = 0; kk < kStageKeys / 16; ++kk) {
           // P (bf16 pairs) sits in the first 64 columns of the stage's S buffer
           const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, kChunkBytes, 1024);
-          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-          umma_bf16_ts(tO, tS[t & 1] + kk * 8, bd, kIdO, acc);
-          umma_bf16_ts(tL, tS[t & 1] + kk * 8, ones, kIdL, acc);
+          umma_bf16_ts(tO[t & 1], tS[t & 1] + kk * 8, bd, kIdO, (t >= 2 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&ctl->v_empty[t & 1]);
-        umma_commit(&ctl->pv_done);
         return true;
       };
       for (int s = 0; ok && s < n_stages; ++s) {
@@ -374,180 +386,209 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
+    const int g = (warp - 2) >> 2;            // group: stages s with s & 1 == g
     const int quad = warp & 3;
-    const int ch = (warp - 2) >> 2;           // column half: keys [64 ch, 64 ch + 64)
     const int row = quad * 32 + lane;         // row within the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const int half = row >> 6;                // query half for 64-row lists
-    float *xmax = sX;                         // [2 tile parity][2 halves][128 rows]
-    float *xsum = sX + 512;                   // [2 halves][128 rows]
-    float m2 = -INFINITY;  // running reference max of scaled logits, log2 units
-    float l = 0.f;         // this thread's share of the unrounded row sum
+    float m2 = -INFINITY;  // this group's running reference max of scaled logits, log2 units
+    float l = 0.f;         // sum of P (fp32) over this group's stages
+    float lr = 0.f;        // sum of the bf16-rounded P over this group's stages
     bool ok = true;
-    for (int t = 0; t < n_stages; ++t) {
-      const int slot = t & 1;
+    const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+    for (int t = g; t < n_stages; t += 2) {
       ok = mbar_wait_warp(&ctl->info_full[t & (kInfoRing - 1)], (t >> 2) & 1, abort, a.timeout_ns, lane);
-      if (ok) ok = mbar_wait_warp(&ctl->s_full[slot], (t >> 1) & 1, abort, a.timeout_ns, lane);
+      if (ok) ok = mbar_wait_warp(&ctl->s_full[g], (t >> 1) & 1, abort, a.timeout_ns, lane);
       if (!ok) break;
       tc_fence_after();
       const StageInfo &inf = ctl->info[t & (kInfoRing - 1)];
-      // this thread's 64 logits: r[c][j] = S[row][64 ch + 32 c + j]
-      uint32_t r[2][32];
-      tmem_ld32(tS[slot] + lane_off + ch * 64, r[0]);
-      tmem_ld32(tS[slot] + lane_off + ch * 64 + 32, r[1]);
+      // the row's 128 logits: r[c][j] = S[row][32 c + j]
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS[g] + lane_off + c * 32, r[c]);
       tmem_ld_wait();
       if (!inf.full) {
-        // cold path: valid columns of this thread's 64 as a bit mask, built
-        // per segment (a used segment's valid keys form one prefix of it)
-        uint64_t vm = 0ull;
+        // cold path: valid columns as a 128-bit mask built per segment (a used
+        // segment's valid keys form one prefix of it)
+        uint64_t vm[2] = {0ull, 0ull};
         const uint32_t mask = inf.mask;
         const int nseg = kStageKeys >> a.seg_shift;
 #pragma unroll 1
         for (int sg = 0; sg < nseg; ++sg) {
           if (!((mask >> (2 * sg + half)) & 1u)) continue;
           const int nv = min(a.seg_keys, max(0, a.n_valid - inf.start[sg]));
-          const int lo = max(0, sg * a.seg_keys - ch * 64);
-          const int hi = min(64, sg * a.seg_keys + nv - ch * 64);
-          if (hi <= lo) continue;
-          const uint64_t upto = hi >= 64 ? ~0ull : ((1ull << hi) - 1ull);
-          vm |= upto & ~((1ull << lo) - 1ull);
-        }
+          const int lo = sg * a.seg_keys, hi = lo + nv;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (!((vm >> j) & 1ull)) r[0][j] = __float_as_uint(-INFINITY);
-          if (!((vm >> (32 + j)) & 1ull)) r[1][j] = __float_as_uint(-INFINITY);
-        }
-      }
-      float rmax = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) rmax = fmaxf(rmax, fmaxf(__uint_as_float(r[0][j]), __uint_as_float(r[1][j])));
-      // exchange the partial row max with the partner warp (same rows, other half)
-      xmax[(t & 1) * 256 + ch * 128 + row] = rmax;
-      mbar_arrive(&ctl->xbar[quad]);
-      ok = mbar_wait_warp(&ctl->xbar[quad], t & 1, abort, a.timeout_ns, lane);
-      if (!ok) break;
-      rmax = fmaxf(rmax, xmax[(t & 1) * 256 + (ch ^ 1) * 128 + row]);
-      const float m_new = fmaxf(m2, rmax * a.scale_log2);
-      const bool need = m_new > m2 + kRescaleThreshold || (m2 == -INFINITY && m_new != -INFINITY);
-      if (t > 0) {
-        ok = mbar_wait_warp(&ctl->pv_done, (t - 1) & 1, abort, a.timeout_ns, lane);
-        if (!ok) break;
-      }
-      if (__any_sync(0xffffffffu, need)) {
-        const float alpha = need ? fast_exp2(m2 - m_new) : 1.f;  // exp2(-inf) = 0
-        if (t > 0) {
-          // cold path: rescale this thread's half of the O row (and, in
-          // half 0, the rounded-P row sum) by alpha
-          tc_fence_after();
-#pragma unroll 1
-          for (int c = 0; c < D / 64 + (ch == 0 ? 1 : 0); ++c) {
-            const uint32_t col = c < D / 64 ? tO + ch * (D / 2) + c * 32 : tL;
-            uint32_t o[32];
-            tmem_ld32(col + lane_off, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-            tmem_st32(col + lane_off, o);
+          for (int w = 0; w < 2; ++w) {
+            const int l0 = max(0, lo - 64 * w), h0 = min(64, hi - 64 * w);
+            if (h0 > l0) {
+              const uint64_t upto = h0 >= 64 ? ~0ull : ((1ull << h0) - 1ull);
+              vm[w] |= upto & ~((1ull << l0) - 1ull);
+            }
           }
         }
-        if (need) {
-          l *= alpha;
-          m2 = m_new;
-        }
-      }
-      // P = exp2(s * scale * log2(e) - m2) as bf16 pairs over this thread's S columns
-      const bool live = m2 != -INFINITY;
-      const float neg_m = live ? -m2 : 0.f;
-      float rs = 0.f;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (!((vm[c >> 1] >> ((c & 1) * 32 + j)) & 1ull)) r[c][j] = __float_as_uint(-INFINITY);
+      }
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        mx[j & 3] = max3f(mx[j & 3], __uint_as_float(r[0][j]), __uint_as_float(r[1][j]));
+        mx[(j + 2) & 3] = max3f(mx[(j + 2) & 3], __uint_as_float(r[2][j]), __uint_as_float(r[3][j]));
+      }
+      const float rmax = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3]));
+      const float m_new = fmaxf(m2, rmax * a.scale_log2);
+      const bool need = m_new > m2 + kRescaleThreshold || (m2 == -INFINITY && m_new != -INFINITY);
+      const bool any_rescale = __any_sync(0xffffffffu, need);
+      float alpha = 1.f;
+      if (need) {
+        alpha = fast_exp2(m2 - m_new);  // exp2(-inf) = 0
+        l *= alpha;
+        lr *= alpha;
+        m2 = m_new;
+      }
+      // P = exp2(s * scale * log2(e) - m2).  While m2 is -inf every logit of
+      // the row is -inf (masked), so the exponent is -inf and P = 0.
+      const float neg_m = m2 != -INFINITY ? -m2 : 0.f;
+      const float2 nm2 = make_float2(neg_m, neg_m);
+      float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      float rr[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const float p0 = live ? fast_exp2(fmaf(__uint_as_float(r[c][2 * j]), a.scale_log2, neg_m)) : 0.f;
-          const float p1 = live ? fast_exp2(fmaf(__uint_as_float(r[c][2 * j + 1]), a.scale_log2, neg_m)) : 0.f;
-          rs += p0 + p1;
-          r[0][c * 16 + j] = pack_bf16x2(p0, p1);
+          const float2 x = ffma2(make_float2(__uint_as_float(r[c][2 * j]), __uint_as_float(r[c][2 * j + 1])), sc2, nm2);
+          const float2 p = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+          rs2[j & 1] = fadd2(rs2[j & 1], p);
+          const uint32_t pk = pack_bf16x2(p.x, p.y);
+          rr[j & 3] = add_bf16x2_f32(rr[j & 3], pk);
+          r[c >> 1][(c & 1) * 16 + j] = pk;  // packed in place over consumed logits
         }
       }
-      l += rs;
-      tmem_st32(tS[slot] + lane_off + ch * 32, r[0]);
+      const float2 rsum = fadd2(rs2[0], rs2[1]);
+      l += rsum.x + rsum.y;
+      lr += (rr[0] + rr[1]) + (rr[2] + rr[3]);
+      if (any_rescale && t >= 2) {
+        // cold path: rescale this group's O row by alpha (1 for rows whose max
+        // stayed).  P.V of stage t-2 was issued before S_t, so the commit that
+        // signalled S_t covers it; P.V of stage t waits for p_full below.
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO[g] + lane_off + c * 32, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          tmem_st32(tO[g] + lane_off + c * 32, o);
+        }
+      }
+      tmem_st32(tS[g] + lane_off + 0, r[0]);
+      tmem_st32(tS[g] + lane_off + 32, r[1]);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&ctl->s_free[slot]);
-      mbar_arrive(&ctl->p_full);
+      mbar_arrive(&ctl->s_free[g]);
+      mbar_arrive(&ctl->p_full[g]);
     }
 
     // ---------------------------------------------------------- epilogue
-    constexpr int DH = D / 2;  // output columns of this thread
-    const int grow = tile * kTileM + row;
-    const size_t orow = (size_t)bh * a.n_pad + grow;
-    float acc[DH];
-    float lr = 0.f;  // row sum of the rounded P (tensor core)
-    bool have = false;
-    if (ok && n_stages > 0) {
-      ok = mbar_wait_warp(&ctl->pv_done, (n_stages - 1) & 1, abort, a.timeout_ns, lane);
-      if (ok) {
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < DH / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + lane_off + ch * DH + c * 32, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) acc[c * 32 + j] = __uint_as_float(o[j]);
-        }
-        uint32_t o[32];
-        tmem_ld32(tL + lane_off, o);
-        tmem_ld_wait();
-        lr = __uint_as_float(o[0]);
-        have = true;
-      }
-    }
-    // full unrounded row sum from the two halves
-    xsum[ch * 128 + row] = l;
-    float lsum = l;
+    // exchange (max, sum, rounded sum) with the other group's thread of this row
+    float *xs = sX;  // [2][3][128]
+    xs[(g * 3 + 0) * 128 + row] = m2;
+    xs[(g * 3 + 1) * 128 + row] = l;
+    xs[(g * 3 + 2) * 128 + row] = lr;
+    float mo = -INFINITY, lo = 0.f, lro = 0.f;
     if (ok) {
       mbar_arrive(&ctl->xbar[quad]);
-      ok = mbar_wait_warp(&ctl->xbar[quad], n_stages & 1, abort, a.timeout_ns, lane);
-      if (ok) lsum += xsum[(ch ^ 1) * 128 + row];
+      ok = mbar_wait_warp(&ctl->xbar[quad], 0, abort, a.timeout_ns, lane);
+      if (ok) {
+        mo = xs[((g ^ 1) * 3 + 0) * 128 + row];
+        lo = xs[((g ^ 1) * 3 + 1) * 128 + row];
+        lro = xs[((g ^ 1) * 3 + 2) * 128 + row];
+      }
     }
-    have = have && ok;
-    const bool row_ok = grow < a.n_valid && have && lsum > 0.f && lr > 0.f;
-    const float inv_l = row_ok ? 1.f / lr : 0.f;
-    float lse = row_ok ? (m2 + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
-#pragma unroll
-    for (int c = 0; c < DH; ++c) acc[c] = row_ok ? acc[c] * inv_l : 0.f;
+    if (ok && n_stages > 0) {
+      // the MMA issuer commits mma_drain after its last P.V: one phase, no ambiguity
+      ok = mbar_wait_warp(&ctl->mma_drain, 0, abort, a.timeout_ns, lane);
+    }
+    // group 0 / 1 partial results -> exact merge
+    const float m0 = g == 0 ? m2 : mo, m1 = g == 0 ? mo : m2;
+    const float l0 = g == 0 ? l : lo, l1 = g == 0 ? lo : l;
+    const float r0 = g == 0 ? lr : lro, r1 = g == 0 ? lro : lr;
+    const float mm = fmaxf(m0, m1);
+    const bool live = ok && n_stages > 0 && mm != -INFINITY;
+    const float w0 = live && m0 != -INFINITY ? fast_exp2(m0 - mm) : 0.f;
+    const float w1 = live && m1 != -INFINITY ? fast_exp2(m1 - mm) : 0.f;
+    const float lsum = l0 * w0 + l1 * w1;
+    const float rsum = r0 * w0 + r1 * w1;
+    const int grow = tile * kTileM + row;
+    const size_t orow = (size_t)bh * a.n_pad + grow;
+    const bool row_ok = live && grow < a.n_valid && lsum > 0.f && rsum > 0.f;
+    const float s0 = row_ok ? w0 / rsum : 0.f, s1 = row_ok ? w1 / rsum : 0.f;
+    float lse = row_ok ? (mm + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
+    MergeWeights mw;
+    mw.wa = 0.f;
+    mw.wb = 1.f;
     if (a.merge_o != nullptr) {
       const float lm = grow < a.n_valid ? a.merge_lse[orow] : -INFINITY;
-      const MergeWeights w = lse_merge_weights(lm, lse);
-      const float4 *mo = reinterpret_cast<const float4 *>(a.merge_o + orow * D + ch * DH);
-#pragma unroll
-      for (int c = 0; c < DH / 4; ++c) {
-        const float4 v = mo[c];
-        acc[4 * c + 0] = w.wa * v.x + w.wb * acc[4 * c + 0];
-        acc[4 * c + 1] = w.wa * v.y + w.wb * acc[4 * c + 1];
-        acc[4 * c + 2] = w.wa * v.z + w.wb * acc[4 * c + 2];
-        acc[4 * c + 3] = w.wa * v.w + w.wb * acc[4 * c + 3];
-      }
-      lse = w.lse;
+      mw = lse_merge_weights(lm, lse);
+      lse = mw.lse;
     }
-    if (a.o_fp32) {
-      float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.o) + orow * D + ch * DH);
+    if (g == 0) a.lse[orow] = lse;
+    if (ok) tc_fence_after();
+    // this group writes columns [g * D/2, (g + 1) * D/2) of the row
+    constexpr int DH = D / 2;
+    // tcgen05.ld is warp-collective: load when any row of the warp needs it
+    const bool warp_loads = __any_sync(0xffffffffu, row_ok);
+#pragma unroll 1
+    for (int c = 0; c < DH / 32; ++c) {
+      const int col = g * DH + c * 32;
+      uint32_t oa[32], ob[32];
+      if (warp_loads) {
+        tmem_ld32(tO[0] + lane_off + col, oa);
+        tmem_ld32(tO[1] + lane_off + col, ob);
+        tmem_ld_wait();
+      }
+      float v[32];
 #pragma unroll
-      for (int c = 0; c < DH / 4; ++c) dst[c] = make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
-    } else {
-      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.o) + orow * D + ch * DH);
+      for (int j = 0; j < 32; ++j) {
+        float x = 0.f;
+        if (row_ok) {
+          // a group without stages never wrote its O: its weight is 0 and its columns are not read
+          x = (s0 > 0.f ? s0 * __uint_as_float(oa[j]) : 0.f) + (s1 > 0.f ? s1 * __uint_as_float(ob[j]) : 0.f);
+        }
+        v[j] = x;
+      }
+      if (a.merge_o != nullptr) {
+        const float4 *mo4 = reinterpret_cast<const float4 *>(a.merge_o + orow * D + col);
 #pragma unroll
-      for (int c = 0; c < DH / 8; ++c) {
-        uint4 pk;
-        pk.x = pack_bf16x2(acc[8 * c + 0], acc[8 * c + 1]);
-        pk.y = pack_bf16x2(acc[8 * c + 2], acc[8 * c + 3]);
-        pk.z = pack_bf16x2(acc[8 * c + 4], acc[8 * c + 5]);
-        pk.w = pack_bf16x2(acc[8 * c + 6], acc[8 * c + 7]);
-        dst[c] = pk;
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 m = mo4[q4];
+          v[4 * q4 + 0] = mw.wa * m.x + mw.wb * v[4 * q4 + 0];
+          v[4 * q4 + 1] = mw.wa * m.y + mw.wb * v[4 * q4 + 1];
+          v[4 * q4 + 2] = mw.wa * m.z + mw.wb * v[4 * q4 + 2];
+          v[4 * q4 + 3] = mw.wa * m.w + mw.wb * v[4 * q4 + 3];
+        }
+      }
+      if (a.o_fp32) {
+        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.o) + orow * D + col);
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+      } else {
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.o) + orow * D + col);
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          uint4 pk;
+          pk.x = pack_bf16x2(v[8 * q8 + 0], v[8 * q8 + 1]);
+          pk.y = pack_bf16x2(v[8 * q8 + 2], v[8 * q8 + 3]);
+          pk.z = pack_bf16x2(v[8 * q8 + 4], v[8 * q8 + 5]);
+          pk.w = pack_bf16x2(v[8 * q8 + 6], v[8 * q8 + 7]);
+          dst[q8] = pk;
+        }
       }
     }
-    if (ch == 0) a.lse[orow] = lse;
   }
 
   // ---------------------------------------------------------------- teardown
