@@ -250,10 +250,13 @@ class SparseVideoAttention:
     reused; outputs of the last call stay readable in ``self.buf``.
     """
 
-    def __init__(self, cfg: PathConfig):
+    def __init__(self, cfg: PathConfig, workspace_for_all_heads: bool = False):
         self.cfg = cfg
         self.buf: Dict[str, torch.Tensor] = {}
         self._key = None
+        # size the Micro workspace as if every head were enabled (callers that
+        # pass different per-call head flags)
+        self._ws_all = workspace_for_all_heads
 
     def _alloc(self, q: torch.Tensor):
         B, H, n_pad, d = q.shape
@@ -276,7 +279,8 @@ class SparseVideoAttention:
             n_r, n_t = n_pad // 64, n_pad // 16
             cap = c.micro_capacity or n_t
             shape = _shape(B, H, c.n_valid, n_pad, d)
-            ws = select_micro_workspace_bytes(shape, c.micro_mode, c.micro_topk, c.micro_percentile, c.micro_heads, cap)
+            ws = select_micro_workspace_bytes(shape, c.micro_mode, c.micro_topk, c.micro_percentile,
+                                              None if self._ws_all else c.micro_heads, cap)
             b.update({
                 "q_pool64": torch.empty(B, H, n_r, d, device=dev, dtype=f32),
                 "k_pool16": torch.empty(B, H, n_t, d, device=dev, dtype=f32),
@@ -290,7 +294,14 @@ class SparseVideoAttention:
         self.buf = b
         self._key = key
 
-    def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None) -> Dict[str, torch.Tensor]:
+    def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None, out_o=None, out_lse=None,
+                 micro_heads=None) -> Dict[str, torch.Tensor]:
+        """Run the whole path on device tensors q, k, v [B, H, n_pad, d] (bf16).
+
+        Outputs go to ``self.buf["o"]`` / ``["lse"]``, or to ``out_o`` /
+        ``out_lse`` when given (same shapes).  ``micro_heads`` overrides the
+        configured per-head Micro flags (length H).
+        """
         c = self.cfg
         self._alloc(q)
         b = self.buf
@@ -299,19 +310,71 @@ class SparseVideoAttention:
         scale = c.scale if c.scale is not None else 1.0 / math.sqrt(d)
         n_k = n_pad // c.bk
         micro = c.micro_mode != 0
+        o = b["o"] if out_o is None else out_o
+        lse = b["lse"] if out_lse is None else out_lse
+        heads = c.micro_heads if micro_heads is None else micro_heads
         pool_qk(q, k, shape, c.bq, c.bk, b["q_pool"], b["k_pool"], b.get("q_pool64"), b.get("k_pool16"), stream)
         select_blocks(b["q_pool"], b["k_pool"], shape, c.bq, c.bk, scale,
                       SelectParams(c.k_min, c.cum_mass, c.fixed_k, c.n_anchor, c.anchor_rot), b["counts"], b["idx"],
                       None, stream)
         if not micro:
-            block_sparse_fwd(q, k, v, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, scale, b["o"], b["lse"],
-                             stream=stream)
+            block_sparse_fwd(q, k, v, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, scale, o, lse, stream=stream)
             return b
         block_sparse_fwd(q, k, v, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, scale, b["o_macro"],
                          b["lse_macro"], stream=stream)
         select_micro(b["q_pool64"], b["k_pool16"], b["counts"], b["idx"], shape, c.bq, c.bk, scale, c.micro_mode,
-                     c.micro_topk, c.micro_percentile, c.micro_heads, self.micro_cap, b["m_counts"], b["m_idx"],
+                     c.micro_topk, c.micro_percentile, heads, self.micro_cap, b["m_counts"], b["m_idx"],
                      b["workspace"], stream)
-        block_sparse_fwd(q, k, v, shape, 64, 16, b["m_counts"], b["m_idx"], self.micro_cap, scale, b["o"], b["lse"],
+        block_sparse_fwd(q, k, v, shape, 64, 16, b["m_counts"], b["m_idx"], self.micro_cap, scale, o, lse,
                          b["o_macro"], b["lse_macro"], stream)
         return b
+
+    def forward_host(self, q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor, o_h: torch.Tensor,
+                     lse_h: torch.Tensor, chunk_heads: int = 4, device=None) -> None:
+        """The whole path on HOST tensors: pinned bf16 q_h, k_h, v_h [B, H, n_pad, d]
+        in, pinned o_h (bf16, same shape) and lse_h (fp32 [B, H, n_pad]) out.
+
+        Every (batch, head) is an independent problem, so the heads are cut into
+        chunks and pipelined over three streams: host-to-device copies of chunk
+        i+1 and device-to-host copies of chunk i-1 overlap the path on chunk i.
+        Results are exactly those of running the path on all heads at once.
+        Returns once the enqueued work is complete.
+        """
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        B, H, n_pad, d = q_h.shape
+        BH = B * H
+        key = (B, H, n_pad, d, dev, chunk_heads)
+        if getattr(self, "_host_key", None) != key:
+            bf = torch.bfloat16
+            self._hbuf = {
+                "q": torch.empty(BH, n_pad, d, device=dev, dtype=bf),
+                "k": torch.empty(BH, n_pad, d, device=dev, dtype=bf),
+                "v": torch.empty(BH, n_pad, d, device=dev, dtype=bf),
+                "o": torch.empty(BH, n_pad, d, device=dev, dtype=bf),
+                "lse": torch.empty(BH, n_pad, device=dev, dtype=torch.float32),
+            }
+            self._chunk = SparseVideoAttention(self.cfg, workspace_for_all_heads=True)
+            self._s_in = torch.cuda.Stream(dev)
+            self._s_out = torch.cuda.Stream(dev)
+            self._host_key = key
+        hb = self._hbuf
+        qf, kf, vf = (x.view(BH, n_pad, d) for x in (q_h, k_h, v_h))
+        of, lf = o_h.view(BH, n_pad, d), lse_h.view(BH, n_pad)
+        flags = None
+        if self.cfg.micro_mode and self.cfg.micro_heads is not None:
+            flags = [int(self.cfg.micro_heads[i % H]) for i in range(BH)]
+        comp = torch.cuda.current_stream(dev)
+        for c0 in range(0, BH, chunk_heads):
+            c1 = min(BH, c0 + chunk_heads)
+            with torch.cuda.stream(self._s_in):
+                for dst, src in ((hb["q"], qf), (hb["k"], kf), (hb["v"], vf)):
+                    dst[c0:c1].copy_(src[c0:c1], non_blocking=True)
+            comp.wait_stream(self._s_in)
+            view = lambda t: t[c0:c1].unsqueeze(0)
+            self._chunk(view(hb["q"]), view(hb["k"]), view(hb["v"]), stream=comp, out_o=view(hb["o"]),
+                        out_lse=view(hb["lse"]), micro_heads=None if flags is None else flags[c0:c1])
+            self._s_out.wait_stream(comp)
+            with torch.cuda.stream(self._s_out):
+                of[c0:c1].copy_(hb["o"][c0:c1], non_blocking=True)
+                lf[c0:c1].copy_(hb["lse"][c0:c1], non_blocking=True)
+        self._s_out.synchronize()

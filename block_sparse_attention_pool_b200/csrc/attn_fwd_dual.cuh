@@ -1,0 +1,422 @@
+// a4 Macro pass, two query tiles per CTA sharing their K/V loads.
+//
+// HyperVAttention section 2 Eq. (4): each query block attends to its selected
+// key blocks; section 4.3: the selected blocks of a row are walked as one
+// packed sequence.  Neighbouring query blocks of a video select overlapping
+// key blocks (spatio-temporal locality), so a CTA that owns two adjacent
+// 128-row query tiles A and B walks the ascending union of their two lists,
+// loads each union block's K and V once, and issues the S and P.V MMAs only
+// for the tile(s) whose list holds that block: every MMA is useful, and each
+// K/V byte feeds up to 256 query rows instead of 128.  This is the layout for
+// 128x128 blocks (list rows = 128, one 128-key list entry per stage).
+//
+// Warp roles (320 threads):
+//   warp 0     TMA producer: Q_A and Q_B once, then K and V of every union
+//              block into 2 + 2 ring slots (rows past n_valid arrive as zeros).
+//   warp 1     MMA issuer: walks the same union (warp-lockstep cursor) and,
+//              per union block s, issues for each tile X that uses it
+//              O_X += P_X(prev) V(prev) for X's previous block when that was
+//              block s-1, then S_X = Q_X K_s^T into TMEM buffer S_X.  Blocks
+//              of A and B interleave on the tensor core, so one tile's MMAs
+//              run while the other tile's softmax works (ping-pong).
+//   warps 2-5  softmax of tile A, warps 6-9 softmax of tile B: one thread
+//              per query row walks its tile's own list, reads the S row from
+//              TMEM, masks keys past n_valid, keeps the running reference max
+//              in the log2 domain with lazy rescale of its TMEM O row (only
+//              when the max grew by more than 2^8), writes P as bf16 pairs back
+//              over the first 64 S columns (the A operand of P.V), and keeps
+//              the fp32 row sum (for LSE) and the rounded-P row sum (to
+//              normalise O: an exact convex combination of the V rows used).
+// TMEM: S_A [0,128), S_B [128,256), O_A [256, 256 + d), O_B [384, 384 + d).
+//
+// Barrier phases: s_full[X] and p_full[X] advance once per block of tile X;
+// S_X of X's next block is issued only after the MMA issuer waited p_full[X]
+// of the current one, so neither can run two phases ahead of its waiter.  The
+// commit that signals S_X(s) also covers P.V of X's previous block (issued
+// before it), which is what a lazy rescale of O_X needs.  The K/V ring slots
+// are released by commits after the last MMA that reads them.
+#pragma once
+
+#include "attn_fwd.cuh"
+
+namespace vsa {
+
+template <int D>
+struct DualSmem {
+  static constexpr int kQBytes = kTileM * D * 2;
+  static constexpr int kKVBytes = kStageKeys * D * 2;
+  static constexpr int kOffQ = 0;                       // Q_A, Q_B
+  static constexpr int kOffK = kOffQ + 2 * kQBytes;
+  static constexpr int kOffV = kOffK + 2 * kKVBytes;
+  static constexpr int kOffCtl = kOffV + 2 * kKVBytes;
+  static constexpr int kBytes = kOffCtl + 512;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+struct DualCtl {
+  uint64_t q_full;
+  uint64_t k_full[2], k_empty[2];
+  uint64_t v_full[2], v_empty[2];
+  uint64_t s_full[2];  // per tile
+  uint64_t p_full[2];  // per tile
+  uint64_t mma_drain;
+  uint32_t tmem_base;
+  int abort;
+  int n_union;
+  int cnt[2];
+};
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_fwd_dual_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
+  using L = DualSmem<D>;
+  extern __shared__ uint8_t dual_smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dual_smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  uint8_t *sQ = smem + L::kOffQ;
+  uint8_t *sK = smem + L::kOffK;
+  uint8_t *sV = smem + L::kOffV;
+  DualCtl *ctl = reinterpret_cast<DualCtl *>(smem + L::kOffCtl);
+  volatile int *abort = &ctl->abort;
+
+  const int pair = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_tiles = a.n_pad / kTileM;
+  const int tile0 = 2 * pair;
+  const bool has_b = tile0 + 1 < n_tiles;
+  const int n_key_blocks = a.n_pad / kStageKeys;
+  const size_t lrow0 = (size_t)bh * n_tiles + tile0;  // list row of tile A (list rows = 128)
+
+  // ---------------------------------------------------------------- setup
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_init(&ctl->q_full, 1);
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&ctl->k_full[i], 1);
+        mbar_init(&ctl->k_empty[i], 1);
+        mbar_init(&ctl->v_full[i], 1);
+        mbar_init(&ctl->v_empty[i], 1);
+        mbar_init(&ctl->s_full[i], 1);
+        mbar_init(&ctl->p_full[i], 128);
+      }
+      mbar_init(&ctl->mma_drain, 1);
+      ctl->abort = 0;
+      fence_barrier_init();
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+    int cnt[2] = {0, 0};
+    bool ok = true;
+    for (int x = 0; x < (has_b ? 2 : 1); ++x) {
+      cnt[x] = __ldg(a.counts + lrow0 + x);
+      if (cnt[x] < 0 || cnt[x] > a.idx_stride) ok = false;
+    }
+    for (int x = 0; x < (has_b ? 2 : 1) && ok; ++x)
+      ok = list_valid(a.idx + (lrow0 + x) * a.idx_stride, cnt[x], n_key_blocks, lane);
+    int n_union = 0;
+    if (!ok) {
+      if (lane == 0) latch_status(VSA_ERR_BAD_INDEX);
+      cnt[0] = cnt[1] = 0;
+    } else {
+      n_union = cnt[0] + cnt[1] -
+                (has_b ? list_intersection(a.idx + lrow0 * a.idx_stride, cnt[0], a.idx + (lrow0 + 1) * a.idx_stride,
+                                           cnt[1], lane)
+                       : 0);
+    }
+    if (lane == 0) {
+      ctl->n_union = n_union;
+      ctl->cnt[0] = cnt[0];
+      ctl->cnt[1] = cnt[1];
+    }
+  } else if (warp == 1) {
+    tmem_alloc(&ctl->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const int n_union = ctl->n_union;
+  const uint32_t tmem = ctl->tmem_base;
+  const uint32_t tS[2] = {tmem, tmem + 128u};
+  const uint32_t tO[2] = {tmem + 256u, tmem + 384u};
+  const int32_t *list[2] = {a.idx + lrow0 * a.idx_stride, a.idx + (lrow0 + 1) * a.idx_stride};
+  const int cnt[2] = {ctl->cnt[0], has_b ? ctl->cnt[1] : 0};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (n_union > 0) {
+      ListCursor cur;
+      cur.init(list[0], cnt[0], has_b ? list[1] : nullptr, cnt[1], has_b ? 2 : 1, lane);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&ctl->q_full, (has_b ? 2 : 1) * L::kQBytes);
+        for (int x = 0; x < (has_b ? 2 : 1); ++x)
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sQ + x * L::kQBytes + c * kChunkBytes, &tm_q, &ctl->q_full, c * 64, (tile0 + x) * kTileM, bh);
+      }
+      int issued = 0;
+      for (int s = 0; s < n_union; ++s) {
+        const int slot = s & 1;
+        const uint32_t use_par = ((s >> 1) - 1) & 1;
+        uint32_t m = 0u;
+        const int blk = cur.next(&m, lane);
+        const int start = blk * kStageKeys;
+        bool ok = true;
+        if (s >= 2) ok = mbar_wait_warp(&ctl->k_empty[slot], use_par, abort, a.timeout_ns, lane);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&ctl->k_full[slot], L::kKVBytes);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sK + slot * L::kKVBytes + c * kChunkBytes, &tm_k, &ctl->k_full[slot], c * 64, start, bh);
+        }
+        if (s >= 2) ok = mbar_wait_warp(&ctl->v_empty[slot], use_par, abort, a.timeout_ns, lane);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&ctl->v_full[slot], L::kKVBytes);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sV + slot * L::kKVBytes + c * kChunkBytes, &tm_v, &ctl->v_full[slot], c * 64, start, bh);
+        }
+        issued = s + 1;
+        __syncwarp();
+      }
+      if (*abort && lane == 0) {
+        mbar_drain(&ctl->q_full, 0, a.timeout_ns);
+        for (int s = max(0, issued - 2); s < issued; ++s) {
+          mbar_drain(&ctl->k_full[s & 1], (s >> 1) & 1, a.timeout_ns);
+          mbar_drain(&ctl->v_full[s & 1], (s >> 1) & 1, a.timeout_ns);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (n_union > 0) {
+      constexpr uint32_t kIdS = idesc_bf16_f32(kTileM, kStageKeys, false);
+      constexpr uint32_t kIdO = idesc_bf16_f32(kTileM, D, true);
+      const uint32_t q_addr = smem_addr(sQ), k_addr = smem_addr(sK), v_addr = smem_addr(sV);
+      ListCursor cur;
+      cur.init(list[0], cnt[0], has_b ? list[1] : nullptr, cnt[1], has_b ? 2 : 1, lane);
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(&ctl->q_full, 0, abort, a.timeout_ns);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      uint32_t prev = 0u;     // usage bits of the previous union block
+      int nx[2] = {0, 0};     // blocks of each tile seen so far
+      int pv_done[2] = {0, 0};  // P.V issued so far per tile
+      auto issue_pv = [&](int x, int s) -> bool {
+        // O_x += P_x(block s) V_s
+        if (!mbar_wait(&ctl->p_full[x], pv_done[x] & 1, abort, a.timeout_ns)) return false;
+        if (!mbar_wait(&ctl->v_full[s & 1], (s >> 1) & 1, abort, a.timeout_ns)) return false;
+        tc_fence_after();
+        const uint32_t vb = v_addr + (s & 1) * L::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < kStageKeys / 16; ++kk) {
+          const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, kChunkBytes, 1024);
+          umma_bf16_ts(tO[x], tS[x] + kk * 8, bd, kIdO, (pv_done[x] > 0 || kk > 0) ? 1u : 0u);
+        }
+        ++pv_done[x];
+        return true;
+      };
+      for (int s = 0; s < n_union; ++s) {
+        uint32_t use = 0u;
+        cur.next(&use, lane);  // whole warp walks the union in lockstep
+        if (!has_b) use &= 1u;  // a single-list cursor tags every block with both bits
+        if (lane == 0 && ok) {
+          bool k_ready = false;
+          for (int x = 0; x < 2 && ok; ++x) {
+            // P.V of x's block s-1 first: S_x(s) overwrites the S buffer that holds P_x(s-1)
+            if ((prev >> x) & 1u) ok = issue_pv(x, s - 1);
+            if (ok && ((use >> x) & 1u)) {
+              if (!k_ready) {
+                ok = mbar_wait(&ctl->k_full[s & 1], (s >> 1) & 1, abort, a.timeout_ns);
+                k_ready = true;
+                if (!ok) break;
+              }
+              tc_fence_after();
+              const uint32_t qb = q_addr + x * L::kQBytes;
+              const uint32_t kb = k_addr + (s & 1) * L::kKVBytes;
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t ad = smem_desc_sw128(qb + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
+                const uint64_t bd = smem_desc_sw128(kb + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
+                umma_bf16_ss(tS[x], ad, bd, kIdS, kk > 0 ? 1u : 0u);
+              }
+              umma_commit(&ctl->s_full[x]);
+              ++nx[x];
+            }
+          }
+          if (ok) {
+            umma_commit(&ctl->k_empty[s & 1]);                 // S MMAs of block s read K_s
+            if (s >= 1) umma_commit(&ctl->v_empty[(s - 1) & 1]);  // P.V of block s-1 read V_{s-1}
+          }
+        }
+        prev = use;
+      }
+      if (lane == 0) {
+        if (ok) {
+          for (int x = 0; x < 2 && ok; ++x)
+            if ((prev >> x) & 1u) ok = issue_pv(x, n_union - 1);
+          if (ok) umma_commit(&ctl->v_empty[(n_union - 1) & 1]);
+        }
+        umma_commit(&ctl->mma_drain);
+        mbar_drain(&ctl->mma_drain, 0, a.timeout_ns);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int x = (warp - 2) >> 2;  // tile
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const bool tile_live = x == 0 || has_b;
+    float m2 = -INFINITY;  // running reference max of scaled logits, log2 units
+    float l = 0.f;         // fp32 row sum of P
+    float lr = 0.f;        // row sum of the bf16-rounded P
+    bool ok = true;
+    const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+    const int n_mine = tile_live && n_union > 0 ? cnt[x] : 0;
+    for (int i = 0; i < n_mine; ++i) {
+      const int key0 = __ldg(list[x] + i) * kStageKeys;
+      ok = mbar_wait_warp(&ctl->s_full[x], i & 1, abort, a.timeout_ns, lane);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS[x] + lane_off + c * 32, r[c]);
+      tmem_ld_wait();
+      const int nv = a.n_valid - key0;  // valid keys of this block
+      if (nv < kStageKeys) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c * 32 + j >= nv) r[c][j] = __float_as_uint(-INFINITY);
+      }
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        mx[j & 3] = max3f(mx[j & 3], __uint_as_float(r[0][j]), __uint_as_float(r[1][j]));
+        mx[(j + 2) & 3] = max3f(mx[(j + 2) & 3], __uint_as_float(r[2][j]), __uint_as_float(r[3][j]));
+      }
+      const float rmax = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3]));
+      const float m_new = fmaxf(m2, rmax * a.scale_log2);
+      const bool need = m_new > m2 + kRescaleThreshold || (m2 == -INFINITY && m_new != -INFINITY);
+      const bool any_rescale = __any_sync(0xffffffffu, need);
+      float alpha = 1.f;
+      if (need) {
+        alpha = fast_exp2(m2 - m_new);  // exp2(-inf) = 0
+        l *= alpha;
+        lr *= alpha;
+        m2 = m_new;
+      }
+      const float neg_m = m2 != -INFINITY ? -m2 : 0.f;
+      const float2 nm2 = make_float2(neg_m, neg_m);
+      float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      float rr[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float2 xx = ffma2(make_float2(__uint_as_float(r[c][2 * j]), __uint_as_float(r[c][2 * j + 1])), sc2, nm2);
+          const float2 p = make_float2(fast_exp2(xx.x), fast_exp2(xx.y));
+          rs2[j & 1] = fadd2(rs2[j & 1], p);
+          const uint32_t pk = pack_bf16x2(p.x, p.y);
+          rr[j & 3] = add_bf16x2_f32(rr[j & 3], pk);
+          r[c >> 1][(c & 1) * 16 + j] = pk;
+        }
+      }
+      const float2 rsum = fadd2(rs2[0], rs2[1]);
+      l += rsum.x + rsum.y;
+      lr += (rr[0] + rr[1]) + (rr[2] + rr[3]);
+      if (any_rescale && i > 0) {
+        // cold path: the commit that signalled this S also covered the P.V of
+        // the tile's previous block, so O_x is settled
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO[x] + lane_off + c * 32, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          tmem_st32(tO[x] + lane_off + c * 32, o);
+        }
+      }
+      tmem_st32(tS[x] + lane_off + 0, r[0]);
+      tmem_st32(tS[x] + lane_off + 32, r[1]);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&ctl->p_full[x]);
+    }
+
+    // ---------------------------------------------------------- epilogue
+    if (tile_live) {
+      if (ok && n_mine > 0) ok = mbar_wait_warp(&ctl->mma_drain, 0, abort, a.timeout_ns, lane);
+      const int grow = (tile0 + x) * kTileM + row;
+      const size_t orow = (size_t)bh * a.n_pad + grow;
+      const bool row_ok = ok && n_mine > 0 && grow < a.n_valid && l > 0.f && lr > 0.f;
+      const float inv = row_ok ? 1.f / lr : 0.f;
+      float lse = row_ok ? (m2 + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      MergeWeights mw;
+      mw.wa = 0.f;
+      mw.wb = 1.f;
+      if (a.merge_o != nullptr) {
+        const float lm = grow < a.n_valid ? a.merge_lse[orow] : -INFINITY;
+        mw = lse_merge_weights(lm, lse);
+        lse = mw.lse;
+      }
+      a.lse[orow] = lse;
+      const bool warp_loads = __any_sync(0xffffffffu, row_ok);
+      if (warp_loads) tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (warp_loads) {
+          tmem_ld32(tO[x] + lane_off + c * 32, o);
+          tmem_ld_wait();
+        }
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = row_ok ? __uint_as_float(o[j]) * inv : 0.f;
+        if (a.merge_o != nullptr) {
+          const float4 *mo4 = reinterpret_cast<const float4 *>(a.merge_o + orow * D + c * 32);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 mm = mo4[q4];
+            v[4 * q4 + 0] = mw.wa * mm.x + mw.wb * v[4 * q4 + 0];
+            v[4 * q4 + 1] = mw.wa * mm.y + mw.wb * v[4 * q4 + 1];
+            v[4 * q4 + 2] = mw.wa * mm.z + mw.wb * v[4 * q4 + 2];
+            v[4 * q4 + 3] = mw.wa * mm.w + mw.wb * v[4 * q4 + 3];
+          }
+        }
+        if (a.o_fp32) {
+          float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.o) + orow * D + c * 32);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+        } else {
+          uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.o) + orow * D + c * 32);
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            uint4 pk;
+            pk.x = pack_bf16x2(v[8 * q8 + 0], v[8 * q8 + 1]);
+            pk.y = pack_bf16x2(v[8 * q8 + 2], v[8 * q8 + 3]);
+            pk.z = pack_bf16x2(v[8 * q8 + 4], v[8 * q8 + 5]);
+            pk.w = pack_bf16x2(v[8 * q8 + 6], v[8 * q8 + 7]);
+            dst[q8] = pk;
+          }
+        }
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace vsa

@@ -23,7 +23,7 @@ namespace vsa {
 
 constexpr int kSelRows = 16;
 constexpr int kSelThreads = 256;
-constexpr int kSelChunk = 32;
+constexpr int kSelChunk = 64;
 
 struct SelectArgs {
   const float *q_pool;  // [BH, n_q, d]
@@ -37,14 +37,42 @@ struct SelectArgs {
   uint8_t *mask;    // [BH, n_q, n_k] or null
 };
 
+// Compare-exchange of the in-register pairs (i, i | J) of a bitonic substage.
+template <int NR, int J>
+__device__ __forceinline__ void bitonic_in_lane(uint64_t (&key)[NR], int lane, int kk) {
+#pragma unroll
+  for (int i = 0; i < NR; ++i) {
+    if ((i & J) == 0) {
+      const bool desc = ((lane * NR + i) & kk) == 0;
+      const uint64_t a = key[i], b = key[i | J];
+      const bool swap = desc ? (a < b) : (a > b);
+      key[i] = swap ? b : a;
+      key[i | J] = swap ? a : b;
+    }
+  }
+}
+
+template <int NR, int J>
+__device__ __forceinline__ void bitonic_in_lane_dispatch(uint64_t (&key)[NR], int lane, int kk, int j) {
+  if constexpr (J >= 1) {
+    if (j == J) {
+      bitonic_in_lane<NR, J>(key, lane, kk);
+      return;
+    }
+    bitonic_in_lane_dispatch<NR, J / 2>(key, lane, kk, j);
+  }
+}
+
 // Bitonic sort, descending, of NR * 32 64-bit keys held NR per lane; the key at
-// sorted position e = lane * NR + i ends in register i of that lane.
+// sorted position e = lane * NR + i ends in register i of that lane.  The
+// stage loops run at run time and only the per-register bodies are unrolled,
+// which keeps the code small enough for the instruction cache.
 template <int NR>
 __device__ __forceinline__ void warp_bitonic_sort_desc(uint64_t (&key)[NR], int lane) {
   constexpr int N = NR * 32;
-#pragma unroll
+#pragma unroll 1
   for (int kk = 2; kk <= N; kk <<= 1) {
-#pragma unroll
+#pragma unroll 1
     for (int j = kk >> 1; j > 0; j >>= 1) {
       if (j >= NR) {
         // partner in lane ^ (j / NR), same register
@@ -52,25 +80,14 @@ __device__ __forceinline__ void warp_bitonic_sort_desc(uint64_t (&key)[NR], int 
         const bool lower = (lane & lx) == 0;
 #pragma unroll
         for (int i = 0; i < NR; ++i) {
-          const int e = lane * NR + i;
-          const bool desc = (e & kk) == 0;
+          const bool desc = ((lane * NR + i) & kk) == 0;
           const uint64_t other = __shfl_xor_sync(0xffffffffu, key[i], lx);
           const uint64_t mx = key[i] > other ? key[i] : other;
           const uint64_t mn = key[i] > other ? other : key[i];
           key[i] = (desc == lower) ? mx : mn;
         }
       } else {
-#pragma unroll
-        for (int i = 0; i < NR; ++i) {
-          if ((i & j) == 0) {
-            const int e = lane * NR + i;
-            const bool desc = (e & kk) == 0;
-            const uint64_t a = key[i], b = key[i | j];
-            const bool swap = desc ? (a < b) : (a > b);
-            key[i] = swap ? b : a;
-            key[i | j] = swap ? a : b;
-          }
-        }
+        bitonic_in_lane_dispatch<NR, (NR > 1 ? NR / 2 : 0)>(key, lane, kk, j);
       }
     }
   }
@@ -125,9 +142,8 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     *reinterpret_cast<float4 *>(qs + r * DP + c4 * 4) = v;
   }
 
-  // ---- logits: thread -> (row t/16, keys (t%16) and (t%16)+16 of the chunk)
-  const int my_row = t >> 4;
-  const int my_key = t & 15;
+  // ---- logits: warp w -> rows 2w, 2w+1; lane -> keys lane, lane + 32 of the chunk
+  const int r0 = 2 * warp;
   for (int k0 = 0; k0 < a.n_k; k0 += kSelChunk) {
     __syncthreads();
     for (int i = t; i < kSelChunk * (D / 4); i += kSelThreads) {
@@ -137,20 +153,28 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
       *reinterpret_cast<float4 *>(ks + r * DP + c4 * 4) = v;
     }
     __syncthreads();
-    float s0 = 0.f, s1 = 0.f;
-    const float *qrow = qs + my_row * DP;
-    const float *k0row = ks + my_key * DP;
-    const float *k1row = ks + (my_key + 16) * DP;
+    float s00 = 0.f, s01 = 0.f, s10 = 0.f, s11 = 0.f;
+    const float *q0 = qs + r0 * DP, *q1 = qs + (r0 + 1) * DP;
+    const float *ka = ks + lane * DP, *kb = ks + (lane + 32) * DP;
 #pragma unroll 8
     for (int c = 0; c < D; c += 4) {
-      const float4 qv = *reinterpret_cast<const float4 *>(qrow + c);
-      const float4 a0 = *reinterpret_cast<const float4 *>(k0row + c);
-      const float4 a1 = *reinterpret_cast<const float4 *>(k1row + c);
-      s0 = fmaf(qv.x, a0.x, s0); s0 = fmaf(qv.y, a0.y, s0); s0 = fmaf(qv.z, a0.z, s0); s0 = fmaf(qv.w, a0.w, s0);
-      s1 = fmaf(qv.x, a1.x, s1); s1 = fmaf(qv.y, a1.y, s1); s1 = fmaf(qv.z, a1.z, s1); s1 = fmaf(qv.w, a1.w, s1);
+      const float4 x0 = *reinterpret_cast<const float4 *>(q0 + c);
+      const float4 x1 = *reinterpret_cast<const float4 *>(q1 + c);
+      const float4 ya = *reinterpret_cast<const float4 *>(ka + c);
+      const float4 yb = *reinterpret_cast<const float4 *>(kb + c);
+      s00 = fmaf(x0.x, ya.x, s00); s00 = fmaf(x0.y, ya.y, s00); s00 = fmaf(x0.z, ya.z, s00); s00 = fmaf(x0.w, ya.w, s00);
+      s01 = fmaf(x0.x, yb.x, s01); s01 = fmaf(x0.y, yb.y, s01); s01 = fmaf(x0.z, yb.z, s01); s01 = fmaf(x0.w, yb.w, s01);
+      s10 = fmaf(x1.x, ya.x, s10); s10 = fmaf(x1.y, ya.y, s10); s10 = fmaf(x1.z, ya.z, s10); s10 = fmaf(x1.w, ya.w, s10);
+      s11 = fmaf(x1.x, yb.x, s11); s11 = fmaf(x1.y, yb.y, s11); s11 = fmaf(x1.z, yb.z, s11); s11 = fmaf(x1.w, yb.w, s11);
     }
-    if (k0 + my_key < nkp) S[my_row * nkp + k0 + my_key] = s0 * a.scale;
-    if (k0 + my_key + 16 < nkp) S[my_row * nkp + k0 + my_key + 16] = s1 * a.scale;
+    if (k0 + lane < nkp) {
+      S[r0 * nkp + k0 + lane] = s00 * a.scale;
+      S[(r0 + 1) * nkp + k0 + lane] = s10 * a.scale;
+    }
+    if (k0 + lane + 32 < nkp) {
+      S[r0 * nkp + k0 + lane + 32] = s01 * a.scale;
+      S[(r0 + 1) * nkp + k0 + lane + 32] = s11 * a.scale;
+    }
   }
   __syncthreads();
 

@@ -16,6 +16,7 @@
 
 #include "../../include/vsa.h"
 #include "attn_fwd.cuh"
+#include "attn_fwd_dual.cuh"
 #include "common.cuh"
 #include "merge.cuh"
 #include "micro.cuh"
@@ -95,6 +96,28 @@ vsa_status launch_attn(const void *q, const void *k, const void *v, const vsa_sh
     return VSA_ERR_CUDA;
   dim3 grid(s->n_pad / vsa::kTileM, s->B * s->H);
   vsa::attn_fwd_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, a);
+  return launch_status();
+}
+
+// 128-row lists of 128-key blocks: two adjacent query tiles per CTA share
+// their K/V loads (attn_fwd_dual_kernel).
+template <int D>
+vsa_status launch_attn_dual(const void *q, const void *k, const void *v, const vsa_shape *s, const AttnArgs &a,
+                            cudaStream_t st) {
+  using L = vsa::DualSmem<D>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err =
+        cudaFuncSetAttribute(vsa::attn_fwd_dual_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  });
+  if (attr_err != cudaSuccess) return VSA_ERR_CUDA;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, s, vsa::kTileM) || !make_map(&mk, k, s, vsa::kStageKeys) || !make_map(&mv, v, s, vsa::kStageKeys))
+    return VSA_ERR_CUDA;
+  const int n_tiles = s->n_pad / vsa::kTileM;
+  dim3 grid((n_tiles + 1) / 2, s->B * s->H);
+  vsa::attn_fwd_dual_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, a);
   return launch_status();
 }
 
@@ -452,6 +475,8 @@ vsa_status vsa_block_sparse_fwd(const void *q, const void *k, const void *v, con
   a.merge_lse = merge_lse;
   a.timeout_ns = kWaitLimitNs;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (list_rows == 128 && seg_keys == 128)
+    return shape->d == 128 ? launch_attn_dual<128>(q, k, v, shape, a, st) : launch_attn_dual<64>(q, k, v, shape, a, st);
   return shape->d == 128 ? launch_attn<128>(q, k, v, shape, a, st) : launch_attn<64>(q, k, v, shape, a, st);
 }
 

@@ -197,29 +197,33 @@ def test_attention_sweep_points(point):
     print(f"\nsweep {w.name} worst:", _attention_case(w, q, k, v, kept, blocks))
 
 
-def test_attention_ragged_and_empty_rows():
+@pytest.mark.parametrize("n_pad,list_rows,seg", [(512, 128, 32), (512, 64, 32), (512, 64, 128), (512, 128, 16),
+                                                 (512, 128, 128), (384, 128, 128), (640, 128, 128)])
+def test_attention_ragged_and_empty_rows(n_pad, list_rows, seg):
     """n_valid not a multiple of the block, a row with an empty list, lists of
-    different lengths in one 128-row tile (64-row lists), 32-key segments."""
-    rng = np.random.default_rng(9)
-    B, H, n_pad, d, n_valid = 1, 2, 512, 128, 437
+    different lengths in one 128-row tile (64-row lists), short segments, and
+    the two-tile 128x128 path with an even and an odd number of query tiles."""
+    rng = np.random.default_rng(9 + n_pad + seg)
+    B, H, d = 1, 2, 128
+    n_valid = n_pad - 75
     q, k, v = (round_to_bf16(rng.standard_normal((B, H, n_pad, d)).astype(np.float32)) for _ in range(3))
     for x in (q, k, v):
         x[:, :, n_valid:] = 0
-    for list_rows, seg in ((128, 32), (64, 32), (64, 128), (128, 16)):
-        n_l, n_s = n_pad // list_rows, n_pad // seg
-        kept = [[[np.sort(rng.choice(n_s, size=int(rng.integers(0, n_s // 2 + 1)), replace=False))
-                  for _ in range(n_l)] for _ in range(H)]]
-        kept[0][0][1] = np.zeros(0, dtype=np.int64)
-        counts, idx = lists_to_dev(kept, n_s, B, H, n_l)
-        shape = vsa.Shape(B, H, n_valid, n_pad, d)
-        o = torch.empty(B, H, n_pad, d, device="cuda")
-        lse = torch.empty(B, H, n_pad, device="cuda")
-        scale = 1 / math.sqrt(d)
-        vsa.block_sparse_fwd(to_dev(q), to_dev(k), to_dev(v), shape, list_rows, seg, counts, idx, n_s, scale, o, lse)
-        assert vsa.read_device_status() == 0
-        mask = orc.token_mask(kept, None, n_pad, list_rows, seg, n_valid)
-        O, L = orc.masked_attention_bruteforce(q, k, v, mask, scale)
-        assert_close_rows(o.cpu().numpy(), lse.cpu().numpy(), O, L, [(0, h, 0, n_pad) for h in range(H)])
+    n_l, n_s = n_pad // list_rows, n_pad // seg
+    kept = [[[np.sort(rng.choice(n_s, size=int(rng.integers(0, n_s // 2 + 1)), replace=False))
+              for _ in range(n_l)] for _ in range(H)]]
+    kept[0][0][1] = np.zeros(0, dtype=np.int64)
+    kept[0][1][0] = np.arange(n_s)                      # one dense row
+    counts, idx = lists_to_dev(kept, n_s, B, H, n_l)
+    shape = vsa.Shape(B, H, n_valid, n_pad, d)
+    o = torch.empty(B, H, n_pad, d, device="cuda")
+    lse = torch.empty(B, H, n_pad, device="cuda")
+    scale = 1 / math.sqrt(d)
+    vsa.block_sparse_fwd(to_dev(q), to_dev(k), to_dev(v), shape, list_rows, seg, counts, idx, n_s, scale, o, lse)
+    assert vsa.read_device_status() == 0
+    mask = orc.token_mask(kept, None, n_pad, list_rows, seg, n_valid)
+    O, L = orc.masked_attention_bruteforce(q, k, v, mask, scale)
+    assert_close_rows(o.cpu().numpy(), lse.cpu().numpy(), O, L, [(0, h, 0, n_pad) for h in range(H)])
 
 
 def test_attention_bad_list_latches_status():
@@ -344,3 +348,28 @@ def test_path_hunyuan_sampled():
     O, L = orc.lse_merge(O_M, L_M, O_u, L_u)
     worst = assert_close_rows(Og, Lg, O, L, [(b, h, i * 128, i * 128 + 128) for b, h, i in rows], bf16_out=True)
     print("\nhunyuan path worst:", worst, "rows", rows)
+
+
+@pytest.mark.parametrize("name,heads,chunk", [("tiny", None, 1), ("hunyuan", (0, 3), 2)])
+def test_forward_host_matches_device_path(name, heads, chunk):
+    """The host-buffer API (chunks of heads pipelined over copy and compute
+    streams) returns exactly what the device path returns for all heads."""
+    w = WORKLOADS[name]
+    q, k, v = inputs(name, heads)
+    H = q.shape[1]
+    flags = micro_heads(w)[:H] if w.micro_mode else None
+    if flags is not None and w.micro_mode == 2:
+        flags = np.array([1] + [0] * (H - 1), dtype=np.uint8)   # at least one Micro head in the cut
+    cfg = vsa.PathConfig.from_workload(w, flags)
+    ref = vsa.SparseVideoAttention(cfg)(to_dev(q), to_dev(k), to_dev(v))
+    o_ref, l_ref = ref["o"].cpu(), ref["lse"].cpu()
+    pin = lambda x: torch.from_numpy(x).to(torch.bfloat16).pin_memory()
+    ho = torch.empty(o_ref.shape, dtype=torch.bfloat16).pin_memory()
+    hl = torch.empty(l_ref.shape, dtype=torch.float32).pin_memory()
+    run = vsa.SparseVideoAttention(cfg)
+    run.forward_host(pin(q), pin(k), pin(v), ho, hl, chunk_heads=chunk)
+    assert vsa.read_device_status() == 0
+    assert torch.equal(ho, o_ref)
+    assert torch.equal(torch.isinf(hl), torch.isinf(l_ref))
+    fin = torch.isfinite(l_ref)
+    assert torch.equal(hl[fin], l_ref[fin])
