@@ -38,7 +38,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from video_inputs import WORKLOADS, make_qkv, micro_heads  # noqa: E402
+from video_inputs import WORKLOADS, make_qkv, micro_heads, sweep_points  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "block-sparse attn ms & effective TFLOP/s (% bf16 peak), speedup vs dense, 1xB200"
@@ -334,7 +334,8 @@ def run_gpu(args, rank, world, local_rank):
         "speedup_vs_dense": round(dense_ms / ms_step, 3),
         "macro_kernel_ms": round(macro_avg_ms, 4),
         "roofline": {
-            "kernel": "attn_fwd_kernel<128> (Macro pass)",
+            "kernel": ("attn_fwd_dual_kernel<%d> (Macro pass)" if (w.bq == 128 and w.bk == 128) else
+                       "attn_fwd_kernel<%d> (Macro pass)") % w.d,
             "bound": "tensor",
             "achieved": round(achieved, 2),
             "peak": peak,
@@ -415,6 +416,56 @@ def run_reference(args, rank, world):
     }
 
 
+def run_sweep(args):
+    """Sparsity sweep on the hunyuan tensors: kept fraction in {100, 50, 25,
+    15, 8}% x blocks {128x128, 64x128}; selection + attention (no Micro),
+    timed with CUDA events; one JSON line per point."""
+    import block_sparse_attention_pool_b200 as vsa
+    from block_sparse_attention_pool_b200 import build as vsa_build
+    vsa_build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    base = WORKLOADS["hunyuan"]
+    q, k, v = make_qkv(base)
+    to_dev = lambda x: torch.from_numpy(x).to(dev).to(torch.bfloat16).contiguous()
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    del q, k, v
+    stream = torch.cuda.current_stream(dev)
+    pk = peaks()
+    dense_ms = {}
+    for frac, w in sweep_points():
+        cfg = vsa.PathConfig(n_valid=w.n_valid, bq=w.bq, bk=w.bk, scale=w.scale, fixed_k=w.fixed_k)
+        run = vsa.SparseVideoAttention(cfg)
+        shape = vsa.Shape(w.B, w.H, w.n_valid, w.n_pad, w.d)
+        run(dq, dk, dv)
+        b = run.buf
+        for _ in range(args.warmup):
+            vsa.block_sparse_fwd(dq, dk, dv, shape, w.bq, w.bk, b["counts"], b["idx"], w.n_pad // w.bk, w.scale,
+                                 b["o"], b["lse"])
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            vsa.block_sparse_fwd(dq, dk, dv, shape, w.bq, w.bk, b["counts"], b["idx"], w.n_pad // w.bk, w.scale,
+                                 b["o"], b["lse"])
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        st = vsa.read_device_status(stream)
+        if st != 0:
+            raise RuntimeError(vsa.status_string(st))
+        ms = e0.elapsed_time(e1) / args.steps
+        flops = macro_flops(b["counts"], w)
+        if frac == 1.0:
+            dense_ms[(w.bq, w.bk)] = ms
+        tf = flops / (ms * 1e-3) / 1e12
+        print(json.dumps({"sweep_point": w.name, "blocks": f"{w.bq}x{w.bk}", "kept_fraction": frac,
+                          "k": w.fixed_k, "attn_ms": round(ms, 3), "effective_tflops": round(tf, 2),
+                          "frac_of_bf16_peak": round(tf / pk["bf16_sustained"], 4),
+                          "peak": f"{pk['bf16_sustained']} TFLOP/s ({pk['source']} bf16 sustained)",
+                          "speedup_vs_dense_same_blocks": round(dense_ms[(w.bq, w.bk)] / ms, 3)}), flush=True)
+        del run
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -425,11 +476,15 @@ def main():
     ap.add_argument("--ref-blocks", type=int, default=6, help="query blocks per oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--chunk-heads", type=int, default=4, help="heads per pipelined chunk of the e2e leg")
+    ap.add_argument("--sweep", action="store_true", help="print the sparsity-sweep lines instead of the bench line")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         line = run_reference(args, rank, world)
         if line is not None:

@@ -24,7 +24,7 @@ import torch
 __all__ = [
     "VsaError", "Shape", "SelectParams", "MicroParams", "lib", "library_path", "EXPORTED",
     "pool_qk", "select_blocks", "mask_to_lists", "select_micro", "select_micro_workspace_bytes", "select_micro_noalloc",
-    "block_sparse_fwd", "lse_merge", "read_device_status", "status_string", "version",
+    "block_sparse_fwd", "lse_merge", "read_device_status", "status_string", "version", "selftest_wait_timeout",
     "PathConfig", "SparseVideoAttention",
 ]
 
@@ -34,7 +34,7 @@ _LIB_PATH = os.path.join(_HERE, "libvsa.so")
 EXPORTED = (
     "vsa_status_string", "vsa_version", "vsa_read_device_status", "vsa_pool_qk", "vsa_select_blocks",
     "vsa_mask_to_lists", "vsa_select_micro_workspace_bytes", "vsa_select_micro", "vsa_select_micro_noalloc",
-    "vsa_block_sparse_fwd", "vsa_lse_merge",
+    "vsa_block_sparse_fwd", "vsa_lse_merge", "vsa_selftest_wait_timeout",
 )
 
 STATUS = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_UNSUPPORTED", 3: "VSA_ERR_CUDA",
@@ -88,6 +88,8 @@ def lib():
     L.vsa_version.argtypes = []
     L.vsa_read_device_status.restype = I
     L.vsa_read_device_status.argtypes = [P]
+    L.vsa_selftest_wait_timeout.restype = I
+    L.vsa_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, P]
     L.vsa_pool_qk.restype = I
     L.vsa_pool_qk.argtypes = [P, P, SP, I, I, P, P, P, P, P]
     L.vsa_select_blocks.restype = I
@@ -142,6 +144,12 @@ def version() -> int:
 
 def read_device_status(stream=None) -> int:
     return lib().vsa_read_device_status(_s(stream))
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Launch the bounded-wait self-test (a wait nothing completes, given up
+    after limit_ns); the device status then reads VSA_ERR_TIMEOUT."""
+    _check(lib().vsa_selftest_wait_timeout(int(limit_ns), _s(stream)), "vsa_selftest_wait_timeout")
 
 
 def pool_qk(q, k, shape: Shape, bq, bk, q_pool, k_pool, q_pool64=None, k_pool16=None, stream=None):

@@ -167,21 +167,6 @@ __device__ __forceinline__ bool list_valid(const int32_t *p, int n, int n_seg_ma
   return __all_sync(0xffffffffu, ok);
 }
 
-// |A intersect B| of two validated ascending lists, warp-parallel binary search.
-__device__ __forceinline__ int list_intersection(const int32_t *a, int na, const int32_t *b, int nb, int lane) {
-  int c = 0;
-  for (int e = lane; e < na; e += 32) {
-    const int v = __ldg(a + e);
-    int lo = 0, hi = nb;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (__ldg(b + mid) < v) lo = mid + 1; else hi = mid;
-    }
-    if (lo < nb && __ldg(b + lo) == v) ++c;
-  }
-  return warp_sum_int(c);
-}
-
 // acc += the two bf16 values packed in pk (fp32 accumulation).
 __device__ __forceinline__ float add_bf16x2_f32(float acc, uint32_t pk) {
   asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
@@ -253,9 +238,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     } else if (n_lists == 1) {
       n_seg = cnt[0];
     } else {
-      n_seg = cnt[0] + cnt[1] -
-              list_intersection(a.idx + lrow0 * a.idx_stride, cnt[0], a.idx + (lrow0 + 1) * a.idx_stride, cnt[1],
-                                lane);
+      // union size by a lockstep walk of the merge (coalesced 32-entry windows)
+      ListCursor cur;
+      cur.init(a.idx + lrow0 * a.idx_stride, cnt[0], a.idx + (lrow0 + 1) * a.idx_stride, cnt[1], 2, lane);
+      uint32_t m;
+      while (cur.next(&m, lane) >= 0) ++n_seg;
     }
     if (lane == 0) ctl->n_seg = n_seg;
   } else if (warp == 1) {

@@ -117,18 +117,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int x = 0; x < (has_b ? 2 : 1) && ok; ++x)
       ok = list_valid(a.idx + (lrow0 + x) * a.idx_stride, cnt[x], n_key_blocks, lane);
-    int n_union = 0;
     if (!ok) {
       if (lane == 0) latch_status(VSA_ERR_BAD_INDEX);
       cnt[0] = cnt[1] = 0;
-    } else {
-      n_union = cnt[0] + cnt[1] -
-                (has_b ? list_intersection(a.idx + lrow0 * a.idx_stride, cnt[0], a.idx + (lrow0 + 1) * a.idx_stride,
-                                           cnt[1], lane)
-                       : 0);
     }
     if (lane == 0) {
-      ctl->n_union = n_union;
+      ctl->n_union = cnt[0] + cnt[1];  // > 0 iff the union is not empty
       ctl->cnt[0] = cnt[0];
       ctl->cnt[1] = cnt[1];
     }
@@ -140,7 +134,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
 
-  const int n_union = ctl->n_union;
+  // The union of the two lists is walked until the cursor runs dry, so its
+  // length never has to be counted up front.
+  const bool any_block = ctl->n_union > 0;
   const uint32_t tmem = ctl->tmem_base;
   const uint32_t tS[2] = {tmem, tmem + 128u};
   const uint32_t tO[2] = {tmem + 256u, tmem + 384u};
@@ -149,7 +145,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (n_union > 0) {
+    if (any_block) {
       ListCursor cur;
       cur.init(list[0], cnt[0], has_b ? list[1] : nullptr, cnt[1], has_b ? 2 : 1, lane);
       if (lane == 0) {
@@ -159,11 +155,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tma_load_3d(sQ + x * L::kQBytes + c * kChunkBytes, &tm_q, &ctl->q_full, c * 64, (tile0 + x) * kTileM, bh);
       }
       int issued = 0;
-      for (int s = 0; s < n_union; ++s) {
+      for (int s = 0;; ++s) {
         const int slot = s & 1;
         const uint32_t use_par = ((s >> 1) - 1) & 1;
         uint32_t m = 0u;
         const int blk = cur.next(&m, lane);
+        if (blk < 0) break;
         const int start = blk * kStageKeys;
         bool ok = true;
         if (s >= 2) ok = mbar_wait_warp(&ctl->k_empty[slot], use_par, abort, a.timeout_ns, lane);
@@ -193,7 +190,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (n_union > 0) {
+    if (any_block) {
       constexpr uint32_t kIdS = idesc_bf16_f32(kTileM, kStageKeys, false);
       constexpr uint32_t kIdO = idesc_bf16_f32(kTileM, D, true);
       const uint32_t q_addr = smem_addr(sQ), k_addr = smem_addr(sK), v_addr = smem_addr(sV);
@@ -219,9 +216,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         ++pv_done[x];
         return true;
       };
-      for (int s = 0; s < n_union; ++s) {
+      int s = 0;
+      for (;; ++s) {
         uint32_t use = 0u;
-        cur.next(&use, lane);  // whole warp walks the union in lockstep
+        if (cur.next(&use, lane) < 0) break;  // whole warp walks the union in lockstep
         if (!has_b) use &= 1u;  // a single-list cursor tags every block with both bits
         if (lane == 0 && ok) {
           bool k_ready = false;
@@ -257,8 +255,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (lane == 0) {
         if (ok) {
           for (int x = 0; x < 2 && ok; ++x)
-            if ((prev >> x) & 1u) ok = issue_pv(x, n_union - 1);
-          if (ok) umma_commit(&ctl->v_empty[(n_union - 1) & 1]);
+            if ((prev >> x) & 1u) ok = issue_pv(x, s - 1);
+          if (ok) umma_commit(&ctl->v_empty[(s - 1) & 1]);
         }
         umma_commit(&ctl->mma_drain);
         mbar_drain(&ctl->mma_drain, 0, a.timeout_ns);
@@ -276,7 +274,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float lr = 0.f;        // row sum of the bf16-rounded P
     bool ok = true;
     const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
-    const int n_mine = tile_live && n_union > 0 ? cnt[x] : 0;
+    const int n_mine = tile_live ? cnt[x] : 0;
     for (int i = 0; i < n_mine; ++i) {
       const int key0 = __ldg(list[x] + i) * kStageKeys;
       ok = mbar_wait_warp(&ctl->s_full[x], i & 1, abort, a.timeout_ns, lane);

@@ -188,6 +188,18 @@ vsa_status noalloc_scratch(void **out) {
   return VSA_OK;
 }
 
+// One thread waits on a barrier that no one arrives at; the bounded wait gives
+// up after limit_ns and latches VSA_ERR_TIMEOUT.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  vsa::mbar_init(&bar, 1);
+  vsa::fence_barrier_init();
+  vsa::mbar_wait(&bar, 0, &abort_flag, limit_ns);
+}
+
 // Per-head slot numbers handed to the device by value (no host-to-device copy).
 struct HeadSlots {
   int16_t slot[kNoallocMaxBH];  // rank among enabled heads, or -1
@@ -232,6 +244,12 @@ vsa_status vsa_read_device_status(void *stream) {
   if (cudaMemcpyToSymbol(vsa::g_status, &zero, sizeof(int)) != cudaSuccess) return VSA_ERR_CUDA;
   if (cudaMemcpyToSymbol(vsa::g_timed_out, &zero, sizeof(int)) != cudaSuccess) return VSA_ERR_CUDA;
   return static_cast<vsa_status>(h);
+}
+
+vsa_status vsa_selftest_wait_timeout(unsigned long long limit_ns, void *stream) {
+  if (limit_ns < 1000ull || limit_ns > 5000000000ull) return VSA_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  return launch_status();
 }
 
 vsa_status vsa_pool_qk(const void *q, const void *k, const vsa_shape *shape, int bq, int bk, float *q_pool,

@@ -129,6 +129,14 @@ VSA_API int vsa_version(void);
  * first device-side error latched since the last call; VSA_OK if none).   */
 VSA_API vsa_status vsa_read_device_status(void *stream);
 
+/* Self-test of the bounded pipeline waits (no counterpart on the pages): one
+ * thread waits on a shared-memory barrier that nothing completes, for at most
+ * limit_ns nanoseconds (1e3 <= limit_ns <= 5e9), then returns.  The status
+ * word then reads VSA_ERR_TIMEOUT and the device stays usable; the kernel
+ * neither faults nor traps.  Like every timeout it also makes other waits
+ * still running give up, until vsa_read_device_status clears it. */
+VSA_API vsa_status vsa_selftest_wait_timeout(unsigned long long limit_ns, void *stream);
+
 /* ---------------------------------------------------------------------------
  * a1 Pooling  ([RSA]: pooled query-key interactions; [HVA] section 4.1: a
  * centroid is the mean of its tokens; [MOD]: fixed non-overlapping blocks.)

@@ -239,6 +239,22 @@ def test_attention_bad_list_latches_status():
     assert vsa.read_device_status() == 0                      # reading clears it
 
 
+def test_bounded_wait_times_out_and_device_stays_usable():
+    """Failure detection without a fault: a wait that nothing completes gives
+    up after its limit, the status reads VSA_ERR_TIMEOUT, reading clears it,
+    and the next attention call runs normally."""
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    vsa.selftest_wait_timeout(50_000_000)          # 50 ms
+    t1.record()
+    assert vsa.read_device_status() == 6
+    assert t0.elapsed_time(t1) >= 45.0
+    assert vsa.read_device_status() == 0
+    test_attention_tiny_all_rows()
+    assert vsa.read_device_status() == 0
+
+
 # ---------------------------------------------------------------------------
 # a6 merge
 # ---------------------------------------------------------------------------
