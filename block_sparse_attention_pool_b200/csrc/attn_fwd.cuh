@@ -333,18 +333,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (n_stages > 0 && lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(kTileM, kStageKeys, false);
       constexpr uint32_t kIdO = idesc_bf16_f32(kTileM, D, true);
-      const uint32_t q_addr = smem_addr(sQ), k_addr = smem_addr(sK), v_addr = smem_addr(sV);
+      // descriptor bases; K steps and ring slots only add to the start address field
+      const uint64_t dQ = smem_desc_sw128(smem_addr(sQ), 16, 1024);
+      const uint64_t dK0 = smem_desc_sw128(smem_addr(sK), 16, 1024);
+      const uint64_t dV0 = smem_desc_sw128(smem_addr(sV), kChunkBytes, 1024);
+      constexpr uint64_t kSlotStep = L::kKVBytes >> 4;
       bool ok = mbar_wait(&ctl->q_full, 0, abort, a.timeout_ns);
       auto issue_pv = [&](int t) -> bool {
         if (!mbar_wait(&ctl->p_full[t & 1], (t >> 1) & 1, abort, a.timeout_ns)) return false;
         if (!mbar_wait(&ctl->v_full[t & 1], (t >> 1) & 1, abort, a.timeout_ns)) return false;
         tc_fence_after();
-        const uint32_t vb = v_addr + (t & 1) * L::kKVBytes;
+        const uint64_t dv = dV0 + (uint64_t)(t & 1) * kSlotStep;
+        const uint32_t to = (t & 1) ? tO[1] : tO[0];
+        const uint32_t ts = (t & 1) ? tS[1] : tS[0];
 #pragma unroll
         for (int kk = 0; kk < kStageKeys / 16; ++kk) {
           // P (bf16 pairs) sits in the first 64 columns of the stage's S buffer
-          const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, kChunkBytes, 1024);
-          umma_bf16_ts(tO[t & 1], tS[t & 1] + kk * 8, bd, kIdO, (t >= 2 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts(to, ts + kk * 8, dv + (uint64_t)(kk * 16 * 128 / 16), kIdO, (t >= 2 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&ctl->v_empty[t & 1]);
         return true;
@@ -355,12 +360,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (ok && s >= 2) ok = mbar_wait(&ctl->s_free[slot], ((s - 2) >> 1) & 1, abort, a.timeout_ns);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t kb = k_addr + slot * L::kKVBytes;
+        const uint64_t dk = dK0 + (uint64_t)slot * kSlotStep;
+        const uint32_t ts = slot ? tS[1] : tS[0];
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(q_addr + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(kb + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
-          umma_bf16_ss(tS[slot], ad, bd, kIdS, kk > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+          umma_bf16_ss(ts, dQ + off, dk + off, kIdS, kk > 0 ? 1u : 0u);
         }
         umma_commit(&ctl->k_empty[slot]);
         umma_commit(&ctl->s_full[slot]);
@@ -378,6 +383,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int row = quad * 32 + lane;         // row within the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const int half = row >> 6;                // query half for 64-row lists
+    const uint32_t tSg = g == 0 ? tS[0] : tS[1];
+    const uint32_t tOg = g == 0 ? tO[0] : tO[1];
     float m2 = -INFINITY;  // this group's running reference max of scaled logits, log2 units
     float l = 0.f;         // sum of P (fp32) over this group's stages
     float lr = 0.f;        // sum of the bf16-rounded P over this group's stages
@@ -392,7 +399,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // the row's 128 logits: r[c][j] = S[row][32 c + j]
       uint32_t r[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS[g] + lane_off + c * 32, r[c]);
+      for (int c = 0; c < 4; ++c) tmem_ld32(tSg + lane_off + c * 32, r[c]);
       tmem_ld_wait();
       if (!inf.full) {
         // cold path: valid columns as a 128-bit mask built per segment (a used
@@ -465,15 +472,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(tO[g] + lane_off + c * 32, o);
+          tmem_ld32(tOg + lane_off + c * 32, o);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-          tmem_st32(tO[g] + lane_off + c * 32, o);
+          tmem_st32(tOg + lane_off + c * 32, o);
         }
       }
-      tmem_st32(tS[g] + lane_off + 0, r[0]);
-      tmem_st32(tS[g] + lane_off + 32, r[1]);
+      tmem_st32(tSg + lane_off + 0, r[0]);
+      tmem_st32(tSg + lane_off + 32, r[1]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&ctl->s_free[g]);

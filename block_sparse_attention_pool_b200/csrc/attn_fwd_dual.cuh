@@ -37,6 +37,8 @@
 // are released by commits after the last MMA that reads them.
 #pragma once
 
+#include <type_traits>
+
 #include "attn_fwd.cuh"
 
 namespace vsa {
@@ -193,28 +195,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (any_block) {
       constexpr uint32_t kIdS = idesc_bf16_f32(kTileM, kStageKeys, false);
       constexpr uint32_t kIdO = idesc_bf16_f32(kTileM, D, true);
-      const uint32_t q_addr = smem_addr(sQ), k_addr = smem_addr(sK), v_addr = smem_addr(sV);
+      // Descriptor bases; a K step or ring slot only adds to the start
+      // address field (bytes >> 4, which never carries out of its 14 bits
+      // inside 227 KB of shared memory).
+      const uint64_t dQ0 = smem_desc_sw128(smem_addr(sQ), 16, 1024);
+      const uint64_t dK0 = smem_desc_sw128(smem_addr(sK), 16, 1024);
+      const uint64_t dV0 = smem_desc_sw128(smem_addr(sV), kChunkBytes, 1024);
+      constexpr uint64_t kQStep = L::kQBytes >> 4, kSlotStep = L::kKVBytes >> 4;
       ListCursor cur;
       cur.init(list[0], cnt[0], has_b ? list[1] : nullptr, cnt[1], has_b ? 2 : 1, lane);
       bool ok = true;
       if (lane == 0) ok = mbar_wait(&ctl->q_full, 0, abort, a.timeout_ns);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       uint32_t prev = 0u;     // usage bits of the previous union block
-      int nx[2] = {0, 0};     // blocks of each tile seen so far
-      int pv_done[2] = {0, 0};  // P.V issued so far per tile
-      auto issue_pv = [&](int x, int s) -> bool {
-        // O_x += P_x(block s) V_s
-        if (!mbar_wait(&ctl->p_full[x], pv_done[x] & 1, abort, a.timeout_ns)) return false;
+      int pv_cnt[2] = {0, 0};  // P.V issued so far per tile
+      // O_x += P_x(block s) V_s
+      auto issue_pv = [&](auto xc, int s) -> bool {
+        constexpr int x = decltype(xc)::value;
+        if (!mbar_wait(&ctl->p_full[x], pv_cnt[x] & 1, abort, a.timeout_ns)) return false;
         if (!mbar_wait(&ctl->v_full[s & 1], (s >> 1) & 1, abort, a.timeout_ns)) return false;
         tc_fence_after();
-        const uint32_t vb = v_addr + (s & 1) * L::kKVBytes;
+        const uint64_t dv = dV0 + (uint64_t)(s & 1) * kSlotStep;
+        const uint32_t first = pv_cnt[x] > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < kStageKeys / 16; ++kk) {
-          const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, kChunkBytes, 1024);
-          umma_bf16_ts(tO[x], tS[x] + kk * 8, bd, kIdO, (pv_done[x] > 0 || kk > 0) ? 1u : 0u);
-        }
-        ++pv_done[x];
+        for (int kk = 0; kk < kStageKeys / 16; ++kk)
+          umma_bf16_ts(tO[x], tS[x] + kk * 8, dv + (uint64_t)(kk * 16 * 128 / 16), kIdO, kk > 0 ? 1u : first);
+        ++pv_cnt[x];
         return true;
+      };
+      // S_x = Q_x K_s^T
+      auto issue_s = [&](auto xc, int s) {
+        constexpr int x = decltype(xc)::value;
+        const uint64_t dq = dQ0 + (uint64_t)x * kQStep;
+        const uint64_t dk = dK0 + (uint64_t)(s & 1) * kSlotStep;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+          umma_bf16_ss(tS[x], dq + off, dk + off, kIdS, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&ctl->s_full[x]);
       };
       int s = 0;
       for (;; ++s) {
@@ -222,27 +241,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (cur.next(&use, lane) < 0) break;  // whole warp walks the union in lockstep
         if (!has_b) use &= 1u;  // a single-list cursor tags every block with both bits
         if (lane == 0 && ok) {
+          // P.V of a tile's block s-1 goes before its S of block s: that S
+          // overwrites the TMEM buffer holding the tile's P.
           bool k_ready = false;
-          for (int x = 0; x < 2 && ok; ++x) {
-            // P.V of x's block s-1 first: S_x(s) overwrites the S buffer that holds P_x(s-1)
-            if ((prev >> x) & 1u) ok = issue_pv(x, s - 1);
-            if (ok && ((use >> x) & 1u)) {
-              if (!k_ready) {
-                ok = mbar_wait(&ctl->k_full[s & 1], (s >> 1) & 1, abort, a.timeout_ns);
-                k_ready = true;
-                if (!ok) break;
-              }
+          if (prev & 1u) ok = issue_pv(std::integral_constant<int, 0>{}, s - 1);
+          if (ok && (use & 1u)) {
+            ok = mbar_wait(&ctl->k_full[s & 1], (s >> 1) & 1, abort, a.timeout_ns);
+            k_ready = true;
+            if (ok) {
               tc_fence_after();
-              const uint32_t qb = q_addr + x * L::kQBytes;
-              const uint32_t kb = k_addr + (s & 1) * L::kKVBytes;
-#pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const uint64_t ad = smem_desc_sw128(qb + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
-                const uint64_t bd = smem_desc_sw128(kb + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
-                umma_bf16_ss(tS[x], ad, bd, kIdS, kk > 0 ? 1u : 0u);
-              }
-              umma_commit(&ctl->s_full[x]);
-              ++nx[x];
+              issue_s(std::integral_constant<int, 0>{}, s);
+            }
+          }
+          if (ok && (prev & 2u)) ok = issue_pv(std::integral_constant<int, 1>{}, s - 1);
+          if (ok && (use & 2u)) {
+            if (!k_ready) ok = mbar_wait(&ctl->k_full[s & 1], (s >> 1) & 1, abort, a.timeout_ns);
+            if (ok) {
+              tc_fence_after();
+              issue_s(std::integral_constant<int, 1>{}, s);
             }
           }
           if (ok) {
@@ -253,11 +269,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         prev = use;
       }
       if (lane == 0) {
-        if (ok) {
-          for (int x = 0; x < 2 && ok; ++x)
-            if ((prev >> x) & 1u) ok = issue_pv(x, s - 1);
-          if (ok) umma_commit(&ctl->v_empty[(s - 1) & 1]);
-        }
+        if (ok && (prev & 1u)) ok = issue_pv(std::integral_constant<int, 0>{}, s - 1);
+        if (ok && (prev & 2u)) ok = issue_pv(std::integral_constant<int, 1>{}, s - 1);
+        if (ok) umma_commit(&ctl->v_empty[(s - 1) & 1]);
         umma_commit(&ctl->mma_drain);
         mbar_drain(&ctl->mma_drain, 0, a.timeout_ns);
       }
@@ -269,20 +283,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int row = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const bool tile_live = x == 0 || has_b;
+    // this group's TMEM buffers and list as scalars (no runtime-indexed arrays)
+    const uint32_t tSx = x == 0 ? tS[0] : tS[1];
+    const uint32_t tOx = x == 0 ? tO[0] : tO[1];
+    const int32_t *listx = x == 0 ? list[0] : list[1];
     float m2 = -INFINITY;  // running reference max of scaled logits, log2 units
     float l = 0.f;         // fp32 row sum of P
     float lr = 0.f;        // row sum of the bf16-rounded P
     bool ok = true;
     const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
-    const int n_mine = tile_live ? cnt[x] : 0;
+    const int n_mine = tile_live ? (x == 0 ? cnt[0] : cnt[1]) : 0;
     for (int i = 0; i < n_mine; ++i) {
-      const int key0 = __ldg(list[x] + i) * kStageKeys;
+      const int key0 = __ldg(listx + i) * kStageKeys;
       ok = mbar_wait_warp(&ctl->s_full[x], i & 1, abort, a.timeout_ns, lane);
       if (!ok) break;
       tc_fence_after();
       uint32_t r[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS[x] + lane_off + c * 32, r[c]);
+      for (int c = 0; c < 4; ++c) tmem_ld32(tSx + lane_off + c * 32, r[c]);
       tmem_ld_wait();
       const int nv = a.n_valid - key0;  // valid keys of this block
       if (nv < kStageKeys) {
@@ -334,15 +352,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(tO[x] + lane_off + c * 32, o);
+          tmem_ld32(tOx + lane_off + c * 32, o);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-          tmem_st32(tO[x] + lane_off + c * 32, o);
+          tmem_st32(tOx + lane_off + c * 32, o);
         }
       }
-      tmem_st32(tS[x] + lane_off + 0, r[0]);
-      tmem_st32(tS[x] + lane_off + 32, r[1]);
+      tmem_st32(tSx + lane_off + 0, r[0]);
+      tmem_st32(tSx + lane_off + 32, r[1]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&ctl->p_full[x]);
@@ -371,7 +389,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         if (warp_loads) {
-          tmem_ld32(tO[x] + lane_off + c * 32, o);
+          tmem_ld32(tOx + lane_off + c * 32, o);
           tmem_ld_wait();
         }
         float v[32];
