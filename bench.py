@@ -188,6 +188,8 @@ def run_gpu(args, rank, world, local_rank):
     # launch inside every step, on the launching stream
     macro_ev = []
 
+    stage_ev = []  # per step: events bracketing pool, select, Macro, Micro select, Micro pass
+
     def run_with_events(qq, kk, vv):
         c = run.cfg
         run._alloc(qq)
@@ -195,25 +197,32 @@ def run_gpu(args, rank, world, local_rank):
         B, H, n_pad, d = qq.shape
         shape = vsa.Shape(B, H, c.n_valid, n_pad, d)
         n_k = n_pad // c.bk
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        ev[0].record(stream)
         vsa.pool_qk(qq, kk, shape, c.bq, c.bk, b["q_pool"], b["k_pool"], b.get("q_pool64"), b.get("k_pool16"))
+        ev[1].record(stream)
         vsa.select_blocks(b["q_pool"], b["k_pool"], shape, c.bq, c.bk, c.scale,
                           vsa.SelectParams(c.k_min, c.cum_mass, c.fixed_k, c.n_anchor, c.anchor_rot), b["counts"],
                           b["idx"])
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+        ev[2].record(stream)
         if c.micro_mode:
             vsa.block_sparse_fwd(qq, kk, vv, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, c.scale, b["o_macro"],
                                  b["lse_macro"])
         else:
             vsa.block_sparse_fwd(qq, kk, vv, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, c.scale, b["o"], b["lse"])
-        e1.record(stream)
-        macro_ev.append((e0, e1))
+        ev[3].record(stream)
         if c.micro_mode:
             vsa.select_micro(b["q_pool64"], b["k_pool16"], b["counts"], b["idx"], shape, c.bq, c.bk, c.scale,
                              c.micro_mode, c.micro_topk, c.micro_percentile, c.micro_heads, run.micro_cap,
                              b["m_counts"], b["m_idx"], b["workspace"])
+            ev[4].record(stream)
             vsa.block_sparse_fwd(qq, kk, vv, shape, 64, 16, b["m_counts"], b["m_idx"], run.micro_cap, c.scale, b["o"],
                                  b["lse"], b["o_macro"], b["lse_macro"])
+        else:
+            ev[4].record(stream)
+        ev[5].record(stream)
+        macro_ev.append((ev[2], ev[3]))
+        stage_ev.append(ev)
         return b
 
     # kernels launched per step by this path (pool, select, Macro; Micro:
@@ -227,6 +236,7 @@ def run_gpu(args, rank, world, local_rank):
     if st != 0:
         raise RuntimeError(f"device status after warm-up: {vsa.status_string(st)}")
     macro_ev.clear()
+    stage_ev.clear()
     fl_macro = macro_flops(run.buf["counts"], w)
     fl_micro = micro_flops(run.buf["m_counts"], w) if w.micro_mode else 0.0
 
@@ -247,6 +257,8 @@ def run_gpu(args, rank, world, local_rank):
     clk = clocks.stop()
     ms_total = t0.elapsed_time(t1)
     macro_ms = [a.elapsed_time(b) for a, b in macro_ev]
+    names = ["pool", "select", "macro_attention", "micro_select", "micro_attention_merge"]
+    stages = {n: round(statistics.mean(e[i].elapsed_time(e[i + 1]) for e in stage_ev), 4) for i, n in enumerate(names)}
     st = vsa.read_device_status(stream)
     if st != 0:
         raise RuntimeError(f"device status after timed steps: {vsa.status_string(st)}")
@@ -333,6 +345,7 @@ def run_gpu(args, rank, world, local_rank):
         "dense_tflops": round(dense_flops / (dense_ms * 1e-3) / 1e12, 2),
         "speedup_vs_dense": round(dense_ms / ms_step, 3),
         "macro_kernel_ms": round(macro_avg_ms, 4),
+        "stages_ms": stages,
         "roofline": {
             "kernel": ("attn_fwd_dual_kernel<%d> (Macro pass)" if (w.bq == 128 and w.bk == 128) else
                        "attn_fwd_kernel<%d> (Macro pass)") % w.d,
