@@ -191,43 +191,20 @@ def run_gpu(args, rank, world, local_rank):
     stage_ev = []  # per step: events bracketing pool, select, Macro, Micro select, Micro pass
 
     def run_with_events(qq, kk, vv):
-        c = run.cfg
-        run._alloc(qq)
-        b = run.buf
-        B, H, n_pad, d = qq.shape
-        shape = vsa.Shape(B, H, c.n_valid, n_pad, d)
-        n_k = n_pad // c.bk
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
-        ev[0].record(stream)
-        vsa.pool_qk(qq, kk, shape, c.bq, c.bk, b["q_pool"], b["k_pool"], b.get("q_pool64"), b.get("k_pool16"))
-        ev[1].record(stream)
-        vsa.select_blocks(b["q_pool"], b["k_pool"], shape, c.bq, c.bk, c.scale,
-                          vsa.SelectParams(c.k_min, c.cum_mass, c.fixed_k, c.n_anchor, c.anchor_rot), b["counts"],
-                          b["idx"])
-        ev[2].record(stream)
-        if c.micro_mode:
-            vsa.block_sparse_fwd(qq, kk, vv, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, c.scale, b["o_macro"],
-                                 b["lse_macro"])
-        else:
-            vsa.block_sparse_fwd(qq, kk, vv, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, c.scale, b["o"], b["lse"])
-        ev[3].record(stream)
-        if c.micro_mode:
-            vsa.select_micro(b["q_pool64"], b["k_pool16"], b["counts"], b["idx"], shape, c.bq, c.bk, c.scale,
-                             c.micro_mode, c.micro_topk, c.micro_percentile, c.micro_heads, run.micro_cap,
-                             b["m_counts"], b["m_idx"], b["workspace"])
-            ev[4].record(stream)
-            vsa.block_sparse_fwd(qq, kk, vv, shape, 64, 16, b["m_counts"], b["m_idx"], run.micro_cap, c.scale, b["o"],
-                                 b["lse"], b["o_macro"], b["lse_macro"])
-        else:
-            ev[4].record(stream)
-        ev[5].record(stream)
+        b = run(qq, kk, vv, stream=stream, on_stage=lambda i: ev[i].record(stream))
         macro_ev.append((ev[2], ev[3]))
         stage_ev.append(ev)
         return b
 
-    # kernels launched per step by this path (pool, select, Macro; Micro:
-    # bitmap, score, 3 rank searches, 2 histograms, compaction, Micro pass)
-    launches_per_step = 3 + (9 if w.micro_mode == 2 else (3 if w.micro_mode == 1 else 0))
+    # kernels launched per step by this path: pooling, selection, the Macro
+    # pass (one launch for the heads without the Micro repair, one for those
+    # with it), Micro selection (percentile: bitmap, score, 3 rank searches,
+    # 2 histograms, compaction; top-k: bitmap, top-k) and the Micro pass
+    n_rep = (sum(1 for f in heads if f) if heads is not None else w.H) if w.micro_mode else 0
+    n_macro = 1 if not w.micro_mode else int(n_rep > 0) + int(n_rep < w.H)
+    n_micro = 0 if not w.micro_mode else (8 if w.micro_mode == 2 else 2) + int(n_rep > 0)
+    launches_per_step = 2 + n_macro + n_micro
 
     for _ in range(args.warmup):
         run_with_events(dq, dk, dv)
@@ -347,8 +324,8 @@ def run_gpu(args, rank, world, local_rank):
         "macro_kernel_ms": round(macro_avg_ms, 4),
         "stages_ms": stages,
         "roofline": {
-            "kernel": ("attn_fwd_dual_kernel<%d> (Macro pass)" if (w.bq == 128 and w.bk == 128) else
-                       "attn_fwd_kernel<%d> (Macro pass)") % w.d,
+            "kernel": ("attn_fwd_dual_kernel<%d> (Macro pass" if (w.bq == 128 and w.bk == 128) else
+                       "attn_fwd_kernel<%d> (Macro pass") % w.d + f", {n_macro} launch(es) per step timed together)",
             "bound": "tensor",
             "achieved": round(achieved, 2),
             "peak": peak,

@@ -34,7 +34,7 @@ _LIB_PATH = os.path.join(_HERE, "libvsa.so")
 EXPORTED = (
     "vsa_status_string", "vsa_version", "vsa_read_device_status", "vsa_pool_qk", "vsa_select_blocks",
     "vsa_mask_to_lists", "vsa_select_micro_workspace_bytes", "vsa_select_micro", "vsa_select_micro_noalloc",
-    "vsa_block_sparse_fwd", "vsa_lse_merge", "vsa_selftest_wait_timeout",
+    "vsa_block_sparse_fwd", "vsa_block_sparse_fwd_heads", "vsa_lse_merge", "vsa_selftest_wait_timeout",
 )
 
 STATUS = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_UNSUPPORTED", 3: "VSA_ERR_CUDA",
@@ -104,6 +104,8 @@ def lib():
     L.vsa_select_micro_noalloc.argtypes = [P, P, P, P, SP, I, I, F, ctypes.POINTER(MicroParams), P, P, P]
     L.vsa_block_sparse_fwd.restype = I
     L.vsa_block_sparse_fwd.argtypes = [P, P, P, SP, I, I, P, P, I, F, P, I, P, P, P, P]
+    L.vsa_block_sparse_fwd_heads.restype = I
+    L.vsa_block_sparse_fwd_heads.argtypes = [P, P, P, SP, I, I, P, P, I, F, P, I, P, P, P, P, I, P]
     L.vsa_lse_merge.restype = I
     L.vsa_lse_merge.argtypes = [P, P, P, P, SP, P, I, P, P]
     _lib = L
@@ -208,11 +210,21 @@ def select_micro_noalloc(q_pool64, k_pool16, counts, idx, shape: Shape, bq, bk, 
 
 
 def block_sparse_fwd(q, k, v, shape: Shape, list_rows, seg_keys, counts, idx, idx_stride, scale, o, lse,
-                     merge_o=None, merge_lse=None, stream=None):
+                     merge_o=None, merge_lse=None, stream=None, heads=None):
+    """``heads``: None (every (batch, head)) or a device int32 tensor of
+    flattened indices b*H + h; only those heads are read and written."""
     o_fp32 = 1 if o.dtype == torch.float32 else 0
-    _check(lib().vsa_block_sparse_fwd(_p(q), _p(k), _p(v), ctypes.byref(shape), int(list_rows), int(seg_keys),
-                                      _p(counts), _p(idx), int(idx_stride), float(scale), _p(o), o_fp32, _p(lse),
-                                      _p(merge_o), _p(merge_lse), _s(stream)), "vsa_block_sparse_fwd")
+    if heads is None:
+        _check(lib().vsa_block_sparse_fwd(_p(q), _p(k), _p(v), ctypes.byref(shape), int(list_rows), int(seg_keys),
+                                          _p(counts), _p(idx), int(idx_stride), float(scale), _p(o), o_fp32, _p(lse),
+                                          _p(merge_o), _p(merge_lse), _s(stream)), "vsa_block_sparse_fwd")
+        return
+    if heads.dtype != torch.int32 or not heads.is_contiguous():
+        raise ValueError("heads must be a contiguous int32 tensor")
+    _check(lib().vsa_block_sparse_fwd_heads(_p(q), _p(k), _p(v), ctypes.byref(shape), int(list_rows),
+                                            int(seg_keys), _p(counts), _p(idx), int(idx_stride), float(scale), _p(o),
+                                            o_fp32, _p(lse), _p(merge_o), _p(merge_lse), _p(heads),
+                                            int(heads.numel()), _s(stream)), "vsa_block_sparse_fwd_heads")
 
 
 def lse_merge(o_a, lse_a, o_b, lse_b, shape: Shape, o_out, lse_out, stream=None):
@@ -302,13 +314,37 @@ class SparseVideoAttention:
         self.buf = b
         self._key = key
 
+    def _head_split(self, B: int, H: int, flags, dev):
+        """Device index lists (b*H + h) of the heads without and with the Micro
+        repair; None stands for "every head", an empty tuple for "no head"."""
+        key = (B, H, None if flags is None else tuple(int(f) for f in flags), dev)
+        cache = self.__dict__.setdefault("_splits", {})
+        if key not in cache:
+            if flags is None:
+                cache[key] = ((), None)
+            else:
+                if len(flags) != H:
+                    raise ValueError(f"micro_heads has {len(flags)} flags for {H} heads")
+                rep = [b * H + h for b in range(B) for h in range(H) if flags[h]]
+                plain = [b * H + h for b in range(B) for h in range(H) if not flags[h]]
+                as_dev = lambda x: torch.tensor(x, dtype=torch.int32, device=dev) if x else ()
+                cache[key] = (None if not rep else as_dev(plain), None if not plain else as_dev(rep))
+        return cache[key]
+
     def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None, out_o=None, out_lse=None,
-                 micro_heads=None) -> Dict[str, torch.Tensor]:
+                 micro_heads=None, on_stage=None) -> Dict[str, torch.Tensor]:
         """Run the whole path on device tensors q, k, v [B, H, n_pad, d] (bf16).
 
         Outputs go to ``self.buf["o"]`` / ``["lse"]``, or to ``out_o`` /
         ``out_lse`` when given (same shapes).  ``micro_heads`` overrides the
-        configured per-head Micro flags (length H).
+        configured per-head Micro flags (length H).  ``on_stage(i)``, when
+        given, is called on the host before the first stage (i = 0) and after
+        each stage: pooling 1, selection 2, Macro pass 3, Micro selection 4,
+        Micro pass 5 (all enqueued, not completed).
+
+        Heads without the Micro repair get their final output from the Macro
+        pass; only heads with it keep a fp32 Macro output, and only they run
+        the Micro pass that merges into it.
         """
         c = self.cfg
         self._alloc(q)
@@ -321,20 +357,36 @@ class SparseVideoAttention:
         o = b["o"] if out_o is None else out_o
         lse = b["lse"] if out_lse is None else out_lse
         heads = c.micro_heads if micro_heads is None else micro_heads
+        stage = on_stage if on_stage is not None else (lambda i: None)
+        stage(0)
         pool_qk(q, k, shape, c.bq, c.bk, b["q_pool"], b["k_pool"], b.get("q_pool64"), b.get("k_pool16"), stream)
+        stage(1)
         select_blocks(b["q_pool"], b["k_pool"], shape, c.bq, c.bk, scale,
                       SelectParams(c.k_min, c.cum_mass, c.fixed_k, c.n_anchor, c.anchor_rot), b["counts"], b["idx"],
                       None, stream)
+        stage(2)
         if not micro:
             block_sparse_fwd(q, k, v, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, scale, o, lse, stream=stream)
+            stage(3)
+            stage(4)
+            stage(5)
             return b
-        block_sparse_fwd(q, k, v, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, scale, b["o_macro"],
-                         b["lse_macro"], stream=stream)
+        plain, rep = self._head_split(B, H, heads, q.device)
+        if not isinstance(plain, tuple):  # heads whose Macro output is final
+            block_sparse_fwd(q, k, v, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, scale, o, lse, stream=stream,
+                             heads=plain)
+        if not isinstance(rep, tuple):    # heads repaired by the Micro pass keep a fp32 Macro output
+            block_sparse_fwd(q, k, v, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, scale, b["o_macro"],
+                             b["lse_macro"], stream=stream, heads=rep)
+        stage(3)
         select_micro(b["q_pool64"], b["k_pool16"], b["counts"], b["idx"], shape, c.bq, c.bk, scale, c.micro_mode,
                      c.micro_topk, c.micro_percentile, heads, self.micro_cap, b["m_counts"], b["m_idx"],
                      b["workspace"], stream)
-        block_sparse_fwd(q, k, v, shape, 64, 16, b["m_counts"], b["m_idx"], self.micro_cap, scale, o, lse,
-                         b["o_macro"], b["lse_macro"], stream)
+        stage(4)
+        if not isinstance(rep, tuple):
+            block_sparse_fwd(q, k, v, shape, 64, 16, b["m_counts"], b["m_idx"], self.micro_cap, scale, o, lse,
+                             b["o_macro"], b["lse_macro"], stream, heads=rep)
+        stage(5)
         return b
 
     def forward_host(self, q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor, o_h: torch.Tensor,

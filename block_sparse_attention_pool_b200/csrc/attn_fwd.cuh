@@ -73,6 +73,8 @@ struct AttnArgs {
   float *lse;
   const float *merge_o;
   const float *merge_lse;
+  const int32_t *heads;  // grid row -> b * H + h, or NULL for grid row = b * H + h
+  int n_bh;              // B * H
   unsigned long long timeout_ns;
 };
 
@@ -192,7 +194,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   volatile int *abort = &ctl->abort;
 
   const int tile = blockIdx.x;
-  const int bh = blockIdx.y;
+  // (batch, head) of this grid row: the caller's head list, or all of them in order.  An
+  // out-of-range entry latches BAD_INDEX before any setup and the whole CTA leaves.
+  const int bh = a.heads ? __ldg(a.heads + blockIdx.y) : static_cast<int>(blockIdx.y);
+  if (bh < 0 || bh >= a.n_bh) {
+    if (threadIdx.x == 0) latch_status(VSA_ERR_BAD_INDEX);
+    return;
+  }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_lists = kTileM / a.list_rows;

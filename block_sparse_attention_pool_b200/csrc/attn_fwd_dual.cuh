@@ -83,7 +83,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   volatile int *abort = &ctl->abort;
 
   const int pair = blockIdx.x;
-  const int bh = blockIdx.y;
+  // (batch, head) of this grid row: the caller's head list, or all of them in order.  An
+  // out-of-range entry latches BAD_INDEX before any setup and the whole CTA leaves.
+  const int bh = a.heads ? __ldg(a.heads + blockIdx.y) : static_cast<int>(blockIdx.y);
+  if (bh < 0 || bh >= a.n_bh) {
+    if (threadIdx.x == 0) latch_status(VSA_ERR_BAD_INDEX);
+    return;
+  }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_tiles = a.n_pad / kTileM;

@@ -83,7 +83,7 @@ bool make_map(CUtensorMap *map, const void *base, const vsa_shape *s, int box_ro
 
 template <int D>
 vsa_status launch_attn(const void *q, const void *k, const void *v, const vsa_shape *s, const AttnArgs &a,
-                       cudaStream_t st) {
+                       int n_heads, cudaStream_t st) {
   using L = vsa::AttnSmem<D>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -94,7 +94,7 @@ vsa_status launch_attn(const void *q, const void *k, const void *v, const vsa_sh
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, s, vsa::kTileM) || !make_map(&mk, k, s, a.seg_keys) || !make_map(&mv, v, s, a.seg_keys))
     return VSA_ERR_CUDA;
-  dim3 grid(s->n_pad / vsa::kTileM, s->B * s->H);
+  dim3 grid(s->n_pad / vsa::kTileM, n_heads);
   vsa::attn_fwd_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, a);
   return launch_status();
 }
@@ -103,7 +103,7 @@ vsa_status launch_attn(const void *q, const void *k, const void *v, const vsa_sh
 // their K/V loads (attn_fwd_dual_kernel).
 template <int D>
 vsa_status launch_attn_dual(const void *q, const void *k, const void *v, const vsa_shape *s, const AttnArgs &a,
-                            cudaStream_t st) {
+                            int n_heads, cudaStream_t st) {
   using L = vsa::DualSmem<D>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -116,7 +116,7 @@ vsa_status launch_attn_dual(const void *q, const void *k, const void *v, const v
   if (!make_map(&mq, q, s, vsa::kTileM) || !make_map(&mk, k, s, vsa::kStageKeys) || !make_map(&mv, v, s, vsa::kStageKeys))
     return VSA_ERR_CUDA;
   const int n_tiles = s->n_pad / vsa::kTileM;
-  dim3 grid((n_tiles + 1) / 2, s->B * s->H);
+  dim3 grid((n_tiles + 1) / 2, n_heads);
   vsa::attn_fwd_dual_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, a);
   return launch_status();
 }
@@ -468,7 +468,20 @@ vsa_status vsa_block_sparse_fwd(const void *q, const void *k, const void *v, con
                                 int seg_keys, const int32_t *counts, const int32_t *idx, int idx_stride, float scale,
                                 void *o, int o_fp32, float *lse, const float *merge_o, const float *merge_lse,
                                 void *stream) {
+  if (!shape_ok(shape)) return VSA_ERR_INVALID_ARG;
+  return vsa_block_sparse_fwd_heads(q, k, v, shape, list_rows, seg_keys, counts, idx, idx_stride, scale, o, o_fp32,
+                                    lse, merge_o, merge_lse, nullptr, shape->B * shape->H, stream);
+}
+
+vsa_status vsa_block_sparse_fwd_heads(const void *q, const void *k, const void *v, const vsa_shape *shape,
+                                      int list_rows, int seg_keys, const int32_t *counts, const int32_t *idx,
+                                      int idx_stride, float scale, void *o, int o_fp32, float *lse,
+                                      const float *merge_o, const float *merge_lse, const int32_t *heads, int n_heads,
+                                      void *stream) {
   if (!shape_ok(shape) || !q || !k || !v || !counts || !idx || !o || !lse) return VSA_ERR_INVALID_ARG;
+  const long long n_bh = (long long)shape->B * shape->H;
+  if (n_heads < 0 || n_heads > n_bh || n_heads > 65535 || (heads == nullptr && n_heads != n_bh))
+    return VSA_ERR_INVALID_ARG;
   if (list_rows != 64 && list_rows != 128) return VSA_ERR_INVALID_ARG;
   if (seg_keys != 16 && seg_keys != 32 && seg_keys != 64 && seg_keys != 128) return VSA_ERR_INVALID_ARG;
   if (idx_stride < 1 || !(scale > 0.f) || !std::isfinite(scale)) return VSA_ERR_INVALID_ARG;
@@ -491,11 +504,15 @@ vsa_status vsa_block_sparse_fwd(const void *q, const void *k, const void *v, con
   a.lse = lse;
   a.merge_o = merge_o;
   a.merge_lse = merge_lse;
+  a.heads = heads;
+  a.n_bh = static_cast<int>(n_bh);
   a.timeout_ns = kWaitLimitNs;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n_heads == 0) return VSA_OK;
   if (list_rows == 128 && seg_keys == 128)
-    return shape->d == 128 ? launch_attn_dual<128>(q, k, v, shape, a, st) : launch_attn_dual<64>(q, k, v, shape, a, st);
-  return shape->d == 128 ? launch_attn<128>(q, k, v, shape, a, st) : launch_attn<64>(q, k, v, shape, a, st);
+    return shape->d == 128 ? launch_attn_dual<128>(q, k, v, shape, a, n_heads, st)
+                             : launch_attn_dual<64>(q, k, v, shape, a, n_heads, st);
+  return shape->d == 128 ? launch_attn<128>(q, k, v, shape, a, n_heads, st) : launch_attn<64>(q, k, v, shape, a, n_heads, st);
 }
 
 vsa_status vsa_lse_merge(const float *o_a, const float *lse_a, const float *o_b, const float *lse_b,

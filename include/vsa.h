@@ -8,6 +8,7 @@
  *   vsa_block_sparse_fwd attention over the kept tiles -> O, LSE    (Macro / Micro pass)
  *   vsa_select_micro     Micro tiles inside omitted blocks          (Micro selection)
  *   vsa_block_sparse_fwd again on the Micro lists, merged by LSE    (Micro pass + merge)
+ *   (vsa_block_sparse_fwd_heads: either pass on a subset of the heads)
  * plus vsa_mask_to_lists (an explicit block mask instead of selection) and
  * vsa_lse_merge (the stand-alone exact merge).
  *
@@ -267,6 +268,30 @@ VSA_API vsa_status vsa_block_sparse_fwd(const void *q, const void *k, const void
                                 int list_rows, int seg_keys, const int32_t *counts, const int32_t *idx,
                                 int idx_stride, float scale, void *o, int o_fp32, float *lse,
                                 const float *merge_o, const float *merge_lse, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * The same forward on a subset of the (batch, head) pairs.  Every (batch,
+ * head) is an independent problem ([HVA] section 2 Eq. (4) is per head), so a
+ * caller may run one pass on some heads and another pass on the rest: the
+ * Micro repair of [HyMoR] (abstract) is applied to some heads only, and those
+ * heads keep their Macro output in fp32 for the merge while the other heads'
+ * Macro output is already final.
+ *
+ * heads   : NULL (then n_heads must be B*H and the call equals
+ *           vsa_block_sparse_fwd), or a DEVICE int32 array of n_heads flattened
+ *           indices b*H + h, each in [0, B*H), no index twice.
+ * n_heads : 0 <= n_heads <= min(B*H, 65535); 0 enqueues nothing.
+ * Only the listed heads are read (their lists, Q/K/V, merge inputs) and
+ * written (their rows of o and lse); every other row of o and lse keeps its
+ * contents.  An out-of-range entry latches VSA_ERR_BAD_INDEX and writes
+ * nothing for that entry; a repeated entry makes two CTAs write the same rows
+ * (undefined result).  All other arguments as for vsa_block_sparse_fwd.
+ * ------------------------------------------------------------------------- */
+VSA_API vsa_status vsa_block_sparse_fwd_heads(const void *q, const void *k, const void *v, const vsa_shape *shape,
+                                              int list_rows, int seg_keys, const int32_t *counts, const int32_t *idx,
+                                              int idx_stride, float scale, void *o, int o_fp32, float *lse,
+                                              const float *merge_o, const float *merge_lse, const int32_t *heads,
+                                              int n_heads, void *stream);
 
 /* ---------------------------------------------------------------------------
  * Stand-alone exact LSE merge of two attention results over disjoint key

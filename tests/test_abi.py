@@ -65,6 +65,14 @@ def test_host_validation_rejects_bad_arguments(L):
     # merge output without its LSE
     assert L.vsa_block_sparse_fwd(fake, fake, fake, ctypes.byref(shape), 128, 128, fake, fake, 2, 0.125, fake, 0,
                                   fake, fake, null, null) == 1
+    # head subsets: negative or too many entries, or no list with fewer than B*H heads
+    fwd_h = L.vsa_block_sparse_fwd_heads
+    for heads, n in ((fake, -1), (fake, 3), (null, 1)):
+        assert fwd_h(fake, fake, fake, ctypes.byref(shape), 128, 128, fake, fake, 2, 0.125, fake, 0, fake, null,
+                     null, heads, n, null) == 1, n
+    # an empty head subset enqueues nothing (and needs no device)
+    assert fwd_h(fake, fake, fake, ctypes.byref(shape), 128, 128, fake, fake, 2, 0.125, fake, 0, fake, null,
+                 null, fake, 0, null) == 0
     # n_valid > n_pad
     bad = vsa.Shape(1, 2, 300, 256, 64)
     assert L.vsa_lse_merge(fake, fake, fake, fake, ctypes.byref(bad), fake, 0, fake, null) == 1

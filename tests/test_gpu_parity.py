@@ -226,6 +226,38 @@ def test_attention_ragged_and_empty_rows(n_pad, list_rows, seg):
     assert_close_rows(o.cpu().numpy(), lse.cpu().numpy(), O, L, [(0, h, 0, n_pad) for h in range(H)])
 
 
+@pytest.mark.parametrize("list_rows,seg", [(128, 128), (64, 16)])
+def test_attention_head_subset(list_rows, seg):
+    """vsa_block_sparse_fwd_heads on some (batch, head) pairs, given in any
+    order, writes for them exactly what the all-heads call writes, leaves the
+    other heads' rows untouched, and an out-of-range entry latches BAD_INDEX
+    without disturbing the valid entries."""
+    rng = np.random.default_rng(21 + seg)
+    B, H, n_pad, d = 2, 3, 640, 128
+    n_valid = n_pad - 40
+    q, k, v = (to_dev(round_to_bf16(rng.standard_normal((B, H, n_pad, d)).astype(np.float32))) for _ in range(3))
+    n_l, n_s = n_pad // list_rows, n_pad // seg
+    kept = [[[np.sort(rng.choice(n_s, size=int(rng.integers(1, n_s // 2 + 1)), replace=False))
+              for _ in range(n_l)] for _ in range(H)] for _ in range(B)]
+    counts, idx = lists_to_dev(kept, n_s, B, H, n_l)
+    shape = vsa.Shape(B, H, n_valid, n_pad, d)
+    scale = 1 / math.sqrt(d)
+    o_all = torch.empty(B * H, n_pad, d, device="cuda")
+    l_all = torch.empty(B * H, n_pad, device="cuda")
+    vsa.block_sparse_fwd(q, k, v, shape, list_rows, seg, counts, idx, n_s, scale, o_all, l_all)
+    for sub, status in (([4, 0, 3], 0), ([5, B * H + 7, 1], 5)):
+        o = torch.full((B * H, n_pad, d), 7.0, device="cuda")
+        lse = torch.full((B * H, n_pad), 5.0, device="cuda")
+        heads = torch.tensor(sub, dtype=torch.int32, device="cuda")
+        vsa.block_sparse_fwd(q, k, v, shape, list_rows, seg, counts, idx, n_s, scale, o, lse, heads=heads)
+        assert vsa.read_device_status() == status
+        for bh in range(B * H):
+            if bh in sub:
+                assert torch.equal(o[bh], o_all[bh]) and torch.equal(lse[bh], l_all[bh]), (sub, bh)
+            else:
+                assert torch.all(o[bh] == 7.0) and torch.all(lse[bh] == 5.0), (sub, bh)
+
+
 def test_attention_bad_list_latches_status():
     B, H, n_pad, d = 1, 1, 256, 128
     q = torch.zeros(B, H, n_pad, d, device="cuda", dtype=torch.bfloat16)
