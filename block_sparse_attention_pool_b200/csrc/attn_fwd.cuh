@@ -10,10 +10,13 @@
 // One CTA = one 128-row query tile of one (batch, head).  The tile's key
 // segments (list entries of seg_keys keys; the union of two 64-row lists
 // when list_rows = 64, each entry tagged with the halves that use it) are
-// packed into 128-key stages.  Warp roles:
+// packed into 128-key stages.  The union is built once, before the pipeline
+// starts, in shared memory (lists of up to kListStage entries; longer lists
+// are merged on the fly from global memory).  Warp roles:
 //   warp 0     TMA producer: Q once, then K and V of each stage into
 //              2 + 2 ring slots (128B-swizzled, one box per segment and
-//              64-column chunk; rows past n_valid arrive as zeros).
+//              64-column chunk, the boxes of a stage issued by one lane
+//              each; rows past n_valid arrive as zeros).
 //   warp 1     MMA issuer (one thread): S_s = Q K_s^T into TMEM buffer S[s&1],
 //              then O[s&1] += P_{s-1} V_{s-1}; tcgen05.commit frees ring slots
 //              and signals the softmax.
@@ -61,6 +64,8 @@ constexpr int kChunkBytes = 128 * 128;  // one 64-column bf16 chunk of a 128-row
 constexpr int kInfoRing = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kListStage = 2048;  // list entries staged in shared memory per list (fast path)
+constexpr int kUnionCap = 2 * kListStage;
 
 struct AttnArgs {
   int n_pad, n_valid;
@@ -82,6 +87,8 @@ struct StageInfo {
   int start[8];   // first key row of each segment of the stage
   uint32_t mask;  // bit 2*s + h: segment s is used by query half h
   int full;       // every column of the stage is used by every row
+  int tail;       // some used segment reaches past n_valid (exact per-column masks)
+  uint32_t use16; // bit 8*h + q: 16-column group q is used by query half h
 };
 
 template <int D>
@@ -92,7 +99,9 @@ struct AttnSmem {
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + 2 * kKVBytes;
   static constexpr int kOffX = kOffV + 2 * kKVBytes;  // epilogue exchange: [2 groups][3][128] floats
-  static constexpr int kOffCtl = kOffX + 4096;
+  static constexpr int kOffU = kOffX + 4096;          // the tile's segment union: [kUnionCap] entries
+  static constexpr int kOffL = kOffU + kUnionCap * 4; // the tile's lists, staged: [2][kListStage]
+  static constexpr int kOffCtl = kOffL + 2 * kListStage * 4;
   static constexpr int kBytes = kOffCtl + 1024;  // barriers, info ring, misc
   static constexpr int kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
 };
@@ -109,7 +118,7 @@ struct AttnCtl {
   uint32_t tmem_base;
   int abort;
   int n_seg;
-  int pad_;
+  int fast;  // the union sits in shared memory (lists short enough to stage)
   StageInfo info[kInfoRing];
 };
 
@@ -156,6 +165,19 @@ struct ListCursor {
     ++pos[0]; ++pos[1]; *m = 3u; return a;
   }
 };
+
+constexpr uint32_t kUnionDropped = 0xffffffffu;  // no real entry: segment indices stay below 2^30
+
+// Number of entries of the ascending array p[0, n) below v.
+__device__ __forceinline__ int lower_bound_smem(const int32_t *p, int n, int v) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (p[mid] < v) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
 
 // Warp-cooperative validation of one list (strictly ascending, in range);
 // returns false on a violation.
@@ -230,7 +252,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
     }
-    // segment count of the tile (union of its lists), with list validation
+    // Segment union of the tile, with list validation.  Fast path (both lists
+    // fit the staging area): the lists are copied to shared memory, checked
+    // there, and merged by rank into the union -- entry i of list 0 lands at
+    // i + #(list-1 entries below it), entry j of list 1 at j + #(list-0
+    // entries at or below it); a list-1 entry equal to a list-0 entry is
+    // dropped and that list-0 entry is tagged for both halves -- then one
+    // compaction pass closes the gaps.  Longer lists are walked from global
+    // memory by ListCursor (count here, segments again in the producer).
     const int n_seg_max = a.n_pad / a.seg_keys;
     int cnt[2] = {0, 0};
     bool ok = true;
@@ -238,21 +267,73 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       cnt[h] = __ldg(a.counts + lrow0 + h);
       if (cnt[h] < 0 || cnt[h] > a.idx_stride) ok = false;
     }
-    for (int h = 0; h < n_lists && ok; ++h)
-      ok = list_valid(a.idx + (lrow0 + h) * a.idx_stride, cnt[h], n_seg_max, lane);
+    const bool fast = ok && cnt[0] <= kListStage && cnt[1] <= kListStage;
     int n_seg = 0;
-    if (!ok) {
-      if (lane == 0) latch_status(VSA_ERR_BAD_INDEX);
-    } else if (n_lists == 1) {
-      n_seg = cnt[0];
-    } else {
-      // union size by a lockstep walk of the merge (coalesced 32-entry windows)
-      ListCursor cur;
-      cur.init(a.idx + lrow0 * a.idx_stride, cnt[0], a.idx + (lrow0 + 1) * a.idx_stride, cnt[1], 2, lane);
-      uint32_t m;
-      while (cur.next(&m, lane) >= 0) ++n_seg;
+    if (fast) {
+      int32_t *sl = reinterpret_cast<int32_t *>(smem + L::kOffL);
+      uint32_t *su = reinterpret_cast<uint32_t *>(smem + L::kOffU);
+      for (int h = 0; h < n_lists; ++h) {
+        const int32_t *src = a.idx + (lrow0 + h) * a.idx_stride;
+        for (int e = lane; e < cnt[h]; e += 32) sl[h * kListStage + e] = __ldg(src + e);
+      }
+      __syncwarp();
+      for (int h = 0; h < n_lists; ++h) {
+        const int32_t *li = sl + h * kListStage;
+        for (int e = lane; e < cnt[h]; e += 32) {
+          const int v = li[e];
+          if (v < 0 || v >= n_seg_max || (e > 0 && li[e - 1] >= v)) ok = false;
+        }
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok && n_lists == 1) {
+        for (int e = lane; e < cnt[0]; e += 32) su[e] = static_cast<uint32_t>(sl[e]) | (3u << 30);
+        n_seg = cnt[0];
+      } else if (ok) {
+        const int32_t *A = sl, *B = sl + kListStage;
+        const int nA = cnt[0], nB = cnt[1];
+        for (int i = lane; i < nA; i += 32) {
+          const int v = A[i];
+          const int r = lower_bound_smem(B, nB, v);
+          const bool d = r < nB && B[r] == v;
+          su[i + r] = static_cast<uint32_t>(v) | ((d ? 3u : 1u) << 30);
+        }
+        for (int j = lane; j < nB; j += 32) {
+          const int v = B[j];
+          const int r = lower_bound_smem(A, nA, v);
+          const bool d = r < nA && A[r] == v;
+          su[j + r + (d ? 1 : 0)] = d ? kUnionDropped : (static_cast<uint32_t>(v) | (2u << 30));
+        }
+        __syncwarp();
+        for (int k0 = 0; k0 < nA + nB; k0 += 32) {
+          const int k = k0 + lane;
+          const uint32_t x = k < nA + nB ? su[k] : kUnionDropped;
+          const uint32_t keep = __ballot_sync(0xffffffffu, x != kUnionDropped);
+          __syncwarp();
+          if (x != kUnionDropped) su[n_seg + __popc(keep & ((1u << lane) - 1u))] = x;
+          n_seg += __popc(keep);
+          __syncwarp();
+        }
+      }
+    } else if (ok) {
+      for (int h = 0; h < n_lists && ok; ++h)
+        ok = list_valid(a.idx + (lrow0 + h) * a.idx_stride, cnt[h], n_seg_max, lane);
+      if (ok && n_lists == 1) {
+        n_seg = cnt[0];
+      } else if (ok) {
+        ListCursor cur;
+        cur.init(a.idx + lrow0 * a.idx_stride, cnt[0], a.idx + (lrow0 + 1) * a.idx_stride, cnt[1], 2, lane);
+        uint32_t m;
+        while (cur.next(&m, lane) >= 0) ++n_seg;
+      }
     }
-    if (lane == 0) ctl->n_seg = n_seg;
+    if (!ok) {
+      n_seg = 0;
+      if (lane == 0) latch_status(VSA_ERR_BAD_INDEX);
+    }
+    if (lane == 0) {
+      ctl->n_seg = n_seg;
+      ctl->fast = fast ? 1 : 0;
+    }
   } else if (warp == 1) {
     tmem_alloc(&ctl->tmem_base, kTmemCols);
     tmem_relinquish();
@@ -270,60 +351,93 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (n_stages > 0) {
+      const bool fast = ctl->fast != 0;
+      const uint32_t *su = reinterpret_cast<const uint32_t *>(smem + L::kOffU);
       ListCursor cur;
-      cur.init(a.idx + lrow0 * a.idx_stride, __ldg(a.counts + lrow0),
-               n_lists > 1 ? a.idx + (lrow0 + 1) * a.idx_stride : nullptr,
-               n_lists > 1 ? __ldg(a.counts + lrow0 + 1) : 0, n_lists, lane);
+      if (!fast)
+        cur.init(a.idx + lrow0 * a.idx_stride, __ldg(a.counts + lrow0),
+                 n_lists > 1 ? a.idx + (lrow0 + 1) * a.idx_stride : nullptr,
+                 n_lists > 1 ? __ldg(a.counts + lrow0 + 1) : 0, n_lists, lane);
       if (lane == 0) {
         mbar_arrive_expect_tx(&ctl->q_full, L::kQBytes);
         for (int c = 0; c < D / 64; ++c)
           tma_load_3d(sQ + c * kChunkBytes, &tm_q, &ctl->q_full, c * 64, tile * kTileM, bh);
       }
+      // copy lane l < seg_per_stage * D/64 moves segment l / (D/64), column chunk l % (D/64)
+      constexpr int kNC = D / 64;
+      const int cp_seg = lane / kNC < 8 ? lane / kNC : 0;
+      const int cp_chunk = lane % kNC;
+      const bool cp_lane = lane < seg_per_stage * kNC;
+      const uint32_t all = seg_per_stage == 8 ? 0xffffu : ((1u << (2 * seg_per_stage)) - 1u);
+      const int g_shift = a.seg_shift - 4;  // 16-column groups per segment = 1 << g_shift
       int issued = 0;
       for (int s = 0; s < n_stages; ++s) {
         const int slot = s & 1;
         const uint32_t use_par = ((s >> 1) - 1) & 1;
-        int start[8];
-        uint32_t mask = 0u;
-        int nseg = 0;
-        for (int i = 0; i < seg_per_stage; ++i) {
-          uint32_t m = 0u;
-          const int sg = (nseg == i) ? cur.next(&m, lane) : -1;
-          if (sg >= 0) {
-            start[i] = sg * a.seg_keys;
-            mask |= m << (2 * i);
-            ++nseg;
-          } else {
-            start[i] = start[0];  // repeat a loaded segment; masked out
+        // this stage's segments: lane i < seg_per_stage holds segment i's first key row
+        int my_start = 0;
+        uint32_t b0 = 0u, b1 = 0u;  // bit i: segment i used by query half 0 / 1
+        if (fast) {
+          const int e = s * seg_per_stage + lane;
+          const bool has = lane < seg_per_stage && e < n_seg;
+          const uint32_t x = has ? su[e] : 0u;
+          const int seg = static_cast<int>(x & 0x3fffffffu);
+          const int seg0 = __shfl_sync(0xffffffffu, seg, 0);  // a stage holds at least one segment
+          my_start = (has ? seg : seg0) * a.seg_keys;
+          b0 = __ballot_sync(0xffffffffu, has && ((x >> 30) & 1u));
+          b1 = __ballot_sync(0xffffffffu, has && ((x >> 31) & 1u));
+        } else {
+          int start0 = 0, nseg = 0;
+          for (int i = 0; i < seg_per_stage; ++i) {
+            uint32_t m = 0u;
+            const int sg = (nseg == i) ? cur.next(&m, lane) : -1;
+            if (sg >= 0) {
+              if (i == 0) start0 = sg * a.seg_keys;
+              if (lane == i) my_start = sg * a.seg_keys;
+              b0 |= (m & 1u) << i;
+              b1 |= ((m >> 1) & 1u) << i;
+              ++nseg;
+            } else if (lane == i) {
+              my_start = start0;  // repeat a loaded segment; masked out
+            }
           }
         }
-        const uint32_t all = seg_per_stage == 8 ? 0xffffu : ((1u << (2 * seg_per_stage)) - 1u);
-        const bool full = (nseg == seg_per_stage) && (mask == all) &&
-                          (start[seg_per_stage - 1] + a.seg_keys <= a.n_valid);
+        const uint32_t used = b0 | b1;
+        const bool tail = __any_sync(0xffffffffu, lane < seg_per_stage && ((used >> lane) & 1u) &&
+                                                      my_start + a.seg_keys > a.n_valid);
+        uint32_t mask = 0u, use16 = 0u;
+        for (int i = 0; i < seg_per_stage; ++i) mask |= (((b0 >> i) & 1u) << (2 * i)) | (((b1 >> i) & 1u) << (2 * i + 1));
+        for (int q = 0; q < 8; ++q)
+          use16 |= (((b0 >> (q >> g_shift)) & 1u) << q) | (((b1 >> (q >> g_shift)) & 1u) << (8 + q));
+        const bool full = mask == all && !tail;
         bool ok = true;
         if (s >= 2) ok = mbar_wait_warp(&ctl->k_empty[slot], use_par, abort, a.timeout_ns, lane);
         if (!ok) break;
+        int st_i[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) st_i[i] = __shfl_sync(0xffffffffu, my_start, i);
         if (lane == 0) {
           StageInfo &inf = ctl->info[s & (kInfoRing - 1)];
-          for (int i = 0; i < 8; ++i) inf.start[i] = i < seg_per_stage ? start[i] : 0;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) inf.start[i] = i < seg_per_stage ? st_i[i] : 0;
           inf.mask = mask;
           inf.full = full ? 1 : 0;
+          inf.tail = tail ? 1 : 0;
+          inf.use16 = use16;
           mbar_arrive(&ctl->info_full[s & (kInfoRing - 1)]);
           mbar_arrive_expect_tx(&ctl->k_full[slot], L::kKVBytes);
-          for (int i = 0; i < seg_per_stage; ++i)
-            for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(sK + slot * L::kKVBytes + c * kChunkBytes + i * a.seg_keys * 128, &tm_k,
-                          &ctl->k_full[slot], c * 64, start[i], bh);
         }
+        __syncwarp();
+        const int cp_row = __shfl_sync(0xffffffffu, my_start, cp_seg);
+        const uint32_t cp_off = cp_chunk * kChunkBytes + cp_seg * a.seg_keys * 128;
+        if (cp_lane)
+          tma_load_3d(sK + slot * L::kKVBytes + cp_off, &tm_k, &ctl->k_full[slot], cp_chunk * 64, cp_row, bh);
         if (s >= 2) ok = mbar_wait_warp(&ctl->v_empty[slot], use_par, abort, a.timeout_ns, lane);
         if (!ok) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&ctl->v_full[slot], L::kKVBytes);
-          for (int i = 0; i < seg_per_stage; ++i)
-            for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(sV + slot * L::kKVBytes + c * kChunkBytes + i * a.seg_keys * 128, &tm_v,
-                          &ctl->v_full[slot], c * 64, start[i], bh);
-        }
+        if (lane == 0) mbar_arrive_expect_tx(&ctl->v_full[slot], L::kKVBytes);
+        __syncwarp();
+        if (cp_lane)
+          tma_load_3d(sV + slot * L::kKVBytes + cp_off, &tm_v, &ctl->v_full[slot], cp_chunk * 64, cp_row, bh);
         issued = s + 1;
         __syncwarp();
       }
@@ -409,9 +523,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tSg + lane_off + c * 32, r[c]);
       tmem_ld_wait();
-      if (!inf.full) {
-        // cold path: valid columns as a 128-bit mask built per segment (a used
-        // segment's valid keys form one prefix of it)
+      if (!inf.full && !inf.tail) {
+        // segments wholly inside n_valid: this half's used 16-column groups
+        const uint32_t u = inf.use16 >> (8 * half);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const bool drop = !((u >> q) & 1u);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (drop) r[q >> 1][(q & 1) * 16 + j] = __float_as_uint(-INFINITY);
+        }
+      } else if (!inf.full) {
+        // a segment reaches past n_valid: valid columns as a 128-bit mask built
+        // per segment (a used segment's valid keys form one prefix of it)
         uint64_t vm[2] = {0ull, 0ull};
         const uint32_t mask = inf.mask;
         const int nseg = kStageKeys >> a.seg_shift;

@@ -258,6 +258,39 @@ def test_attention_head_subset(list_rows, seg):
                 assert torch.all(o[bh] == 7.0) and torch.all(lse[bh] == 5.0), (sub, bh)
 
 
+def test_attention_long_lists_both_union_paths():
+    """64-row lists of 16-key segments as long as the sequence allows: tiles
+    whose two lists fit the shared-memory staging (up to 2048 entries each,
+    union up to 4096) take the staged union; a tile with a longer list is
+    merged from global memory.  Rows of both kinds, and a short neighbour,
+    are compared with the oracle."""
+    rng = np.random.default_rng(77)
+    B, H, d, seg, list_rows = 1, 1, 128, 16, 64
+    n_pad = seg * 2304
+    n_valid = n_pad - 9
+    q, k, v = (round_to_bf16(rng.standard_normal((B, H, n_pad, d)).astype(np.float32)) for _ in range(3))
+    n_l, n_s = n_pad // list_rows, n_pad // seg
+    pick = lambda n: np.sort(rng.choice(n_s, size=n, replace=False))
+    kept = [[[pick(int(rng.integers(0, 40))) for _ in range(n_l)]]]
+    sizes = {2: 2100, 3: 50,            # tile 1: one list past the staging size (global merge)
+             10: 2048, 11: 2048,        # tile 5: both at the staging size (staged union)
+             20: 2300, 21: 2200,        # tile 10: both long
+             n_l - 2: 1500, n_l - 1: 2048}
+    for r, n in sizes.items():
+        kept[0][0][r] = pick(n)
+    counts, idx = lists_to_dev(kept, n_s, B, H, n_l)
+    shape = vsa.Shape(B, H, n_valid, n_pad, d)
+    o = torch.empty(B, H, n_pad, d, device="cuda")
+    lse = torch.empty(B, H, n_pad, device="cuda")
+    scale = 1 / math.sqrt(d)
+    vsa.block_sparse_fwd(to_dev(q), to_dev(k), to_dev(v), shape, list_rows, seg, counts, idx, n_s, scale, o, lse)
+    assert vsa.read_device_status() == 0
+    rows = [(0, 0, r) for r in sorted(set(sizes) | {0, 1, 30})]
+    O, L = orc.block_sparse_attention(q, k, v, kept, list_rows, seg, n_valid, scale, rows=rows)
+    assert_close_rows(o.cpu().numpy(), lse.cpu().numpy(), O, L,
+                      [(b, h, r * list_rows, (r + 1) * list_rows) for b, h, r in rows])
+
+
 def test_attention_bad_list_latches_status():
     B, H, n_pad, d = 1, 1, 256, 128
     q = torch.zeros(B, H, n_pad, d, device="cuda", dtype=torch.bfloat16)
