@@ -15,6 +15,10 @@
 // sorted in registers (32 keys per lane at most, n_k <= 1024), the sorted
 // weights are exponentiated and prefix-summed, and the kept prefix plus the
 // anchors is written out as an ascending index list with ballot compaction.
+// A fixed count (fixed_k > 0) needs the set of the k largest weights only: that
+// instantiation keeps 32-bit keys, finds the k-th largest by a bitwise search
+// and marks the set without sorting (same set as the sort, ties to the lower
+// block index).
 #pragma once
 
 #include "common.cuh"
@@ -93,6 +97,39 @@ __device__ __forceinline__ void warp_bitonic_sort_desc(uint64_t (&key)[NR], int 
   }
 }
 
+// Fixed count: mark in the warp bitmap the m largest of the row's score keys
+// (element j = 32 i + lane in register i; equal keys go to the lower j;
+// 1 <= m <= number of real elements, padding keys are 0).  The set needs no
+// order, so instead of a sort the m-th largest key H is found bit by bit
+// (the largest H with #(key >= H) >= m), and of the keys equal to H the
+// lowest-index ones fill the rank.  Word i of the bitmap is register i's ballot.
+template <int NR>
+__device__ __forceinline__ void mark_top_m(const uint32_t (&hk)[NR], int m, int lane, uint32_t *bits) {
+  uint32_t H = 0u;
+#pragma unroll 1
+  for (int b = 31; b >= 0; --b) {
+    const uint32_t cand = H | (1u << b);
+    unsigned c = 0u;
+#pragma unroll
+    for (int i = 0; i < NR; ++i) c += hk[i] >= cand ? 1u : 0u;
+    if (static_cast<int>(__reduce_add_sync(0xffffffffu, c)) >= m) H = cand;
+  }
+  unsigned above = 0u;
+#pragma unroll
+  for (int i = 0; i < NR; ++i) above += hk[i] > H ? 1u : 0u;
+  const int need = m - static_cast<int>(__reduce_add_sync(0xffffffffu, above));
+  const uint32_t lt = (1u << lane) - 1u;
+  int before = 0;  // keys equal to H at lower element indices
+#pragma unroll
+  for (int i = 0; i < NR; ++i) {
+    const uint32_t eq = __ballot_sync(0xffffffffu, hk[i] == H);
+    const bool sel = hk[i] > H || (hk[i] == H && before + __popc(eq & lt) < need);
+    const uint32_t word = __ballot_sync(0xffffffffu, sel);
+    if (lane == (i & 31)) bits[i] = word;
+    before += __popc(eq);
+  }
+}
+
 // Emit the ascending index list of the set bits of a per-warp bitmap of n bits
 // (word w covers indices [32w, 32w + 32)); returns the count.
 __device__ __forceinline__ int emit_bitmap_list(const uint32_t *bits, int n, int lane, int32_t *dst,
@@ -119,7 +156,7 @@ __device__ __forceinline__ int emit_bitmap_list(const uint32_t *bits, int n, int
   return total;
 }
 
-template <int D, int NR>
+template <int D, int NR, bool BY_RANK>
 __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a) {
   constexpr int DP = D + 4;  // padded row stride (floats)
   extern __shared__ __align__(16) float sel_smem[];
@@ -190,78 +227,105 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     uint8_t *mrow = a.mask ? a.mask + orow * a.n_k : nullptr;
     const bool q_has_rows = qi * a.bq < a.n_valid;
 
-    // Load: element j = i*32 + lane goes to register i (any start placement
-    // sorts to the same result).
-    uint64_t key[NR];
-#pragma unroll
-    for (int i = 0; i < NR; ++i) {
-      const int j = i * 32 + lane;
-      if (j < a.n_k) {
-        const int sj = min(a.bk, max(0, a.n_valid - j * a.bk));
-        const float w = sj > 0 ? S[r * nkp + j] + (sj == a.bk ? ln_bk : logf((float)sj)) : -INFINITY;
-        key[i] = ((uint64_t)float_key(w) << 32) | (uint64_t)(0xffffffffu - (uint32_t)j);
-      } else {
-        key[i] = 0ull;
-      }
-    }
-    warp_bitonic_sort_desc<NR>(key, lane);
-
-    int m = 0;
-    if (q_has_rows) {
-      if (a.fixed_k > 0) {
-        m = min(a.fixed_k, a.n_k);
-      } else {
-        int m_p = 0;
-        if (a.cum_mass > 0.f) {
-          const float wmax = key_float((uint32_t)(__shfl_sync(0xffffffffu, key[0], 0) >> 32));
-          float p[NR];
-          float lsum = 0.f;
-#pragma unroll
-          for (int i = 0; i < NR; ++i) {
-            const bool real = key[i] != 0ull;
-            const float w = key_float((uint32_t)(key[i] >> 32));
-            p[i] = (real && w != -INFINITY) ? expf(w - wmax) : 0.f;
-            lsum += p[i];
-            p[i] = lsum;  // inclusive lane-local prefix
-          }
-          // exclusive prefix of lane totals
-          float base = lsum;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const float y = __shfl_up_sync(0xffffffffu, base, o);
-            if (lane >= o) base += y;
-          }
-          const float total = __shfl_sync(0xffffffffu, base, 31);
-          base -= lsum;
-          const float target = a.cum_mass * total;
-          int first = 0x7fffffff;
-#pragma unroll
-          for (int i = NR - 1; i >= 0; --i)
-            if (base + p[i] >= target) first = lane * NR + i;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) first = min(first, __shfl_xor_sync(0xffffffffu, first, o));
-          m_p = first == 0x7fffffff ? a.n_k : first + 1;
-        }
-        m = min(a.n_k, max(a.k_min, m_p));
-      }
-    }
-
-    // mark the kept prefix and the anchors
-    bits[lane] = 0u;
-    __syncwarp();
-    if (q_has_rows) {
+    if constexpr (BY_RANK) {
+      // fixed count (fixed_k > 0): the k largest log-weights, no order needed
+      uint32_t hk[NR];
 #pragma unroll
       for (int i = 0; i < NR; ++i) {
-        if (lane * NR + i < m) {
-          const int j = (int)(0xffffffffu - (uint32_t)(key[i] & 0xffffffffull));
-          atomicOr(&bits[j >> 5], 1u << (j & 31));
+        const int j = i * 32 + lane;
+        uint32_t kv = 0u;
+        if (j < a.n_k) {
+          const int sj = min(a.bk, max(0, a.n_valid - j * a.bk));
+          const float w = sj > 0 ? S[r * nkp + j] + (sj == a.bk ? ln_bk : logf((float)sj)) : -INFINITY;
+          kv = float_key(w);
         }
+        hk[i] = kv;
       }
-      if (lane == 0 && a.n_anchor > 0) {
+      bits[lane] = 0u;
+      __syncwarp();
+      if (q_has_rows) mark_top_m<NR>(hk, min(a.fixed_k, a.n_k), lane, bits);
+      __syncwarp();
+      if (q_has_rows && lane == 0 && a.n_anchor > 0) {
         const int step = a.n_k / a.n_anchor;
         for (int tt = 0; tt < a.n_anchor; ++tt) {
           const int j = (int)(((long long)a.anchor_rot + (long long)tt * step) % a.n_k);
           atomicOr(&bits[j >> 5], 1u << (j & 31));
+        }
+      }
+    } else {
+      // Load: element j = i*32 + lane goes to register i (any start placement
+      // sorts to the same result).
+      uint64_t key[NR];
+  #pragma unroll
+      for (int i = 0; i < NR; ++i) {
+        const int j = i * 32 + lane;
+        if (j < a.n_k) {
+          const int sj = min(a.bk, max(0, a.n_valid - j * a.bk));
+          const float w = sj > 0 ? S[r * nkp + j] + (sj == a.bk ? ln_bk : logf((float)sj)) : -INFINITY;
+          key[i] = ((uint64_t)float_key(w) << 32) | (uint64_t)(0xffffffffu - (uint32_t)j);
+        } else {
+          key[i] = 0ull;
+        }
+      }
+      warp_bitonic_sort_desc<NR>(key, lane);
+
+      int m = 0;
+      if (q_has_rows) {
+        if (a.fixed_k > 0) {
+          m = min(a.fixed_k, a.n_k);
+        } else {
+          int m_p = 0;
+          if (a.cum_mass > 0.f) {
+            const float wmax = key_float((uint32_t)(__shfl_sync(0xffffffffu, key[0], 0) >> 32));
+            float p[NR];
+            float lsum = 0.f;
+  #pragma unroll
+            for (int i = 0; i < NR; ++i) {
+              const bool real = key[i] != 0ull;
+              const float w = key_float((uint32_t)(key[i] >> 32));
+              p[i] = (real && w != -INFINITY) ? expf(w - wmax) : 0.f;
+              lsum += p[i];
+              p[i] = lsum;  // inclusive lane-local prefix
+            }
+            // exclusive prefix of lane totals
+            float base = lsum;
+  #pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const float y = __shfl_up_sync(0xffffffffu, base, o);
+              if (lane >= o) base += y;
+            }
+            const float total = __shfl_sync(0xffffffffu, base, 31);
+            base -= lsum;
+            const float target = a.cum_mass * total;
+            int first = 0x7fffffff;
+  #pragma unroll
+            for (int i = NR - 1; i >= 0; --i)
+              if (base + p[i] >= target) first = lane * NR + i;
+  #pragma unroll
+            for (int o = 16; o > 0; o >>= 1) first = min(first, __shfl_xor_sync(0xffffffffu, first, o));
+            m_p = first == 0x7fffffff ? a.n_k : first + 1;
+          }
+          m = min(a.n_k, max(a.k_min, m_p));
+        }
+      }
+
+      // mark the kept prefix and the anchors
+      bits[lane] = 0u;
+      __syncwarp();
+      if (q_has_rows) {
+  #pragma unroll
+        for (int i = 0; i < NR; ++i) {
+          if (lane * NR + i < m) {
+            const int j = (int)(0xffffffffu - (uint32_t)(key[i] & 0xffffffffull));
+            atomicOr(&bits[j >> 5], 1u << (j & 31));
+          }
+        }
+        if (lane == 0 && a.n_anchor > 0) {
+          const int step = a.n_k / a.n_anchor;
+          for (int tt = 0; tt < a.n_anchor; ++tt) {
+            const int j = (int)(((long long)a.anchor_rot + (long long)tt * step) % a.n_k);
+            atomicOr(&bits[j >> 5], 1u << (j & 31));
+          }
         }
       }
     }

@@ -290,9 +290,10 @@ vsa_status vsa_select_blocks(const float *q_pool, const float *k_pool, const vsa
   const size_t smem = (size_t)(vsa::kSelRows + vsa::kSelChunk) * dp * 4 + (size_t)vsa::kSelRows * nkp * 4 + 8 * 32 * 4;
   dim3 grid((n_q + vsa::kSelRows - 1) / vsa::kSelRows, shape->B * shape->H);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool by_rank = params->fixed_k > 0;  // a fixed count needs no sort
 #define VSA_SEL_CASE(DD, NR)                                                                                  \
   {                                                                                                           \
-    auto kern = vsa::select_blocks_kernel<DD, NR>;                                                            \
+    auto kern = by_rank ? vsa::select_blocks_kernel<DD, NR, true> : vsa::select_blocks_kernel<DD, NR, false>; \
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) \
       return VSA_ERR_CUDA;                                                                                    \
     kern<<<grid, vsa::kSelThreads, smem, st>>>(a);                                                            \
