@@ -179,6 +179,66 @@ __device__ __forceinline__ int lower_bound_smem(const int32_t *p, int n, int v) 
   return lo;
 }
 
+// Warp-cooperative: stages one or two ascending lists (n0, n1 entries, each
+// at most `stride`) in shared memory at sl and sl + stride, checks them
+// (entries strictly ascending, in [0, n_max)), and writes their union to su,
+// ascending, each entry = index | (lists holding it) << 30 (bit 30: list 0,
+// bit 31: list 1; a lone list gets single_tag).  Two lists are merged by rank
+// -- entry i of list 0 lands at i + #(list-1 entries below it), entry j of
+// list 1 at j + #(list-0 entries at or below it); a list-1 entry equal to a
+// list-0 entry is dropped and that list-0 entry is tagged for both -- and one
+// compaction pass closes the gaps.  Returns the union size, or -1 when a
+// list is invalid.  su holds n0 + n1 entries of scratch.
+__device__ __forceinline__ int stage_union(const int32_t *g0, int n0, const int32_t *g1, int n1, int n_lists,
+                                           int n_max, int32_t *sl, int stride, uint32_t *su, uint32_t single_tag,
+                                           int lane) {
+  const int cnt[2] = {n0, n_lists > 1 ? n1 : 0};
+  const int32_t *src[2] = {g0, g1};
+  for (int h = 0; h < n_lists; ++h)
+    for (int e = lane; e < cnt[h]; e += 32) sl[h * stride + e] = __ldg(src[h] + e);
+  __syncwarp();
+  bool ok = true;
+  for (int h = 0; h < n_lists; ++h) {
+    const int32_t *li = sl + h * stride;
+    for (int e = lane; e < cnt[h]; e += 32) {
+      const int v = li[e];
+      if (v < 0 || v >= n_max || (e > 0 && li[e - 1] >= v)) ok = false;
+    }
+  }
+  if (!__all_sync(0xffffffffu, ok)) return -1;
+  if (n_lists == 1) {
+    for (int e = lane; e < cnt[0]; e += 32) su[e] = static_cast<uint32_t>(sl[e]) | (single_tag << 30);
+    __syncwarp();
+    return cnt[0];
+  }
+  const int32_t *A = sl, *B = sl + stride;
+  const int nA = cnt[0], nB = cnt[1];
+  for (int i = lane; i < nA; i += 32) {
+    const int v = A[i];
+    const int r = lower_bound_smem(B, nB, v);
+    const bool d = r < nB && B[r] == v;
+    su[i + r] = static_cast<uint32_t>(v) | ((d ? 3u : 1u) << 30);
+  }
+  for (int j = lane; j < nB; j += 32) {
+    const int v = B[j];
+    const int r = lower_bound_smem(A, nA, v);
+    const bool d = r < nA && A[r] == v;
+    su[j + r + (d ? 1 : 0)] = d ? kUnionDropped : (static_cast<uint32_t>(v) | (2u << 30));
+  }
+  __syncwarp();
+  int n = 0;
+  for (int k0 = 0; k0 < nA + nB; k0 += 32) {
+    const int k = k0 + lane;
+    const uint32_t x = k < nA + nB ? su[k] : kUnionDropped;
+    const uint32_t keep = __ballot_sync(0xffffffffu, x != kUnionDropped);
+    __syncwarp();
+    if (x != kUnionDropped) su[n + __popc(keep & ((1u << lane) - 1u))] = x;
+    n += __popc(keep);
+    __syncwarp();
+  }
+  return n;
+}
+
 // Warp-cooperative validation of one list (strictly ascending, in range);
 // returns false on a violation.
 __device__ __forceinline__ bool list_valid(const int32_t *p, int n, int n_seg_max, int lane) {
@@ -270,50 +330,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const bool fast = ok && cnt[0] <= kListStage && cnt[1] <= kListStage;
     int n_seg = 0;
     if (fast) {
-      int32_t *sl = reinterpret_cast<int32_t *>(smem + L::kOffL);
-      uint32_t *su = reinterpret_cast<uint32_t *>(smem + L::kOffU);
-      for (int h = 0; h < n_lists; ++h) {
-        const int32_t *src = a.idx + (lrow0 + h) * a.idx_stride;
-        for (int e = lane; e < cnt[h]; e += 32) sl[h * kListStage + e] = __ldg(src + e);
-      }
-      __syncwarp();
-      for (int h = 0; h < n_lists; ++h) {
-        const int32_t *li = sl + h * kListStage;
-        for (int e = lane; e < cnt[h]; e += 32) {
-          const int v = li[e];
-          if (v < 0 || v >= n_seg_max || (e > 0 && li[e - 1] >= v)) ok = false;
-        }
-      }
-      ok = __all_sync(0xffffffffu, ok);
-      if (ok && n_lists == 1) {
-        for (int e = lane; e < cnt[0]; e += 32) su[e] = static_cast<uint32_t>(sl[e]) | (3u << 30);
-        n_seg = cnt[0];
-      } else if (ok) {
-        const int32_t *A = sl, *B = sl + kListStage;
-        const int nA = cnt[0], nB = cnt[1];
-        for (int i = lane; i < nA; i += 32) {
-          const int v = A[i];
-          const int r = lower_bound_smem(B, nB, v);
-          const bool d = r < nB && B[r] == v;
-          su[i + r] = static_cast<uint32_t>(v) | ((d ? 3u : 1u) << 30);
-        }
-        for (int j = lane; j < nB; j += 32) {
-          const int v = B[j];
-          const int r = lower_bound_smem(A, nA, v);
-          const bool d = r < nA && A[r] == v;
-          su[j + r + (d ? 1 : 0)] = d ? kUnionDropped : (static_cast<uint32_t>(v) | (2u << 30));
-        }
-        __syncwarp();
-        for (int k0 = 0; k0 < nA + nB; k0 += 32) {
-          const int k = k0 + lane;
-          const uint32_t x = k < nA + nB ? su[k] : kUnionDropped;
-          const uint32_t keep = __ballot_sync(0xffffffffu, x != kUnionDropped);
-          __syncwarp();
-          if (x != kUnionDropped) su[n_seg + __popc(keep & ((1u << lane) - 1u))] = x;
-          n_seg += __popc(keep);
-          __syncwarp();
-        }
-      }
+      n_seg = stage_union(a.idx + lrow0 * a.idx_stride, cnt[0], a.idx + (lrow0 + 1) * a.idx_stride, cnt[1],
+                          n_lists, n_seg_max, reinterpret_cast<int32_t *>(smem + L::kOffL), kListStage,
+                          reinterpret_cast<uint32_t *>(smem + L::kOffU), 3u, lane);
+      ok = n_seg >= 0;
     } else if (ok) {
       for (int h = 0; h < n_lists && ok; ++h)
         ok = list_valid(a.idx + (lrow0 + h) * a.idx_stride, cnt[h], n_seg_max, lane);

@@ -29,7 +29,10 @@
 //              normalise O: an exact convex combination of the V rows used).
 // TMEM: S_A [0,128), S_B [128,256), O_A [256, 256 + d), O_B [384, 384 + d).
 //
-// Barrier phases: s_full[X] and p_full[X] advance once per block of tile X;
+// P of a block goes to TMEM in two halves: p_half[X] signals keys 0-63, so the
+// first half of the block's P.V runs while the softmax exponentiates keys
+// 64-127, and p_full[X] signals the rest.
+// Barrier phases: s_full[X], p_half[X] and p_full[X] advance once per block of tile X;
 // S_X of X's next block is issued only after the MMA issuer waited p_full[X]
 // of the current one, so neither can run two phases ahead of its waiter.  The
 // commit that signals S_X(s) also covers P.V of X's previous block (issued
@@ -43,6 +46,8 @@
 
 namespace vsa {
 
+constexpr int kDualList = 1024;  // list entries staged per tile (every list of n_k <= 1024 blocks)
+
 template <int D>
 struct DualSmem {
   static constexpr int kQBytes = kTileM * D * 2;
@@ -50,7 +55,9 @@ struct DualSmem {
   static constexpr int kOffQ = 0;                       // Q_A, Q_B
   static constexpr int kOffK = kOffQ + 2 * kQBytes;
   static constexpr int kOffV = kOffK + 2 * kKVBytes;
-  static constexpr int kOffCtl = kOffV + 2 * kKVBytes;
+  static constexpr int kOffU = kOffV + 2 * kKVBytes;          // union of the two lists [kDualList * 2]
+  static constexpr int kOffL = kOffU + 2 * kDualList * 4;     // the two lists, staged [2][kDualList]
+  static constexpr int kOffCtl = kOffL + 2 * kDualList * 4;
   static constexpr int kBytes = kOffCtl + 512;
   static constexpr int kAlloc = kBytes + 1024;
 };
@@ -60,12 +67,14 @@ struct DualCtl {
   uint64_t k_full[2], k_empty[2];
   uint64_t v_full[2], v_empty[2];
   uint64_t s_full[2];  // per tile
-  uint64_t p_full[2];  // per tile
+  uint64_t p_full[2];  // per tile: P of the block's keys 64-127 written (and its keys 0-63 before)
+  uint64_t p_half[2];  // per tile: P of the block's keys 0-63 written
   uint64_t mma_drain;
   uint32_t tmem_base;
   int abort;
   int n_union;
   int cnt[2];
+  int fast;  // union and lists staged in shared memory
 };
 
 template <int D>
@@ -109,6 +118,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_init(&ctl->v_empty[i], 1);
         mbar_init(&ctl->s_full[i], 1);
         mbar_init(&ctl->p_full[i], 128);
+        mbar_init(&ctl->p_half[i], 128);
       }
       mbar_init(&ctl->mma_drain, 1);
       ctl->abort = 0;
@@ -123,16 +133,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       cnt[x] = __ldg(a.counts + lrow0 + x);
       if (cnt[x] < 0 || cnt[x] > a.idx_stride) ok = false;
     }
-    for (int x = 0; x < (has_b ? 2 : 1) && ok; ++x)
-      ok = list_valid(a.idx + (lrow0 + x) * a.idx_stride, cnt[x], n_key_blocks, lane);
+    // lists short enough to stage: validated and merged into the union in
+    // shared memory once; otherwise validated here and walked from global
+    // memory by ListCursor
+    const bool fast = ok && cnt[0] <= kDualList && cnt[1] <= kDualList;
+    int n_union = cnt[0] + cnt[1];  // cursor path: > 0 iff the union is not empty
+    if (fast) {
+      n_union = stage_union(a.idx + lrow0 * a.idx_stride, cnt[0], a.idx + (lrow0 + 1) * a.idx_stride, cnt[1],
+                            has_b ? 2 : 1, n_key_blocks, reinterpret_cast<int32_t *>(smem + L::kOffL), kDualList,
+                            reinterpret_cast<uint32_t *>(smem + L::kOffU), 1u, lane);
+      ok = n_union >= 0;
+    } else {
+      for (int x = 0; x < (has_b ? 2 : 1) && ok; ++x)
+        ok = list_valid(a.idx + (lrow0 + x) * a.idx_stride, cnt[x], n_key_blocks, lane);
+    }
     if (!ok) {
       if (lane == 0) latch_status(VSA_ERR_BAD_INDEX);
       cnt[0] = cnt[1] = 0;
+      n_union = 0;
     }
     if (lane == 0) {
-      ctl->n_union = cnt[0] + cnt[1];  // > 0 iff the union is not empty
+      ctl->n_union = n_union;
       ctl->cnt[0] = cnt[0];
       ctl->cnt[1] = cnt[1];
+      ctl->fast = fast ? 1 : 0;
     }
   } else if (warp == 1) {
     tmem_alloc(&ctl->tmem_base, kTmemCols);
@@ -150,12 +174,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tO[2] = {tmem + 256u, tmem + 384u};
   const int32_t *list[2] = {a.idx + lrow0 * a.idx_stride, a.idx + (lrow0 + 1) * a.idx_stride};
   const int cnt[2] = {ctl->cnt[0], has_b ? ctl->cnt[1] : 0};
+  const bool fast = ctl->fast != 0;
+  const int n_union = ctl->n_union;
+  const uint32_t *su = reinterpret_cast<const uint32_t *>(smem + L::kOffU);
+  const int32_t *sl = reinterpret_cast<const int32_t *>(smem + L::kOffL);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (any_block) {
       ListCursor cur;
-      cur.init(list[0], cnt[0], has_b ? list[1] : nullptr, cnt[1], has_b ? 2 : 1, lane);
+      if (!fast) cur.init(list[0], cnt[0], has_b ? list[1] : nullptr, cnt[1], has_b ? 2 : 1, lane);
       if (lane == 0) {
         mbar_arrive_expect_tx(&ctl->q_full, (has_b ? 2 : 1) * L::kQBytes);
         for (int x = 0; x < (has_b ? 2 : 1); ++x)
@@ -167,8 +195,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int slot = s & 1;
         const uint32_t use_par = ((s >> 1) - 1) & 1;
         uint32_t m = 0u;
-        const int blk = cur.next(&m, lane);
-        if (blk < 0) break;
+        int blk;
+        if (fast) {
+          if (s >= n_union) break;
+          blk = static_cast<int>(su[s] & 0x3fffffffu);
+        } else {
+          blk = cur.next(&m, lane);
+          if (blk < 0) break;
+        }
         const int start = blk * kStageKeys;
         bool ok = true;
         if (s >= 2) ok = mbar_wait_warp(&ctl->k_empty[slot], use_par, abort, a.timeout_ns, lane);
@@ -209,7 +243,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t dV0 = smem_desc_sw128(smem_addr(sV), kChunkBytes, 1024);
       constexpr uint64_t kQStep = L::kQBytes >> 4, kSlotStep = L::kKVBytes >> 4;
       ListCursor cur;
-      cur.init(list[0], cnt[0], has_b ? list[1] : nullptr, cnt[1], has_b ? 2 : 1, lane);
+      if (!fast) cur.init(list[0], cnt[0], has_b ? list[1] : nullptr, cnt[1], has_b ? 2 : 1, lane);
       bool ok = true;
       if (lane == 0) ok = mbar_wait(&ctl->q_full, 0, abort, a.timeout_ns);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -218,14 +252,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // O_x += P_x(block s) V_s
       auto issue_pv = [&](auto xc, int s) -> bool {
         constexpr int x = decltype(xc)::value;
-        if (!mbar_wait(&ctl->p_full[x], pv_cnt[x] & 1, abort, a.timeout_ns)) return false;
+        // keys 0-63 of the block as soon as their P is in TMEM, keys 64-127 after
+        if (!mbar_wait(&ctl->p_half[x], pv_cnt[x] & 1, abort, a.timeout_ns)) return false;
         if (!mbar_wait(&ctl->v_full[s & 1], (s >> 1) & 1, abort, a.timeout_ns)) return false;
         tc_fence_after();
         const uint64_t dv = dV0 + (uint64_t)(s & 1) * kSlotStep;
         const uint32_t first = pv_cnt[x] > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < kStageKeys / 16; ++kk)
+        for (int kk = 0; kk < kStageKeys / 32; ++kk)
           umma_bf16_ts(tO[x], tS[x] + kk * 8, dv + (uint64_t)(kk * 16 * 128 / 16), kIdO, kk > 0 ? 1u : first);
+        if (!mbar_wait(&ctl->p_full[x], pv_cnt[x] & 1, abort, a.timeout_ns)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = kStageKeys / 32; kk < kStageKeys / 16; ++kk)
+          umma_bf16_ts(tO[x], tS[x] + kk * 8, dv + (uint64_t)(kk * 16 * 128 / 16), kIdO, 1u);
         ++pv_cnt[x];
         return true;
       };
@@ -244,8 +284,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int s = 0;
       for (;; ++s) {
         uint32_t use = 0u;
-        if (cur.next(&use, lane) < 0) break;  // whole warp walks the union in lockstep
-        if (!has_b) use &= 1u;  // a single-list cursor tags every block with both bits
+        if (fast) {
+          if (s >= n_union) break;
+          use = su[s] >> 30;
+        } else {
+          if (cur.next(&use, lane) < 0) break;  // whole warp walks the union in lockstep
+          if (!has_b) use &= 1u;  // a single-list cursor tags every block with both bits
+        }
         if (lane == 0 && ok) {
           // P.V of a tile's block s-1 goes before its S of block s: that S
           // overwrites the TMEM buffer holding the tile's P.
@@ -300,7 +345,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
     const int n_mine = tile_live ? (x == 0 ? cnt[0] : cnt[1]) : 0;
     for (int i = 0; i < n_mine; ++i) {
-      const int key0 = __ldg(listx + i) * kStageKeys;
+      const int key0 = (fast ? sl[x * kDualList + i] : __ldg(listx + i)) * kStageKeys;
       ok = mbar_wait_warp(&ctl->s_full[x], i & 1, abort, a.timeout_ns, lane);
       if (!ok) break;
       tc_fence_after();
@@ -337,8 +382,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float2 nm2 = make_float2(neg_m, neg_m);
       float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       float rr[4] = {0.f, 0.f, 0.f, 0.f};
+      // P of keys 0-63 (logit chunks 0, 1), packed into r[0]
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const float2 xx = ffma2(make_float2(__uint_as_float(r[c][2 * j]), __uint_as_float(r[c][2 * j + 1])), sc2, nm2);
@@ -346,30 +392,48 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           rs2[j & 1] = fadd2(rs2[j & 1], p);
           const uint32_t pk = pack_bf16x2(p.x, p.y);
           rr[j & 3] = add_bf16x2_f32(rr[j & 3], pk);
-          r[c >> 1][(c & 1) * 16 + j] = pk;
+          r[0][c * 16 + j] = pk;
         }
       }
-      const float2 rsum = fadd2(rs2[0], rs2[1]);
-      l += rsum.x + rsum.y;
-      lr += (rr[0] + rr[1]) + (rr[2] + rr[3]);
       if (any_rescale && i > 0) {
-        // cold path: the commit that signalled this S also covered the P.V of
-        // the tile's previous block, so O_x is settled
+        // cold path, before any P.V of this block: the commit that signalled
+        // this S also covered the P.V of the tile's previous block, so O_x is
+        // settled
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tOx + lane_off + c * 32, o);
+        for (int c = 0; c < D / 8; ++c) {  // 8 columns at a time: the logits of keys 64-127 are still live
+          uint32_t o[8];
+          tmem_ld8(tOx + lane_off + c * 8, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-          tmem_st32(tOx + lane_off + c * 32, o);
+          for (int j = 0; j < 8; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          tmem_st8(tOx + lane_off + c * 8, o);
         }
       }
+      // keys 0-63 handed to the tensor core first: their P.V overlaps the
+      // exponentials of keys 64-127
       tmem_st32(tSx + lane_off + 0, r[0]);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&ctl->p_half[x]);
+#pragma unroll
+      for (int c = 2; c < 4; ++c) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float2 xx = ffma2(make_float2(__uint_as_float(r[c][2 * j]), __uint_as_float(r[c][2 * j + 1])), sc2, nm2);
+          const float2 p = make_float2(fast_exp2(xx.x), fast_exp2(xx.y));
+          rs2[j & 1] = fadd2(rs2[j & 1], p);
+          const uint32_t pk = pack_bf16x2(p.x, p.y);
+          rr[j & 3] = add_bf16x2_f32(rr[j & 3], pk);
+          r[1][(c - 2) * 16 + j] = pk;
+        }
+      }
       tmem_st32(tSx + lane_off + 32, r[1]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&ctl->p_full[x]);
+      const float2 rsum = fadd2(rs2[0], rs2[1]);
+      l += rsum.x + rsum.y;
+      lr += (rr[0] + rr[1]) + (rr[2] + rr[3]);
     }
 
     // ---------------------------------------------------------- epilogue
