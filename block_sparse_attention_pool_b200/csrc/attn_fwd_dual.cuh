@@ -37,7 +37,13 @@
 // of the current one, so neither can run two phases ahead of its waiter.  The
 // commit that signals S_X(s) also covers P.V of X's previous block (issued
 // before it), which is what a lazy rescale of O_X needs.  The K/V ring slots
-// are released by commits after the last MMA that reads them.
+// are released by one commit per union block s (into kv_free[s & 1]), issued
+// after the block's S MMAs, which follow the P.V of block s-1: it frees K_s and
+// V_{s-1}.  The producer waits on it for K_{s+2} and, one block later, for
+// V_{s+1}; block s+2 cannot commit before K_{s+2} is loaded, so the wait stays
+// unambiguous.  Issuing a tcgen05.mma costs the issuing thread most of the
+// MMA's execution time, so the issuer does as few waits and commits per
+// block as it can.
 #pragma once
 
 #include <type_traits>
@@ -64,8 +70,8 @@ struct DualSmem {
 
 struct DualCtl {
   uint64_t q_full;
-  uint64_t k_full[2], k_empty[2];
-  uint64_t v_full[2], v_empty[2];
+  uint64_t k_full[2], v_full[2];
+  uint64_t kv_free[2];  // one commit per union block s into kv_free[s & 1]: K_s and V_{s-1} are free
   uint64_t s_full[2];  // per tile
   uint64_t p_full[2];  // per tile: P of the block's keys 64-127 written (and its keys 0-63 before)
   uint64_t p_half[2];  // per tile: P of the block's keys 0-63 written
@@ -113,9 +119,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&ctl->q_full, 1);
       for (int i = 0; i < 2; ++i) {
         mbar_init(&ctl->k_full[i], 1);
-        mbar_init(&ctl->k_empty[i], 1);
+        mbar_init(&ctl->kv_free[i], 1);
         mbar_init(&ctl->v_full[i], 1);
-        mbar_init(&ctl->v_empty[i], 1);
         mbar_init(&ctl->s_full[i], 1);
         mbar_init(&ctl->p_full[i], 128);
         mbar_init(&ctl->p_half[i], 128);
@@ -205,14 +210,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         const int start = blk * kStageKeys;
         bool ok = true;
-        if (s >= 2) ok = mbar_wait_warp(&ctl->k_empty[slot], use_par, abort, a.timeout_ns, lane);
+        if (s >= 2) ok = mbar_wait_warp(&ctl->kv_free[slot], use_par, abort, a.timeout_ns, lane);  // K_{s-2} read
         if (!ok) break;
         if (lane == 0) {
           mbar_arrive_expect_tx(&ctl->k_full[slot], L::kKVBytes);
           for (int c = 0; c < D / 64; ++c)
             tma_load_3d(sK + slot * L::kKVBytes + c * kChunkBytes, &tm_k, &ctl->k_full[slot], c * 64, start, bh);
         }
-        if (s >= 2) ok = mbar_wait_warp(&ctl->v_empty[slot], use_par, abort, a.timeout_ns, lane);
+        // V_{s-2} read: committed with block s-1
+        if (s >= 2) ok = mbar_wait_warp(&ctl->kv_free[slot ^ 1], ((s - 1) >> 1) & 1, abort, a.timeout_ns, lane);
         if (!ok) break;
         if (lane == 0) {
           mbar_arrive_expect_tx(&ctl->v_full[slot], L::kKVBytes);
@@ -250,11 +256,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       uint32_t prev = 0u;     // usage bits of the previous union block
       int pv_cnt[2] = {0, 0};  // P.V issued so far per tile
       // O_x += P_x(block s) V_s
-      auto issue_pv = [&](auto xc, int s) -> bool {
+      auto issue_pv = [&](auto xc, int s, bool &v_ready) -> bool {
         constexpr int x = decltype(xc)::value;
         // keys 0-63 of the block as soon as their P is in TMEM, keys 64-127 after
         if (!mbar_wait(&ctl->p_half[x], pv_cnt[x] & 1, abort, a.timeout_ns)) return false;
-        if (!mbar_wait(&ctl->v_full[s & 1], (s >> 1) & 1, abort, a.timeout_ns)) return false;
+        if (!v_ready) {
+          if (!mbar_wait(&ctl->v_full[s & 1], (s >> 1) & 1, abort, a.timeout_ns)) return false;
+          v_ready = true;
+        }
         tc_fence_after();
         const uint64_t dv = dV0 + (uint64_t)(s & 1) * kSlotStep;
         const uint32_t first = pv_cnt[x] > 0 ? 1u : 0u;
@@ -294,8 +303,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (lane == 0 && ok) {
           // P.V of a tile's block s-1 goes before its S of block s: that S
           // overwrites the TMEM buffer holding the tile's P.
-          bool k_ready = false;
-          if (prev & 1u) ok = issue_pv(std::integral_constant<int, 0>{}, s - 1);
+          bool k_ready = false, v_ready = false;
+          if (prev & 1u) ok = issue_pv(std::integral_constant<int, 0>{}, s - 1, v_ready);
           if (ok && (use & 1u)) {
             ok = mbar_wait(&ctl->k_full[s & 1], (s >> 1) & 1, abort, a.timeout_ns);
             k_ready = true;
@@ -304,7 +313,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               issue_s(std::integral_constant<int, 0>{}, s);
             }
           }
-          if (ok && (prev & 2u)) ok = issue_pv(std::integral_constant<int, 1>{}, s - 1);
+          if (ok && (prev & 2u)) ok = issue_pv(std::integral_constant<int, 1>{}, s - 1, v_ready);
           if (ok && (use & 2u)) {
             if (!k_ready) ok = mbar_wait(&ctl->k_full[s & 1], (s >> 1) & 1, abort, a.timeout_ns);
             if (ok) {
@@ -313,16 +322,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
           }
           if (ok) {
-            umma_commit(&ctl->k_empty[s & 1]);                 // S MMAs of block s read K_s
-            if (s >= 1) umma_commit(&ctl->v_empty[(s - 1) & 1]);  // P.V of block s-1 read V_{s-1}
+            umma_commit(&ctl->kv_free[s & 1]);  // the S MMAs of block s read K_s, the P.V of block s-1 V_{s-1}
           }
         }
         prev = use;
       }
       if (lane == 0) {
-        if (ok && (prev & 1u)) ok = issue_pv(std::integral_constant<int, 0>{}, s - 1);
-        if (ok && (prev & 2u)) ok = issue_pv(std::integral_constant<int, 1>{}, s - 1);
-        if (ok) umma_commit(&ctl->v_empty[(s - 1) & 1]);
+        bool v_ready = false;
+        if (ok && (prev & 1u)) ok = issue_pv(std::integral_constant<int, 0>{}, s - 1, v_ready);
+        if (ok && (prev & 2u)) ok = issue_pv(std::integral_constant<int, 1>{}, s - 1, v_ready);
         umma_commit(&ctl->mma_drain);
         mbar_drain(&ctl->mma_drain, 0, a.timeout_ns);
       }
