@@ -290,42 +290,49 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         umma_commit(&ctl->s_full[x]);
       };
+      // one union block: P.V of a tile's block s-1 goes before its S of block
+      // s (that S overwrites the TMEM buffer holding the tile's P)
+      auto step = [&](int s, uint32_t use) {
+        bool k_ready = false, v_ready = false;
+        if (prev & 1u) ok = issue_pv(std::integral_constant<int, 0>{}, s - 1, v_ready);
+        if (ok && (use & 1u)) {
+          ok = mbar_wait(&ctl->k_full[s & 1], (s >> 1) & 1, abort, a.timeout_ns);
+          k_ready = true;
+          if (ok) {
+            tc_fence_after();
+            issue_s(std::integral_constant<int, 0>{}, s);
+          }
+        }
+        if (ok && (prev & 2u)) ok = issue_pv(std::integral_constant<int, 1>{}, s - 1, v_ready);
+        if (ok && (use & 2u)) {
+          if (!k_ready) ok = mbar_wait(&ctl->k_full[s & 1], (s >> 1) & 1, abort, a.timeout_ns);
+          if (ok) {
+            tc_fence_after();
+            issue_s(std::integral_constant<int, 1>{}, s);
+          }
+        }
+        if (ok) umma_commit(&ctl->kv_free[s & 1]);  // the S MMAs of block s read K_s, the P.V of block s-1 V_{s-1}
+        prev = use;
+      };
       int s = 0;
-      for (;; ++s) {
-        uint32_t use = 0u;
-        if (fast) {
-          if (s >= n_union) break;
-          use = su[s] >> 30;
-        } else {
+      if (fast) {
+        // the union sits in shared memory: lane 0 walks it alone
+        if (lane == 0) {
+          uint32_t e = n_union > 0 ? su[0] : 0u;
+          for (; s < n_union && ok; ++s) {
+            const uint32_t cur_e = e;
+            if (s + 1 < n_union) e = su[s + 1];  // next entry, loaded while this block issues
+            step(s, cur_e >> 30);
+          }
+        }
+      } else {
+        for (;; ++s) {
+          uint32_t use = 0u;
           if (cur.next(&use, lane) < 0) break;  // whole warp walks the union in lockstep
           if (!has_b) use &= 1u;  // a single-list cursor tags every block with both bits
+          if (lane == 0 && ok) step(s, use);
+          prev = use;
         }
-        if (lane == 0 && ok) {
-          // P.V of a tile's block s-1 goes before its S of block s: that S
-          // overwrites the TMEM buffer holding the tile's P.
-          bool k_ready = false, v_ready = false;
-          if (prev & 1u) ok = issue_pv(std::integral_constant<int, 0>{}, s - 1, v_ready);
-          if (ok && (use & 1u)) {
-            ok = mbar_wait(&ctl->k_full[s & 1], (s >> 1) & 1, abort, a.timeout_ns);
-            k_ready = true;
-            if (ok) {
-              tc_fence_after();
-              issue_s(std::integral_constant<int, 0>{}, s);
-            }
-          }
-          if (ok && (prev & 2u)) ok = issue_pv(std::integral_constant<int, 1>{}, s - 1, v_ready);
-          if (ok && (use & 2u)) {
-            if (!k_ready) ok = mbar_wait(&ctl->k_full[s & 1], (s >> 1) & 1, abort, a.timeout_ns);
-            if (ok) {
-              tc_fence_after();
-              issue_s(std::integral_constant<int, 1>{}, s);
-            }
-          }
-          if (ok) {
-            umma_commit(&ctl->kv_free[s & 1]);  // the S MMAs of block s read K_s, the P.V of block s-1 V_{s-1}
-          }
-        }
-        prev = use;
       }
       if (lane == 0) {
         bool v_ready = false;
