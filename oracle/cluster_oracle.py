@@ -1,0 +1,198 @@
+"""fp64 CPU oracle of 3D local-window clustering and the cluster permutation.
+
+TEST INFRASTRUCTURE.  Like vsa_oracle, this file is the independent statement
+of what the CUDA library computes, used only by the tests, the package smoke
+check and the benchmark's CPU-baseline leg.  It shares no code with the CUDA
+path.  Plain NumPy in float64.
+
+Source: HyperVAttention: Efficient Sparse Attention with Spatio-Temporal
+Clustering for Video Diffusion (arXiv 2607.03012v1), "HVA" below:
+
+* §2 Eq. (1): the query and key tokens are reordered by permutations Pi^q
+  and Pi^k so that the tokens of a cluster are contiguous (V follows K);
+* §2 Eq. (4): attention runs on the reordered tensors and the output is put
+  back in token order, O = (Pi^q)^-1 O';
+* §4.1 Eq. (5): the T x H x W token lattice is cut into regular cells of
+  (k_t, k_h, k_w) tokens, one centroid per cell, initialised from the token
+  at the centre of the cell; a token is assigned to the nearest (squared
+  Euclidean) centroid among the cells of a (w_t, w_h, w_w) window around its
+  own cell; a centroid is then the mean of the tokens assigned to it; the
+  cells never move, and the two steps repeat.
+
+Readings taken where the page is silent (listed in the design notes too):
+
+ C1 cell counts per axis are ceil(T / k_t) etc.; a cell at the far edge of
+    an axis holds the remaining tokens;
+ C2 the "token at the centre" of a cell with extent e along an axis is at
+    offset (e - 1) // 2 from the cell's start (the lower middle);
+ C3 the window of w cells along an axis spans cell offsets
+    -((w - 1) // 2) .. w // 2 around the token's cell, clipped to the grid
+    (symmetric for odd w; one more cell on the far side for even w);
+ C4 ties in the assignment go to the lower flat cell index (t-major, then h,
+    then w);
+ C5 a centroid that receives no token keeps its previous value;
+ C6 one iteration = assignment of every token, then the centroid update;
+    the returned assignment is that of the last iteration and the returned
+    centroids are those of its update;
+ C7 within a cluster the permutation keeps the original token order, and the
+    clusters follow each other in flat cell order; padding rows (at or past
+    N_valid) stay where they are;
+ C8 blocks of the permuted sequence are the attention blocks: the permuted
+    Q', K', V' go through the same pooling, selection and attention as the
+    unpermuted path (fixed block sizes).  Cluster-aligned variable blocks
+    (padding or merging clusters to tile sizes, HVA §4.3) are a later step.
+"""
+from __future__ import annotations
+
+from typing import Dict, Sequence, Tuple
+
+import numpy as np
+
+__all__ = [
+    "cell_counts", "token_cells", "initial_centroids", "window_offsets", "window_cells",
+    "local_window_clustering", "clustering_objective", "cluster_permutation", "permute_rows",
+    "unpermute_rows", "forward_clustered",
+]
+
+
+def cell_counts(grid: Sequence[int], cell: Sequence[int]) -> Tuple[int, int, int]:
+    """Cells per axis (reading C1)."""
+    return tuple(-(-g // c) for g, c in zip(grid, cell))
+
+
+def token_cells(grid, cell) -> np.ndarray:
+    """g(l) of Eq. (5) for every token l of the T x H x W lattice in frame-first
+    order, as a flat cell index (t-major)."""
+    T, H, W = grid
+    CT, CH, CW = cell_counts(grid, cell)
+    t, h, w = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")
+    ct, ch, cw = t // cell[0], h // cell[1], w // cell[2]
+    return ((ct * CH + ch) * CW + cw).reshape(-1)
+
+
+def initial_centroids(x: np.ndarray, grid, cell) -> np.ndarray:
+    """One centroid per cell: the embedding of the cell's centre token
+    (reading C2).  x: [N, d] with N = T*H*W in frame-first order."""
+    T, H, W = grid
+    CT, CH, CW = cell_counts(grid, cell)
+    mu = np.zeros((CT * CH * CW, x.shape[1]))
+    for ct in range(CT):
+        for ch in range(CH):
+            for cw in range(CW):
+                start = (ct * cell[0], ch * cell[1], cw * cell[2])
+                ext = (min(cell[0], T - start[0]), min(cell[1], H - start[1]), min(cell[2], W - start[2]))
+                t, h, w = (s + (e - 1) // 2 for s, e in zip(start, ext))
+                mu[(ct * CH + ch) * CW + cw] = x[(t * H + h) * W + w]
+    return mu
+
+
+def window_offsets(w: int) -> range:
+    """Cell offsets of a window of w cells along one axis (reading C3)."""
+    return range(-((w - 1) // 2), w // 2 + 1)
+
+
+def window_cells(cell_coord, counts, window) -> np.ndarray:
+    """Flat indices of the cells of the window around one cell, ascending."""
+    CT, CH, CW = counts
+    out = []
+    for dt in window_offsets(window[0]):
+        for dh in window_offsets(window[1]):
+            for dw in window_offsets(window[2]):
+                t, h, w = cell_coord[0] + dt, cell_coord[1] + dh, cell_coord[2] + dw
+                if 0 <= t < CT and 0 <= h < CH and 0 <= w < CW:
+                    out.append((t * CH + h) * CW + w)
+    return np.array(sorted(out), dtype=np.int64)
+
+
+def local_window_clustering(x: np.ndarray, grid, cell, window, n_iter: int) -> Tuple[np.ndarray, np.ndarray]:
+    """HVA §4.1 Eq. (5), n_iter rounds of (assignment, centroid update).
+
+    x: [N, d] token embeddings (N = T*H*W, frame-first order).  Returns the
+    assignment a [N] (flat cell index of each token's centroid) and the
+    centroids mu [n_cells, d].
+    """
+    x = np.asarray(x, dtype=np.float64)
+    counts = cell_counts(grid, cell)
+    CT, CH, CW = counts
+    g = token_cells(grid, cell)
+    mu = initial_centroids(x, grid, cell)
+    a = np.zeros(x.shape[0], dtype=np.int64)
+    # the tokens of each cell share one window
+    cell_tokens = [np.nonzero(g == u)[0] for u in range(CT * CH * CW)]
+    windows = [window_cells((u // (CH * CW), (u // CW) % CH, u % CW), counts, window) for u in range(CT * CH * CW)]
+    for _ in range(n_iter):
+        for u, toks in enumerate(cell_tokens):
+            if toks.size == 0:
+                continue
+            cand = windows[u]
+            diff = x[toks][:, None, :] - mu[cand][None, :, :]
+            dist = np.einsum("tcd,tcd->tc", diff, diff)
+            a[toks] = cand[np.argmin(dist, axis=1)]  # argmin keeps the first minimum: lower cell (C4)
+        for u in range(mu.shape[0]):
+            members = a == u
+            if members.any():
+                mu[u] = x[members].mean(axis=0)
+    return a, mu
+
+
+def clustering_objective(x: np.ndarray, a: np.ndarray, mu: np.ndarray) -> float:
+    """Sum over tokens of the squared distance to the assigned centroid."""
+    diff = np.asarray(x, dtype=np.float64) - mu[a]
+    return float(np.einsum("nd,nd->", diff, diff))
+
+
+def cluster_permutation(a: np.ndarray, n_cells: int, n_pad: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Pi of Eq. (1) as a gather index: row i of the permuted sequence is
+    token perm[i].  Tokens of cluster 0 first, then cluster 1, ...; original
+    order within a cluster; padding rows N..n_pad-1 stay in place (C7).
+    Returns (perm [n_pad], sizes [n_cells])."""
+    N = a.shape[0]
+    order = np.argsort(a, kind="stable")
+    perm = np.concatenate([order, np.arange(N, n_pad)]).astype(np.int64)
+    sizes = np.bincount(a, minlength=n_cells).astype(np.int64)
+    return perm, sizes
+
+
+def permute_rows(x: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    """x' = Pi x along the token axis (the last-but-one axis for 2-D rows)."""
+    return x[perm]
+
+
+def unpermute_rows(y: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    """x = Pi^-1 y: row perm[i] of the result is row i of y (Eq. (4))."""
+    out = np.empty_like(y)
+    out[perm] = y
+    return out
+
+
+def forward_clustered(q, k, v, w, cell, window, n_iter, head_enable=None) -> Dict[str, object]:
+    """Cluster Q and K per (batch, head), permute (Eq. (1)), run the
+    unpermuted path's oracle (vsa_oracle.forward) on Q', K', V', and put O and
+    LSE back in token order (Eq. (4)).  Reading C8."""
+    from .vsa_oracle import forward
+    B, H, n_pad, d = q.shape
+    N = w.n_valid
+    grid = w.grid
+    n_cells = int(np.prod(cell_counts(grid, cell)))
+    qp, kp, vp = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    perms = {"q": np.zeros((B, H, n_pad), dtype=np.int64), "k": np.zeros((B, H, n_pad), dtype=np.int64)}
+    assign = {"q": np.zeros((B, H, N), dtype=np.int64), "k": np.zeros((B, H, N), dtype=np.int64)}
+    for b in range(B):
+        for h in range(H):
+            for name, x in (("q", q), ("k", k)):
+                a, _ = local_window_clustering(x[b, h, :N], grid, cell, window, n_iter)
+                perm, _ = cluster_permutation(a, n_cells, n_pad)
+                perms[name][b, h] = perm
+                assign[name][b, h] = a
+            qp[b, h] = permute_rows(q[b, h], perms["q"][b, h])
+            kp[b, h] = permute_rows(k[b, h], perms["k"][b, h])
+            vp[b, h] = permute_rows(v[b, h], perms["k"][b, h])
+    res = forward(qp, kp, vp, w, head_enable=head_enable)
+    O = np.empty_like(res["O"])
+    L = np.empty_like(res["LSE"])
+    for b in range(B):
+        for h in range(H):
+            O[b, h] = unpermute_rows(res["O"][b, h], perms["q"][b, h])
+            L[b, h] = unpermute_rows(res["LSE"][b, h], perms["q"][b, h])
+    return {"perm_q": perms["q"], "perm_k": perms["k"], "assign_q": assign["q"], "assign_k": assign["k"],
+            "permuted": res, "O": O, "LSE": L}
