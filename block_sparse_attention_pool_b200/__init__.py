@@ -25,7 +25,7 @@ __all__ = [
     "VsaError", "Shape", "SelectParams", "MicroParams", "lib", "library_path", "EXPORTED",
     "pool_qk", "select_blocks", "mask_to_lists", "select_micro", "select_micro_workspace_bytes", "select_micro_noalloc",
     "block_sparse_fwd", "lse_merge", "read_device_status", "status_string", "version", "selftest_wait_timeout",
-    "PathConfig", "SparseVideoAttention",
+    "PathConfig", "SparseVideoAttention", "ClusterParams", "cluster_count", "cluster_tokens", "permute_rows",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -35,6 +35,7 @@ EXPORTED = (
     "vsa_status_string", "vsa_version", "vsa_read_device_status", "vsa_pool_qk", "vsa_select_blocks",
     "vsa_mask_to_lists", "vsa_select_micro_workspace_bytes", "vsa_select_micro", "vsa_select_micro_noalloc",
     "vsa_block_sparse_fwd", "vsa_block_sparse_fwd_heads", "vsa_lse_merge", "vsa_selftest_wait_timeout",
+    "vsa_cluster_count", "vsa_cluster_tokens", "vsa_permute_rows",
 )
 
 STATUS = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_UNSUPPORTED", 3: "VSA_ERR_CUDA",
@@ -53,6 +54,17 @@ class VsaError(RuntimeError):
 class Shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("n_valid", ctypes.c_int), ("n_pad", ctypes.c_int),
                 ("d", ctypes.c_int)]
+
+
+class ClusterParams(ctypes.Structure):
+    """vsa_cluster_params: token lattice, cell extents (tokens), window (cells), rounds."""
+    _fields_ = [("lattice_t", ctypes.c_int), ("lattice_h", ctypes.c_int), ("lattice_w", ctypes.c_int),
+                ("cell_t", ctypes.c_int), ("cell_h", ctypes.c_int), ("cell_w", ctypes.c_int),
+                ("win_t", ctypes.c_int), ("win_h", ctypes.c_int), ("win_w", ctypes.c_int), ("iters", ctypes.c_int)]
+
+    @staticmethod
+    def make(lattice, cell, window, iters) -> "ClusterParams":
+        return ClusterParams(*[int(v) for v in (*lattice, *cell, *window, iters)])
 
 
 class SelectParams(ctypes.Structure):
@@ -108,6 +120,12 @@ def lib():
     L.vsa_block_sparse_fwd_heads.argtypes = [P, P, P, SP, I, I, P, P, I, F, P, I, P, P, P, P, I, P]
     L.vsa_lse_merge.restype = I
     L.vsa_lse_merge.argtypes = [P, P, P, P, SP, P, I, P, P]
+    L.vsa_cluster_count.restype = I
+    L.vsa_cluster_count.argtypes = [ctypes.POINTER(ClusterParams)]
+    L.vsa_cluster_tokens.restype = I
+    L.vsa_cluster_tokens.argtypes = [P, SP, ctypes.POINTER(ClusterParams), P, P, P, P, P]
+    L.vsa_permute_rows.restype = I
+    L.vsa_permute_rows.argtypes = [P, P, I, I, I, I, P, P]
     _lib = L
     return L
 
@@ -227,6 +245,24 @@ def block_sparse_fwd(q, k, v, shape: Shape, list_rows, seg_keys, counts, idx, id
                                             int(heads.numel()), _s(stream)), "vsa_block_sparse_fwd_heads")
 
 
+def cluster_count(params: ClusterParams) -> int:
+    return int(lib().vsa_cluster_count(ctypes.byref(params)))
+
+
+def cluster_tokens(x, shape: Shape, params: ClusterParams, assign, centroids, sizes, perm, stream=None):
+    _check(lib().vsa_cluster_tokens(_p(x), ctypes.byref(shape), ctypes.byref(params), _p(assign), _p(centroids),
+                                    _p(sizes), _p(perm), _s(stream)), "vsa_cluster_tokens")
+
+
+def permute_rows(src, perm, dst, inverse: bool = False, stream=None):
+    """Rows of src [B, H, n_pad, ...] gathered by perm [B, H, n_pad] into dst
+    (inverse: scattered)."""
+    B, H, n_pad = perm.shape
+    row_bytes = src[0, 0, 0].numel() * src.element_size() if src.dim() > 3 else src.element_size()
+    _check(lib().vsa_permute_rows(_p(src), _p(perm), B * H, n_pad, row_bytes, 1 if inverse else 0, _p(dst),
+                                  _s(stream)), "vsa_permute_rows")
+
+
 def lse_merge(o_a, lse_a, o_b, lse_b, shape: Shape, o_out, lse_out, stream=None):
     out_fp32 = 1 if o_out.dtype == torch.float32 else 0
     _check(lib().vsa_lse_merge(_p(o_a), _p(lse_a), _p(o_b), _p(lse_b), ctypes.byref(shape), _p(o_out), out_fp32,
@@ -254,6 +290,14 @@ class PathConfig:
     micro_percentile: float = 0.0
     micro_heads: Optional[Sequence[int]] = None
     micro_capacity: int = 0          # 0: every tile of the row fits (no overflow possible)
+    # cluster-permuted layout (HyperVAttention Eq. (1), (4), (5)): None = tokens in their own order
+    cluster_lattice: Optional[Sequence[int]] = None   # (T, H, W) with T*H*W == n_valid
+    cluster_cell: Sequence[int] = (3, 5, 8)
+    cluster_window: Sequence[int] = (3, 5, 5)
+    cluster_iters: int = 3
+
+    def cluster_params(self) -> "ClusterParams":
+        return ClusterParams.make(self.cluster_lattice, self.cluster_cell, self.cluster_window, self.cluster_iters)
 
     @staticmethod
     def from_workload(w, micro_heads=None) -> "PathConfig":
@@ -311,6 +355,23 @@ class SparseVideoAttention:
                 "workspace": torch.empty(max(16, ws), device=dev, dtype=torch.uint8),
             })
             self.micro_cap = cap
+        if c.cluster_lattice is not None:
+            G = cluster_count(c.cluster_params())
+            if G <= 0:
+                raise ValueError("invalid clustering parameters")
+            bf = torch.bfloat16
+            b.update({
+                "qp": torch.empty(B, H, n_pad, d, device=dev, dtype=bf),
+                "kp": torch.empty(B, H, n_pad, d, device=dev, dtype=bf),
+                "vp": torch.empty(B, H, n_pad, d, device=dev, dtype=bf),
+                "op": torch.empty(B, H, n_pad, d, device=dev, dtype=bf),
+                "lp": torch.empty(B, H, n_pad, device=dev, dtype=f32),
+            })
+            for name in ("q", "k"):
+                b["assign_" + name] = torch.empty(B, H, c.n_valid, device=dev, dtype=i32)
+                b["centroids_" + name] = torch.empty(B, H, G, d, device=dev, dtype=f32)
+                b["sizes_" + name] = torch.empty(B, H, G, device=dev, dtype=i32)
+                b["perm_" + name] = torch.empty(B, H, n_pad, device=dev, dtype=i32)
         self.buf = b
         self._key = key
 
@@ -333,6 +394,34 @@ class SparseVideoAttention:
 
     def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None, out_o=None, out_lse=None,
                  micro_heads=None, on_stage=None) -> Dict[str, torch.Tensor]:
+        """Run the path on device tensors q, k, v [B, H, n_pad, d] (bf16).
+
+        With ``cfg.cluster_lattice`` set, Q and K are first clustered per
+        (batch, head) by 3D local-window clustering, Q', K', V' are the
+        cluster-ordered rows (Eq. (1)), the path below runs on them, and O
+        and LSE are put back in token order (Eq. (4)); the permutations stay
+        in ``self.buf["perm_q"]`` / ``["perm_k"]``.  Otherwise see _run.
+        """
+        if self.cfg.cluster_lattice is None:
+            return self._run(q, k, v, stream, out_o, out_lse, micro_heads, on_stage)
+        self._alloc(q)
+        b = self.buf
+        B, H, n_pad, d = q.shape
+        shape = _shape(B, H, self.cfg.n_valid, n_pad, d)
+        params = self.cfg.cluster_params()
+        for name, x in (("q", q), ("k", k)):
+            cluster_tokens(x, shape, params, b["assign_" + name], b["centroids_" + name], b["sizes_" + name],
+                           b["perm_" + name], stream)
+        permute_rows(q, b["perm_q"], b["qp"], stream=stream)
+        permute_rows(k, b["perm_k"], b["kp"], stream=stream)
+        permute_rows(v, b["perm_k"], b["vp"], stream=stream)
+        self._run(b["qp"], b["kp"], b["vp"], stream, b["op"], b["lp"], micro_heads, on_stage)
+        permute_rows(b["op"], b["perm_q"], b["o"] if out_o is None else out_o, inverse=True, stream=stream)
+        permute_rows(b["lp"], b["perm_q"], b["lse"] if out_lse is None else out_lse, inverse=True, stream=stream)
+        return b
+
+    def _run(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None, out_o=None, out_lse=None,
+             micro_heads=None, on_stage=None) -> Dict[str, torch.Tensor]:
         """Run the whole path on device tensors q, k, v [B, H, n_pad, d] (bf16).
 
         Outputs go to ``self.buf["o"]`` / ``["lse"]``, or to ``out_o`` /

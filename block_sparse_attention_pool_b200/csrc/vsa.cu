@@ -11,12 +11,14 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 #include <vector>
 
 #include "../../include/vsa.h"
 #include "attn_fwd.cuh"
 #include "attn_fwd_dual.cuh"
+#include "cluster.cuh"
 #include "common.cuh"
 #include "merge.cuh"
 #include "micro.cuh"
@@ -213,6 +215,77 @@ __global__ void noalloc_slot_fill_kernel(HeadSlots hs, int32_t *slot_of_bh) {
   const int b = bh / hs.H, h = bh % hs.H;
   const int r = hs.slot[h];
   slot_of_bh[bh] = r < 0 ? -1 : b * hs.n_enabled + r;
+}
+
+
+// ---- clustering --------------------------------------------------------------
+
+// Geometry of valid clustering parameters, or false.
+bool cluster_geom(const vsa_cluster_params *p, vsa::ClusterGeom *g) {
+  if (!p) return false;
+  const int v[10] = {p->lattice_t, p->lattice_h, p->lattice_w, p->cell_t, p->cell_h, p->cell_w,
+                     p->win_t,     p->win_h,     p->win_w,     p->iters};
+  for (int i = 0; i < 10; ++i)
+    if (v[i] < 1) return false;
+  if (p->iters > 64) return false;
+  if ((long long)p->cell_t * p->cell_h * p->cell_w > vsa::kClusterMaxTokens) return false;
+  if ((long long)p->win_t * p->win_h * p->win_w > vsa::kClusterMaxWindow) return false;
+  const long long n = (long long)p->lattice_t * p->lattice_h * p->lattice_w;
+  if (n > (1ll << 30)) return false;
+  g->T = p->lattice_t;
+  g->H = p->lattice_h;
+  g->W = p->lattice_w;
+  g->kt = p->cell_t;
+  g->kh = p->cell_h;
+  g->kw = p->cell_w;
+  g->CT = (g->T + g->kt - 1) / g->kt;
+  g->CH = (g->H + g->kh - 1) / g->kh;
+  g->CW = (g->W + g->kw - 1) / g->kw;
+  g->wt = p->win_t;
+  g->wh = p->win_h;
+  g->ww = p->win_w;
+  const long long cells = (long long)g->CT * g->CH * g->CW;
+  if (cells > (1ll << 30)) return false;
+  g->n_cells = (int)cells;
+  g->n_valid = (int)n;
+  g->n_pad = 0;
+  return true;
+}
+
+// Tokens of the largest reverse-window box (the member-list capacity).
+int cluster_box_tokens(const vsa::ClusterGeom &g) {
+  const long long t = std::min((long long)g.wt * g.kt, (long long)g.T);
+  const long long h = std::min((long long)g.wh * g.kh, (long long)g.H);
+  const long long w = std::min((long long)g.ww * g.kw, (long long)g.W);
+  return (int)(t * h * w);
+}
+
+template <int D>
+vsa_status launch_cluster(const __nv_bfloat16 *x, const vsa::ClusterGeom &g, int iters, int BH, int32_t *assign,
+                          float *mu, int32_t *sizes, int32_t *perm, cudaStream_t st) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  constexpr int kAssignSmem = (int)sizeof(vsa::AssignSmem<D>);
+  constexpr int kListMax = 128 + 4 * vsa::kClusterMaxTokens * vsa::kClusterMaxWindow;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(vsa::cluster_assign_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kAssignSmem);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(vsa::cluster_update_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      kListMax);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(vsa::cluster_perm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kListMax);
+  });
+  if (attr_err != cudaSuccess) return VSA_ERR_CUDA;
+  const int list_smem = 128 + 4 * cluster_box_tokens(g);
+  const dim3 grid(g.n_cells, BH);
+  vsa::cluster_init_kernel<D><<<grid, 128, 0, st>>>(x, g, mu);
+  for (int it = 0; it < iters; ++it) {
+    vsa::cluster_assign_kernel<D><<<grid, vsa::kClusterThreads, kAssignSmem, st>>>(x, g, mu, assign);
+    vsa::cluster_update_kernel<D><<<grid, vsa::kClusterThreads, list_smem, st>>>(x, g, assign, mu, sizes);
+  }
+  vsa::cluster_perm_kernel<<<grid, vsa::kClusterThreads, list_smem, st>>>(g, assign, sizes, perm);
+  return launch_status();
 }
 
 }  // namespace
@@ -527,6 +600,48 @@ vsa_status vsa_lse_merge(const float *o_a, const float *lse_a, const float *o_b,
     vsa::lse_merge_kernel<128><<<blocks, 256, 0, st>>>(o_a, lse_a, o_b, lse_b, rows, o_out, o_out_fp32, lse_out);
   else
     vsa::lse_merge_kernel<64><<<blocks, 256, 0, st>>>(o_a, lse_a, o_b, lse_b, rows, o_out, o_out_fp32, lse_out);
+  return launch_status();
+}
+
+
+int vsa_cluster_count(const vsa_cluster_params *params) {
+  vsa::ClusterGeom g;
+  return cluster_geom(params, &g) ? g.n_cells : 0;
+}
+
+vsa_status vsa_cluster_tokens(const void *x, const vsa_shape *shape, const vsa_cluster_params *params,
+                              int32_t *assign, float *centroids, int32_t *sizes, int32_t *perm, void *stream) {
+  if (!shape_ok(shape) || !x || !assign || !centroids || !sizes || !perm) return VSA_ERR_INVALID_ARG;
+  vsa::ClusterGeom g;
+  if (!cluster_geom(params, &g) || g.n_valid != shape->n_valid) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(centroids)) return VSA_ERR_INVALID_ARG;
+  g.n_pad = shape->n_pad;
+  const int BH = shape->B * shape->H;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+  return shape->d == 128 ? launch_cluster<128>(xb, g, params->iters, BH, assign, centroids, sizes, perm, st)
+                         : launch_cluster<64>(xb, g, params->iters, BH, assign, centroids, sizes, perm, st);
+}
+
+vsa_status vsa_permute_rows(const void *src, const int32_t *perm, int batch_heads, int n_pad, int row_bytes,
+                            int inverse, void *dst, void *stream) {
+  if (!src || !perm || !dst || src == dst) return VSA_ERR_INVALID_ARG;
+  if (batch_heads < 1 || n_pad < 1 || row_bytes < 4 || row_bytes % 4 != 0) return VSA_ERR_INVALID_ARG;
+  const bool wide = row_bytes % 16 == 0;
+  const uintptr_t mask = wide ? 15u : 3u;
+  if ((reinterpret_cast<uintptr_t>(src) & mask) || (reinterpret_cast<uintptr_t>(dst) & mask) ||
+      (reinterpret_cast<uintptr_t>(perm) & 3u))
+    return VSA_ERR_INVALID_ARG;
+  const long long rows = (long long)batch_heads * n_pad;
+  const long long span = rows * row_bytes;
+  const char *s8 = static_cast<const char *>(src);
+  const char *d8 = static_cast<const char *>(dst);
+  if (s8 < d8 + span && d8 < s8 + span) return VSA_ERR_INVALID_ARG;  // overlapping buffers
+  const long long blocks = (rows + 7) / 8;
+  if (blocks > 0x7fffffffll) return VSA_ERR_UNSUPPORTED;
+  vsa::permute_rows_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint32_t *>(src), perm, n_pad, rows, row_bytes / 4, inverse ? 1 : 0,
+      static_cast<uint32_t *>(dst));
   return launch_status();
 }
 

@@ -9,6 +9,7 @@
  *   vsa_select_micro     Micro tiles inside omitted blocks          (Micro selection)
  *   vsa_block_sparse_fwd again on the Micro lists, merged by LSE    (Micro pass + merge)
  *   (vsa_block_sparse_fwd_heads: either pass on a subset of the heads)
+ * and, for the cluster-permuted layout, vsa_cluster_tokens + vsa_permute_rows.
  * plus vsa_mask_to_lists (an explicit block mask instead of selection) and
  * vsa_lse_merge (the stand-alone exact merge).
  *
@@ -302,6 +303,55 @@ VSA_API vsa_status vsa_block_sparse_fwd_heads(const void *q, const void *k, cons
  * ------------------------------------------------------------------------- */
 VSA_API vsa_status vsa_lse_merge(const float *o_a, const float *lse_a, const float *o_b, const float *lse_b,
                          const vsa_shape *shape, void *o_out, int o_out_fp32, float *lse_out, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Cluster-permuted layout ([HVA] §4.1 Eq. (5) 3D local-window clustering;
+ * §2 Eq. (1) the permutation that makes each cluster's tokens contiguous;
+ * Eq. (4) the output put back in token order).
+ *
+ * The n_valid = lattice_t * lattice_h * lattice_w valid tokens of every
+ * (batch, head) form a T x H x W lattice in frame-first order.  The lattice is
+ * cut into cells of (cell_t, cell_h, cell_w) tokens (ceil per axis; an edge
+ * cell holds the rest), one centroid per cell initialised from the cell's
+ * centre token (offset (e-1)/2 along an axis of extent e).  Each of `iters`
+ * rounds assigns every token to the nearest centroid (squared Euclidean,
+ * fp32, ties to the lower cell) among the cells of a (win_t, win_h, win_w)
+ * window around its own cell (offsets -((w-1)/2) .. w/2, clipped), then sets
+ * every centroid to the mean of its tokens (an empty cluster keeps its
+ * centroid).  The permutation lists the tokens cluster by cluster (cells in
+ * flat t-major order), in token order inside a cluster; padding rows
+ * n_valid .. n_pad-1 stay in place.  Everything is deterministic.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int lattice_t, lattice_h, lattice_w; /* lattice_t*lattice_h*lattice_w == n_valid */
+  int cell_t, cell_h, cell_w;          /* >= 1; cell_t*cell_h*cell_w <= 128 */
+  int win_t, win_h, win_w;             /* >= 1; win_t*win_h*win_w <= 128 */
+  int iters;                           /* 1 .. 64 */
+} vsa_cluster_params;
+
+/* Number of cells (clusters) of the parameters, 0 if they are invalid.  Host only. */
+VSA_API int vsa_cluster_count(const vsa_cluster_params *params);
+
+/* x: bf16 [B, H, n_pad, d] (Q or K).  Outputs, caller-allocated DEVICE memory:
+ *   assign    int32 [B, H, n_valid]   cluster (flat cell index) of each token
+ *   centroids fp32  [B, H, n_cells, d]
+ *   sizes     int32 [B, H, n_cells]   tokens per cluster
+ *   perm      int32 [B, H, n_pad]     row i of the permuted sequence is token perm[i]
+ * Invalid parameters or a lattice that does not match n_valid return
+ * VSA_ERR_INVALID_ARG; d must be 64 or 128. */
+VSA_API vsa_status vsa_cluster_tokens(const void *x, const vsa_shape *shape, const vsa_cluster_params *params,
+                                      int32_t *assign, float *centroids, int32_t *sizes, int32_t *perm,
+                                      void *stream);
+
+/* Row permutation along the token axis of [B*H, n_pad, row] data (rows of
+ * row_bytes, a multiple of 4, 16-byte aligned when a multiple of 16):
+ *   inverse = 0: dst[bh][i] = src[bh][perm[bh][i]]   (Eq. (1): X' = Pi X)
+ *   inverse = 1: dst[bh][perm[bh][i]] = src[bh][i]   (Eq. (4): O = Pi^-1 O')
+ * perm is int32 [B*H, n_pad], each row a permutation of 0 .. n_pad-1; an entry
+ * out of range latches VSA_ERR_BAD_INDEX and that row is not copied.
+ * src and dst must not overlap. */
+VSA_API vsa_status vsa_permute_rows(const void *src, const int32_t *perm, int batch_heads, int n_pad, int row_bytes,
+                                    int inverse, void *dst, void *stream);
 
 #ifdef __cplusplus
 }
