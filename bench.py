@@ -456,6 +456,97 @@ def run_sweep(args):
         del run
 
 
+def run_cluster(args):
+    """The cluster-permuted layout on the chosen workload (HyperVAttention
+    Eq. (1), (4), (5)): 3D local-window clustering of Q and K, row
+    permutation, the path on the permuted rows, and the output put back in
+    token order.  One JSON line with the per-stage times (CUDA events), the
+    step's effective TFLOP/s over kept tiles, and the relative L2 error of
+    the final output against dense attention (the same kernel with every
+    block kept) for the token-order and the cluster-permuted layouts."""
+    import dataclasses
+    import block_sparse_attention_pool_b200 as vsa
+    from block_sparse_attention_pool_b200 import build as vsa_build
+    vsa_build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    q, k, v = make_qkv(w)
+    to_dev = lambda x: torch.from_numpy(x).to(dev).to(torch.bfloat16).contiguous()
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    del q, k, v
+    stream = torch.cuda.current_stream(dev)
+    heads = micro_heads(w) if w.micro_mode else None
+    cfg = vsa.PathConfig.from_workload(w, heads)
+    cfg.cluster_lattice = w.grid
+    cfg.cluster_cell, cfg.cluster_window, cfg.cluster_iters = args.cluster_cell, args.cluster_window, args.cluster_iters
+    run = vsa.SparseVideoAttention(cfg)
+    B, H, n_pad, d = dq.shape
+    shape = vsa.Shape(B, H, w.n_valid, n_pad, d)
+    params = cfg.cluster_params()
+
+    def step(ev):
+        b = run.buf
+        ev[0].record(stream)
+        for name, x in (("q", dq), ("k", dk)):
+            vsa.cluster_tokens(x, shape, params, b["assign_" + name], b["centroids_" + name], b["sizes_" + name],
+                               b["perm_" + name], stream)
+        ev[1].record(stream)
+        vsa.permute_rows(dq, b["perm_q"], b["qp"], stream=stream)
+        vsa.permute_rows(dk, b["perm_k"], b["kp"], stream=stream)
+        vsa.permute_rows(dv, b["perm_k"], b["vp"], stream=stream)
+        ev[2].record(stream)
+        run._run(b["qp"], b["kp"], b["vp"], stream, b["op"], b["lp"])
+        ev[3].record(stream)
+        vsa.permute_rows(b["op"], b["perm_q"], b["o"], inverse=True, stream=stream)
+        vsa.permute_rows(b["lp"], b["perm_q"], b["lse"], inverse=True, stream=stream)
+        ev[4].record(stream)
+
+    run(dq, dk, dv)  # buffers
+    evs = []
+    for i in range(args.warmup + args.steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        step(ev)
+        if i >= args.warmup:
+            evs.append(ev)
+    torch.cuda.synchronize(dev)
+    st = vsa.read_device_status(stream)
+    if st != 0:
+        raise RuntimeError(vsa.status_string(st))
+    names = ["cluster_qk", "permute_in", "path", "permute_out"]
+    stages = {n: round(statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs), 4) for i, n in enumerate(names)}
+    ms = statistics.mean(e[0].elapsed_time(e[4]) for e in evs)
+    flops = macro_flops(run.buf["counts"], w) + (micro_flops(run.buf["m_counts"], w) if w.micro_mode else 0.0)
+    o_clu = run.buf["o"].float().clone()
+    # the same path in token order, and dense attention of the same kernel
+    plain = vsa.SparseVideoAttention(vsa.PathConfig.from_workload(w, heads))
+    o_tok = plain(dq, dk, dv)["o"].float().clone()
+    del plain
+    dense = vsa.SparseVideoAttention(vsa.PathConfig(n_valid=w.n_valid, bq=w.bq, bk=w.bk, scale=w.scale,
+                                                    fixed_k=n_pad // w.bk))
+    o_ref = dense(dq, dk, dv)["o"].float()
+    nv = w.n_valid
+    rel = lambda o: float(torch.linalg.vector_norm(o[:, :, :nv] - o_ref[:, :, :nv]) /
+                          torch.linalg.vector_norm(o_ref[:, :, :nv]))
+    sizes = run.buf["sizes_q"].float()
+    line = {
+        "metric": METRIC + " (cluster-permuted layout)",
+        "value": round(flops / (ms * 1e-3) / 1e12, 3),
+        "unit": "TFLOP/s",
+        "ms_per_step": round(ms, 4),
+        "stages_ms": stages,
+        "config": {"workload": workload_label(w), "lattice": list(w.grid), "cell": list(args.cluster_cell),
+                   "window": list(args.cluster_window), "iters": args.cluster_iters,
+                   "clusters_per_head": int(sizes.shape[-1]),
+                   "cluster_size_mean_max": [round(float(sizes.mean()), 1), int(sizes.max())],
+                   "kept_fraction_macro": round(float(run.buf["counts"].sum().item()) /
+                                                (w.B * w.H * ((w.n_valid + w.bq - 1) // w.bq) * (n_pad // w.bk)), 4)},
+        "rel_l2_error_vs_dense": {"token_order": round(rel(o_tok), 5), "cluster_permuted": round(rel(o_clu), 5)},
+        "data": "synthetic (seeded video-shaped Q/K/V, no model weights)",
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -467,6 +558,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--chunk-heads", type=int, default=4, help="heads per pipelined chunk of the e2e leg")
     ap.add_argument("--sweep", action="store_true", help="print the sparsity-sweep lines instead of the bench line")
+    ap.add_argument("--cluster", action="store_true",
+                    help="print the cluster-permuted-layout line (3D local-window clustering) instead of the bench line")
+    ap.add_argument("--cluster-cell", type=int, nargs=3, default=(3, 5, 8))
+    ap.add_argument("--cluster-window", type=int, nargs=3, default=(3, 5, 5))
+    ap.add_argument("--cluster-iters", type=int, default=3)
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -474,6 +570,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.sweep:
         run_sweep(args)
+        return
+    if args.cluster:
+        run_cluster(args)
         return
     if args.impl == "reference":
         line = run_reference(args, rank, world)

@@ -12,7 +12,7 @@
 // Kernels (one (batch, head) per blockIdx.y):
 //   cluster_init_kernel    centroid u = the centre token of cell u
 //   cluster_assign_kernel  one CTA per cell: the cell's tokens (<= 128) x the
-//                          window's centroids (<= 128, in chunks of 32) as an
+//                          window's centroids (<= 128, staged once) as an
 //                          fp32 register-tiled GEMM on shared memory;
 //                          distance = |mu|^2 - 2 x.mu (|x|^2 is common to all
 //                          candidates of a token); argmin with ties to the
@@ -40,7 +40,6 @@ namespace vsa {
 constexpr int kClusterThreads = 256;
 constexpr int kClusterMaxTokens = 128;  // tokens per cell
 constexpr int kClusterMaxWindow = 128;  // cells per window
-constexpr int kClusterChunk = 32;       // window centroids per shared-memory chunk
 
 struct ClusterGeom {
   int T, H, W;        // token lattice
@@ -89,124 +88,148 @@ __global__ void cluster_init_kernel(const __nv_bfloat16 *__restrict__ x, Cluster
   for (int k = threadIdx.x; k < D; k += blockDim.x) dst[k] = __bfloat162float(x[row * D + k]);
 }
 
+// Shared memory of the assignment kernel: the cell's tokens and the window's
+// centroids as fp32 rows (row stride D + 4 floats, 16-byte aligned) and the
+// window's cell indices.  The centroid block is sized
+// by the window (n_win rows, rounded up to 16).
 template <int D>
-struct AssignSmem {
+struct AssignLayout {
   static constexpr int kLd = D + 4;
-  float X[kClusterMaxTokens][kLd];
-  float C[kClusterChunk][kLd];
-  float cnorm[kClusterChunk];
-  int win[kClusterMaxWindow];
-  int n_win;
+  static constexpr int kOffX = 0;
+  static constexpr int kOffC = kOffX + kClusterMaxTokens * kLd * 4;
+  static __host__ __device__ int off_win(int win_rows) { return kOffC + win_rows * kLd * 4; }
+  static __host__ __device__ int bytes(int win_rows) { return off_win(win_rows) + kClusterMaxWindow * 4 + 16; }
 };
 
-template <int D>
+// One CTA per cell.  Thread (ty, tx) scores tokens ty + 16 a (a < 8) against
+// centroids tx + 16 b (b < NB): each 4-wide step of d loads 8 + NB float4 and
+// issues 32 NB FMAs.  NB = ceil(window cells / 16) is a template parameter.
+template <int D, int NB>
 __global__ void __launch_bounds__(kClusterThreads) cluster_assign_kernel(const __nv_bfloat16 *__restrict__ x,
                                                                          ClusterGeom g, const float *__restrict__ mu,
                                                                          int32_t *__restrict__ assign) {
+  using L = AssignLayout<D>;
+  constexpr int kLd = L::kLd;
+  constexpr int kRows = 16 * NB;
   extern __shared__ __align__(16) uint8_t cluster_smem_raw[];
-  AssignSmem<D> &sm = *reinterpret_cast<AssignSmem<D> *>(cluster_smem_raw);
+  float(*sX)[kLd] = reinterpret_cast<float(*)[kLd]>(cluster_smem_raw + L::kOffX);
+  float(*sC)[kLd] = reinterpret_cast<float(*)[kLd]>(cluster_smem_raw + L::kOffC);
+  int *win = reinterpret_cast<int *>(cluster_smem_raw + L::off_win(kRows));
+  __shared__ int s_tok[kClusterMaxTokens];  // lattice index of the cell's i-th token
+  __shared__ int s_wcnt[kClusterMaxWindow / 32];
   const int u0 = blockIdx.x, bh = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int cw = u0 % g.CW, ch = (u0 / g.CW) % g.CH, ct = u0 / (g.CW * g.CH);
   const TokBox box = cell_box(ct, ct + 1, ch, ch + 1, cw, cw + 1, g);
   const int n_tok = box.size();
 
-  // window cells, ascending flat index (t-major loops)
-  if (tid == 0) {
-    int n = 0;
-    for (int dt = win_lo(g.wt); dt <= win_hi(g.wt); ++dt)
-      for (int dh = win_lo(g.wh); dh <= win_hi(g.wh); ++dh)
-        for (int dw = win_lo(g.ww); dw <= win_hi(g.ww); ++dw) {
-          const int t = ct + dt, h = ch + dh, w = cw + dw;
-          if (t >= 0 && t < g.CT && h >= 0 && h < g.CH && w >= 0 && w < g.CW && n < kClusterMaxWindow)
-            sm.win[n++] = (t * g.CH + h) * g.CW + w;
-        }
-    sm.n_win = n;
-  }
-  // the cell's tokens as fp32 rows (zero rows past n_tok)
-  const __nv_bfloat16 *xb = x + (size_t)bh * g.n_pad * D;
-  for (int e = tid; e < kClusterMaxTokens * (D / 2); e += kClusterThreads) {
-    const int i = e / (D / 2), k2 = e % (D / 2);
-    float2 v = make_float2(0.f, 0.f);
-    if (i < n_tok) {
-      const __nv_bfloat162 p = reinterpret_cast<const __nv_bfloat162 *>(xb + (size_t)box.token(i, g) * D)[k2];
-      v = __bfloat1622float2(p);
+  // token table; window cells in (t, h, w) loop order = ascending flat index,
+  // compacted by ballot over the first four warps
+  int wcell = -1;
+  if (tid < kClusterMaxTokens) s_tok[tid] = tid < n_tok ? box.token(tid, g) : -1;
+  if (tid < kClusterMaxWindow) {
+    if (tid < g.wt * g.wh * g.ww) {
+      const int dw = tid % g.ww, dh = (tid / g.ww) % g.wh, dt = tid / (g.ww * g.wh);
+      const int t = ct + win_lo(g.wt) + dt, h = ch + win_lo(g.wh) + dh, w = cw + win_lo(g.ww) + dw;
+      if (t >= 0 && t < g.CT && h >= 0 && h < g.CH && w >= 0 && w < g.CW) wcell = (t * g.CH + h) * g.CW + w;
     }
-    sm.X[i][2 * k2] = v.x;
-    sm.X[i][2 * k2 + 1] = v.y;
+    const uint32_t bal = __ballot_sync(0xffffffffu, wcell >= 0);
+    if (lane == 0) s_wcnt[warp] = __popc(bal);
+    __syncwarp();
+    wcell = wcell >= 0 ? (wcell | (__popc(bal & ((1u << lane) - 1u)) << 24)) : -1;  // rank inside the warp
   }
   __syncthreads();
-  const int n_win = sm.n_win;
-  const float *mub = mu + (size_t)bh * g.n_cells * D;
+  int n_win = 0;
+#pragma unroll
+  for (int w = 0; w < kClusterMaxWindow / 32; ++w) n_win += s_wcnt[w];
+  if (tid < kClusterMaxWindow && wcell >= 0) {
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += s_wcnt[w];
+    const int pos = before + (wcell >> 24);
+    if (pos < kRows) win[pos] = wcell & 0xffffff;
+  }
+  n_win = min(n_win, kRows);
+  __syncthreads();
 
+  // the cell's tokens (zero rows past n_tok) and the window's centroids (zero
+  // rows past n_win), fp32
+  const __nv_bfloat16 *xb = x + (size_t)bh * g.n_pad * D;
+  for (int e = tid; e < kClusterMaxTokens * (D / 8); e += kClusterThreads) {
+    const int i = e / (D / 8), k8 = e % (D / 8);
+    const int tok = s_tok[i];
+    float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
+    if (tok >= 0) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(xb + (size_t)tok * D) + k8);
+      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+      const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+      const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.z));
+      const float2 d = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.w));
+      lo = make_float4(a.x, a.y, b.x, b.y);
+      hi = make_float4(c.x, c.y, d.x, d.y);
+    }
+    *reinterpret_cast<float4 *>(&sX[i][8 * k8]) = lo;
+    *reinterpret_cast<float4 *>(&sX[i][8 * k8 + 4]) = hi;
+  }
+  const float *mub = mu + (size_t)bh * g.n_cells * D;
+  for (int e = tid; e < kRows * (D / 4); e += kClusterThreads) {
+    const int j = e / (D / 4), k4 = e % (D / 4);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (j < n_win) v = __ldg(reinterpret_cast<const float4 *>(mub + (size_t)win[j] * D) + k4);
+    *reinterpret_cast<float4 *>(&sC[j][4 * k4]) = v;
+  }
+  __syncthreads();
+
+  // dot products and, alongside, |mu|^2 of this thread's centroids (every
+  // thread that holds a centroid sums it in the same order)
   const int ty = tid >> 4, tx = tid & 15;
-  float best_d[8];
-  int best_c[8];
+  float acc[8][NB], cn[NB];
 #pragma unroll
-  for (int a = 0; a < 8; ++a) {
-    best_d[a] = INFINITY;
-    best_c[a] = 0x7fffffff;
+  for (int b = 0; b < NB; ++b) {
+    cn[b] = 0.f;
+#pragma unroll
+    for (int a = 0; a < 8; ++a) acc[a][b] = 0.f;
   }
-  for (int c0 = 0; c0 < n_win; c0 += kClusterChunk) {
-    __syncthreads();  // the previous chunk's centroids are consumed
-    for (int e = tid; e < kClusterChunk * (D / 4); e += kClusterThreads) {
-      const int j = e / (D / 4), k4 = e % (D / 4);
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c0 + j < n_win) v = reinterpret_cast<const float4 *>(mub + (size_t)sm.win[c0 + j] * D)[k4];
-      *reinterpret_cast<float4 *>(&sm.C[j][4 * k4]) = v;
+#pragma unroll 2
+  for (int k = 0; k < D; k += 4) {
+    float4 cv[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      cv[b] = *reinterpret_cast<const float4 *>(&sC[tx + 16 * b][k]);
+      cn[b] = fmaf(cv[b].x, cv[b].x, cn[b]);
+      cn[b] = fmaf(cv[b].y, cv[b].y, cn[b]);
+      cn[b] = fmaf(cv[b].z, cv[b].z, cn[b]);
+      cn[b] = fmaf(cv[b].w, cv[b].w, cn[b]);
     }
-    __syncthreads();
-    // |mu|^2 of the chunk: warp w reduces rows 4w .. 4w+3 in a fixed order
-    for (int j = warp * 4; j < warp * 4 + 4; ++j) {
-      float s = 0.f;
-      for (int k = lane; k < D; k += 32) s = fmaf(sm.C[j][k], sm.C[j][k], s);
-      s = warp_sum(s);
-      if (lane == 0) sm.cnorm[j] = s;
-    }
-    float acc[8][2];
 #pragma unroll
-    for (int a = 0; a < 8; ++a) acc[a][0] = acc[a][1] = 0.f;
-#pragma unroll 4
-    for (int k = 0; k < D; k += 4) {
-      const float4 b0 = *reinterpret_cast<const float4 *>(&sm.C[tx][k]);
-      const float4 b1 = *reinterpret_cast<const float4 *>(&sm.C[tx + 16][k]);
+    for (int a = 0; a < 8; ++a) {
+      const float4 xv = *reinterpret_cast<const float4 *>(&sX[ty + 16 * a][k]);
 #pragma unroll
-      for (int a = 0; a < 8; ++a) {
-        const float4 xv = *reinterpret_cast<const float4 *>(&sm.X[ty + 16 * a][k]);
-        acc[a][0] = fmaf(xv.x, b0.x, acc[a][0]);
-        acc[a][0] = fmaf(xv.y, b0.y, acc[a][0]);
-        acc[a][0] = fmaf(xv.z, b0.z, acc[a][0]);
-        acc[a][0] = fmaf(xv.w, b0.w, acc[a][0]);
-        acc[a][1] = fmaf(xv.x, b1.x, acc[a][1]);
-        acc[a][1] = fmaf(xv.y, b1.y, acc[a][1]);
-        acc[a][1] = fmaf(xv.z, b1.z, acc[a][1]);
-        acc[a][1] = fmaf(xv.w, b1.w, acc[a][1]);
-      }
-    }
-    __syncthreads();  // cnorm written by other warps
-#pragma unroll
-    for (int bb = 0; bb < 2; ++bb) {
-      const int j = tx + 16 * bb;
-      if (c0 + j < n_win) {
-        const int cell = sm.win[c0 + j];
-        const float cn = sm.cnorm[j];
-#pragma unroll
-        for (int a = 0; a < 8; ++a) {
-          const float dist = fmaf(-2.f, acc[a][bb], cn);
-          if (dist < best_d[a] || (dist == best_d[a] && cell < best_c[a])) {
-            best_d[a] = dist;
-            best_c[a] = cell;
-          }
-        }
+      for (int b = 0; b < NB; ++b) {
+        acc[a][b] = fmaf(xv.x, cv[b].x, acc[a][b]);
+        acc[a][b] = fmaf(xv.y, cv[b].y, acc[a][b]);
+        acc[a][b] = fmaf(xv.z, cv[b].z, acc[a][b]);
+        acc[a][b] = fmaf(xv.w, cv[b].w, acc[a][b]);
       }
     }
   }
-  // argmin across the 16 threads (tx) that share a token
   int32_t *ab = assign + (size_t)bh * g.n_valid;
 #pragma unroll
   for (int a = 0; a < 8; ++a) {
-    float d = best_d[a];
-    int c = best_c[a];
+    float d = INFINITY;
+    int c = 0x7fffffff;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const int j = tx + 16 * b;
+      if (j < n_win) {
+        const float dist = fmaf(-2.f, acc[a][b], cn[b]);
+        const int cell = win[j];
+        if (dist < d || (dist == d && cell < c)) {
+          d = dist;
+          c = cell;
+        }
+      }
+    }
+    // argmin across the 16 threads (tx) that share a token
 #pragma unroll
     for (int o = 1; o < 16; o <<= 1) {
       const float od = __shfl_xor_sync(0xffffffffu, d, o);
@@ -217,7 +240,7 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_assign_kernel(const _
       }
     }
     const int i = ty + 16 * a;
-    if (tx == 0 && i < n_tok) ab[box.token(i, g)] = c;
+    if (tx == 0 && i < n_tok) ab[s_tok[i]] = c;
   }
 }
 

@@ -245,7 +245,7 @@ bool cluster_geom(const vsa_cluster_params *p, vsa::ClusterGeom *g) {
   g->wh = p->win_h;
   g->ww = p->win_w;
   const long long cells = (long long)g->CT * g->CH * g->CW;
-  if (cells > (1ll << 30)) return false;
+  if (cells > (1ll << 24)) return false;  // cell indices travel in 24 bits inside the assignment kernel
   g->n_cells = (int)cells;
   g->n_valid = (int)n;
   g->n_pad = 0;
@@ -260,19 +260,43 @@ int cluster_box_tokens(const vsa::ClusterGeom &g) {
   return (int)(t * h * w);
 }
 
+// The assignment kernel for windows of up to 16 * NB cells; its shared
+// memory is set once per instantiation.
+template <int D, int NB>
+vsa_status launch_assign(const __nv_bfloat16 *x, const vsa::ClusterGeom &g, dim3 grid, const float *mu,
+                         int32_t *assign, cudaStream_t st) {
+  static const int bytes = vsa::AssignLayout<D>::bytes(16 * NB);
+  static const cudaError_t attr =
+      cudaFuncSetAttribute(vsa::cluster_assign_kernel<D, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (attr != cudaSuccess) return VSA_ERR_CUDA;
+  vsa::cluster_assign_kernel<D, NB><<<grid, vsa::kClusterThreads, bytes, st>>>(x, g, mu, assign);
+  return VSA_OK;
+}
+
+template <int D>
+vsa_status launch_assign_any(const __nv_bfloat16 *x, const vsa::ClusterGeom &g, dim3 grid, const float *mu,
+                             int32_t *assign, cudaStream_t st) {
+  switch ((g.wt * g.wh * g.ww + 15) / 16) {
+    case 1: return launch_assign<D, 1>(x, g, grid, mu, assign, st);
+    case 2: return launch_assign<D, 2>(x, g, grid, mu, assign, st);
+    case 3: return launch_assign<D, 3>(x, g, grid, mu, assign, st);
+    case 4: return launch_assign<D, 4>(x, g, grid, mu, assign, st);
+    case 5: return launch_assign<D, 5>(x, g, grid, mu, assign, st);
+    case 6: return launch_assign<D, 6>(x, g, grid, mu, assign, st);
+    case 7: return launch_assign<D, 7>(x, g, grid, mu, assign, st);
+    default: return launch_assign<D, 8>(x, g, grid, mu, assign, st);
+  }
+}
+
 template <int D>
 vsa_status launch_cluster(const __nv_bfloat16 *x, const vsa::ClusterGeom &g, int iters, int BH, int32_t *assign,
                           float *mu, int32_t *sizes, int32_t *perm, cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
-  constexpr int kAssignSmem = (int)sizeof(vsa::AssignSmem<D>);
   constexpr int kListMax = 128 + 4 * vsa::kClusterMaxTokens * vsa::kClusterMaxWindow;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(vsa::cluster_assign_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    kAssignSmem);
-    if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(vsa::cluster_update_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      kListMax);
+    attr_err = cudaFuncSetAttribute(vsa::cluster_update_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kListMax);
     if (attr_err == cudaSuccess)
       attr_err = cudaFuncSetAttribute(vsa::cluster_perm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kListMax);
   });
@@ -281,7 +305,8 @@ vsa_status launch_cluster(const __nv_bfloat16 *x, const vsa::ClusterGeom &g, int
   const dim3 grid(g.n_cells, BH);
   vsa::cluster_init_kernel<D><<<grid, 128, 0, st>>>(x, g, mu);
   for (int it = 0; it < iters; ++it) {
-    vsa::cluster_assign_kernel<D><<<grid, vsa::kClusterThreads, kAssignSmem, st>>>(x, g, mu, assign);
+    const vsa_status as = launch_assign_any<D>(x, g, grid, mu, assign, st);
+    if (as != VSA_OK) return as;
     vsa::cluster_update_kernel<D><<<grid, vsa::kClusterThreads, list_smem, st>>>(x, g, assign, mu, sizes);
   }
   vsa::cluster_perm_kernel<<<grid, vsa::kClusterThreads, list_smem, st>>>(g, assign, sizes, perm);
