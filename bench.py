@@ -556,7 +556,7 @@ def main():
     ap.add_argument("--workload", default="hunyuan", choices=sorted(WORKLOADS))
     ap.add_argument("--ref-blocks", type=int, default=6, help="query blocks per oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--chunk-heads", type=int, default=4, help="heads per pipelined chunk of the e2e leg")
+    ap.add_argument("--chunk-heads", type=int, default=2, help="heads per pipelined chunk of the e2e leg")
     ap.add_argument("--sweep", action="store_true", help="print the sparsity-sweep lines instead of the bench line")
     ap.add_argument("--cluster", action="store_true",
                     help="print the cluster-permuted-layout line (3D local-window clustering) instead of the bench line")

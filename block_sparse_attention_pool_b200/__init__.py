@@ -479,7 +479,7 @@ class SparseVideoAttention:
         return b
 
     def forward_host(self, q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor, o_h: torch.Tensor,
-                     lse_h: torch.Tensor, chunk_heads: int = 4, device=None) -> None:
+                     lse_h: torch.Tensor, chunk_heads: int = 2, device=None) -> None:
         """The whole path on HOST tensors: pinned bf16 q_h, k_h, v_h [B, H, n_pad, d]
         in, pinned o_h (bf16, same shape) and lse_h (fp32 [B, H, n_pad]) out.
 
