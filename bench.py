@@ -43,6 +43,30 @@ from video_inputs import WORKLOADS, make_qkv, micro_heads, sweep_points  # noqa:
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "block-sparse attn ms & effective TFLOP/s (% bf16 peak), speedup vs dense, 1xB200"
 
+# DRAM bytes (read + write) of the Macro pass per hunyuan step, from the
+# one-pass ncu capture summarised in profiles/attn_fwd_dual_hunyuan_traffic.md,
+# valid only while the kernel sources hash to the value it was taken with.
+MACRO_TRAFFIC = {
+    "sources": ["csrc/attn_fwd_dual.cuh", "csrc/attn_fwd.cuh", "csrc/common.cuh"],
+    "sha256_16": "12d517136229b172",
+    "workload": "hunyuan",
+    "bytes_per_step": 3319685376 + 890615040,
+}
+
+
+def macro_traffic(workload: str):
+    """The captured Macro-pass DRAM bytes per step, or None when the workload
+    differs or the kernel sources changed since the capture."""
+    import hashlib
+    if workload != MACRO_TRAFFIC["workload"]:
+        return None
+    h = hashlib.sha256()
+    pkg = os.path.join(os.path.dirname(os.path.abspath(__file__)), "block_sparse_attention_pool_b200")
+    for rel in MACRO_TRAFFIC["sources"]:
+        with open(os.path.join(pkg, rel), "rb") as f:
+            h.update(f.read())
+    return MACRO_TRAFFIC["bytes_per_step"] if h.hexdigest()[:16] == MACRO_TRAFFIC["sha256_16"] else None
+
 
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -331,7 +355,7 @@ def run_gpu(args, rank, world, local_rank):
             "peak": peak,
             "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
-            "traffic": None,
+            "traffic": macro_traffic(args.workload),
         },
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 3),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -348,6 +348,33 @@ def test_lse_merge_kernel():
 # whole path
 # ---------------------------------------------------------------------------
 
+@pytest.mark.parametrize("micro_mode", [1, 2])
+def test_path_two_batches_every_row(micro_mode):
+    """B = 2 through the whole path: batch-major (batch, head) indexing in
+    every kernel, Micro head flags repeated per batch element, the per-head
+    percentile taken per (batch, head) slot, and the Micro pass and its fp32
+    Macro output restricted to the flagged heads of both batch elements."""
+    import dataclasses
+    w = dataclasses.replace(WORKLOADS["tiny"], B=2, micro_mode=micro_mode, micro_percentile=0.9, fixed_k=2)
+    q, k, v = make_qkv(w)
+    assert q.shape[0] == 2 and not np.array_equal(q[0], q[1])
+    heads = np.array([1, 0], dtype=np.uint8) if micro_mode == 2 else micro_heads(w)
+    res = orc.forward(q, k, v, w, head_enable=heads)
+    run = vsa.SparseVideoAttention(vsa.PathConfig.from_workload(w, heads))
+    out = run(to_dev(q), to_dev(k), to_dev(v))
+    assert vsa.read_device_status() == 0
+    counts, idx = out["counts"].cpu().numpy(), out["idx"].cpu().numpy()
+    mc, mi = out["m_counts"].cpu().numpy(), out["m_idx"].cpu().numpy()
+    for b in range(2):
+        for h in range(w.H):
+            for i in range(w.n_q):
+                assert np.array_equal(idx[b, h, i, :counts[b, h, i]], res["kept"][b][h][i]), (b, h, i)
+            for r in range(w.n_pad // 64):
+                assert np.array_equal(mi[b, h, r, :mc[b, h, r]], res["tiles"][b][h][r]), (b, h, r)
+    assert_close_rows(out["o"].float().cpu().numpy(), out["lse"].cpu().numpy(), res["O"], res["LSE"],
+                      [(b, h, 0, w.n_pad) for b in range(2) for h in range(w.H)], bf16_out=True)
+
+
 def test_path_tiny_every_row():
     w = WORKLOADS["tiny"]
     q, k, v = inputs("tiny")
