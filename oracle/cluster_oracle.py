@@ -44,14 +44,15 @@ Readings taken where the page is silent (listed in the design notes too):
 """
 from __future__ import annotations
 
-from typing import Dict, Sequence, Tuple
+from typing import Dict, List, Sequence, Tuple
 
 import numpy as np
 
 __all__ = [
     "cell_counts", "token_cells", "initial_centroids", "window_offsets", "window_cells",
     "local_window_clustering", "clustering_objective", "cluster_permutation", "permute_rows",
-    "unpermute_rows", "forward_clustered",
+    "unpermute_rows", "forward_clustered", "select_clusters", "tile_cost", "merge_clusters", "total_cost",
+    "forward_cluster_blocks",
 ]
 
 
@@ -196,3 +197,135 @@ def forward_clustered(q, k, v, w, cell, window, n_iter, head_enable=None) -> Dic
             L[b, h] = unpermute_rows(res["LSE"][b, h], perms["q"][b, h])
     return {"perm_q": perms["q"], "perm_k": perms["k"], "assign_q": assign["q"], "assign_k": assign["k"],
             "permuted": res, "O": O, "LSE": L}
+
+
+# ---------------------------------------------------------------------------
+# Cluster-aligned blocks (HVA §2 Eq. (2)-(4) on clusters, §4.3 Eq. (7)-(10),
+# Algorithm 1 "Parallel Agglomerative Merging")
+#
+# Further readings (C9-C14):
+#  C9  cluster-level selection is the path's selection on centroids: logits
+#      S_ij = <mu_i^q, mu_j^k> / sqrt(d), weights s_j^k = key-cluster sizes,
+#      the same Top-p / Min-kc / fixed-k rule and ties (R3, R4); a query
+#      cluster with no token keeps nothing; anchors are not used;
+#  C10 the random bipartition of round r is given as one bit per query
+#      cluster (an input array); a group takes the bit of its lowest member;
+#  C11 pi(A) = argmin over B of dC(A, B), ties to the group with the lower
+#      lowest member; among the A that chose the same B the smallest dC wins,
+#      ties to the lower lowest member; only dC < 0 is applied (Alg. 1 l.14);
+#  C12 a group's query tokens are its clusters' tokens, clusters in ascending
+#      index, each in its permutation order, padded to a multiple of tau_q;
+#      groups follow each other in ascending lowest member;
+#  C13 a key cluster occupies ceil(s_j / seg) segments of seg keys, clusters in
+#      ascending index; the last segment of a cluster holds s_j mod seg keys
+#      (the rest is padding, never attended);
+#  C14 every query token of group S attends to the keys of the union of the
+#      key clusters selected by S's members (chi(S) of Eq. (8)).
+# ---------------------------------------------------------------------------
+
+def select_clusters(mu_q, mu_k, sizes_q, sizes_k, scale, k_min, cum_mass, fixed_k):
+    """C9: kept key clusters per query cluster (ascending arrays)."""
+    from .vsa_oracle import size_weighted_probs, select_row
+    S = (np.asarray(mu_q, dtype=np.float64) @ np.asarray(mu_k, dtype=np.float64).T) * scale
+    P, w = size_weighted_probs(S, np.asarray(sizes_k, dtype=np.float64))
+    kept = []
+    for i in range(S.shape[0]):
+        if sizes_q[i] <= 0:
+            kept.append(np.zeros(0, dtype=np.int64))
+        else:
+            kept.append(select_row(w[i], P[i], k_min, cum_mass, fixed_k)[0])
+    return kept
+
+
+def tile_cost(sq: int, wk: int, tau_q: int, tau_k: int) -> int:
+    """Eq. (7) / (8): CTA-aligned query rows times CTA-aligned packed keys."""
+    return (tau_q * (-(-sq // tau_q))) * (tau_k * (-(-wk // tau_k)))
+
+
+def merge_clusters(sizes_q, sizes_k, kept, tau_q: int, tau_k: int, sides) -> List[List[int]]:
+    """Algorithm 1 (Eq. (9), (10)) with the bipartitions ``sides`` [R, N_q]
+    (readings C10, C11).  Returns the groups (ascending member lists),
+    ordered by their lowest member."""
+    nq = len(sizes_q)
+    sk = np.asarray(sizes_k, dtype=np.int64)
+    groups = {i: [i] for i in range(nq)}              # keyed by lowest member
+    chi = {i: set(int(j) for j in kept[i]) for i in range(nq)}
+    sq = {i: int(sizes_q[i]) for i in range(nq)}
+    wk = lambda keys: int(sum(sk[j] for j in keys))
+    cost = lambda g: tile_cost(sq[g], wk(chi[g]), tau_q, tau_k)
+    for r in range(len(sides)):
+        leaders = sorted(groups)
+        A = [g for g in leaders if sides[r][g] == 0]
+        B = [g for g in leaders if sides[r][g] != 0]
+        if not A or not B:
+            continue
+        choice = {}
+        for a in A:
+            best = None
+            for b in B:
+                merged = tile_cost(sq[a] + sq[b], wk(chi[a] | chi[b]), tau_q, tau_k)
+                d = merged - cost(a) - cost(b)
+                if best is None or d < best[0]:
+                    best = (d, b)
+            choice[a] = best
+        accepted = {}
+        for a in A:
+            d, b = choice[a]
+            if d < 0 and (b not in accepted or d < accepted[b][0]):
+                accepted[b] = (d, a)
+        for b, (d, a) in accepted.items():
+            lead = min(a, b)
+            other = b if lead == a else a
+            groups[lead] = sorted(groups[a] + groups[b])
+            chi[lead] = chi[a] | chi[b]
+            sq[lead] = sq[a] + sq[b]
+            del groups[other], chi[other], sq[other]
+    return [groups[g] for g in sorted(groups)]
+
+
+def total_cost(groups, sizes_q, sizes_k, kept, tau_q, tau_k) -> int:
+    sk = np.asarray(sizes_k, dtype=np.int64)
+    tot = 0
+    for g in groups:
+        keys = set()
+        for i in g:
+            keys |= set(int(j) for j in kept[i])
+        tot += tile_cost(int(sum(sizes_q[i] for i in g)), int(sum(sk[j] for j in keys)), tau_q, tau_k)
+    return tot
+
+
+def forward_cluster_blocks(q, k, v, n_valid, grid, cell, window, n_iter, scale, k_min, cum_mass, fixed_k,
+                           tau_q=128, tau_k=128, sides=None) -> Dict[str, object]:
+    """The cluster-aligned pipeline, per (batch, head): cluster Q and K
+    (Eq. (5)), select key clusters per query cluster on centroids (C9),
+    merge query clusters (Algorithm 1, when ``sides`` is given), and attend
+    each query token to the keys of its group's selected clusters (C14).
+    Returns O [B, H, N_pad, d], LSE [B, H, N_pad] in token order plus the
+    per-head clusters, selections and groups."""
+    from .vsa_oracle import attention_rows, NEG_INF
+    B, H, n_pad, d = q.shape
+    O = np.zeros((B, H, n_pad, d))
+    L = np.full((B, H, n_pad), NEG_INF)
+    info = []
+    for b in range(B):
+        for h in range(H):
+            aq, muq = local_window_clustering(q[b, h, :n_valid], grid, cell, window, n_iter)
+            ak, muk = local_window_clustering(k[b, h, :n_valid], grid, cell, window, n_iter)
+            G = muq.shape[0]
+            sq = np.bincount(aq, minlength=G)
+            sk = np.bincount(ak, minlength=G)
+            kept = select_clusters(muq, muk, sq, sk, scale, k_min, cum_mass, fixed_k)
+            groups = merge_clusters(sq, sk, kept, tau_q, tau_k, sides[b][h]) if sides is not None else \
+                [[i] for i in range(G)]
+            for g in groups:
+                rows = np.nonzero(np.isin(aq, g))[0]
+                if rows.size == 0:
+                    continue
+                sel = sorted(set().union(*[set(int(j) for j in kept[i]) for i in g]))
+                keys = np.nonzero(np.isin(ak, sel))[0]
+                o, lse = attention_rows(q[b, h, rows], k[b, h, keys], v[b, h, keys], scale)
+                O[b, h, rows] = o
+                L[b, h, rows] = lse
+            info.append({"assign_q": aq, "assign_k": ak, "mu_q": muq, "mu_k": muk, "sizes_q": sq, "sizes_k": sk,
+                         "kept": kept, "groups": groups})
+    return {"O": O, "LSE": L, "heads": info}

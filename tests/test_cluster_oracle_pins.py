@@ -139,3 +139,57 @@ def test_dense_selection_is_invariant_to_the_permutation():
     assert np.allclose(res["O"], O, atol=1e-12)
     fin = np.isfinite(L)
     assert np.allclose(res["LSE"][fin], L[fin], atol=1e-12)
+
+
+def test_hand_worked_merging():
+    """tests/golden/cluster_hand.txt, "Hardware-aware merging"."""
+    sq, sk = [3, 1, 2, 2], [2, 2, 4]
+    kept = [np.array([0]), np.array([0]), np.array([1, 2]), np.array([2])]
+    assert orc.total_cost([[0], [1], [2], [3]], sq, sk, kept, 4, 4) == 80
+    g1 = orc.merge_clusters(sq, sk, kept, 4, 4, [[0, 1, 0, 1]])
+    assert g1 == [[0, 1], [2], [3]] and orc.total_cost(g1, sq, sk, kept, 4, 4) == 64
+    g2 = orc.merge_clusters(sq, sk, kept, 4, 4, [[0, 1, 0, 1], [1, 0, 0, 1]])
+    assert g2 == [[0, 1], [2, 3]] and orc.total_cost(g2, sq, sk, kept, 4, 4) == 48
+
+
+def test_merging_partitions_and_never_raises_the_cost():
+    rng = np.random.default_rng(21)
+    nq, nk = 60, 40
+    sq = rng.integers(0, 200, size=nq)
+    sk = rng.integers(1, 200, size=nk)
+    kept = [np.sort(rng.choice(nk, size=int(rng.integers(1, 12)), replace=False)) for _ in range(nq)]
+    sides = rng.integers(0, 2, size=(8, nq))
+    prev = orc.total_cost([[i] for i in range(nq)], sq, sk, kept, 128, 128)
+    for r in range(1, 9):
+        groups = orc.merge_clusters(sq, sk, kept, 128, 128, sides[:r])
+        assert sorted(i for g in groups for i in g) == list(range(nq))
+        cost = orc.total_cost(groups, sq, sk, kept, 128, 128)
+        assert cost <= prev
+        prev = cost
+    assert prev < orc.total_cost([[i] for i in range(nq)], sq, sk, kept, 128, 128)
+
+
+def test_cluster_selection_with_equal_sizes_is_top_k_of_the_logits():
+    """With every key cluster the same size, Eq. (2)'s weights are a common
+    factor and fixed-k selection keeps the k largest centroid logits."""
+    rng = np.random.default_rng(22)
+    muq, muk = rng.standard_normal((5, 8)), rng.standard_normal((9, 8))
+    kept = orc.select_clusters(muq, muk, [3, 0, 4, 4, 1], [7] * 9, 0.3, 0, 0.0, 4)
+    for i in range(5):
+        expect = [] if i == 1 else sorted(np.argsort(-(muq[i] @ muk.T), kind="stable")[:4].tolist())
+        assert kept[i].tolist() == expect
+
+
+def test_cluster_blocks_with_everything_kept_is_dense_attention():
+    """Every key cluster kept (fixed k = all): each token attends to all keys,
+    whatever the clusters and the merging, so the result is dense attention."""
+    w = WORKLOADS["tiny"]
+    q, k, v = make_qkv(w)
+    G = int(np.prod(orc.cell_counts(w.grid, (2, 2, 2))))
+    sides = np.random.default_rng(3).integers(0, 2, size=(w.B, w.H, 4, G))
+    res = orc.forward_cluster_blocks(q, k, v, w.n_valid, w.grid, (2, 2, 2), (3, 3, 3), 2, w.scale, 0, 0.0, G,
+                                     sides=sides)
+    assert any(len(g) > 1 for g in res["heads"][0]["groups"])
+    mask = np.ones((w.n_pad, w.n_pad), dtype=bool)
+    O, L = orc.masked_attention_bruteforce(q, k, v, np.broadcast_to(mask, (w.B, w.H, w.n_pad, w.n_pad)), w.scale)
+    assert np.allclose(res["O"], O, atol=1e-12) and np.allclose(res["LSE"], L, atol=1e-12)
