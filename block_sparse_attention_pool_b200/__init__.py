@@ -26,6 +26,7 @@ __all__ = [
     "pool_qk", "select_blocks", "mask_to_lists", "select_micro", "select_micro_workspace_bytes", "select_micro_noalloc",
     "block_sparse_fwd", "lse_merge", "read_device_status", "status_string", "version", "selftest_wait_timeout",
     "PathConfig", "SparseVideoAttention", "ClusterParams", "cluster_count", "cluster_tokens", "permute_rows",
+    "select_clusters", "merge_clusters", "merge_clusters_workspace_bytes",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -35,7 +36,8 @@ EXPORTED = (
     "vsa_status_string", "vsa_version", "vsa_read_device_status", "vsa_pool_qk", "vsa_select_blocks",
     "vsa_mask_to_lists", "vsa_select_micro_workspace_bytes", "vsa_select_micro", "vsa_select_micro_noalloc",
     "vsa_block_sparse_fwd", "vsa_block_sparse_fwd_heads", "vsa_lse_merge", "vsa_selftest_wait_timeout",
-    "vsa_cluster_count", "vsa_cluster_tokens", "vsa_permute_rows",
+    "vsa_cluster_count", "vsa_cluster_tokens", "vsa_permute_rows", "vsa_select_clusters",
+    "vsa_merge_clusters_workspace_bytes", "vsa_merge_clusters",
 )
 
 STATUS = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_UNSUPPORTED", 3: "VSA_ERR_CUDA",
@@ -126,6 +128,12 @@ def lib():
     L.vsa_cluster_tokens.argtypes = [P, SP, ctypes.POINTER(ClusterParams), P, P, P, P, P]
     L.vsa_permute_rows.restype = I
     L.vsa_permute_rows.argtypes = [P, P, I, I, I, I, P, P]
+    L.vsa_select_clusters.restype = I
+    L.vsa_merge_clusters_workspace_bytes.restype = S
+    L.vsa_merge_clusters_workspace_bytes.argtypes = [I, I]
+    L.vsa_merge_clusters.restype = I
+    L.vsa_merge_clusters.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, S, P, P, P, P]
+    L.vsa_select_clusters.argtypes = [P, P, P, P, I, I, I, I, F, ctypes.POINTER(SelectParams), P, P, P]
     _lib = L
     return L
 
@@ -182,6 +190,30 @@ def select_blocks(q_pool, k_pool, shape: Shape, bq, bk, scale, params: SelectPar
     _check(lib().vsa_select_blocks(_p(q_pool), _p(k_pool), ctypes.byref(shape), bq, bk, float(scale),
                                    ctypes.byref(params), _p(counts), _p(idx), _p(mask), _s(stream)),
            "vsa_select_blocks")
+
+
+def select_clusters(mu_q, mu_k, sizes_q, sizes_k, scale, params: SelectParams, counts, idx, stream=None):
+    """Cluster-level selection; mu_* fp32 [B, H, n, d], sizes_* int32 [B, H, n]."""
+    bh = mu_q.shape[0] * mu_q.shape[1]
+    _check(lib().vsa_select_clusters(_p(mu_q), _p(mu_k), _p(sizes_q), _p(sizes_k), bh, mu_q.shape[2],
+                                     mu_k.shape[2], mu_q.shape[3], float(scale), ctypes.byref(params), _p(counts),
+                                     _p(idx), _s(stream)), "vsa_select_clusters")
+
+
+def merge_clusters_workspace_bytes(batch_heads: int, n_q: int) -> int:
+    return int(lib().vsa_merge_clusters_workspace_bytes(batch_heads, n_q))
+
+
+def merge_clusters(sizes_q, sizes_k, counts, idx, sides, tau_q, tau_k, workspace, group_of, g_counts, g_idx,
+                   stream=None):
+    """Algorithm 1 merging; sizes_* int32 [B, H, n], sides uint8 [B, H, R, n_q]
+    (or None for R = 0), workspace a uint8 device buffer."""
+    bh = sizes_q.shape[0] * sizes_q.shape[1]
+    rounds = 0 if sides is None else sides.shape[2]
+    _check(lib().vsa_merge_clusters(_p(sizes_q), _p(sizes_k), _p(counts), _p(idx), _p(sides), bh, sizes_q.shape[2],
+                                    sizes_k.shape[2], rounds, int(tau_q), int(tau_k), _p(workspace),
+                                    workspace.numel() * workspace.element_size(), _p(group_of), _p(g_counts),
+                                    _p(g_idx), _s(stream)), "vsa_merge_clusters")
 
 
 def mask_to_lists(mask, shape: Shape, bq, bk, counts, idx, stream=None):

@@ -81,6 +81,15 @@ struct AttnArgs {
   const int32_t *heads;  // grid row -> b * H + h, or NULL for grid row = b * H + h
   int n_bh;              // B * H
   unsigned long long timeout_ns;
+  // Cluster-group mode (tile_list non-null; list_rows 128, seg_keys 16): tile T of
+  // head bh uses list row tile_list[bh][T] (-1: no such tile, the CTA leaves at
+  // once), whose entries are key clusters j < n_kc; cluster j is the K/V rows
+  // [kc_off[j], kc_off[j] + kc_size[j]), walked as 16-key segments of which the
+  // last may be partial.  Query and output rows per head: n_rows_q.
+  const int32_t *tile_list;  // [BH][n_tiles]
+  const int32_t *kc_off;     // [BH][n_kc]
+  const int32_t *kc_size;    // [BH][n_kc]
+  int n_kc, n_lists_bh, n_tiles, n_rows_q;
 };
 
 struct StageInfo {
@@ -89,6 +98,7 @@ struct StageInfo {
   int full;       // every column of the stage is used by every row
   int tail;       // some used segment reaches past n_valid (exact per-column masks)
   uint32_t use16; // bit 8*h + q: 16-column group q is used by query half h
+  uint32_t len4;  // cluster-group mode: bits [4s, 4s + 4) = 16 - valid keys of segment s
 };
 
 template <int D>
@@ -118,6 +128,7 @@ struct AttnCtl {
   uint32_t tmem_base;
   int abort;
   int n_seg;
+  int n_ent;  // cluster-group mode: key clusters of the tile's list
   int fast;  // the union sits in shared memory (lists short enough to stage)
   StageInfo info[kInfoRing];
 };
@@ -285,10 +296,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const bool groups = a.tile_list != nullptr;
+  int group_row = 0;
+  if (groups) {
+    group_row = __ldg(a.tile_list + (size_t)bh * a.n_tiles + tile);
+    if (group_row < 0) return;  // no tile here
+    if (group_row >= a.n_lists_bh) {
+      if (threadIdx.x == 0) latch_status(VSA_ERR_BAD_INDEX);
+      return;
+    }
+  }
   const int n_lists = kTileM / a.list_rows;
-  const int lists_per_bh = a.n_pad / a.list_rows;
+  const int lists_per_bh = groups ? a.n_lists_bh : a.n_pad / a.list_rows;
   const int seg_per_stage = kStageKeys / a.seg_keys;
-  const size_t lrow0 = (size_t)bh * lists_per_bh + (size_t)tile * n_lists;
+  const size_t lrow0 = (size_t)bh * lists_per_bh + (groups ? (size_t)group_row : (size_t)tile * n_lists);
+  const int n_rows_q = groups ? a.n_rows_q : a.n_pad;
+  const int q_valid = groups ? a.n_rows_q : a.n_valid;
 
   // ---------------------------------------------------------------- setup
   if (warp == 0) {
@@ -329,7 +352,41 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     const bool fast = ok && cnt[0] <= kListStage && cnt[1] <= kListStage;
     int n_seg = 0;
-    if (fast) {
+    if (groups) {
+      // the group's key clusters: ids at sl[e], first rows at sl[kListStage + e],
+      // sizes at su[kListStage + e], inclusive prefix of their 16-key segment counts at su[e]
+      int32_t *sl = reinterpret_cast<int32_t *>(smem + L::kOffL);
+      uint32_t *su = reinterpret_cast<uint32_t *>(smem + L::kOffU);
+      ok = ok && fast;
+      const int n = ok ? cnt[0] : 0;
+      const int32_t *li = a.idx + lrow0 * a.idx_stride;
+      for (int e = lane; e < n; e += 32) sl[e] = __ldg(li + e);
+      __syncwarp();
+      int carry = 0;
+      for (int e0 = 0; e0 < n; e0 += 32) {
+        const int e = e0 + lane;
+        int segs = 0;
+        if (e < n) {
+          const int j = sl[e];
+          if (j < 0 || j >= a.n_kc || (e > 0 && sl[e - 1] >= j)) {
+            ok = false;
+          } else {
+            const int off = __ldg(a.kc_off + (size_t)bh * a.n_kc + j);
+            const int sz = __ldg(a.kc_size + (size_t)bh * a.n_kc + j);
+            if (off < 0 || sz < 0 || (long long)off + sz > a.n_pad) ok = false;
+            segs = ok ? (sz + 15) >> 4 : 0;
+            sl[kListStage + e] = off;
+            su[kListStage + e] = static_cast<uint32_t>(ok ? sz : 0);
+          }
+        }
+        const int incl = warp_exclusive_scan(segs, lane) + segs + carry;
+        if (e < n) su[e] = static_cast<uint32_t>(incl);
+        carry = __shfl_sync(0xffffffffu, incl, 31);
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      n_seg = ok ? carry : 0;
+      __syncwarp();
+    } else if (fast) {
       n_seg = stage_union(a.idx + lrow0 * a.idx_stride, cnt[0], a.idx + (lrow0 + 1) * a.idx_stride, cnt[1],
                           n_lists, n_seg_max, reinterpret_cast<int32_t *>(smem + L::kOffL), kListStage,
                           reinterpret_cast<uint32_t *>(smem + L::kOffU), 3u, lane);
@@ -352,6 +409,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     if (lane == 0) {
       ctl->n_seg = n_seg;
+      ctl->n_ent = cnt[0];
       ctl->fast = fast ? 1 : 0;
     }
   } else if (warp == 1) {
@@ -397,7 +455,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // this stage's segments: lane i < seg_per_stage holds segment i's first key row
         int my_start = 0;
         uint32_t b0 = 0u, b1 = 0u;  // bit i: segment i used by query half 0 / 1
-        if (fast) {
+        uint32_t my_len4 = 0u;
+        if (groups) {
+          // segment g of the group's packed key stream: entry e with su[e-1] <= g < su[e]
+          const int g = s * seg_per_stage + lane;
+          const bool has = lane < seg_per_stage && g < n_seg;
+          int start = 0;
+          if (has) {
+            const int n_ent = ctl->n_ent;
+            int lo = 0, hi = n_ent - 1;
+            while (lo < hi) {
+              const int mid = (lo + hi) >> 1;
+              if (static_cast<int>(su[mid]) > g) hi = mid;
+              else lo = mid + 1;
+            }
+            const int k = g - (lo > 0 ? static_cast<int>(su[lo - 1]) : 0);
+            const int32_t *sl = reinterpret_cast<const int32_t *>(smem + L::kOffL);
+            start = sl[kListStage + lo] + 16 * k;
+            const int len = min(16, static_cast<int>(su[kListStage + lo]) - 16 * k);
+            my_len4 = static_cast<uint32_t>(16 - len) << (4 * lane);
+          }
+          const int start0 = __shfl_sync(0xffffffffu, start, 0);
+          my_start = has ? start : start0;
+          b0 = b1 = __ballot_sync(0xffffffffu, has);
+          my_len4 = __reduce_or_sync(0xffffffffu, my_len4);
+        } else if (fast) {
           const int e = s * seg_per_stage + lane;
           const bool has = lane < seg_per_stage && e < n_seg;
           const uint32_t x = has ? su[e] : 0u;
@@ -423,8 +505,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
         const uint32_t used = b0 | b1;
-        const bool tail = __any_sync(0xffffffffu, lane < seg_per_stage && ((used >> lane) & 1u) &&
-                                                      my_start + a.seg_keys > a.n_valid);
+        const bool tail = groups ? my_len4 != 0u
+                                 : __any_sync(0xffffffffu, lane < seg_per_stage && ((used >> lane) & 1u) &&
+                                                               my_start + a.seg_keys > a.n_valid);
         uint32_t mask = 0u, use16 = 0u;
         for (int i = 0; i < seg_per_stage; ++i) mask |= (((b0 >> i) & 1u) << (2 * i)) | (((b1 >> i) & 1u) << (2 * i + 1));
         for (int q = 0; q < 8; ++q)
@@ -444,6 +527,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           inf.full = full ? 1 : 0;
           inf.tail = tail ? 1 : 0;
           inf.use16 = use16;
+          inf.len4 = my_len4;
           mbar_arrive(&ctl->info_full[s & (kInfoRing - 1)]);
           mbar_arrive_expect_tx(&ctl->k_full[slot], L::kKVBytes);
         }
@@ -562,7 +646,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll 1
         for (int sg = 0; sg < nseg; ++sg) {
           if (!((mask >> (2 * sg + half)) & 1u)) continue;
-          const int nv = min(a.seg_keys, max(0, a.n_valid - inf.start[sg]));
+          const int nv = groups ? 16 - static_cast<int>((inf.len4 >> (4 * sg)) & 15u)
+                                : min(a.seg_keys, max(0, a.n_valid - inf.start[sg]));
           const int lo = sg * a.seg_keys, hi = lo + nv;
 #pragma unroll
           for (int w = 0; w < 2; ++w) {
@@ -670,8 +755,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const float lsum = l0 * w0 + l1 * w1;
     const float rsum = r0 * w0 + r1 * w1;
     const int grow = tile * kTileM + row;
-    const size_t orow = (size_t)bh * a.n_pad + grow;
-    const bool row_ok = live && grow < a.n_valid && lsum > 0.f && rsum > 0.f;
+    const size_t orow = (size_t)bh * n_rows_q + grow;
+    const bool row_ok = live && grow < q_valid && lsum > 0.f && rsum > 0.f;
     const float s0 = row_ok ? w0 / rsum : 0.f, s1 = row_ok ? w1 / rsum : 0.f;
     float lse = row_ok ? (mm + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
     MergeWeights mw;

@@ -39,6 +39,11 @@ struct SelectArgs {
   int32_t *counts;  // [BH, n_q]
   int32_t *idx;     // [BH, n_q, n_k]
   uint8_t *mask;    // [BH, n_q, n_k] or null
+  // cluster mode (HyperVAttention Eq. (2) on clusters): explicit sizes of the
+  // query and key units [BH, n_q] / [BH, n_k] replace the block sizes implied
+  // by n_valid; null in block mode
+  const int32_t *q_sizes;
+  const int32_t *k_sizes;
 };
 
 // Compare-exchange of the in-register pairs (i, i | J) of a bitonic substage.
@@ -225,7 +230,7 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     const size_t orow = (size_t)bh * a.n_q + qi;
     int32_t *dst = a.idx + orow * a.n_k;
     uint8_t *mrow = a.mask ? a.mask + orow * a.n_k : nullptr;
-    const bool q_has_rows = qi * a.bq < a.n_valid;
+    const bool q_has_rows = a.q_sizes ? __ldg(a.q_sizes + orow) > 0 : qi * a.bq < a.n_valid;
 
     if constexpr (BY_RANK) {
       // fixed count (fixed_k > 0): the k largest log-weights, no order needed
@@ -235,7 +240,7 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
         const int j = i * 32 + lane;
         uint32_t kv = 0u;
         if (j < a.n_k) {
-          const int sj = min(a.bk, max(0, a.n_valid - j * a.bk));
+          const int sj = a.k_sizes ? __ldg(a.k_sizes + (size_t)bh * a.n_k + j) : min(a.bk, max(0, a.n_valid - j * a.bk));
           const float w = sj > 0 ? S[r * nkp + j] + (sj == a.bk ? ln_bk : logf((float)sj)) : -INFINITY;
           kv = float_key(w);
         }
@@ -260,7 +265,7 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
       for (int i = 0; i < NR; ++i) {
         const int j = i * 32 + lane;
         if (j < a.n_k) {
-          const int sj = min(a.bk, max(0, a.n_valid - j * a.bk));
+          const int sj = a.k_sizes ? __ldg(a.k_sizes + (size_t)bh * a.n_k + j) : min(a.bk, max(0, a.n_valid - j * a.bk));
           const float w = sj > 0 ? S[r * nkp + j] + (sj == a.bk ? ln_bk : logf((float)sj)) : -INFINITY;
           key[i] = ((uint64_t)float_key(w) << 32) | (uint64_t)(0xffffffffu - (uint32_t)j);
         } else {

@@ -19,6 +19,8 @@
 #include "attn_fwd.cuh"
 #include "attn_fwd_dual.cuh"
 #include "cluster.cuh"
+#include "cluster_merge.cuh"
+#include "cluster_plan.cuh"
 #include "common.cuh"
 #include "merge.cuh"
 #include "micro.cuh"
@@ -81,6 +83,47 @@ bool make_map(CUtensorMap *map, const void *base, const vsa_shape *s, int box_ro
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// [BH][rows][d] bf16, all rows inside the tensor.
+bool make_map_rows(CUtensorMap *map, const void *base, int rows, int d, int BH, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D>
+vsa_status set_attn_smem() {
+  using L = vsa::AttnSmem<D>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(vsa::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  });
+  return attr_err == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+// Cluster-group mode: Q rows of the group layout ([BH][n_rows_q][d]), K/V in the
+// key cluster permutation ([BH][n_pad][d], 16-row boxes).
+template <int D>
+vsa_status launch_attn_groups(const void *q, const void *k, const void *v, const vsa_shape *s, const AttnArgs &a,
+                              cudaStream_t st) {
+  using L = vsa::AttnSmem<D>;
+  if (set_attn_smem<D>() != VSA_OK) return VSA_ERR_CUDA;
+  const int BH = s->B * s->H;
+  CUtensorMap mq, mk, mv;
+  if (!make_map_rows(&mq, q, a.n_rows_q, D, BH, vsa::kTileM) || !make_map(&mk, k, s, 16) || !make_map(&mv, v, s, 16))
+    return VSA_ERR_CUDA;
+  dim3 grid(a.n_tiles, BH);
+  vsa::attn_fwd_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, a);
+  return launch_status();
 }
 
 template <int D>
@@ -313,6 +356,70 @@ vsa_status launch_cluster(const __nv_bfloat16 *x, const vsa::ClusterGeom &g, int
   return launch_status();
 }
 
+bool select_params_ok(float scale, const vsa_select_params *params) {
+  if (!(scale > 0.f) || !std::isfinite(scale)) return false;
+  return params->k_min >= 0 && params->fixed_k >= 0 && params->n_anchor >= 0 && params->anchor_rot >= 0 &&
+         std::isfinite(params->cum_mass);
+}
+
+// Selection over n_q query units x n_k key units (blocks, or clusters with
+// explicit sizes), one CTA per 16 query units of one (batch, head).
+vsa_status launch_select(const vsa::SelectArgs &a, int d, int BH, bool by_rank, cudaStream_t st) {
+  const int n_q = a.n_q, n_k = a.n_k;
+  int nkp = 32;
+  while (nkp < n_k) nkp <<= 1;
+  const int dp = d + 4;
+  const size_t smem = (size_t)(vsa::kSelRows + vsa::kSelChunk) * dp * 4 + (size_t)vsa::kSelRows * nkp * 4 + 8 * 32 * 4;
+  dim3 grid((n_q + vsa::kSelRows - 1) / vsa::kSelRows, BH);
+#define VSA_SEL_CASE(DD, NR)                                                                                  \
+  {                                                                                                           \
+    auto kern = by_rank ? vsa::select_blocks_kernel<DD, NR, true> : vsa::select_blocks_kernel<DD, NR, false>; \
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) \
+      return VSA_ERR_CUDA;                                                                                    \
+    kern<<<grid, vsa::kSelThreads, smem, st>>>(a);                                                            \
+  }
+#define VSA_SEL_NR(DD)                     \
+  switch (nkp / 32) {                      \
+    case 1: VSA_SEL_CASE(DD, 1) break;     \
+    case 2: VSA_SEL_CASE(DD, 2) break;     \
+    case 4: VSA_SEL_CASE(DD, 4) break;     \
+    case 8: VSA_SEL_CASE(DD, 8) break;     \
+    case 16: VSA_SEL_CASE(DD, 16) break;   \
+    default: VSA_SEL_CASE(DD, 32) break;   \
+  }
+  if (d == 128) {
+    VSA_SEL_NR(128)
+  } else {
+    VSA_SEL_NR(64)
+  }
+#undef VSA_SEL_NR
+#undef VSA_SEL_CASE
+  return launch_status();
+}
+
+// Workspace of the cluster merging, carved from one caller buffer (256-byte
+// aligned arrays).  Returns the bytes needed; fills *ws when base is non-null.
+size_t merge_ws_layout(int BH, int nq, void *base, vsa::MergeWs *ws) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> void * {
+    void *p = base ? static_cast<char *>(base) + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  const size_t n = (size_t)BH * nq;
+  vsa::MergeWs w;
+  w.lead = static_cast<int32_t *>(take(n * 4));
+  w.gsq = static_cast<int32_t *>(take(n * 4));
+  w.gwk = static_cast<int32_t *>(take(n * 4));
+  w.chi = static_cast<uint32_t *>(take(n * vsa::kMergeWords * 4));
+  w.list = static_cast<int32_t *>(take(2 * n * 4));
+  w.nlist = static_cast<int32_t *>(take((size_t)BH * 2 * 4));
+  w.best = static_cast<unsigned long long *>(take(n * 8));
+  w.passes = static_cast<int32_t *>(take((size_t)BH * 4));
+  if (ws) *ws = w;
+  return off;
+}
+
 }  // namespace
 
 extern "C" {
@@ -374,45 +481,25 @@ vsa_status vsa_select_blocks(const float *q_pool, const float *k_pool, const vsa
   if (!shape_ok(shape) || !q_pool || !k_pool || !params || !counts || !idx) return VSA_ERR_INVALID_ARG;
   if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return VSA_ERR_INVALID_ARG;
   if (!aligned16(q_pool) || !aligned16(k_pool)) return VSA_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || !std::isfinite(scale)) return VSA_ERR_INVALID_ARG;
-  if (params->k_min < 0 || params->fixed_k < 0 || params->n_anchor < 0 || params->anchor_rot < 0 ||
-      !std::isfinite(params->cum_mass))
-    return VSA_ERR_INVALID_ARG;
+  if (!select_params_ok(scale, params)) return VSA_ERR_INVALID_ARG;
   const int n_q = shape->n_pad / bq, n_k = shape->n_pad / bk;
   if (n_k > 1024) return VSA_ERR_UNSUPPORTED;
   vsa::SelectArgs a{q_pool, k_pool, n_q, n_k, bq, bk, shape->n_valid, scale, params->k_min, params->fixed_k,
-                    params->n_anchor, params->anchor_rot, params->cum_mass, counts, idx, mask};
-  int nkp = 32;
-  while (nkp < n_k) nkp <<= 1;
-  const int dp = shape->d + 4;
-  const size_t smem = (size_t)(vsa::kSelRows + vsa::kSelChunk) * dp * 4 + (size_t)vsa::kSelRows * nkp * 4 + 8 * 32 * 4;
-  dim3 grid((n_q + vsa::kSelRows - 1) / vsa::kSelRows, shape->B * shape->H);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const bool by_rank = params->fixed_k > 0;  // a fixed count needs no sort
-#define VSA_SEL_CASE(DD, NR)                                                                                  \
-  {                                                                                                           \
-    auto kern = by_rank ? vsa::select_blocks_kernel<DD, NR, true> : vsa::select_blocks_kernel<DD, NR, false>; \
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) \
-      return VSA_ERR_CUDA;                                                                                    \
-    kern<<<grid, vsa::kSelThreads, smem, st>>>(a);                                                            \
-  }
-#define VSA_SEL_NR(DD)                     \
-  switch (nkp / 32) {                      \
-    case 1: VSA_SEL_CASE(DD, 1) break;     \
-    case 2: VSA_SEL_CASE(DD, 2) break;     \
-    case 4: VSA_SEL_CASE(DD, 4) break;     \
-    case 8: VSA_SEL_CASE(DD, 8) break;     \
-    case 16: VSA_SEL_CASE(DD, 16) break;   \
-    default: VSA_SEL_CASE(DD, 32) break;   \
-  }
-  if (shape->d == 128) {
-    VSA_SEL_NR(128)
-  } else {
-    VSA_SEL_NR(64)
-  }
-#undef VSA_SEL_NR
-#undef VSA_SEL_CASE
-  return launch_status();
+                    params->n_anchor, params->anchor_rot, params->cum_mass, counts, idx, mask, nullptr, nullptr};
+  return launch_select(a, shape->d, shape->B * shape->H, params->fixed_k > 0, static_cast<cudaStream_t>(stream));
+}
+
+vsa_status vsa_select_clusters(const float *mu_q, const float *mu_k, const int32_t *sizes_q, const int32_t *sizes_k,
+                               int batch_heads, int n_q, int n_k, int d, float scale,
+                               const vsa_select_params *params, int32_t *counts, int32_t *idx, void *stream) {
+  if (!mu_q || !mu_k || !sizes_q || !sizes_k || !params || !counts || !idx) return VSA_ERR_INVALID_ARG;
+  if (batch_heads < 1 || batch_heads > 65535 || n_q < 1 || n_k < 1 || (d != 64 && d != 128)) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(mu_q) || !aligned16(mu_k)) return VSA_ERR_INVALID_ARG;
+  if (!select_params_ok(scale, params) || params->n_anchor != 0) return VSA_ERR_INVALID_ARG;
+  if (n_k > 1024) return VSA_ERR_UNSUPPORTED;
+  vsa::SelectArgs a{mu_q, mu_k, n_q, n_k, 1, 1, 0, scale, params->k_min, params->fixed_k,
+                    0, 0, params->cum_mass, counts, idx, nullptr, sizes_q, sizes_k};
+  return launch_select(a, d, batch_heads, params->fixed_k > 0, static_cast<cudaStream_t>(stream));
 }
 
 vsa_status vsa_mask_to_lists(const uint8_t *mask, const vsa_shape *shape, int bq, int bk, int32_t *counts,
@@ -588,7 +675,7 @@ vsa_status vsa_block_sparse_fwd_heads(const void *q, const void *k, const void *
   if (merge_o && static_cast<const void *>(merge_o) == o) return VSA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (merge_o && !aligned16(merge_o)))
     return VSA_ERR_INVALID_ARG;
-  AttnArgs a;
+  AttnArgs a{};
   a.n_pad = shape->n_pad;
   a.n_valid = shape->n_valid;
   a.list_rows = list_rows;
@@ -668,6 +755,139 @@ vsa_status vsa_permute_rows(const void *src, const int32_t *perm, int batch_head
       static_cast<const uint32_t *>(src), perm, n_pad, rows, row_bytes / 4, inverse ? 1 : 0,
       static_cast<uint32_t *>(dst));
   return launch_status();
+}
+
+size_t vsa_merge_clusters_workspace_bytes(int batch_heads, int n_q) {
+  if (batch_heads < 1 || n_q < 1) return 0;
+  return merge_ws_layout(batch_heads, n_q, nullptr, nullptr);
+}
+
+vsa_status vsa_merge_clusters(const int32_t *sizes_q, const int32_t *sizes_k, const int32_t *counts,
+                              const int32_t *idx, const uint8_t *sides, int batch_heads, int n_q, int n_k,
+                              int rounds, int tau_q, int tau_k, void *workspace, size_t workspace_bytes,
+                              int32_t *group_of, int32_t *g_counts, int32_t *g_idx, void *stream) {
+  if (!sizes_q || !sizes_k || !counts || !idx || !workspace || !group_of || !g_counts || !g_idx)
+    return VSA_ERR_INVALID_ARG;
+  if (batch_heads < 1 || batch_heads > 65535 || n_q < 1 || n_k < 1 || rounds < 0 || rounds > 64)
+    return VSA_ERR_INVALID_ARG;
+  if (rounds > 0 && !sides) return VSA_ERR_INVALID_ARG;
+  if (tau_q < 1 || tau_k < 1 || tau_q > (1 << 20) || tau_k > (1 << 20)) return VSA_ERR_INVALID_ARG;
+  if (n_q > vsa::kMergeMaxClusters || n_k > vsa::kMergeMaxClusters) return VSA_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return VSA_ERR_INVALID_ARG;
+  if (workspace_bytes < merge_ws_layout(batch_heads, n_q, nullptr, nullptr)) return VSA_ERR_INVALID_ARG;
+  vsa::MergeArgs a{};
+  a.sizes_q = sizes_q;
+  a.sizes_k = sizes_k;
+  a.counts = counts;
+  a.idx = idx;
+  a.sides = sides;
+  a.nq = n_q;
+  a.nk = n_k;
+  a.rounds = rounds;
+  a.tau_q = tau_q;
+  a.tau_k = tau_k;
+  a.inv_tau_q = 1.0f / (float)tau_q;
+  a.inv_tau_k = 1.0f / (float)tau_k;
+  a.group_of = group_of;
+  a.g_counts = g_counts;
+  a.g_idx = g_idx;
+  merge_ws_layout(batch_heads, n_q, workspace, &a.ws);
+  a.timeout_ns = kWaitLimitNs;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  vsa::merge_init_kernel<<<batch_heads, vsa::kMergeHeadThreads, 0, st>>>(a);
+  if (rounds > 0) {
+    const int smem = vsa::MergeSmem::kAlloc;
+    if (cudaFuncSetAttribute(vsa::merge_pairs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return VSA_ERR_CUDA;
+    const int tiles = (n_q + vsa::kMergeTile - 1) / vsa::kMergeTile;
+    for (int r = 0; r < rounds; ++r) {
+      vsa::merge_pairs_kernel<<<dim3(tiles, tiles, batch_heads), vsa::kMergeThreads, smem, st>>>(a);
+      vsa::merge_apply_kernel<<<batch_heads, vsa::kMergeHeadThreads, 0, st>>>(a, r);
+    }
+  }
+  return launch_status();
+}
+
+int vsa_cluster_rows_capacity(int n_valid, int n_q) {
+  if (n_valid < 1 || n_q < 1) return 0;
+  const long long rows = ((long long)n_valid + 127ll * n_q + 127) / 128 * 128;
+  return rows > 0x7fffffffll ? 0 : static_cast<int>(rows);
+}
+
+vsa_status vsa_cluster_plan(const int32_t *group_of, const int32_t *sizes_q, const int32_t *perm_q,
+                            const int32_t *sizes_k, int batch_heads, int n_q, int n_k, int n_valid, int n_pad,
+                            int n_rows, int32_t *qmap, int32_t *qinv, int32_t *tile_list, int32_t *kc_off,
+                            void *stream) {
+  if (!group_of || !sizes_q || !perm_q || !sizes_k || !qmap || !qinv || !tile_list || !kc_off)
+    return VSA_ERR_INVALID_ARG;
+  if (batch_heads < 1 || batch_heads > 65535 || n_q < 1 || n_k < 1 || n_valid < 1 || n_pad < n_valid)
+    return VSA_ERR_INVALID_ARG;
+  if (n_rows < 128 || n_rows % 128 != 0) return VSA_ERR_INVALID_ARG;
+  if (n_q > vsa::kPlanMaxClusters || n_k > vsa::kPlanMaxClusters) return VSA_ERR_UNSUPPORTED;
+  vsa::PlanArgs a{group_of, sizes_q, perm_q, sizes_k, n_q, n_k, n_valid, n_pad, n_rows, qmap, qinv, tile_list, kc_off};
+  vsa::cluster_plan_kernel<<<batch_heads, vsa::kPlanThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  return launch_status();
+}
+
+vsa_status vsa_gather_rows(const void *src, const int32_t *map, int batch_heads, int n_src, int n_dst,
+                           int row_bytes, uint32_t fill, void *dst, void *stream) {
+  if (!src || !map || !dst || src == dst) return VSA_ERR_INVALID_ARG;
+  if (batch_heads < 1 || n_src < 1 || n_dst < 1 || row_bytes < 4 || row_bytes % 4 != 0) return VSA_ERR_INVALID_ARG;
+  const bool wide = row_bytes % 16 == 0;
+  const uintptr_t mask = wide ? 15u : 3u;
+  if ((reinterpret_cast<uintptr_t>(src) & mask) || (reinterpret_cast<uintptr_t>(dst) & mask) ||
+      (reinterpret_cast<uintptr_t>(map) & 3u))
+    return VSA_ERR_INVALID_ARG;
+  const char *s8 = static_cast<const char *>(src);
+  const char *d8 = static_cast<const char *>(dst);
+  const long long src_span = (long long)batch_heads * n_src * row_bytes;
+  const long long dst_span = (long long)batch_heads * n_dst * row_bytes;
+  if (s8 < d8 + dst_span && d8 < s8 + src_span) return VSA_ERR_INVALID_ARG;
+  const long long rows = (long long)batch_heads * n_dst;
+  const long long blocks = (rows + 7) / 8;
+  if (blocks > 0x7fffffffll) return VSA_ERR_UNSUPPORTED;
+  vsa::gather_rows_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint32_t *>(src), map, n_src, n_dst, rows, row_bytes / 4, fill, static_cast<uint32_t *>(dst));
+  return launch_status();
+}
+
+vsa_status vsa_cluster_group_fwd(const void *q_rows, const void *k, const void *v, const vsa_shape *shape,
+                                 int n_rows, const int32_t *tile_list, const int32_t *kc_off,
+                                 const int32_t *kc_size, int n_kc, const int32_t *counts, const int32_t *idx,
+                                 int n_lists, float scale, void *o, int o_fp32, float *lse, void *stream) {
+  if (!shape_ok(shape) || !q_rows || !k || !v || !tile_list || !kc_off || !kc_size || !counts || !idx || !o || !lse)
+    return VSA_ERR_INVALID_ARG;
+  if (n_rows < 128 || n_rows % 128 != 0 || n_kc < 1 || n_lists < 1) return VSA_ERR_INVALID_ARG;
+  if (n_kc > vsa::kListStage) return VSA_ERR_UNSUPPORTED;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(q_rows) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return VSA_ERR_INVALID_ARG;
+  if ((long long)n_rows * shape->d * shape->B * shape->H >= (1ll << 40)) return VSA_ERR_UNSUPPORTED;
+  AttnArgs a{};
+  a.n_pad = shape->n_pad;
+  a.n_valid = shape->n_valid;
+  a.list_rows = 128;
+  a.seg_keys = 16;
+  a.seg_shift = 4;
+  a.idx_stride = n_kc;
+  a.counts = counts;
+  a.idx = idx;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.o = o;
+  a.o_fp32 = o_fp32 ? 1 : 0;
+  a.lse = lse;
+  a.n_bh = shape->B * shape->H;
+  a.timeout_ns = kWaitLimitNs;
+  a.tile_list = tile_list;
+  a.kc_off = kc_off;
+  a.kc_size = kc_size;
+  a.n_kc = n_kc;
+  a.n_lists_bh = n_lists;
+  a.n_tiles = n_rows / 128;
+  a.n_rows_q = n_rows;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return shape->d == 128 ? launch_attn_groups<128>(q_rows, k, v, shape, a, st)
+                         : launch_attn_groups<64>(q_rows, k, v, shape, a, st);
 }
 
 }  // extern "C"

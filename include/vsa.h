@@ -175,6 +175,31 @@ VSA_API vsa_status vsa_select_blocks(const float *q_pool, const float *k_pool, c
                              int32_t *idx, uint8_t *mask, void *stream);
 
 /* ---------------------------------------------------------------------------
+ * Cluster-level selection ([HVA] section 2 Eq. (2) and Eq. (3) with query and
+ * key clusters as the units: the logits are centroid products, s_j is the
+ * size of key cluster j).
+ *
+ * Per (batch-head, query cluster i): S_ij = mu_q_i . mu_k_j * scale; the same
+ * ranking (descending S_ij + ln s_j, ties to the lower j, s_j = 0 ranks last)
+ * and the same Top-p / Min-kc / fixed-k rule as vsa_select_blocks; anchors are
+ * not used (params->n_anchor must be 0).  A query cluster of size 0 keeps
+ * nothing.
+ *
+ * mu_q    : fp32 [batch_heads, n_q, d]  query centroids (16-byte aligned).
+ * mu_k    : fp32 [batch_heads, n_k, d]  key centroids.
+ * sizes_q : int32 [batch_heads, n_q]    tokens per query cluster.
+ * sizes_k : int32 [batch_heads, n_k]    tokens per key cluster.
+ * d in {64, 128}; n_k <= 1024 (VSA_ERR_UNSUPPORTED above).
+ * counts  : int32 [batch_heads, n_q]       kept key clusters per query cluster.
+ * idx     : int32 [batch_heads, n_q, n_k]  kept key-cluster indices, ascending,
+ *           in the first counts[row] slots of the row.
+ * ------------------------------------------------------------------------- */
+VSA_API vsa_status vsa_select_clusters(const float *mu_q, const float *mu_k, const int32_t *sizes_q,
+                                       const int32_t *sizes_k, int batch_heads, int n_q, int n_k, int d,
+                                       float scale, const vsa_select_params *params, int32_t *counts,
+                                       int32_t *idx, void *stream);
+
+/* ---------------------------------------------------------------------------
  * Explicit block mask -> lists (the mask-passed-in path of the same
  * attention, [HVA] section 2: m_ij = 1 iff key block j is attended by row i).
  *
@@ -352,6 +377,47 @@ VSA_API vsa_status vsa_cluster_tokens(const void *x, const vsa_shape *shape, con
  * src and dst must not overlap. */
 VSA_API vsa_status vsa_permute_rows(const void *src, const int32_t *perm, int batch_heads, int n_pad, int row_bytes,
                                     int inverse, void *dst, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Hardware-aware cluster merging ([HVA] section 4.3, Eq. (7)-(10), Algorithm 1
+ * "Parallel Agglomerative Merging").
+ *
+ * Query clusters are merged into groups S; a group's cost is
+ * C(S) = tau_q ceil(s_q(S) / tau_q) * tau_k ceil(w_k(S) / tau_k), s_q(S) its
+ * query tokens and w_k(S) the summed sizes of chi(S), the union of the key
+ * clusters its members kept (Eq. (8)).  Starting from singletons, each of
+ * `rounds` rounds splits the current groups by sides[r][leader] (0 = side A,
+ * else B; the leader of a group is its lowest member), lets every A group
+ * pick the B group of smallest dC = C(A u B) - C(A) - C(B) (ties to the lower
+ * leader), keeps for every B the picking A of smallest dC (ties to the lower
+ * leader), and merges the kept pairs with dC < 0.  The random bipartition is
+ * an input so that runs are reproducible.  A query cluster of size 0 never
+ * merges.  All arithmetic is integer: the result is exact.
+ *
+ * sizes_q : int32 [batch_heads, n_q]        tokens per query cluster (>= 0).
+ * sizes_k : int32 [batch_heads, n_k]        tokens per key cluster (>= 0).
+ * counts, idx : the kept lists (vsa_select_clusters layout; idx row stride n_k).
+ * sides   : uint8 [batch_heads, rounds, n_q] bipartition bits; may be NULL when
+ *           rounds == 0.
+ * n_q, n_k <= 1024 (VSA_ERR_UNSUPPORTED above); 0 <= rounds <= 64;
+ * 1 <= tau_q, tau_k <= 2^20.
+ * workspace : device scratch of vsa_merge_clusters_workspace_bytes() bytes,
+ *           256-byte aligned; its content on entry is irrelevant.
+ * Outputs:
+ *   group_of : int32 [batch_heads, n_q]       leader of each cluster's group.
+ *   g_counts : int32 [batch_heads, n_q]       at a leader: |chi(S)|; else 0.
+ *   g_idx    : int32 [batch_heads, n_q, n_k]  at a leader: chi(S) ascending in
+ *              the first g_counts slots (other rows untouched).
+ * An invalid kept list (not strictly ascending, out of range) or a negative
+ * size latches VSA_ERR_BAD_INDEX; that list counts as empty.
+ * ------------------------------------------------------------------------- */
+VSA_API size_t vsa_merge_clusters_workspace_bytes(int batch_heads, int n_q);
+
+VSA_API vsa_status vsa_merge_clusters(const int32_t *sizes_q, const int32_t *sizes_k, const int32_t *counts,
+                                      const int32_t *idx, const uint8_t *sides, int batch_heads, int n_q,
+                                      int n_k, int rounds, int tau_q, int tau_k, void *workspace,
+                                      size_t workspace_bytes, int32_t *group_of, int32_t *g_counts,
+                                      int32_t *g_idx, void *stream);
 
 #ifdef __cplusplus
 }

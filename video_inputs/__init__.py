@@ -295,3 +295,16 @@ def make_qkv(w: Workload, heads: Optional[Tuple[int, int]] = None):
         with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as ex:
             list(ex.map(lambda bh: one_head(*bh), jobs))
     return tuple(out)
+
+
+def merge_sides(w: Workload, rounds: int, n_clusters: int, heads: Optional[Tuple[int, int]] = None) -> np.ndarray:
+    """uint8 [B, H, rounds, n_clusters] random bipartition bits of the cluster
+    merging rounds (one bit per query cluster and round; a group takes the
+    bit of its lowest member), drawn from an RNG stream of their own."""
+    h0, h1 = (0, w.H) if heads is None else heads
+    out = np.zeros((w.B, h1 - h0, rounds, n_clusters), dtype=np.uint8)
+    for b in range(w.B):
+        for h in range(h0, h1):
+            rng = np.random.default_rng([w.seed, 4, b, h])
+            out[b, h - h0] = rng.integers(0, 2, size=(rounds, n_clusters), dtype=np.uint8)
+    return out
