@@ -26,7 +26,8 @@ __all__ = [
     "pool_qk", "select_blocks", "mask_to_lists", "select_micro", "select_micro_workspace_bytes", "select_micro_noalloc",
     "block_sparse_fwd", "lse_merge", "read_device_status", "status_string", "version", "selftest_wait_timeout",
     "PathConfig", "SparseVideoAttention", "ClusterParams", "cluster_count", "cluster_tokens", "permute_rows",
-    "select_clusters", "merge_clusters", "merge_clusters_workspace_bytes",
+    "select_clusters", "merge_clusters", "merge_clusters_workspace_bytes", "cluster_rows_capacity", "cluster_plan",
+    "gather_rows", "cluster_group_fwd", "ClusterBlockConfig", "ClusterBlockAttention",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -37,7 +38,8 @@ EXPORTED = (
     "vsa_mask_to_lists", "vsa_select_micro_workspace_bytes", "vsa_select_micro", "vsa_select_micro_noalloc",
     "vsa_block_sparse_fwd", "vsa_block_sparse_fwd_heads", "vsa_lse_merge", "vsa_selftest_wait_timeout",
     "vsa_cluster_count", "vsa_cluster_tokens", "vsa_permute_rows", "vsa_select_clusters",
-    "vsa_merge_clusters_workspace_bytes", "vsa_merge_clusters",
+    "vsa_merge_clusters_workspace_bytes", "vsa_merge_clusters", "vsa_cluster_rows_capacity", "vsa_cluster_plan",
+    "vsa_gather_rows", "vsa_cluster_group_fwd",
 )
 
 STATUS = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_UNSUPPORTED", 3: "VSA_ERR_CUDA",
@@ -133,6 +135,14 @@ def lib():
     L.vsa_merge_clusters_workspace_bytes.argtypes = [I, I]
     L.vsa_merge_clusters.restype = I
     L.vsa_merge_clusters.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, S, P, P, P, P]
+    L.vsa_cluster_rows_capacity.restype = I
+    L.vsa_cluster_rows_capacity.argtypes = [I, I]
+    L.vsa_cluster_plan.restype = I
+    L.vsa_cluster_plan.argtypes = [P, P, P, P, I, I, I, I, I, I, P, P, P, P, P]
+    L.vsa_gather_rows.restype = I
+    L.vsa_gather_rows.argtypes = [P, P, I, I, I, I, ctypes.c_uint32, P, P]
+    L.vsa_cluster_group_fwd.restype = I
+    L.vsa_cluster_group_fwd.argtypes = [P, P, P, SP, I, P, P, P, I, P, P, I, F, P, I, P, P]
     L.vsa_select_clusters.argtypes = [P, P, P, P, I, I, I, I, F, ctypes.POINTER(SelectParams), P, P, P]
     _lib = L
     return L
@@ -214,6 +224,40 @@ def merge_clusters(sizes_q, sizes_k, counts, idx, sides, tau_q, tau_k, workspace
                                     sizes_k.shape[2], rounds, int(tau_q), int(tau_k), _p(workspace),
                                     workspace.numel() * workspace.element_size(), _p(group_of), _p(g_counts),
                                     _p(g_idx), _s(stream)), "vsa_merge_clusters")
+
+
+def cluster_rows_capacity(n_valid: int, n_q: int) -> int:
+    return int(lib().vsa_cluster_rows_capacity(n_valid, n_q))
+
+
+def cluster_plan(group_of, sizes_q, perm_q, sizes_k, n_valid, qmap, qinv, tile_list, kc_off, stream=None):
+    """Query-layout plan of the groups; group_of/sizes_* int32 [B, H, n], perm_q
+    int32 [B, H, n_pad], qmap [B, H, n_rows], qinv [B, H, n_pad], tile_list
+    [B, H, n_rows/128], kc_off [B, H, n_k]."""
+    B, H, nq = sizes_q.shape
+    _check(lib().vsa_cluster_plan(_p(group_of), _p(sizes_q), _p(perm_q), _p(sizes_k), B * H, nq, sizes_k.shape[2],
+                                  int(n_valid), perm_q.shape[2], qmap.shape[2], _p(qmap), _p(qinv), _p(tile_list),
+                                  _p(kc_off), _s(stream)), "vsa_cluster_plan")
+
+
+def gather_rows(src, mp, dst, fill: int = 0, stream=None):
+    """dst[b, h, i] = src[b, h, mp[b, h, i]] (-1: fill word, -2: untouched); rows
+    are the trailing dimensions after [B, H, n]."""
+    B, H, n_src = src.shape[:3]
+    n_dst = dst.shape[2]
+    row_bytes = (src.numel() // (B * H * n_src)) * src.element_size()
+    _check(lib().vsa_gather_rows(_p(src), _p(mp), B * H, n_src, n_dst, row_bytes, ctypes.c_uint32(fill & 0xffffffff),
+                                 _p(dst), _s(stream)), "vsa_gather_rows")
+
+
+def cluster_group_fwd(q_rows, k, v, shape: Shape, tile_list, kc_off, kc_size, counts, idx, scale, o, lse,
+                      stream=None):
+    """Attention of the query layout's tiles to their groups' key clusters."""
+    n_rows = q_rows.shape[2]
+    _check(lib().vsa_cluster_group_fwd(_p(q_rows), _p(k), _p(v), ctypes.byref(shape), n_rows, _p(tile_list),
+                                       _p(kc_off), _p(kc_size), kc_size.shape[2], _p(counts), _p(idx),
+                                       counts.shape[2], float(scale), _p(o), 1 if o.dtype == torch.float32 else 0,
+                                       _p(lse), _s(stream)), "vsa_cluster_group_fwd")
 
 
 def mask_to_lists(mask, shape: Shape, bq, bk, counts, idx, stream=None):
@@ -559,3 +603,116 @@ class SparseVideoAttention:
                 of[c0:c1].copy_(hb["o"][c0:c1], non_blocking=True)
                 lf[c0:c1].copy_(hb["lse"][c0:c1], non_blocking=True)
         self._s_out.synchronize()
+
+
+@dataclass
+class ClusterBlockConfig:
+    """Cluster-aligned blocks (HyperVAttention §2 Eq. (1)-(4) on clusters,
+    §4.1 Eq. (5), §4.3 Eq. (7)-(10), Algorithm 1)."""
+    n_valid: int
+    lattice: Sequence[int]            # (T, H, W) with T*H*W == n_valid
+    cell: Sequence[int] = (3, 5, 8)
+    window: Sequence[int] = (3, 5, 5)
+    iters: int = 3
+    scale: Optional[float] = None
+    k_min: int = 0
+    cum_mass: float = 0.0
+    fixed_k: int = 0
+    rounds: int = 3                   # merging rounds R (App. A.1: 3)
+    tau_q: int = 128                  # CTA tile sizes of the cost model (Eq. (7))
+    tau_k: int = 128
+
+    def cluster_params(self) -> "ClusterParams":
+        return ClusterParams.make(self.lattice, self.cell, self.window, self.iters)
+
+
+class ClusterBlockAttention:
+    """Cluster Q and K -> select key clusters per query cluster -> merge query
+    clusters (Algorithm 1) -> group layout -> attention per group tile ->
+    output back in token order.  Every stage is a libvsa kernel; buffers are
+    allocated once per input shape and stay readable in ``self.buf``."""
+
+    STAGES = ("cluster_qk", "select", "merge", "plan", "gather_in", "attention", "gather_out")
+
+    def __init__(self, cfg: ClusterBlockConfig):
+        self.cfg = cfg
+        self.buf: Dict[str, torch.Tensor] = {}
+        self._key = None
+
+    def _alloc(self, q: torch.Tensor):
+        B, H, n_pad, d = q.shape
+        key = (B, H, n_pad, d, q.device)
+        if key == self._key:
+            return
+        c = self.cfg
+        G = cluster_count(c.cluster_params())
+        if G < 1:
+            raise VsaError(1, "ClusterBlockAttention: invalid clustering parameters")
+        rows = cluster_rows_capacity(c.n_valid, G)
+        dev = q.device
+        i32, f32 = torch.int32, torch.float32
+        b = {}
+        for n in ("q", "k"):
+            b["assign_" + n] = torch.empty(B, H, c.n_valid, device=dev, dtype=i32)
+            b["centroids_" + n] = torch.empty(B, H, G, d, device=dev, dtype=f32)
+            b["sizes_" + n] = torch.empty(B, H, G, device=dev, dtype=i32)
+            b["perm_" + n] = torch.empty(B, H, n_pad, device=dev, dtype=i32)
+        b["counts"] = torch.empty(B, H, G, device=dev, dtype=i32)
+        b["idx"] = torch.empty(B, H, G, G, device=dev, dtype=i32)
+        b["merge_ws"] = torch.empty(merge_clusters_workspace_bytes(B * H, G), device=dev, dtype=torch.uint8)
+        b["group_of"] = torch.empty(B, H, G, device=dev, dtype=i32)
+        b["g_counts"] = torch.empty(B, H, G, device=dev, dtype=i32)
+        b["g_idx"] = torch.empty(B, H, G, G, device=dev, dtype=i32)
+        b["qmap"] = torch.empty(B, H, rows, device=dev, dtype=i32)
+        b["qinv"] = torch.empty(B, H, n_pad, device=dev, dtype=i32)
+        b["tile_list"] = torch.empty(B, H, rows // 128, device=dev, dtype=i32)
+        b["kc_off"] = torch.empty(B, H, G, device=dev, dtype=i32)
+        b["q_rows"] = torch.empty(B, H, rows, d, device=dev, dtype=torch.bfloat16)
+        b["kp"] = torch.empty(B, H, n_pad, d, device=dev, dtype=torch.bfloat16)
+        b["vp"] = torch.empty(B, H, n_pad, d, device=dev, dtype=torch.bfloat16)
+        b["o_rows"] = torch.empty(B, H, rows, d, device=dev, dtype=torch.bfloat16)
+        b["lse_rows"] = torch.empty(B, H, rows, device=dev, dtype=f32)
+        b["o"] = torch.empty(B, H, n_pad, d, device=dev, dtype=torch.bfloat16)
+        b["lse"] = torch.empty(B, H, n_pad, device=dev, dtype=f32)
+        self.buf = b
+        self._key = key
+
+    def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, sides: Optional[torch.Tensor] = None,
+                 stream=None, on_stage=None) -> Dict[str, torch.Tensor]:
+        """q, k, v: bf16 device tensors [B, H, n_pad, d].  sides: uint8 device
+        tensor [B, H, rounds, G] of bipartition bits (the random draws of
+        Algorithm 1), or None for no merging.  ``on_stage(i)`` is called on
+        the host before the first stage (i = 0) and after each of STAGES."""
+        c = self.cfg
+        self._alloc(q)
+        b = self.buf
+        B, H, n_pad, d = q.shape
+        shape = _shape(B, H, c.n_valid, n_pad, d)
+        scale = c.scale if c.scale is not None else 1.0 / math.sqrt(d)
+        stage = on_stage if on_stage is not None else (lambda i: None)
+        stage(0)
+        params = c.cluster_params()
+        for name, x in (("q", q), ("k", k)):
+            cluster_tokens(x, shape, params, b["assign_" + name], b["centroids_" + name], b["sizes_" + name],
+                           b["perm_" + name], stream)
+        stage(1)
+        select_clusters(b["centroids_q"], b["centroids_k"], b["sizes_q"], b["sizes_k"], scale,
+                        SelectParams(c.k_min, c.cum_mass, c.fixed_k, 0, 0), b["counts"], b["idx"], stream)
+        stage(2)
+        merge_clusters(b["sizes_q"], b["sizes_k"], b["counts"], b["idx"], sides, c.tau_q, c.tau_k, b["merge_ws"],
+                       b["group_of"], b["g_counts"], b["g_idx"], stream)
+        stage(3)
+        cluster_plan(b["group_of"], b["sizes_q"], b["perm_q"], b["sizes_k"], c.n_valid, b["qmap"], b["qinv"],
+                     b["tile_list"], b["kc_off"], stream)
+        stage(4)
+        gather_rows(q, b["qmap"], b["q_rows"], 0, stream)
+        permute_rows(k, b["perm_k"], b["kp"], stream=stream)
+        permute_rows(v, b["perm_k"], b["vp"], stream=stream)
+        stage(5)
+        cluster_group_fwd(b["q_rows"], b["kp"], b["vp"], shape, b["tile_list"], b["kc_off"], b["sizes_k"],
+                          b["g_counts"], b["g_idx"], scale, b["o_rows"], b["lse_rows"], stream)
+        stage(6)
+        gather_rows(b["o_rows"], b["qinv"], b["o"], 0, stream)
+        gather_rows(b["lse_rows"], b["qinv"], b["lse"], 0xff800000, stream)
+        stage(7)
+        return b

@@ -9,7 +9,9 @@
  *   vsa_select_micro     Micro tiles inside omitted blocks          (Micro selection)
  *   vsa_block_sparse_fwd again on the Micro lists, merged by LSE    (Micro pass + merge)
  *   (vsa_block_sparse_fwd_heads: either pass on a subset of the heads)
- * and, for the cluster-permuted layout, vsa_cluster_tokens + vsa_permute_rows.
+ * and, for the cluster-permuted layout, vsa_cluster_tokens + vsa_permute_rows;
+ * for cluster-aligned blocks, vsa_select_clusters, vsa_merge_clusters,
+ * vsa_cluster_plan, vsa_gather_rows and vsa_cluster_group_fwd.
  * plus vsa_mask_to_lists (an explicit block mask instead of selection) and
  * vsa_lse_merge (the stand-alone exact merge).
  *
@@ -418,6 +420,75 @@ VSA_API vsa_status vsa_merge_clusters(const int32_t *sizes_q, const int32_t *siz
                                       int n_k, int rounds, int tau_q, int tau_k, void *workspace,
                                       size_t workspace_bytes, int32_t *group_of, int32_t *g_counts,
                                       int32_t *g_idx, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Cluster-aligned blocks: layout and attention ([HVA] section 2 Eq. (1), (4):
+ * attention runs on the cluster-permuted tokens and the output is put back in
+ * token order; section 4.3: each group of query clusters is one block row,
+ * executed in whole CTA tiles, its selected key clusters packed one after the
+ * other).
+ *
+ * Query rows: groups in ascending leader order; a group's rows are its member
+ * clusters in ascending order, each cluster's tokens in the order of the query
+ * permutation (vsa_cluster_tokens), padded with rows of zeros to a multiple of
+ * 128.  Key rows: the key permutation itself (clusters one after the other).
+ *
+ * vsa_cluster_rows_capacity: rows per head that the query layout can need,
+ * 128 * ceil((n_valid + 127 * n_q) / 128) (0 on invalid input).  Host only.
+ *
+ * vsa_cluster_plan (n_q, n_k <= 1024):
+ *   group_of : int32 [BH, n_q]  (vsa_merge_clusters; group_of[i] = i for no merging)
+ *   sizes_q  : int32 [BH, n_q];  perm_q : int32 [BH, n_pad]  (vsa_cluster_tokens of Q)
+ *   sizes_k  : int32 [BH, n_k]
+ *   n_rows   : rows per head of the query layout, a multiple of 128 (the capacity).
+ * Outputs:
+ *   qmap      int32 [BH, n_rows]      token of each layout row; -1 = padding row of
+ *             a group, -2 = row of an unused tile past the last group.
+ *   qinv      int32 [BH, n_pad]       layout row of each token; -1 at or past n_valid.
+ *   tile_list int32 [BH, n_rows/128]  group (leader) of each 128-row tile, -1 unused.
+ *   kc_off    int32 [BH, n_k]         first row of key cluster j in the key
+ *             permutation (the exclusive prefix sum of sizes_k).
+ * More rows needed than n_rows latches VSA_ERR_CAPACITY; a group_of entry that
+ * is not a leader, or a perm_q entry outside [0, n_valid), VSA_ERR_BAD_INDEX.
+ *
+ * vsa_gather_rows: dst[bh][i] = src[bh][map[bh][i]] for rows of row_bytes (a
+ * multiple of 4; 16-byte aligned buffers when a multiple of 16); map -1 writes
+ * the 32-bit word `fill` over the row, map -2 leaves the row untouched; any
+ * other entry outside [0, n_src) latches VSA_ERR_BAD_INDEX.  src [BH, n_src],
+ * dst [BH, n_dst]; the buffers must not overlap.  Used for Q -> query layout
+ * (qmap, fill 0) and for the output back to token order (qinv; fill 0 for O,
+ * 0xff800000 = -inf for LSE).
+ *
+ * vsa_cluster_group_fwd: attention of every query layout tile to the keys of
+ * its group's key clusters.
+ *   q_rows : bf16 [B, H, n_rows, d]  the query layout.
+ *   k, v   : bf16 [B, H, n_pad, d]   keys / values in the key permutation.
+ *   tile_list, kc_off : from vsa_cluster_plan;  kc_size : sizes_k.
+ *   counts, idx : int32 [BH, n_lists], [BH, n_lists, n_kc]: the key clusters of
+ *            each group at its leader's row, ascending (vsa_merge_clusters'
+ *            g_counts / g_idx, or vsa_select_clusters' lists without merging).
+ *   n_kc <= 2048.
+ *   o      : [B, H, n_rows, d] bf16 (o_fp32 = 0) or fp32;  lse : fp32 [B, H, n_rows].
+ * A key cluster is walked as 16-key segments, the last one partial; keys are
+ * rows [kc_off[j], kc_off[j] + kc_size[j]) of K and V.  Rows of unused tiles
+ * are not written; padding rows of a group are computed like any other row
+ * (zero queries) and are dropped by the gather back to token order.
+ * ------------------------------------------------------------------------- */
+VSA_API int vsa_cluster_rows_capacity(int n_valid, int n_q);
+
+VSA_API vsa_status vsa_cluster_plan(const int32_t *group_of, const int32_t *sizes_q, const int32_t *perm_q,
+                                    const int32_t *sizes_k, int batch_heads, int n_q, int n_k, int n_valid,
+                                    int n_pad, int n_rows, int32_t *qmap, int32_t *qinv, int32_t *tile_list,
+                                    int32_t *kc_off, void *stream);
+
+VSA_API vsa_status vsa_gather_rows(const void *src, const int32_t *map, int batch_heads, int n_src, int n_dst,
+                                   int row_bytes, uint32_t fill, void *dst, void *stream);
+
+VSA_API vsa_status vsa_cluster_group_fwd(const void *q_rows, const void *k, const void *v, const vsa_shape *shape,
+                                         int n_rows, const int32_t *tile_list, const int32_t *kc_off,
+                                         const int32_t *kc_size, int n_kc, const int32_t *counts,
+                                         const int32_t *idx, int n_lists, float scale, void *o, int o_fp32,
+                                         float *lse, void *stream);
 
 #ifdef __cplusplus
 }

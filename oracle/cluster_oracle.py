@@ -52,7 +52,7 @@ __all__ = [
     "cell_counts", "token_cells", "initial_centroids", "window_offsets", "window_cells",
     "local_window_clustering", "clustering_objective", "cluster_permutation", "permute_rows",
     "unpermute_rows", "forward_clustered", "select_clusters", "tile_cost", "merge_clusters", "total_cost",
-    "forward_cluster_blocks",
+    "forward_cluster_blocks", "attend_cluster_groups",
 ]
 
 
@@ -294,6 +294,26 @@ def total_cost(groups, sizes_q, sizes_k, kept, tau_q, tau_k) -> int:
     return tot
 
 
+def attend_cluster_groups(q, k, v, aq, ak, kept, groups, scale, O, L, only=None) -> None:
+    """C14 for one (batch, head): every query token of group S attends to the
+    key tokens of the clusters in chi(S) (Eq. (4) on the groups).  q, k, v
+    [N_pad, d]; aq, ak the token clusters [N_valid]; writes the rows of O
+    [N_pad, d] and L [N_pad] that belong to the groups (all, or the group
+    indices in ``only``)."""
+    from .vsa_oracle import attention_rows
+    for gi, g in enumerate(groups):
+        if only is not None and gi not in only:
+            continue
+        rows = np.nonzero(np.isin(aq, g))[0]
+        if rows.size == 0:
+            continue
+        sel = sorted(set().union(*[set(int(j) for j in kept[i]) for i in g]))
+        keys = np.nonzero(np.isin(ak, sel))[0]
+        o, lse = attention_rows(q[rows], k[keys], v[keys], scale)
+        O[rows] = o
+        L[rows] = lse
+
+
 def forward_cluster_blocks(q, k, v, n_valid, grid, cell, window, n_iter, scale, k_min, cum_mass, fixed_k,
                            tau_q=128, tau_k=128, sides=None) -> Dict[str, object]:
     """The cluster-aligned pipeline, per (batch, head): cluster Q and K
@@ -302,7 +322,7 @@ def forward_cluster_blocks(q, k, v, n_valid, grid, cell, window, n_iter, scale, 
     each query token to the keys of its group's selected clusters (C14).
     Returns O [B, H, N_pad, d], LSE [B, H, N_pad] in token order plus the
     per-head clusters, selections and groups."""
-    from .vsa_oracle import attention_rows, NEG_INF
+    from .vsa_oracle import NEG_INF
     B, H, n_pad, d = q.shape
     O = np.zeros((B, H, n_pad, d))
     L = np.full((B, H, n_pad), NEG_INF)
@@ -317,15 +337,7 @@ def forward_cluster_blocks(q, k, v, n_valid, grid, cell, window, n_iter, scale, 
             kept = select_clusters(muq, muk, sq, sk, scale, k_min, cum_mass, fixed_k)
             groups = merge_clusters(sq, sk, kept, tau_q, tau_k, sides[b][h]) if sides is not None else \
                 [[i] for i in range(G)]
-            for g in groups:
-                rows = np.nonzero(np.isin(aq, g))[0]
-                if rows.size == 0:
-                    continue
-                sel = sorted(set().union(*[set(int(j) for j in kept[i]) for i in g]))
-                keys = np.nonzero(np.isin(ak, sel))[0]
-                o, lse = attention_rows(q[b, h, rows], k[b, h, keys], v[b, h, keys], scale)
-                O[b, h, rows] = o
-                L[b, h, rows] = lse
+            attend_cluster_groups(q[b, h], k[b, h], v[b, h], aq, ak, kept, groups, scale, O[b, h], L[b, h])
             info.append({"assign_q": aq, "assign_k": ak, "mu_q": muq, "mu_k": muk, "sizes_q": sq, "sizes_k": sk,
                          "kept": kept, "groups": groups})
     return {"O": O, "LSE": L, "heads": info}

@@ -25,7 +25,7 @@ import block_sparse_attention_pool_b200 as vsa
 import oracle as orc
 from video_inputs import WORKLOADS, make_qkv
 
-from gpu_helpers import compare_selection, to_dev
+from gpu_helpers import assert_close_rows, compare_selection, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -232,3 +232,97 @@ def test_merge_clusters_rejects_bad_lists():
     vsa.merge_clusters(sq, sk, counts, idx, None, 16, 16, ws, outs[0], outs[1], g_idx)
     assert vsa.read_device_status() == 5
     assert outs[1][0, 0, 3].item() == 0
+
+
+def _run_cluster_blocks(w, heads, cell, window, iters, rule, rounds, taus=(128, 128)):
+    q, k, v = make_qkv(w, heads=heads)
+    H = q.shape[1]
+    k_min, cum_mass, fixed_k = rule
+    cfg = vsa.ClusterBlockConfig(n_valid=w.n_valid, lattice=w.grid, cell=cell, window=window, iters=iters,
+                                 scale=w.scale, k_min=k_min, cum_mass=cum_mass, fixed_k=fixed_k, rounds=rounds,
+                                 tau_q=taus[0], tau_k=taus[1])
+    G = vsa.cluster_count(cfg.cluster_params())
+    from video_inputs import merge_sides
+    sides = torch.from_numpy(merge_sides(w, rounds, G, heads)).cuda() if rounds else None
+    run = vsa.ClusterBlockAttention(cfg)
+    b = run(to_dev(q), to_dev(k), to_dev(v), sides=sides)
+    torch.cuda.synchronize()
+    assert vsa.read_device_status() == 0
+    host = {n: t.cpu() for n, t in b.items() if n not in ("q_rows", "kp", "vp", "o_rows", "merge_ws")}
+    return q, k, v, H, G, host, (None if sides is None else sides.cpu().numpy())
+
+
+def _groups_of(group_of_row):
+    groups = {}
+    for i, l in enumerate(group_of_row.tolist()):
+        groups.setdefault(l, []).append(i)
+    return [groups[l] for l in sorted(groups)]
+
+
+def _check_plan(h, w, G, host, groups):
+    """The query layout: every valid token on exactly one row, groups in
+    leader order, members ascending, each cluster in permutation order, 128-row
+    padding, tiles naming their group."""
+    qmap, qinv = host["qmap"][0, h].numpy(), host["qinv"][0, h].numpy()
+    tiles = host["tile_list"][0, h].numpy()
+    sq = host["sizes_q"][0, h].numpy()
+    perm = host["perm_q"][0, h].numpy()
+    off = np.concatenate([[0], np.cumsum(sq)])
+    row = 0
+    for g in groups:
+        n = int(sq[g].sum())
+        want = np.concatenate([perm[off[i]:off[i + 1]] for i in g]) if n else np.zeros(0, dtype=np.int64)
+        assert np.array_equal(qmap[row:row + n], want)
+        pad = -(-n // 128) * 128
+        assert np.all(qmap[row + n:row + pad] == -1)
+        assert np.all(tiles[row // 128:(row + pad) // 128] == min(g))
+        row += pad
+    assert np.all(qmap[row:] == -2) and np.all(tiles[row // 128:] == -1)
+    valid = qmap[qmap >= 0]
+    assert np.array_equal(np.sort(valid), np.arange(w.n_valid))
+    assert np.array_equal(qinv[valid], np.nonzero(qmap >= 0)[0])
+    assert np.all(qinv[w.n_valid:] == -1)
+    kc = host["kc_off"][0, h].numpy()
+    assert np.array_equal(kc, np.concatenate([[0], np.cumsum(host["sizes_k"][0, h].numpy())[:-1]]))
+
+
+@pytest.mark.parametrize("name,heads,cell,window,iters,rule,rounds,n_check", [
+    ("tiny", None, (2, 2, 2), (3, 3, 3), 2, (2, 0.9, 0), 3, None),
+    ("tiny", None, (1, 4, 3), (1, 2, 4), 2, (0, 0.0, 5), 0, None),      # no merging
+    ("tiny", None, (1, 1, 1), (1, 3, 3), 1, (1, 0.5, 0), 3, None),      # one-token clusters
+    ("wan13b", (3, 4), (3, 5, 8), (3, 5, 5), 3, (1, 0.95, 0), 3, 40),
+])
+def test_cluster_block_path_matches_the_oracle(name, heads, cell, window, iters, rule, rounds, n_check):
+    w = WORKLOADS[name]
+    q, k, v, H, G, host, sides = _run_cluster_blocks(w, heads, cell, window, iters, rule, rounds)
+    for h in range(H):
+        group_of = host["group_of"][0, h].numpy()
+        groups = _groups_of(group_of)
+        counts, idx = host["counts"][0, h].numpy(), host["idx"][0, h].numpy()
+        kept = [idx[i, :counts[i]].astype(np.int64) for i in range(G)]
+        # the merge on these lists is the oracle's
+        s = sides[0, h] if sides is not None else np.zeros((0, G), dtype=np.uint8)
+        assert [sorted(g) for g in groups] == orc.merge_clusters(host["sizes_q"][0, h].numpy(),
+                                                                 host["sizes_k"][0, h].numpy(), kept, 128, 128, s)
+        _check_plan(h, w, G, host, groups)
+        # attention: the oracle on the GPU's assignment, lists and groups
+        aq, ak = host["assign_q"][0, h].numpy(), host["assign_k"][0, h].numpy()
+        O = np.zeros((w.n_pad, w.d))
+        L = np.full(w.n_pad, -np.inf)
+        if n_check is None:
+            only = None
+        else:
+            rng = np.random.default_rng(7 + h)
+            only = set(rng.choice(len(groups), size=min(n_check, len(groups)), replace=False).tolist())
+            only |= {0, len(groups) - 1}
+        orc.attend_cluster_groups(q[0, h].astype(np.float64), k[0, h].astype(np.float64),
+                                  v[0, h].astype(np.float64), aq, ak, kept, groups, w.scale, O, L, only=only)
+        og = host["o"][0, h].float().numpy()
+        lg = host["lse"][0, h].numpy()
+        if only is None:
+            rows = np.arange(w.n_pad)
+        else:
+            rows = np.nonzero(np.isin(aq, [i for gi in only for i in groups[gi]]))[0]
+            rows = np.concatenate([rows, np.arange(w.n_valid, w.n_pad)])
+        assert_close_rows(og[None, None, rows], lg[None, None, rows], O[None, None, rows], L[None, None, rows],
+                          [(0, 0, 0, rows.size)], bf16_out=True)
