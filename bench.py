@@ -571,6 +571,120 @@ def run_cluster(args):
     print(json.dumps(line), flush=True)
 
 
+def run_cluster_blocks(args):
+    """Cluster-aligned blocks on the chosen workload (HyperVAttention Eq. (1)-
+    (5), (7)-(10), Algorithm 1): clustering, cluster-level selection, merging
+    of query clusters, the group layout, attention per group tile, and the
+    output back in token order, all on the device.  One JSON line: per-stage
+    times (CUDA events), the attention kernel's tensor throughput over the
+    tiles it executes, the cost model's CTA density and token density with
+    and without merging, and the relative L2 error against dense attention."""
+    import block_sparse_attention_pool_b200 as vsa
+    from block_sparse_attention_pool_b200 import build as vsa_build
+    from video_inputs import merge_sides
+    vsa_build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    q, k, v = make_qkv(w)
+    to_dev = lambda x: torch.from_numpy(x).to(dev).to(torch.bfloat16).contiguous()
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    del q, k, v
+    stream = torch.cuda.current_stream(dev)
+    B, H, n_pad, d = dq.shape
+    rule = dict(k_min=w.k_min, cum_mass=w.cum_mass, fixed_k=0)
+    if w.fixed_k:
+        rule = dict(k_min=0, cum_mass=0.0, fixed_k=w.fixed_k)
+    if args.cluster_cum_mass > 0:
+        rule = dict(k_min=1, cum_mass=args.cluster_cum_mass, fixed_k=0)
+    cfg = vsa.ClusterBlockConfig(n_valid=w.n_valid, lattice=w.grid, cell=args.cluster_cell,
+                                 window=args.cluster_window, iters=args.cluster_iters, scale=w.scale,
+                                 rounds=args.merge_rounds, **rule)
+    G = vsa.cluster_count(cfg.cluster_params())
+    if rule["fixed_k"]:
+        cfg.fixed_k = max(1, min(G, int(round(rule["fixed_k"] * G / (n_pad // w.bk)))))
+    sides = torch.from_numpy(merge_sides(w, args.merge_rounds, G)).to(dev) if args.merge_rounds else None
+    run = vsa.ClusterBlockAttention(cfg)
+    n_st = len(run.STAGES)
+
+    def step(ev):
+        run(dq, dk, dv, sides=sides, stream=stream, on_stage=lambda i: ev[i].record(stream))
+
+    evs = []
+    for i in range(args.warmup + args.steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_st + 1)]
+        step(ev)
+        if i >= args.warmup:
+            evs.append(ev)
+    torch.cuda.synchronize(dev)
+    st = vsa.read_device_status(stream)
+    if st != 0:
+        raise RuntimeError(vsa.status_string(st))
+    stages = {n: round(statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs), 4) for i, n in enumerate(run.STAGES)}
+    ms = statistics.mean(e[0].elapsed_time(e[n_st]) for e in evs)
+    b = run.buf
+
+    def densities(buf):
+        """Per head: groups' query tokens s_q(S), key tokens w_k(S), executed
+        128 x 128 tiles (16-key segments packed per group) -> token density,
+        CTA density of the cost model (Eq. (7)/(8)), executed tiles."""
+        sq = buf["sizes_q"].long()
+        sk = buf["sizes_k"].long()
+        gof = buf["group_of"].long()
+        cnt = buf["g_counts"].long()
+        Gn = sq.shape[-1]
+        valid = torch.arange(Gn, device=dev)[None, None, None, :] < cnt[..., None]
+        # only the first g_counts entries of a row are written: index 0 elsewhere
+        idx = torch.where(valid, buf["g_idx"].long(), 0).clamp(0, Gn - 1)
+        wk = (torch.gather(sk[:, :, None, :].expand(-1, -1, Gn, -1), 3, idx) * valid).sum(-1)
+        segs = (torch.gather(((sk + 15) // 16)[:, :, None, :].expand(-1, -1, Gn, -1), 3, idx) * valid).sum(-1)
+        gsq = torch.zeros_like(sq).scatter_add_(2, gof, sq)
+        lead = gof == torch.arange(Gn, device=dev)[None, None, :]
+        gsq, wk, segs = gsq * lead, wk * lead, segs * lead
+        nn = float(w.n_valid) ** 2 * B * H
+        tok = float((gsq * wk).sum()) / nn
+        cta = float((((gsq + 127) // 128) * ((wk + 127) // 128)).sum()) * 128 * 128 / nn
+        tiles = int((((gsq + 127) // 128) * ((segs * 16 + 127) // 128)).sum())
+        return tok, cta, tiles, int(lead.sum())
+
+    tok_m, cta_m, tiles_m, n_groups = densities(b)
+    o_merged = b["o"].float().clone()
+    # the same path without merging (every query cluster its own group)
+    run0 = vsa.ClusterBlockAttention(cfg)
+    run0(dq, dk, dv, sides=None, stream=stream)
+    torch.cuda.synchronize(dev)
+    tok_0, cta_0, tiles_0, _ = densities(run0.buf)
+    o_single = run0.buf["o"].float().clone()
+    del run0
+    dense = vsa.SparseVideoAttention(vsa.PathConfig(n_valid=w.n_valid, bq=w.bq, bk=w.bk, scale=w.scale,
+                                                    fixed_k=n_pad // w.bk))
+    o_ref = dense(dq, dk, dv)["o"].float()
+    nv = w.n_valid
+    rel = lambda o: float(torch.linalg.vector_norm(o[:, :, :nv] - o_ref[:, :, :nv]) /
+                          torch.linalg.vector_norm(o_ref[:, :, :nv]))
+    attn_ms = stages["attention"]
+    tile_flops = 4.0 * d * 128 * 128 * tiles_m
+    sizes = b["sizes_q"].float()
+    line = {
+        "metric": METRIC + " (cluster-aligned blocks)",
+        "value": round(tile_flops / (attn_ms * 1e-3) / 1e12, 3),
+        "unit": "TFLOP/s (attention kernel, executed 128x128 tiles)",
+        "ms_per_step": round(ms, 4),
+        "stages_ms": stages,
+        "config": {"workload": workload_label(w), "lattice": list(w.grid), "cell": list(args.cluster_cell),
+                   "window": list(args.cluster_window), "iters": args.cluster_iters, "rounds": args.merge_rounds,
+                   "tau": [cfg.tau_q, cfg.tau_k], "rule": {"k_min": cfg.k_min, "cum_mass": cfg.cum_mass,
+                                                           "fixed_k": cfg.fixed_k},
+                   "clusters_per_head": G, "groups_per_head_mean": round(n_groups / (B * H), 1),
+                   "cluster_size_mean_max": [round(float(sizes.mean()), 1), int(sizes.max())]},
+        "density": {"merged": {"token": round(tok_m, 4), "cta_cost_model": round(cta_m, 4), "tiles": tiles_m},
+                    "unmerged": {"token": round(tok_0, 4), "cta_cost_model": round(cta_0, 4), "tiles": tiles_0}},
+        "rel_l2_error_vs_dense": {"merged": round(rel(o_merged), 5), "unmerged": round(rel(o_single), 5)},
+        "data": "synthetic (seeded video-shaped Q/K/V, no model weights)",
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -587,6 +701,11 @@ def main():
     ap.add_argument("--cluster-cell", type=int, nargs=3, default=(3, 5, 8))
     ap.add_argument("--cluster-window", type=int, nargs=3, default=(3, 5, 5))
     ap.add_argument("--cluster-iters", type=int, default=3)
+    ap.add_argument("--cluster-blocks", action="store_true",
+                    help="print the cluster-aligned-blocks line (selection on clusters, merging, group tiles)")
+    ap.add_argument("--merge-rounds", type=int, default=3)
+    ap.add_argument("--cluster-cum-mass", type=float, default=0.0,
+                    help="cluster selection by cumulative mass instead of the workload's rule")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -597,6 +716,9 @@ def main():
         return
     if args.cluster:
         run_cluster(args)
+        return
+    if args.cluster_blocks:
+        run_cluster_blocks(args)
         return
     if args.impl == "reference":
         line = run_reference(args, rank, world)
