@@ -271,10 +271,18 @@ __device__ __forceinline__ float add_bf16x2_f32(float acc, uint32_t pk) {
   return acc;
 }
 
+// Taller K / V boxes of cluster-group mode: [0] 32 rows, [1] 64 rows (a run of
+// consecutive segments of one key cluster is contiguous in memory).
+struct alignas(64) GroupMaps {
+  CUtensorMap k[2];
+  CUtensorMap v[2];
+};
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ GroupMaps xm,
+                    const AttnArgs a) {
   using L = AttnSmem<D>;
   extern __shared__ uint8_t attn_smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(attn_smem_raw) + 1023) &
@@ -448,6 +456,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const bool cp_lane = lane < seg_per_stage * kNC;
       const uint32_t all = seg_per_stage == 8 ? 0xffffu : ((1u << (2 * seg_per_stage)) - 1u);
       const int g_shift = a.seg_shift - 4;  // 16-column groups per segment = 1 << g_shift
+      const int n_ent = ctl->n_ent;
+      int cur_e = 0, cur_k = 0;  // cluster-group mode: the next stage's first segment
       int issued = 0;
       for (int s = 0; s < n_stages; ++s) {
         const int slot = s & 1;
@@ -456,29 +466,50 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         int my_start = 0;
         uint32_t b0 = 0u, b1 = 0u;  // bit i: segment i used by query half 0 / 1
         uint32_t my_len4 = 0u;
+        int my_box = 1;  // segments covered by this lane's K / V box (0: inside another lane's box)
         if (groups) {
-          // segment g of the group's packed key stream: entry e with su[e-1] <= g < su[e]
+          // lane i < seg_per_stage: segment i of the stage, counted on from the stage's
+          // first segment (segment cur_k of entry cur_e); su[e] is the inclusive prefix
+          // of the entries' segment counts
           const int g = s * seg_per_stage + lane;
           const bool has = lane < seg_per_stage && g < n_seg;
-          int start = 0;
+          int e = cur_e, k = cur_k + lane, start = 0;
           if (has) {
-            const int n_ent = ctl->n_ent;
-            int lo = 0, hi = n_ent - 1;
-            while (lo < hi) {
-              const int mid = (lo + hi) >> 1;
-              if (static_cast<int>(su[mid]) > g) hi = mid;
-              else lo = mid + 1;
-            }
-            const int k = g - (lo > 0 ? static_cast<int>(su[lo - 1]) : 0);
             const int32_t *sl = reinterpret_cast<const int32_t *>(smem + L::kOffL);
-            start = sl[kListStage + lo] + 16 * k;
-            const int len = min(16, static_cast<int>(su[kListStage + lo]) - 16 * k);
+            for (;;) {
+              const int ns = static_cast<int>(su[e]) - (e > 0 ? static_cast<int>(su[e - 1]) : 0);
+              if (k < ns || e >= n_ent - 1) break;
+              k -= ns;
+              ++e;
+            }
+            start = sl[kListStage + e] + 16 * k;
+            const int len = min(16, static_cast<int>(su[kListStage + e]) - 16 * k);
             my_len4 = static_cast<uint32_t>(16 - len) << (4 * lane);
           }
+          cur_e = __shfl_sync(0xffffffffu, e, seg_per_stage - 1);
+          cur_k = __shfl_sync(0xffffffffu, k, seg_per_stage - 1) + 1;
           const int start0 = __shfl_sync(0xffffffffu, start, 0);
           my_start = has ? start : start0;
           b0 = b1 = __ballot_sync(0xffffffffu, has);
           my_len4 = __reduce_or_sync(0xffffffffu, my_len4);
+          // runs of consecutive segments of one entry are contiguous rows: cover each
+          // run greedily with 64-, 32- and 16-row boxes
+          const int e_up = __shfl_up_sync(0xffffffffu, e, 1), k_up = __shfl_up_sync(0xffffffffu, k, 1);
+          const uint32_t cont = __ballot_sync(0xffffffffu, has && lane > 0 && e_up == e && k_up + 1 == k);
+          const uint32_t starts = b0 & ~cont;
+          if (has) {
+            const uint32_t upto = (2u << lane) - 1u;
+            const int rs = 31 - __clz(starts & upto);
+            const uint32_t enders = ((starts | ~b0) & ~upto) | (1u << seg_per_stage);
+            const int re = __ffs(enders) - 1;
+            const int run = re - rs, p = lane - rs, n64 = run >> 2;
+            if (p < 4 * n64) {
+              my_box = (p & 3) == 0 ? 4 : 0;
+            } else {
+              const int q = p - 4 * n64, rem = run - 4 * n64;
+              my_box = rem >= 2 ? (q == 0 ? 2 : (q == 2 ? 1 : 0)) : (q == 0 ? 1 : 0);
+            }
+          }
         } else if (fast) {
           const int e = s * seg_per_stage + lane;
           const bool has = lane < seg_per_stage && e < n_seg;
@@ -509,9 +540,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                  : __any_sync(0xffffffffu, lane < seg_per_stage && ((used >> lane) & 1u) &&
                                                                my_start + a.seg_keys > a.n_valid);
         uint32_t mask = 0u, use16 = 0u;
-        for (int i = 0; i < seg_per_stage; ++i) mask |= (((b0 >> i) & 1u) << (2 * i)) | (((b1 >> i) & 1u) << (2 * i + 1));
-        for (int q = 0; q < 8; ++q)
-          use16 |= (((b0 >> (q >> g_shift)) & 1u) << q) | (((b1 >> (q >> g_shift)) & 1u) << (8 + q));
+        if (groups) {
+          // both halves use every segment: spread bit i of b0 to bits 2i, 2i + 1
+          uint32_t x = b0 & 0xffu;
+          x = (x | (x << 4)) & 0x0f0fu;
+          x = (x | (x << 2)) & 0x3333u;
+          x = (x | (x << 1)) & 0x5555u;
+          mask = x | (x << 1);
+          use16 = (b0 & 0xffu) | ((b0 & 0xffu) << 8);
+        } else {
+          for (int i = 0; i < seg_per_stage; ++i)
+            mask |= (((b0 >> i) & 1u) << (2 * i)) | (((b1 >> i) & 1u) << (2 * i + 1));
+          for (int q = 0; q < 8; ++q)
+            use16 |= (((b0 >> (q >> g_shift)) & 1u) << q) | (((b1 >> (q >> g_shift)) & 1u) << (8 + q));
+        }
         const bool full = mask == all && !tail;
         bool ok = true;
         if (s >= 2) ok = mbar_wait_warp(&ctl->k_empty[slot], use_par, abort, a.timeout_ns, lane);
@@ -533,15 +575,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         __syncwarp();
         const int cp_row = __shfl_sync(0xffffffffu, my_start, cp_seg);
+        const int cp_box = __shfl_sync(0xffffffffu, my_box, cp_seg);
         const uint32_t cp_off = cp_chunk * kChunkBytes + cp_seg * a.seg_keys * 128;
-        if (cp_lane)
-          tma_load_3d(sK + slot * L::kKVBytes + cp_off, &tm_k, &ctl->k_full[slot], cp_chunk * 64, cp_row, bh);
+        const CUtensorMap *map_k = cp_box == 4 ? &xm.k[1] : (cp_box == 2 ? &xm.k[0] : &tm_k);
+        const CUtensorMap *map_v = cp_box == 4 ? &xm.v[1] : (cp_box == 2 ? &xm.v[0] : &tm_v);
+        if (cp_lane && cp_box > 0)
+          tma_load_3d(sK + slot * L::kKVBytes + cp_off, map_k, &ctl->k_full[slot], cp_chunk * 64, cp_row, bh);
         if (s >= 2) ok = mbar_wait_warp(&ctl->v_empty[slot], use_par, abort, a.timeout_ns, lane);
         if (!ok) break;
         if (lane == 0) mbar_arrive_expect_tx(&ctl->v_full[slot], L::kKVBytes);
         __syncwarp();
-        if (cp_lane)
-          tma_load_3d(sV + slot * L::kKVBytes + cp_off, &tm_v, &ctl->v_full[slot], cp_chunk * 64, cp_row, bh);
+        if (cp_lane && cp_box > 0)
+          tma_load_3d(sV + slot * L::kKVBytes + cp_off, map_v, &ctl->v_full[slot], cp_chunk * 64, cp_row, bh);
         issued = s + 1;
         __syncwarp();
       }
@@ -627,17 +672,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tSg + lane_off + c * 32, r[c]);
       tmem_ld_wait();
-      if (!inf.full && !inf.tail) {
-        // segments wholly inside n_valid: this half's used 16-column groups
-        const uint32_t u = inf.use16 >> (8 * half);
+      if (!inf.full && (!inf.tail || groups)) {
+        // whole 16-column groups this half does not use
+        const uint32_t u = (inf.use16 >> (8 * half)) & 0xffu;
+        if (u != 0xffu) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const bool drop = !((u >> q) & 1u);
+          for (int q = 0; q < 8; ++q) {
+            const bool drop = !((u >> q) & 1u);
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (drop) r[q >> 1][(q & 1) * 16 + j] = __float_as_uint(-INFINITY);
+            for (int j = 0; j < 16; ++j)
+              if (drop) r[q >> 1][(q & 1) * 16 + j] = __float_as_uint(-INFINITY);
+          }
         }
-      } else if (!inf.full) {
+      }
+      if (!inf.full && inf.tail && groups) {
+        // partial segments (the last one of a key cluster): columns past its valid keys
+        uint32_t part = inf.len4;
+        while (part != 0u) {
+          const int sg = (__ffs(part) - 1) >> 2;
+          const int nv = 16 - static_cast<int>((part >> (4 * sg)) & 15u);
+          part &= ~(0xfu << (4 * sg));
+          switch (sg) {
+#define VSA_MASK_SEG(K)                                                                      \
+  case K: {                                                                                  \
+    _Pragma("unroll") for (int j = 0; j < 16; ++j) if (j >= nv) r[(K) >> 1][((K) & 1) * 16 + j] = \
+        __float_as_uint(-INFINITY);                                                          \
+  } break;
+            VSA_MASK_SEG(0)
+            VSA_MASK_SEG(1)
+            VSA_MASK_SEG(2)
+            VSA_MASK_SEG(3)
+            VSA_MASK_SEG(4)
+            VSA_MASK_SEG(5)
+            VSA_MASK_SEG(6)
+            VSA_MASK_SEG(7)
+#undef VSA_MASK_SEG
+            default: break;
+          }
+        }
+      } else if (!inf.full && inf.tail) {
         // a segment reaches past n_valid: valid columns as a 128-bit mask built
         // per segment (a used segment's valid keys form one prefix of it)
         uint64_t vm[2] = {0ull, 0ull};
@@ -646,8 +719,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll 1
         for (int sg = 0; sg < nseg; ++sg) {
           if (!((mask >> (2 * sg + half)) & 1u)) continue;
-          const int nv = groups ? 16 - static_cast<int>((inf.len4 >> (4 * sg)) & 15u)
-                                : min(a.seg_keys, max(0, a.n_valid - inf.start[sg]));
+          const int nv = min(a.seg_keys, max(0, a.n_valid - inf.start[sg]));
           const int lo = sg * a.seg_keys, hi = lo + nv;
 #pragma unroll
           for (int w = 0; w < 2; ++w) {

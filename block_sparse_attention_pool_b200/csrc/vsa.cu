@@ -119,10 +119,13 @@ vsa_status launch_attn_groups(const void *q, const void *k, const void *v, const
   if (set_attn_smem<D>() != VSA_OK) return VSA_ERR_CUDA;
   const int BH = s->B * s->H;
   CUtensorMap mq, mk, mv;
-  if (!make_map_rows(&mq, q, a.n_rows_q, D, BH, vsa::kTileM) || !make_map(&mk, k, s, 16) || !make_map(&mv, v, s, 16))
+  vsa::GroupMaps xm;
+  if (!make_map_rows(&mq, q, a.n_rows_q, D, BH, vsa::kTileM) || !make_map(&mk, k, s, 16) || !make_map(&mv, v, s, 16) ||
+      !make_map(&xm.k[0], k, s, 32) || !make_map(&xm.k[1], k, s, 64) || !make_map(&xm.v[0], v, s, 32) ||
+      !make_map(&xm.v[1], v, s, 64))
     return VSA_ERR_CUDA;
   dim3 grid(a.n_tiles, BH);
-  vsa::attn_fwd_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, a);
+  vsa::attn_fwd_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, xm, a);
   return launch_status();
 }
 
@@ -140,7 +143,10 @@ vsa_status launch_attn(const void *q, const void *k, const void *v, const vsa_sh
   if (!make_map(&mq, q, s, vsa::kTileM) || !make_map(&mk, k, s, a.seg_keys) || !make_map(&mv, v, s, a.seg_keys))
     return VSA_ERR_CUDA;
   dim3 grid(s->n_pad / vsa::kTileM, n_heads);
-  vsa::attn_fwd_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, a);
+  vsa::GroupMaps xm;  // unused outside cluster-group mode
+  xm.k[0] = xm.k[1] = mk;
+  xm.v[0] = xm.v[1] = mv;
+  vsa::attn_fwd_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, xm, a);
   return launch_status();
 }
 
