@@ -6,3 +6,4 @@ calls into it and it shares no code with the CUDA library.
 """
 from .vsa_oracle import *  # noqa: F401,F403
 from .cluster_oracle import *  # noqa: F401,F403
+from .rectify_oracle import *  # noqa: F401,F403
