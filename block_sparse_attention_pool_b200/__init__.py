@@ -28,6 +28,7 @@ __all__ = [
     "PathConfig", "SparseVideoAttention", "ClusterParams", "cluster_count", "cluster_tokens", "permute_rows",
     "select_clusters", "merge_clusters", "merge_clusters_workspace_bytes", "cluster_rows_capacity", "cluster_plan",
     "gather_rows", "cluster_group_fwd", "ClusterBlockConfig", "ClusterBlockAttention",
+    "pool_kv_bf16", "rectify_fwd",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -39,7 +40,7 @@ EXPORTED = (
     "vsa_block_sparse_fwd", "vsa_block_sparse_fwd_heads", "vsa_lse_merge", "vsa_selftest_wait_timeout",
     "vsa_cluster_count", "vsa_cluster_tokens", "vsa_permute_rows", "vsa_select_clusters",
     "vsa_merge_clusters_workspace_bytes", "vsa_merge_clusters", "vsa_cluster_rows_capacity", "vsa_cluster_plan",
-    "vsa_gather_rows", "vsa_cluster_group_fwd",
+    "vsa_gather_rows", "vsa_cluster_group_fwd", "vsa_pool_kv_bf16", "vsa_rectify_fwd",
 )
 
 STATUS = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_UNSUPPORTED", 3: "VSA_ERR_CUDA",
@@ -143,6 +144,10 @@ def lib():
     L.vsa_gather_rows.argtypes = [P, P, I, I, I, I, ctypes.c_uint32, P, P]
     L.vsa_cluster_group_fwd.restype = I
     L.vsa_cluster_group_fwd.argtypes = [P, P, P, SP, I, P, P, P, I, P, P, I, F, P, I, P, P]
+    L.vsa_pool_kv_bf16.restype = I
+    L.vsa_pool_kv_bf16.argtypes = [P, P, SP, I, I, P, P, P]
+    L.vsa_rectify_fwd.restype = I
+    L.vsa_rectify_fwd.argtypes = [P, P, P, SP, I, I, I, P, P, I, F, P, P, P, I, P, P, I, P]
     L.vsa_select_clusters.argtypes = [P, P, P, P, I, I, I, I, F, ctypes.POINTER(SelectParams), P, P, P]
     _lib = L
     return L
@@ -260,6 +265,25 @@ def cluster_group_fwd(q_rows, k, v, shape: Shape, tile_list, kc_off, kc_size, co
                                        _p(lse), _s(stream)), "vsa_cluster_group_fwd")
 
 
+def pool_kv_bf16(k, v, shape: Shape, bk, k_bar, v_bar, stream=None):
+    """bf16 block means of K and V: k_bar, v_bar [B, H, n_rows, d]."""
+    _check(lib().vsa_pool_kv_bf16(_p(k), _p(v), ctypes.byref(shape), bk, k_bar.shape[2], _p(k_bar), _p(v_bar),
+                                  _s(stream)), "vsa_pool_kv_bf16")
+
+
+def rectify_fwd(q, k_bar, v_bar, shape: Shape, bq, bk, counts, idx, idx_stride, scale, o, lse, merge_o=None,
+                merge_lse=None, heads=None, stream=None):
+    """Pooled pass over the omitted blocks, merged into (merge_o, merge_lse)."""
+    if heads is None:
+        hp, nh = None, shape.B * shape.H
+    else:
+        hp, nh = _p(heads), heads.numel()
+    _check(lib().vsa_rectify_fwd(_p(q), _p(k_bar), _p(v_bar), ctypes.byref(shape), bq, bk, k_bar.shape[2],
+                                 _p(counts), _p(idx), idx_stride, float(scale), _p(merge_o), _p(merge_lse), _p(o),
+                                 1 if o.dtype == torch.float32 else 0, _p(lse), hp, nh, _s(stream)),
+           "vsa_rectify_fwd")
+
+
 def mask_to_lists(mask, shape: Shape, bq, bk, counts, idx, stream=None):
     _check(lib().vsa_mask_to_lists(_p(mask), ctypes.byref(shape), bq, bk, _p(counts), _p(idx), _s(stream)),
            "vsa_mask_to_lists")
@@ -366,6 +390,9 @@ class PathConfig:
     micro_percentile: float = 0.0
     micro_heads: Optional[Sequence[int]] = None
     micro_capacity: int = 0          # 0: every tile of the row fits (no overflow possible)
+    # pooled rectification of the omitted blocks (Rectified SpaAttn; replaces the Micro repair)
+    rectify: bool = False
+    rectify_heads: Optional[Sequence[int]] = None   # per-head flags; None = every head
     # cluster-permuted layout (HyperVAttention Eq. (1), (4), (5)): None = tokens in their own order
     cluster_lattice: Optional[Sequence[int]] = None   # (T, H, W) with T*H*W == n_valid
     cluster_cell: Sequence[int] = (3, 5, 8)
@@ -431,6 +458,16 @@ class SparseVideoAttention:
                 "workspace": torch.empty(max(16, ws), device=dev, dtype=torch.uint8),
             })
             self.micro_cap = cap
+        if c.rectify:
+            if c.micro_mode:
+                raise ValueError("rectification replaces the Micro repair: set micro_mode = 0")
+            n_rows = -(-n_k // 128) * 128
+            b.update({
+                "k_bar": torch.empty(B, H, n_rows, d, device=dev, dtype=torch.bfloat16),
+                "v_bar": torch.empty(B, H, n_rows, d, device=dev, dtype=torch.bfloat16),
+                "o_macro": torch.empty(B, H, n_pad, d, device=dev, dtype=f32),
+                "lse_macro": torch.empty(B, H, n_pad, device=dev, dtype=f32),
+            })
         if c.cluster_lattice is not None:
             G = cluster_count(c.cluster_params())
             if G <= 0:
@@ -452,8 +489,9 @@ class SparseVideoAttention:
         self._key = key
 
     def _head_split(self, B: int, H: int, flags, dev):
-        """Device index lists (b*H + h) of the heads without and with the Micro
-        repair; None stands for "every head", an empty tuple for "no head"."""
+        """Device index lists (b*H + h) of the heads without and with the
+        repair (Micro or rectification); None stands for "every head", an empty
+        tuple for "no head"."""
         key = (B, H, None if flags is None else tuple(int(f) for f in flags), dev)
         cache = self.__dict__.setdefault("_splits", {})
         if key not in cache:
@@ -461,7 +499,7 @@ class SparseVideoAttention:
                 cache[key] = ((), None)
             else:
                 if len(flags) != H:
-                    raise ValueError(f"micro_heads has {len(flags)} flags for {H} heads")
+                    raise ValueError(f"{len(flags)} head flags for {H} heads")
                 rep = [b * H + h for b in range(B) for h in range(H) if flags[h]]
                 plain = [b * H + h for b in range(B) for h in range(H) if not flags[h]]
                 as_dev = lambda x: torch.tensor(x, dtype=torch.int32, device=dev) if x else ()
@@ -530,6 +568,24 @@ class SparseVideoAttention:
                       SelectParams(c.k_min, c.cum_mass, c.fixed_k, c.n_anchor, c.anchor_rot), b["counts"], b["idx"],
                       None, stream)
         stage(2)
+        if c.rectify:
+            # kept blocks exactly (Macro), then the omitted blocks as pooled keys, merged by LSE
+            plain, rep = self._head_split(B, H, c.rectify_heads, q.device)
+            if not isinstance(plain, tuple):
+                block_sparse_fwd(q, k, v, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, scale, o, lse,
+                                 stream=stream, heads=plain)
+            if not isinstance(rep, tuple):
+                block_sparse_fwd(q, k, v, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, scale, b["o_macro"],
+                                 b["lse_macro"], stream=stream, heads=rep)
+            stage(3)
+            if not isinstance(rep, tuple):
+                pool_kv_bf16(k, v, shape, c.bk, b["k_bar"], b["v_bar"], stream)
+            stage(4)
+            if not isinstance(rep, tuple):
+                rectify_fwd(q, b["k_bar"], b["v_bar"], shape, c.bq, c.bk, b["counts"], b["idx"], n_k, scale, o, lse,
+                            b["o_macro"], b["lse_macro"], heads=rep, stream=stream)
+            stage(5)
+            return b
         if not micro:
             block_sparse_fwd(q, k, v, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, scale, o, lse, stream=stream)
             stage(3)

@@ -90,6 +90,12 @@ struct AttnArgs {
   const int32_t *kc_off;     // [BH][n_kc]
   const int32_t *kc_size;    // [BH][n_kc]
   int n_kc, n_lists_bh, n_tiles, n_rows_q;
+  // Pooled-rectification mode (pool_nk > 0; seg_keys 128): the keys are the bf16
+  // means of the pool_nk key blocks (K / V maps of pooled rows), key block j
+  // weighted by its valid key count s_j = clamp(pool_nvalid - j * pool_bk, 0,
+  // pool_bk); the lists (counts / idx, list_rows query rows each) name the kept
+  // blocks, which this pass skips.
+  int pool_nk, pool_bk, pool_nvalid;
 };
 
 struct StageInfo {
@@ -305,6 +311,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const bool groups = a.tile_list != nullptr;
+  const bool pooled = a.pool_nk > 0;
   int group_row = 0;
   if (groups) {
     group_row = __ldg(a.tile_list + (size_t)bh * a.n_tiles + tile);
@@ -360,7 +367,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     const bool fast = ok && cnt[0] <= kListStage && cnt[1] <= kListStage;
     int n_seg = 0;
-    if (groups) {
+    if (pooled) {
+      // kept-block bitmaps of the tile's query blocks (one per list) in shared memory
+      uint32_t *sb = reinterpret_cast<uint32_t *>(smem + L::kOffL);
+      sb[lane] = 0u;
+      sb[32 + lane] = 0u;
+      __syncwarp();
+      for (int h = 0; h < n_lists && ok; ++h) {
+        const int32_t *li = a.idx + (lrow0 + h) * a.idx_stride;
+        for (int e = lane; e < cnt[h]; e += 32) {
+          const int j = __ldg(li + e);
+          if (j < 0 || j >= a.pool_nk) ok = false;
+          else atomicOr(&sb[h * 32 + (j >> 5)], 1u << (j & 31));
+        }
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      __syncwarp();
+      n_seg = ok ? (a.pool_nk + kStageKeys - 1) / kStageKeys : 0;
+    } else if (groups) {
       // the group's key clusters: ids at sl[e], first rows at sl[kListStage + e],
       // sizes at su[kListStage + e], inclusive prefix of their 16-key segment counts at su[e]
       int32_t *sl = reinterpret_cast<int32_t *>(smem + L::kOffL);
@@ -467,7 +491,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         uint32_t b0 = 0u, b1 = 0u;  // bit i: segment i used by query half 0 / 1
         uint32_t my_len4 = 0u;
         int my_box = 1;  // segments covered by this lane's K / V box (0: inside another lane's box)
-        if (groups) {
+        if (pooled) {
+          my_start = s * kStageKeys;
+          b0 = b1 = 1u;
+        } else if (groups) {
           // lane i < seg_per_stage: segment i of the stage, counted on from the stage's
           // first segment (segment cur_k of entry cur_e); su[e] is the inclusive prefix
           // of the entries' segment counts
@@ -536,7 +563,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
         const uint32_t used = b0 | b1;
-        const bool tail = groups ? my_len4 != 0u
+        const bool tail = pooled ? false
+                        : groups ? my_len4 != 0u
                                  : __any_sync(0xffffffffu, lane < seg_per_stage && ((used >> lane) & 1u) &&
                                                                my_start + a.seg_keys > a.n_valid);
         uint32_t mask = 0u, use16 = 0u;
@@ -554,7 +582,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int q = 0; q < 8; ++q)
             use16 |= (((b0 >> (q >> g_shift)) & 1u) << q) | (((b1 >> (q >> g_shift)) & 1u) << (8 + q));
         }
-        const bool full = mask == all && !tail;
+        const bool full = pooled || (mask == all && !tail);
         bool ok = true;
         if (s >= 2) ok = mbar_wait_warp(&ctl->k_empty[slot], use_par, abort, a.timeout_ns, lane);
         if (!ok) break;
@@ -660,7 +688,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float l = 0.f;         // sum of P (fp32) over this group's stages
     float lr = 0.f;        // sum of the bf16-rounded P over this group's stages
     bool ok = true;
-    const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+    const float sl2 = pooled ? 1.f : a.scale_log2;  // pooled logits arrive scaled
+    const float2 sc2 = make_float2(sl2, sl2);
     for (int t = g; t < n_stages; t += 2) {
       ok = mbar_wait_warp(&ctl->info_full[t & (kInfoRing - 1)], (t >> 2) & 1, abort, a.timeout_ns, lane);
       if (ok) ok = mbar_wait_warp(&ctl->s_full[g], (t >> 1) & 1, abort, a.timeout_ns, lane);
@@ -736,6 +765,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int j = 0; j < 32; ++j)
             if (!((vm[c >> 1] >> ((c & 1) * 32 + j)) & 1ull)) r[c][j] = __float_as_uint(-INFINITY);
       }
+      if (pooled) {
+        // logit * scale * log2(e) + log2(s_j), -inf for kept blocks and blocks without keys
+        const uint32_t *sb = reinterpret_cast<const uint32_t *>(smem + L::kOffL) + (n_lists > 1 ? half * 32 : 0);
+        const uint32_t w4[4] = {sb[4 * t], sb[4 * t + 1], sb[4 * t + 2], sb[4 * t + 3]};
+        const int n_full = a.pool_nvalid / a.pool_bk, rem = a.pool_nvalid - n_full * a.pool_bk;
+        const int lim = n_full - kStageKeys * t;  // columns below lim are full-size blocks
+        const float lb = log2f(static_cast<float>(a.pool_bk));
+        const float lr = rem > 0 ? log2f(static_cast<float>(rem)) : -INFINITY;
+        if (lim >= kStageKeys) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              r[c][j] = ((w4[c] >> j) & 1u) ? __float_as_uint(-INFINITY)
+                                            : __float_as_uint(fmaf(__uint_as_float(r[c][j]), a.scale_log2, lb));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int col = 32 * c + j;
+              const float b = col < lim ? lb : (col == lim ? lr : -INFINITY);
+              r[c][j] = ((w4[c] >> j) & 1u) ? __float_as_uint(-INFINITY)
+                                            : __float_as_uint(fmaf(__uint_as_float(r[c][j]), a.scale_log2, b));
+            }
+        }
+      }
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
@@ -743,7 +799,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mx[(j + 2) & 3] = max3f(mx[(j + 2) & 3], __uint_as_float(r[2][j]), __uint_as_float(r[3][j]));
       }
       const float rmax = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3]));
-      const float m_new = fmaxf(m2, rmax * a.scale_log2);
+      const float m_new = fmaxf(m2, rmax * sl2);
       const bool need = m_new > m2 + kRescaleThreshold || (m2 == -INFINITY && m_new != -INFINITY);
       const bool any_rescale = __any_sync(0xffffffffu, need);
       float alpha = 1.f;

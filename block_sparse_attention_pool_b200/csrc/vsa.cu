@@ -25,6 +25,7 @@
 #include "merge.cuh"
 #include "micro.cuh"
 #include "pool.cuh"
+#include "rectify.cuh"
 #include "select.cuh"
 
 namespace {
@@ -125,6 +126,26 @@ vsa_status launch_attn_groups(const void *q, const void *k, const void *v, const
       !make_map(&xm.v[1], v, s, 64))
     return VSA_ERR_CUDA;
   dim3 grid(a.n_tiles, BH);
+  vsa::attn_fwd_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, xm, a);
+  return launch_status();
+}
+
+// Pooled-rectification pass: Q tiles of the layer, keys = the n_rows pooled rows
+// ([BH][n_rows][d], the first n_k holding block means), 128-row boxes.
+template <int D>
+vsa_status launch_attn_pooled(const void *q, const void *kb, const void *vb, const vsa_shape *s, int n_rows,
+                              const AttnArgs &a, int n_heads, cudaStream_t st) {
+  using L = vsa::AttnSmem<D>;
+  if (set_attn_smem<D>() != VSA_OK) return VSA_ERR_CUDA;
+  const int BH = s->B * s->H;
+  CUtensorMap mq, mk, mv;
+  vsa::GroupMaps xm;
+  if (!make_map(&mq, q, s, vsa::kTileM) || !make_map_rows(&mk, kb, n_rows, D, BH, vsa::kStageKeys) ||
+      !make_map_rows(&mv, vb, n_rows, D, BH, vsa::kStageKeys))
+    return VSA_ERR_CUDA;
+  xm.k[0] = xm.k[1] = mk;
+  xm.v[0] = xm.v[1] = mv;
+  dim3 grid(s->n_pad / vsa::kTileM, n_heads);
   vsa::attn_fwd_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, xm, a);
   return launch_status();
 }
@@ -894,6 +915,68 @@ vsa_status vsa_cluster_group_fwd(const void *q_rows, const void *k, const void *
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return shape->d == 128 ? launch_attn_groups<128>(q_rows, k, v, shape, a, st)
                          : launch_attn_groups<64>(q_rows, k, v, shape, a, st);
+}
+
+vsa_status vsa_pool_kv_bf16(const void *k, const void *v, const vsa_shape *shape, int bk, int n_rows, void *k_bar,
+                            void *v_bar, void *stream) {
+  if (!shape_ok(shape) || !k || !v || !k_bar || !v_bar) return VSA_ERR_INVALID_ARG;
+  if (bk != 64 && bk != 128) return VSA_ERR_INVALID_ARG;
+  if (n_rows < shape->n_pad / bk || n_rows % 128 != 0) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_bar) || !aligned16(v_bar)) return VSA_ERR_INVALID_ARG;
+  dim3 grid(n_rows, shape->B * shape->H, 2);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const __nv_bfloat16 *kb = static_cast<const __nv_bfloat16 *>(k), *vb = static_cast<const __nv_bfloat16 *>(v);
+  __nv_bfloat16 *ko = static_cast<__nv_bfloat16 *>(k_bar), *vo = static_cast<__nv_bfloat16 *>(v_bar);
+  if (shape->d == 128)
+    vsa::pool_kv_bf16_kernel<128><<<grid, vsa::kPoolBfThreads, 0, st>>>(kb, vb, shape->n_pad, shape->n_valid, bk,
+                                                                        n_rows, ko, vo);
+  else
+    vsa::pool_kv_bf16_kernel<64><<<grid, vsa::kPoolBfThreads, 0, st>>>(kb, vb, shape->n_pad, shape->n_valid, bk,
+                                                                       n_rows, ko, vo);
+  return launch_status();
+}
+
+vsa_status vsa_rectify_fwd(const void *q, const void *k_bar, const void *v_bar, const vsa_shape *shape, int bq,
+                           int bk, int n_rows, const int32_t *counts, const int32_t *idx, int idx_stride,
+                           float scale, const float *merge_o, const float *merge_lse, void *o, int o_fp32,
+                           float *lse, const int32_t *heads, int n_heads, void *stream) {
+  if (!shape_ok(shape) || !q || !k_bar || !v_bar || !counts || !idx || !o || !lse) return VSA_ERR_INVALID_ARG;
+  const long long n_bh = (long long)shape->B * shape->H;
+  if (n_heads < 0 || n_heads > n_bh || (heads == nullptr && n_heads != n_bh)) return VSA_ERR_INVALID_ARG;
+  if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return VSA_ERR_INVALID_ARG;
+  const int n_k = shape->n_pad / bk;
+  if (n_k > 1024) return VSA_ERR_UNSUPPORTED;
+  if (n_rows < n_k || n_rows % 128 != 0 || idx_stride < 1) return VSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return VSA_ERR_INVALID_ARG;
+  if ((merge_o == nullptr) != (merge_lse == nullptr)) return VSA_ERR_INVALID_ARG;
+  if (merge_o && static_cast<const void *>(merge_o) == o) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_bar) || !aligned16(v_bar) || !aligned16(o) || (merge_o && !aligned16(merge_o)))
+    return VSA_ERR_INVALID_ARG;
+  AttnArgs a{};
+  a.n_pad = shape->n_pad;
+  a.n_valid = shape->n_valid;
+  a.list_rows = bq;
+  a.seg_keys = 128;
+  a.seg_shift = 7;
+  a.idx_stride = idx_stride;
+  a.counts = counts;
+  a.idx = idx;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.o = o;
+  a.o_fp32 = o_fp32 ? 1 : 0;
+  a.lse = lse;
+  a.merge_o = merge_o;
+  a.merge_lse = merge_lse;
+  a.heads = heads;
+  a.n_bh = static_cast<int>(n_bh);
+  a.timeout_ns = kWaitLimitNs;
+  a.pool_nk = n_k;
+  a.pool_bk = bk;
+  a.pool_nvalid = shape->n_valid;
+  if (n_heads == 0) return VSA_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return shape->d == 128 ? launch_attn_pooled<128>(q, k_bar, v_bar, shape, n_rows, a, n_heads, st)
+                         : launch_attn_pooled<64>(q, k_bar, v_bar, shape, n_rows, a, n_heads, st);
 }
 
 }  // extern "C"

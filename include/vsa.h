@@ -11,7 +11,8 @@
  *   (vsa_block_sparse_fwd_heads: either pass on a subset of the heads)
  * and, for the cluster-permuted layout, vsa_cluster_tokens + vsa_permute_rows;
  * for cluster-aligned blocks, vsa_select_clusters, vsa_merge_clusters,
- * vsa_cluster_plan, vsa_gather_rows and vsa_cluster_group_fwd.
+ * vsa_cluster_plan, vsa_gather_rows and vsa_cluster_group_fwd; for pooled
+ * rectification of omitted blocks, vsa_pool_kv_bf16 + vsa_rectify_fwd.
  * plus vsa_mask_to_lists (an explicit block mask instead of selection) and
  * vsa_lse_merge (the stand-alone exact merge).
  *
@@ -489,6 +490,42 @@ VSA_API vsa_status vsa_cluster_group_fwd(const void *q_rows, const void *k, cons
                                          const int32_t *kc_size, int n_kc, const int32_t *counts,
                                          const int32_t *idx, int n_lists, float scale, void *o, int o_fp32,
                                          float *lse, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Pooled rectification of omitted blocks ([RSA] abstract: sparse attention
+ * amplifies the kept keys' weights and drops the omitted keys' weight; both
+ * are rectified from pooled query-key interactions).  Readings (the page has
+ * no formulas): an omitted key block j of query block i stands for s_j copies
+ * of its mean key and mean value, s_j its valid key count; every query row of
+ * block i gets s_j exp(scale q.kbar_j) vbar_j in the numerator and
+ * s_j exp(scale q.kbar_j) in the denominator of its softmax, which the kept
+ * keys share, so their weights are no longer amplified.  Every omitted block
+ * with a valid key is rectified.  Used instead of the Micro repair.
+ *
+ * vsa_pool_kv_bf16: k_bar, v_bar bf16 [B, H, n_rows, d] = the means of the
+ * valid rows of each bk-row key block of K and V (fp32 sums, one rounding to
+ * bf16); rows past the last key block are zeros.  n_rows is a multiple of 128
+ * and at least n_pad / bk.
+ *
+ * vsa_rectify_fwd: the pooled pass of the query tiles of the given heads:
+ *   q       : bf16 [B, H, n_pad, d];  k_bar, v_bar : from vsa_pool_kv_bf16.
+ *   counts, idx : the kept lists (vsa_select_blocks layout: bq-row lists,
+ *             idx row stride idx_stride); the pass attends to the other blocks.
+ *   merge_o, merge_lse : fp32 [B, H, n_pad, d] / [B, H, n_pad] output of the
+ *             kept blocks (vsa_block_sparse_fwd with o_fp32 = 1), merged exactly
+ *             by LSE into the result (NULL: the pooled terms alone).
+ *   o, lse  : the rectified output (bf16 or fp32) and its LSE.
+ *   heads, n_heads : as vsa_block_sparse_fwd_heads.
+ *   n_pad / bk <= 1024.
+ * ------------------------------------------------------------------------- */
+VSA_API vsa_status vsa_pool_kv_bf16(const void *k, const void *v, const vsa_shape *shape, int bk, int n_rows,
+                                    void *k_bar, void *v_bar, void *stream);
+
+VSA_API vsa_status vsa_rectify_fwd(const void *q, const void *k_bar, const void *v_bar, const vsa_shape *shape,
+                                   int bq, int bk, int n_rows, const int32_t *counts, const int32_t *idx,
+                                   int idx_stride, float scale, const float *merge_o, const float *merge_lse,
+                                   void *o, int o_fp32, float *lse, const int32_t *heads, int n_heads,
+                                   void *stream);
 
 #ifdef __cplusplus
 }
