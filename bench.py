@@ -756,6 +756,91 @@ def run_rectify(args):
     print(json.dumps(line), flush=True)
 
 
+def run_reuse(args):
+    """Cross-step mask reuse over simulated denoising steps (MOD-DiT pattern
+    refresh every delta-t steps; HyperVAttention section 3 temporal
+    stability).  Step t's inputs are the workload's tensors plus a seeded drift,
+    x_t = x_0 + drift * t * eps with eps ~ N(0, 1) per element (drawn on the
+    device from a fixed seed).  SelectionSchedule(0, refresh) decides per step
+    whether the path selects or reuses the last lists.  One JSON line: per
+    step the mode, the path time (CUDA events), the relative L2 error against
+    dense attention of that step with the scheduled lists and with a fresh
+    selection, and the overlap (Jaccard) of the kept blocks."""
+    import block_sparse_attention_pool_b200 as vsa
+    from block_sparse_attention_pool_b200 import build as vsa_build
+    vsa_build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    q, k, v = make_qkv(w)
+    to_dev = lambda x: torch.from_numpy(x).to(dev).to(torch.bfloat16).contiguous()
+    x0 = [to_dev(x) for x in (q, k, v)]
+    del q, k, v
+    gen = torch.Generator(device=dev).manual_seed(1000 + w.seed)
+    eps = [torch.randn(x.shape, generator=gen, device=dev, dtype=torch.float32) for x in x0]
+    stream = torch.cuda.current_stream(dev)
+    heads = micro_heads(w) if w.micro_mode else None
+    run = vsa.SparseVideoAttention(vsa.PathConfig.from_workload(w, heads))
+    fresh = vsa.SparseVideoAttention(vsa.PathConfig.from_workload(w, heads))
+    n_pad = x0[0].shape[2]
+    dense = vsa.SparseVideoAttention(vsa.PathConfig(n_valid=w.n_valid, bq=w.bq, bk=w.bk, scale=w.scale,
+                                                    fixed_k=n_pad // w.bk))
+    sched = vsa.SelectionSchedule(0, args.reuse_refresh)
+    nv = w.n_valid
+    rel = lambda o, ref: float(torch.linalg.vector_norm(o[:, :, :nv] - ref[:, :, :nv]) /
+                               torch.linalg.vector_norm(ref[:, :, :nv]))
+
+    def kept_mask(buf):
+        n_k = buf["idx"].shape[-1]
+        valid = torch.arange(n_k, device=dev)[None, None, None, :] < buf["counts"][..., None]
+        # unused list slots scatter into a spare column n_k
+        m = torch.zeros(buf["idx"].shape[:-1] + (n_k + 1,), dtype=torch.bool, device=dev)
+        m.scatter_(3, torch.where(valid, buf["idx"].long(), n_k), True)
+        return m[..., :n_k]
+
+    steps = []
+    for t in range(args.reuse_steps):
+        xt = [(x.float() + args.reuse_drift * t * e).to(torch.bfloat16) for x, e in zip(x0, eps)]
+        mode = sched.mode(t)
+        for _ in range(args.warmup if t == 0 else 0):
+            run(*xt)
+        ms = []
+        for _ in range(args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            run(*xt, reuse_selection=(mode == "reuse"))
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ms.append(e0.elapsed_time(e1))
+        o_sched = run.buf["o"].float().clone()
+        fresh(*xt)
+        ref = dense(*xt)["o"].float()
+        a, b = kept_mask(run.buf), kept_mask(fresh.buf)
+        jac = float((a & b).sum()) / max(1.0, float((a | b).sum()))
+        steps.append({"t": t, "mode": mode, "ms": round(statistics.mean(ms), 4),
+                      "rel_l2_error_vs_dense": round(rel(o_sched, ref), 5),
+                      "rel_l2_error_fresh_selection": round(rel(fresh.buf["o"].float(), ref), 5),
+                      "kept_jaccard_vs_fresh": round(jac, 4)})
+        del xt, ref
+    st = vsa.read_device_status(stream)
+    if st != 0:
+        raise RuntimeError(vsa.status_string(st))
+    sel = [x["ms"] for x in steps if x["mode"] == "select"]
+    reu = [x["ms"] for x in steps if x["mode"] == "reuse"]
+    line = {
+        "metric": METRIC + " (cross-step mask reuse)",
+        "value": round(statistics.mean(sel) - statistics.mean(reu), 4) if reu else 0.0,
+        "unit": "ms saved per reuse step",
+        "config": {"workload": workload_label(w), "refresh": args.reuse_refresh, "drift_per_step": args.reuse_drift,
+                   "steps": args.reuse_steps},
+        "ms_select_step": round(statistics.mean(sel), 4),
+        "ms_reuse_step": round(statistics.mean(reu), 4) if reu else None,
+        "per_step": steps,
+        "data": "synthetic (seeded video-shaped Q/K/V plus seeded per-step drift, no model weights)",
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -775,6 +860,11 @@ def main():
     ap.add_argument("--cluster-blocks", action="store_true",
                     help="print the cluster-aligned-blocks line (selection on clusters, merging, group tiles)")
     ap.add_argument("--merge-rounds", type=int, default=3)
+    ap.add_argument("--reuse", action="store_true",
+                    help="print the cross-step mask reuse line (simulated denoising steps) instead of the bench line")
+    ap.add_argument("--reuse-refresh", type=int, default=2)
+    ap.add_argument("--reuse-steps", type=int, default=6)
+    ap.add_argument("--reuse-drift", type=float, default=0.05)
     ap.add_argument("--rectify", action="store_true",
                     help="print the pooled-rectification line (omitted blocks as pooled keys) instead of the bench line")
     ap.add_argument("--cluster-cum-mass", type=float, default=0.0,
@@ -795,6 +885,9 @@ def main():
         return
     if args.rectify:
         run_rectify(args)
+        return
+    if args.reuse:
+        run_reuse(args)
         return
     if args.impl == "reference":
         line = run_reference(args, rank, world)

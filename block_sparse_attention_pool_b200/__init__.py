@@ -28,7 +28,7 @@ __all__ = [
     "PathConfig", "SparseVideoAttention", "ClusterParams", "cluster_count", "cluster_tokens", "permute_rows",
     "select_clusters", "merge_clusters", "merge_clusters_workspace_bytes", "cluster_rows_capacity", "cluster_plan",
     "gather_rows", "cluster_group_fwd", "ClusterBlockConfig", "ClusterBlockAttention",
-    "pool_kv_bf16", "rectify_fwd",
+    "pool_kv_bf16", "rectify_fwd", "SelectionSchedule",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -421,6 +421,7 @@ class SparseVideoAttention:
         self.cfg = cfg
         self.buf: Dict[str, torch.Tensor] = {}
         self._key = None
+        self._selected = None  # shape of the last call that ran selection
         # size the Micro workspace as if every head were enabled (callers that
         # pass different per-call head flags)
         self._ws_all = workspace_for_all_heads
@@ -430,6 +431,7 @@ class SparseVideoAttention:
         key = (B, H, n_pad, d, q.device)
         if key == self._key:
             return
+        self._selected = None
         c = self.cfg
         dev = q.device
         n_q, n_k = n_pad // c.bq, n_pad // c.bk
@@ -507,8 +509,12 @@ class SparseVideoAttention:
         return cache[key]
 
     def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None, out_o=None, out_lse=None,
-                 micro_heads=None, on_stage=None) -> Dict[str, torch.Tensor]:
+                 micro_heads=None, on_stage=None, reuse_selection: bool = False) -> Dict[str, torch.Tensor]:
         """Run the path on device tensors q, k, v [B, H, n_pad, d] (bf16).
+
+        ``reuse_selection``: skip pooling and selection (block and Micro) and
+        attend with the lists of the last call that selected (cross-step reuse
+        of the mask, see SelectionSchedule).
 
         With ``cfg.cluster_lattice`` set, Q and K are first clustered per
         (batch, head) by 3D local-window clustering, Q', K', V' are the
@@ -517,7 +523,9 @@ class SparseVideoAttention:
         in ``self.buf["perm_q"]`` / ``["perm_k"]``.  Otherwise see _run.
         """
         if self.cfg.cluster_lattice is None:
-            return self._run(q, k, v, stream, out_o, out_lse, micro_heads, on_stage)
+            return self._run(q, k, v, stream, out_o, out_lse, micro_heads, on_stage, reuse_selection)
+        if reuse_selection:
+            raise ValueError("reuse_selection applies to the token-order layout")
         self._alloc(q)
         b = self.buf
         B, H, n_pad, d = q.shape
@@ -535,7 +543,7 @@ class SparseVideoAttention:
         return b
 
     def _run(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None, out_o=None, out_lse=None,
-             micro_heads=None, on_stage=None) -> Dict[str, torch.Tensor]:
+             micro_heads=None, on_stage=None, reuse: bool = False) -> Dict[str, torch.Tensor]:
         """Run the whole path on device tensors q, k, v [B, H, n_pad, d] (bf16).
 
         Outputs go to ``self.buf["o"]`` / ``["lse"]``, or to ``out_o`` /
@@ -562,11 +570,16 @@ class SparseVideoAttention:
         heads = c.micro_heads if micro_heads is None else micro_heads
         stage = on_stage if on_stage is not None else (lambda i: None)
         stage(0)
-        pool_qk(q, k, shape, c.bq, c.bk, b["q_pool"], b["k_pool"], b.get("q_pool64"), b.get("k_pool16"), stream)
+        if reuse and self._selected != (B, H, n_pad, d):
+            raise ValueError("reuse_selection needs a previous call with fresh selection on this shape")
+        if not reuse:
+            pool_qk(q, k, shape, c.bq, c.bk, b["q_pool"], b["k_pool"], b.get("q_pool64"), b.get("k_pool16"), stream)
         stage(1)
-        select_blocks(b["q_pool"], b["k_pool"], shape, c.bq, c.bk, scale,
-                      SelectParams(c.k_min, c.cum_mass, c.fixed_k, c.n_anchor, c.anchor_rot), b["counts"], b["idx"],
-                      None, stream)
+        if not reuse:
+            select_blocks(b["q_pool"], b["k_pool"], shape, c.bq, c.bk, scale,
+                          SelectParams(c.k_min, c.cum_mass, c.fixed_k, c.n_anchor, c.anchor_rot), b["counts"],
+                          b["idx"], None, stream)
+            self._selected = (B, H, n_pad, d)
         stage(2)
         if c.rectify:
             # kept blocks exactly (Macro), then the omitted blocks as pooled keys, merged by LSE
@@ -600,9 +613,10 @@ class SparseVideoAttention:
             block_sparse_fwd(q, k, v, shape, c.bq, c.bk, b["counts"], b["idx"], n_k, scale, b["o_macro"],
                              b["lse_macro"], stream=stream, heads=rep)
         stage(3)
-        select_micro(b["q_pool64"], b["k_pool16"], b["counts"], b["idx"], shape, c.bq, c.bk, scale, c.micro_mode,
-                     c.micro_topk, c.micro_percentile, heads, self.micro_cap, b["m_counts"], b["m_idx"],
-                     b["workspace"], stream)
+        if not reuse:
+            select_micro(b["q_pool64"], b["k_pool16"], b["counts"], b["idx"], shape, c.bq, c.bk, scale,
+                         c.micro_mode, c.micro_topk, c.micro_percentile, heads, self.micro_cap, b["m_counts"],
+                         b["m_idx"], b["workspace"], stream)
         stage(4)
         if not isinstance(rep, tuple):
             block_sparse_fwd(q, k, v, shape, 64, 16, b["m_counts"], b["m_idx"], self.micro_cap, scale, o, lse,
@@ -772,3 +786,31 @@ class ClusterBlockAttention:
         gather_rows(b["lse_rows"], b["qinv"], b["lse"], 0xff800000, stream)
         stage(7)
         return b
+
+
+class SelectionSchedule:
+    """Cross-step reuse of the block mask over denoising steps.
+
+    MOD-DiT (section on linear pattern prediction): sparsity patterns drift
+    slowly and piecewise linearly in the mid-late denoising steps, a full
+    attention warm-up comes first, and the pattern is refreshed every
+    delta-t steps; HyperVAttention section 3: cluster assignments stay stable
+    across adjacent steps.  Reading taken here: the first ``warmup`` steps run
+    dense attention, the selection runs at step ``warmup`` and every
+    ``refresh`` steps after it, and the steps in between attend with the last
+    selected lists (no linear prediction of pattern intensities).
+    """
+
+    def __init__(self, warmup: int = 0, refresh: int = 2):
+        if warmup < 0 or refresh < 1:
+            raise ValueError("warmup >= 0 and refresh >= 1")
+        self.warmup = warmup
+        self.refresh = refresh
+
+    def mode(self, step: int) -> str:
+        """'dense', 'select' or 'reuse' for denoising step ``step`` (0-based)."""
+        if step < 0:
+            raise ValueError("step >= 0")
+        if step < self.warmup:
+            return "dense"
+        return "select" if (step - self.warmup) % self.refresh == 0 else "reuse"
