@@ -52,7 +52,8 @@ __all__ = [
     "cell_counts", "token_cells", "initial_centroids", "window_offsets", "window_cells",
     "local_window_clustering", "clustering_objective", "cluster_permutation", "permute_rows",
     "unpermute_rows", "forward_clustered", "select_clusters", "tile_cost", "merge_clusters", "total_cost",
-    "forward_cluster_blocks", "attend_cluster_groups",
+    "forward_cluster_blocks", "attend_cluster_groups", "lowe_ratio", "ambiguous_subset", "hybrid_anchor",
+    "hybrid_update",
 ]
 
 
@@ -341,3 +342,85 @@ def forward_cluster_blocks(q, k, v, n_valid, grid, cell, window, n_iter, scale, 
             info.append({"assign_q": aq, "assign_k": ak, "mu_q": muq, "mu_k": muk, "sizes_q": sq, "sizes_k": sk,
                          "kept": kept, "groups": groups})
     return {"O": O, "LSE": L, "heads": info}
+
+
+# ---------------------------------------------------------------------------
+# Hybrid clustering across denoising steps (HVA §4.2, Eq. (6); App. A.1: full
+# clustering every two steps, the 15% most ambiguous tokens cached)
+#
+# Further readings (C15-C19):
+#  C15 Lowe's ratio rho_l = d1 / d2 (Eq. (6), Euclidean distances) is taken
+#      over the centroids the token's last local assignment compared -- the
+#      centroids of its window before the anchor step's final update -- with
+#      u* that assignment's argmin (ties to the lower cell); a window of one
+#      centroid gives rho = 0, d1 = d2 = 0 gives rho = 1;
+#  C16 the cached subset is the ceil(frac * N) tokens of largest rho, ties to
+#      the lower token index, listed in ascending token order;
+#  C17 at an intermediate step each cached token is reassigned, with its
+#      current embedding, to the nearest centroid of the whole current set
+#      (squared Euclidean, ties to the lower cell); other tokens keep theirs;
+#  C18 "updating the corresponding centroids": a cluster that gained or lost a
+#      token is set to the mean of its members' current embeddings (an emptied
+#      one keeps its centroid); every other centroid is unchanged;
+#  C19 sizes and permutation follow the new assignment (C7).
+# ---------------------------------------------------------------------------
+
+def lowe_ratio(x: np.ndarray, mu: np.ndarray, grid, cell, window) -> np.ndarray:
+    """C15: rho of every token against the centroids mu of its window."""
+    x = np.asarray(x, dtype=np.float64)
+    counts = cell_counts(grid, cell)
+    CT, CH, CW = counts
+    g = token_cells(grid, cell)
+    rho = np.zeros(x.shape[0])
+    for u in range(CT * CH * CW):
+        toks = np.nonzero(g == u)[0]
+        if toks.size == 0:
+            continue
+        cand = window_cells((u // (CH * CW), (u // CW) % CH, u % CW), counts, window)
+        diff = x[toks][:, None, :] - mu[cand][None, :, :]
+        dist = np.sqrt(np.einsum("tcd,tcd->tc", diff, diff))
+        if cand.size == 1:
+            continue  # rho = 0
+        best = np.argmin(dist, axis=1)
+        d1 = dist[np.arange(toks.size), best]
+        rest = dist.copy()
+        rest[np.arange(toks.size), best] = np.inf
+        d2 = rest.min(axis=1)
+        rho[toks] = np.where(d2 > 0, d1 / np.where(d2 > 0, d2, 1.0), 1.0)
+    return rho
+
+
+def ambiguous_subset(rho: np.ndarray, frac: float) -> np.ndarray:
+    """C16: the ceil(frac * N) largest rho, ties to the lower index, ascending."""
+    n = int(np.ceil(frac * rho.shape[0]))
+    order = np.lexsort((np.arange(rho.shape[0]), -rho))
+    return np.sort(order[:n])
+
+
+def hybrid_anchor(x: np.ndarray, grid, cell, window, n_iter: int, frac: float):
+    """An anchor step: full local-window clustering (n_iter >= 1 rounds), Lowe's
+    ratio from the last round's comparison (C15) and the cached subset (C16).
+    Returns (a, mu, rho, subset)."""
+    a, mu = local_window_clustering(x, grid, cell, window, n_iter)
+    _, mu_last = local_window_clustering(x, grid, cell, window, n_iter - 1) if n_iter > 1 else \
+        (None, initial_centroids(np.asarray(x, dtype=np.float64), grid, cell))
+    rho = lowe_ratio(x, mu_last, grid, cell, window)
+    return a, mu, rho, ambiguous_subset(rho, frac)
+
+
+def hybrid_update(x_new: np.ndarray, a_prev: np.ndarray, mu_prev: np.ndarray, subset: np.ndarray):
+    """An intermediate step (C17, C18): returns (a, mu, changed clusters)."""
+    x_new = np.asarray(x_new, dtype=np.float64)
+    a = np.array(a_prev, dtype=np.int64, copy=True)
+    mu = np.array(mu_prev, dtype=np.float64, copy=True)
+    if subset.size:
+        diff = x_new[subset][:, None, :] - mu_prev[None, :, :]
+        dist = np.einsum("tcd,tcd->tc", diff, diff)
+        a[subset] = np.argmin(dist, axis=1)  # first minimum: lower cell
+    moved = subset[a[subset] != a_prev[subset]]
+    changed = np.unique(np.concatenate([a_prev[moved], a[moved]])).astype(np.int64)
+    for u in changed:
+        members = a == u
+        if members.any():
+            mu[u] = x_new[members].mean(axis=0)
+    return a, mu, changed
