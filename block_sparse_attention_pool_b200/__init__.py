@@ -28,7 +28,8 @@ __all__ = [
     "PathConfig", "SparseVideoAttention", "ClusterParams", "cluster_count", "cluster_tokens", "permute_rows",
     "select_clusters", "merge_clusters", "merge_clusters_workspace_bytes", "cluster_rows_capacity", "cluster_plan",
     "gather_rows", "cluster_group_fwd", "ClusterBlockConfig", "ClusterBlockAttention",
-    "pool_kv_bf16", "rectify_fwd", "SelectionSchedule",
+    "pool_kv_bf16", "rectify_fwd", "SelectionSchedule", "cluster_anchor", "cluster_refine",
+    "cluster_refine_workspace_bytes", "subset_size",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -40,7 +41,8 @@ EXPORTED = (
     "vsa_block_sparse_fwd", "vsa_block_sparse_fwd_heads", "vsa_lse_merge", "vsa_selftest_wait_timeout",
     "vsa_cluster_count", "vsa_cluster_tokens", "vsa_permute_rows", "vsa_select_clusters",
     "vsa_merge_clusters_workspace_bytes", "vsa_merge_clusters", "vsa_cluster_rows_capacity", "vsa_cluster_plan",
-    "vsa_gather_rows", "vsa_cluster_group_fwd", "vsa_pool_kv_bf16", "vsa_rectify_fwd",
+    "vsa_gather_rows", "vsa_cluster_group_fwd", "vsa_pool_kv_bf16", "vsa_rectify_fwd", "vsa_cluster_anchor",
+    "vsa_cluster_refine_workspace_bytes", "vsa_cluster_refine",
 )
 
 STATUS = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_UNSUPPORTED", 3: "VSA_ERR_CUDA",
@@ -144,6 +146,12 @@ def lib():
     L.vsa_gather_rows.argtypes = [P, P, I, I, I, I, ctypes.c_uint32, P, P]
     L.vsa_cluster_group_fwd.restype = I
     L.vsa_cluster_group_fwd.argtypes = [P, P, P, SP, I, P, P, P, I, P, P, I, F, P, I, P, P]
+    L.vsa_cluster_anchor.restype = I
+    L.vsa_cluster_anchor.argtypes = [P, SP, ctypes.POINTER(ClusterParams), I, P, P, P, P, P, P, P]
+    L.vsa_cluster_refine_workspace_bytes.restype = S
+    L.vsa_cluster_refine_workspace_bytes.argtypes = [SP, ctypes.POINTER(ClusterParams)]
+    L.vsa_cluster_refine.restype = I
+    L.vsa_cluster_refine.argtypes = [P, SP, ctypes.POINTER(ClusterParams), P, I, P, P, P, P, P, S, P]
     L.vsa_pool_kv_bf16.restype = I
     L.vsa_pool_kv_bf16.argtypes = [P, P, SP, I, I, P, P, P]
     L.vsa_rectify_fwd.restype = I
@@ -282,6 +290,33 @@ def rectify_fwd(q, k_bar, v_bar, shape: Shape, bq, bk, counts, idx, idx_stride, 
                                  _p(counts), _p(idx), idx_stride, float(scale), _p(merge_o), _p(merge_lse), _p(o),
                                  1 if o.dtype == torch.float32 else 0, _p(lse), hp, nh, _s(stream)),
            "vsa_rectify_fwd")
+
+
+def subset_size(n_valid: int, frac: float) -> int:
+    """ceil(frac * n_valid): the cached subset of the hybrid clustering."""
+    return int(math.ceil(frac * n_valid))
+
+
+def cluster_anchor(x, shape: Shape, params: "ClusterParams", assign, centroids, sizes, perm, ratio, subset,
+                   stream=None):
+    """Anchor step: full clustering plus Lowe's ratio and the cached subset
+    (subset int32 [B, H, n_sub])."""
+    _check(lib().vsa_cluster_anchor(_p(x), ctypes.byref(shape), ctypes.byref(params), subset.shape[2], _p(assign),
+                                    _p(centroids), _p(sizes), _p(perm), _p(ratio), _p(subset), _s(stream)),
+           "vsa_cluster_anchor")
+
+
+def cluster_refine_workspace_bytes(shape: Shape, params: "ClusterParams") -> int:
+    return int(lib().vsa_cluster_refine_workspace_bytes(ctypes.byref(shape), ctypes.byref(params)))
+
+
+def cluster_refine(x, shape: Shape, params: "ClusterParams", subset, assign, centroids, sizes, perm, workspace,
+                   stream=None):
+    """Intermediate step: global reassignment of the cached subset, update of the
+    touched centroids, sizes and permutation rebuilt (assign, centroids in place)."""
+    _check(lib().vsa_cluster_refine(_p(x), ctypes.byref(shape), ctypes.byref(params), _p(subset), subset.shape[2],
+                                    _p(assign), _p(centroids), _p(sizes), _p(perm), _p(workspace),
+                                    workspace.numel() * workspace.element_size(), _s(stream)), "vsa_cluster_refine")
 
 
 def mask_to_lists(mask, shape: Shape, bq, bk, counts, idx, stream=None):
@@ -691,6 +726,7 @@ class ClusterBlockConfig:
     rounds: int = 3                   # merging rounds R (App. A.1: 3)
     tau_q: int = 128                  # CTA tile sizes of the cost model (Eq. (7))
     tau_k: int = 128
+    hybrid_frac: float = 0.15         # cached share of tokens at anchor steps (App. A.1: 15%)
 
     def cluster_params(self) -> "ClusterParams":
         return ClusterParams.make(self.lattice, self.cell, self.window, self.iters)
@@ -727,6 +763,13 @@ class ClusterBlockAttention:
             b["centroids_" + n] = torch.empty(B, H, G, d, device=dev, dtype=f32)
             b["sizes_" + n] = torch.empty(B, H, G, device=dev, dtype=i32)
             b["perm_" + n] = torch.empty(B, H, n_pad, device=dev, dtype=i32)
+        n_sub = subset_size(c.n_valid, c.hybrid_frac)
+        shape = _shape(B, H, c.n_valid, n_pad, d)
+        for n in ("q", "k"):
+            b["ratio_" + n] = torch.empty(B, H, c.n_valid, device=dev, dtype=f32)
+            b["subset_" + n] = torch.empty(B, H, max(1, n_sub), device=dev, dtype=i32)
+        b["refine_ws"] = torch.empty(cluster_refine_workspace_bytes(shape, c.cluster_params()), device=dev,
+                                     dtype=torch.uint8)
         b["counts"] = torch.empty(B, H, G, device=dev, dtype=i32)
         b["idx"] = torch.empty(B, H, G, G, device=dev, dtype=i32)
         b["merge_ws"] = torch.empty(merge_clusters_workspace_bytes(B * H, G), device=dev, dtype=torch.uint8)
@@ -746,13 +789,18 @@ class ClusterBlockAttention:
         b["lse"] = torch.empty(B, H, n_pad, device=dev, dtype=f32)
         self.buf = b
         self._key = key
+        self._anchored = False
 
     def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, sides: Optional[torch.Tensor] = None,
-                 stream=None, on_stage=None) -> Dict[str, torch.Tensor]:
+                 stream=None, on_stage=None, cluster_step: str = "full") -> Dict[str, torch.Tensor]:
         """q, k, v: bf16 device tensors [B, H, n_pad, d].  sides: uint8 device
         tensor [B, H, rounds, G] of bipartition bits (the random draws of
-        Algorithm 1), or None for no merging.  ``on_stage(i)`` is called on
-        the host before the first stage (i = 0) and after each of STAGES."""
+        Algorithm 1), or None for no merging.  ``cluster_step``: "full" (3D
+        local-window clustering), "anchor" (the same, plus Lowe's ratio and the
+        cached subset of the hybrid strategy) or "refine" (an intermediate
+        step: only the cached subset is revisited; needs an earlier anchor).
+        ``on_stage(i)`` is called on the host before the first stage (i = 0)
+        and after each of STAGES."""
         c = self.cfg
         self._alloc(q)
         b = self.buf
@@ -760,11 +808,25 @@ class ClusterBlockAttention:
         shape = _shape(B, H, c.n_valid, n_pad, d)
         scale = c.scale if c.scale is not None else 1.0 / math.sqrt(d)
         stage = on_stage if on_stage is not None else (lambda i: None)
+        if cluster_step not in ("full", "anchor", "refine"):
+            raise ValueError("cluster_step is 'full', 'anchor' or 'refine'")
+        if cluster_step == "refine" and not self._anchored:
+            raise ValueError("a refine step needs an earlier anchor step on this shape")
         stage(0)
         params = c.cluster_params()
         for name, x in (("q", q), ("k", k)):
-            cluster_tokens(x, shape, params, b["assign_" + name], b["centroids_" + name], b["sizes_" + name],
-                           b["perm_" + name], stream)
+            args = (b["assign_" + name], b["centroids_" + name], b["sizes_" + name], b["perm_" + name])
+            if cluster_step == "full":
+                cluster_tokens(x, shape, params, *args, stream)
+            elif cluster_step == "anchor":
+                cluster_anchor(x, shape, params, *args, b["ratio_" + name], b["subset_" + name], stream)
+            else:
+                cluster_refine(x, shape, params, b["subset_" + name], b["assign_" + name], b["centroids_" + name],
+                               b["sizes_" + name], b["perm_" + name], b["refine_ws"], stream)
+        if cluster_step == "anchor":
+            self._anchored = True
+        elif cluster_step == "full":
+            self._anchored = False
         stage(1)
         select_clusters(b["centroids_q"], b["centroids_k"], b["sizes_q"], b["sizes_k"], scale,
                         SelectParams(c.k_min, c.cum_mass, c.fixed_k, 0, 0), b["counts"], b["idx"], stream)

@@ -104,10 +104,14 @@ struct AssignLayout {
 // One CTA per cell.  Thread (ty, tx) scores tokens ty + 16 a (a < 8) against
 // centroids tx + 16 b (b < NB): each 4-wide step of d loads 8 + NB float4 and
 // issues 32 NB FMAs.  NB = ceil(window cells / 16) is a template parameter.
-template <int D, int NB>
+// RATIO: also write each token's Lowe ratio rho = d1 / d2 (HyperVAttention
+// Eq. (6): Euclidean distances to the nearest and the second-nearest centroid
+// of the window; 0 for a window of one centroid, 1 when both are 0).
+template <int D, int NB, bool RATIO = false>
 __global__ void __launch_bounds__(kClusterThreads) cluster_assign_kernel(const __nv_bfloat16 *__restrict__ x,
                                                                          ClusterGeom g, const float *__restrict__ mu,
-                                                                         int32_t *__restrict__ assign) {
+                                                                         int32_t *__restrict__ assign,
+                                                                         float *__restrict__ ratio) {
   using L = AssignLayout<D>;
   constexpr int kLd = L::kLd;
   constexpr int kRows = 16 * NB;
@@ -182,7 +186,9 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_assign_kernel(const _
   // dot products and, alongside, |mu|^2 of this thread's centroids (every
   // thread that holds a centroid sums it in the same order)
   const int ty = tid >> 4, tx = tid & 15;
-  float acc[8][NB], cn[NB];
+  float acc[8][NB], cn[NB], xn[8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a) xn[a] = 0.f;
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
     cn[b] = 0.f;
@@ -203,6 +209,12 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_assign_kernel(const _
 #pragma unroll
     for (int a = 0; a < 8; ++a) {
       const float4 xv = *reinterpret_cast<const float4 *>(&sX[ty + 16 * a][k]);
+      if constexpr (RATIO) {
+        xn[a] = fmaf(xv.x, xv.x, xn[a]);
+        xn[a] = fmaf(xv.y, xv.y, xn[a]);
+        xn[a] = fmaf(xv.z, xv.z, xn[a]);
+        xn[a] = fmaf(xv.w, xv.w, xn[a]);
+      }
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
         acc[a][b] = fmaf(xv.x, cv[b].x, acc[a][b]);
@@ -215,7 +227,7 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_assign_kernel(const _
   int32_t *ab = assign + (size_t)bh * g.n_valid;
 #pragma unroll
   for (int a = 0; a < 8; ++a) {
-    float d = INFINITY;
+    float d = INFINITY, d2 = INFINITY;  // best and second-best |mu|^2 - 2 x.mu
     int c = 0x7fffffff;
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
@@ -224,23 +236,36 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_assign_kernel(const _
         const float dist = fmaf(-2.f, acc[a][b], cn[b]);
         const int cell = win[j];
         if (dist < d || (dist == d && cell < c)) {
+          d2 = d;
           d = dist;
           c = cell;
+        } else {
+          d2 = fminf(d2, dist);
         }
       }
     }
-    // argmin across the 16 threads (tx) that share a token
+    // argmin across the 16 threads (tx) that share a token; the second best is
+    // the smaller of the losing best and the two second bests
 #pragma unroll
     for (int o = 1; o < 16; o <<= 1) {
       const float od = __shfl_xor_sync(0xffffffffu, d, o);
       const int oc = __shfl_xor_sync(0xffffffffu, c, o);
+      const float od2 = __shfl_xor_sync(0xffffffffu, d2, o);
+      d2 = fminf(fminf(d2, od2), fmaxf(d, od));
       if (od < d || (od == d && oc < c)) {
         d = od;
         c = oc;
       }
     }
     const int i = ty + 16 * a;
-    if (tx == 0 && i < n_tok) ab[s_tok[i]] = c;
+    if (tx == 0 && i < n_tok) {
+      ab[s_tok[i]] = c;
+      if constexpr (RATIO) {
+        const float e1 = fmaxf(0.f, xn[a] + d), e2 = d2 == INFINITY ? INFINITY : fmaxf(0.f, xn[a] + d2);
+        const float rho = e2 == INFINITY ? 0.f : (e2 > 0.f ? sqrtf(e1) / sqrtf(e2) : 1.f);
+        ratio[(size_t)bh * g.n_valid + s_tok[i]] = rho;
+      }
+    }
   }
 }
 

@@ -19,6 +19,7 @@
 #include "attn_fwd.cuh"
 #include "attn_fwd_dual.cuh"
 #include "cluster.cuh"
+#include "cluster_hybrid.cuh"
 #include "cluster_merge.cuh"
 #include "cluster_plan.cuh"
 #include "common.cuh"
@@ -334,33 +335,38 @@ int cluster_box_tokens(const vsa::ClusterGeom &g) {
 // memory is set once per instantiation.
 template <int D, int NB>
 vsa_status launch_assign(const __nv_bfloat16 *x, const vsa::ClusterGeom &g, dim3 grid, const float *mu,
-                         int32_t *assign, cudaStream_t st) {
+                         int32_t *assign, float *ratio, cudaStream_t st) {
   static const int bytes = vsa::AssignLayout<D>::bytes(16 * NB);
   static const cudaError_t attr =
-      cudaFuncSetAttribute(vsa::cluster_assign_kernel<D, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (attr != cudaSuccess) return VSA_ERR_CUDA;
-  vsa::cluster_assign_kernel<D, NB><<<grid, vsa::kClusterThreads, bytes, st>>>(x, g, mu, assign);
+      cudaFuncSetAttribute(vsa::cluster_assign_kernel<D, NB, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  static const cudaError_t attr_r =
+      cudaFuncSetAttribute(vsa::cluster_assign_kernel<D, NB, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (attr != cudaSuccess || attr_r != cudaSuccess) return VSA_ERR_CUDA;
+  if (ratio)
+    vsa::cluster_assign_kernel<D, NB, true><<<grid, vsa::kClusterThreads, bytes, st>>>(x, g, mu, assign, ratio);
+  else
+    vsa::cluster_assign_kernel<D, NB, false><<<grid, vsa::kClusterThreads, bytes, st>>>(x, g, mu, assign, nullptr);
   return VSA_OK;
 }
 
 template <int D>
 vsa_status launch_assign_any(const __nv_bfloat16 *x, const vsa::ClusterGeom &g, dim3 grid, const float *mu,
-                             int32_t *assign, cudaStream_t st) {
+                             int32_t *assign, float *ratio, cudaStream_t st) {
   switch ((g.wt * g.wh * g.ww + 15) / 16) {
-    case 1: return launch_assign<D, 1>(x, g, grid, mu, assign, st);
-    case 2: return launch_assign<D, 2>(x, g, grid, mu, assign, st);
-    case 3: return launch_assign<D, 3>(x, g, grid, mu, assign, st);
-    case 4: return launch_assign<D, 4>(x, g, grid, mu, assign, st);
-    case 5: return launch_assign<D, 5>(x, g, grid, mu, assign, st);
-    case 6: return launch_assign<D, 6>(x, g, grid, mu, assign, st);
-    case 7: return launch_assign<D, 7>(x, g, grid, mu, assign, st);
-    default: return launch_assign<D, 8>(x, g, grid, mu, assign, st);
+    case 1: return launch_assign<D, 1>(x, g, grid, mu, assign, ratio, st);
+    case 2: return launch_assign<D, 2>(x, g, grid, mu, assign, ratio, st);
+    case 3: return launch_assign<D, 3>(x, g, grid, mu, assign, ratio, st);
+    case 4: return launch_assign<D, 4>(x, g, grid, mu, assign, ratio, st);
+    case 5: return launch_assign<D, 5>(x, g, grid, mu, assign, ratio, st);
+    case 6: return launch_assign<D, 6>(x, g, grid, mu, assign, ratio, st);
+    case 7: return launch_assign<D, 7>(x, g, grid, mu, assign, ratio, st);
+    default: return launch_assign<D, 8>(x, g, grid, mu, assign, ratio, st);
   }
 }
 
 template <int D>
 vsa_status launch_cluster(const __nv_bfloat16 *x, const vsa::ClusterGeom &g, int iters, int BH, int32_t *assign,
-                          float *mu, int32_t *sizes, int32_t *perm, cudaStream_t st) {
+                          float *mu, int32_t *sizes, int32_t *perm, float *ratio, cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   constexpr int kListMax = 128 + 4 * vsa::kClusterMaxTokens * vsa::kClusterMaxWindow;
@@ -375,7 +381,8 @@ vsa_status launch_cluster(const __nv_bfloat16 *x, const vsa::ClusterGeom &g, int
   const dim3 grid(g.n_cells, BH);
   vsa::cluster_init_kernel<D><<<grid, 128, 0, st>>>(x, g, mu);
   for (int it = 0; it < iters; ++it) {
-    const vsa_status as = launch_assign_any<D>(x, g, grid, mu, assign, st);
+    // the last round's assignment also yields Lowe's ratio when asked
+    const vsa_status as = launch_assign_any<D>(x, g, grid, mu, assign, it == iters - 1 ? ratio : nullptr, st);
     if (as != VSA_OK) return as;
     vsa::cluster_update_kernel<D><<<grid, vsa::kClusterThreads, list_smem, st>>>(x, g, assign, mu, sizes);
   }
@@ -758,8 +765,8 @@ vsa_status vsa_cluster_tokens(const void *x, const vsa_shape *shape, const vsa_c
   const int BH = shape->B * shape->H;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
-  return shape->d == 128 ? launch_cluster<128>(xb, g, params->iters, BH, assign, centroids, sizes, perm, st)
-                         : launch_cluster<64>(xb, g, params->iters, BH, assign, centroids, sizes, perm, st);
+  return shape->d == 128 ? launch_cluster<128>(xb, g, params->iters, BH, assign, centroids, sizes, perm, nullptr, st)
+                         : launch_cluster<64>(xb, g, params->iters, BH, assign, centroids, sizes, perm, nullptr, st);
 }
 
 vsa_status vsa_permute_rows(const void *src, const int32_t *perm, int batch_heads, int n_pad, int row_bytes,
@@ -977,6 +984,85 @@ vsa_status vsa_rectify_fwd(const void *q, const void *k_bar, const void *v_bar, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return shape->d == 128 ? launch_attn_pooled<128>(q, k_bar, v_bar, shape, n_rows, a, n_heads, st)
                          : launch_attn_pooled<64>(q, k_bar, v_bar, shape, n_rows, a, n_heads, st);
+}
+
+vsa_status vsa_cluster_anchor(const void *x, const vsa_shape *shape, const vsa_cluster_params *params, int n_sub,
+                              int32_t *assign, float *centroids, int32_t *sizes, int32_t *perm, float *ratio,
+                              int32_t *subset, void *stream) {
+  if (!shape_ok(shape) || !x || !assign || !centroids || !sizes || !perm || !ratio || !subset)
+    return VSA_ERR_INVALID_ARG;
+  vsa::ClusterGeom g;
+  if (!cluster_geom(params, &g) || g.n_valid != shape->n_valid) return VSA_ERR_INVALID_ARG;
+  if (params->iters < 1 || n_sub < 1 || n_sub > shape->n_valid) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(centroids)) return VSA_ERR_INVALID_ARG;
+  g.n_pad = shape->n_pad;
+  const int BH = shape->B * shape->H;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+  const vsa_status r = shape->d == 128
+                           ? launch_cluster<128>(xb, g, params->iters, BH, assign, centroids, sizes, perm, ratio, st)
+                           : launch_cluster<64>(xb, g, params->iters, BH, assign, centroids, sizes, perm, ratio, st);
+  if (r != VSA_OK) return r;
+  vsa::subset_select_kernel<<<BH, vsa::kHybThreads, 0, st>>>(ratio, shape->n_valid, n_sub, subset);
+  return launch_status();
+}
+
+size_t vsa_cluster_refine_workspace_bytes(const vsa_shape *shape, const vsa_cluster_params *params) {
+  vsa::ClusterGeom g;
+  if (!shape_ok(shape) || !cluster_geom(params, &g)) return 0;
+  const size_t BH = (size_t)shape->B * shape->H;
+  const size_t n_chunks = (shape->n_valid + vsa::kSortChunk - 1) / vsa::kSortChunk;
+  return align256(BH * g.n_cells * n_chunks * 4) + align256(BH * g.n_cells * 4);
+}
+
+vsa_status vsa_cluster_refine(const void *x, const vsa_shape *shape, const vsa_cluster_params *params,
+                              const int32_t *subset, int n_sub, int32_t *assign, float *centroids, int32_t *sizes,
+                              int32_t *perm, void *workspace, size_t workspace_bytes, void *stream) {
+  if (!shape_ok(shape) || !x || !subset || !assign || !centroids || !sizes || !perm || !workspace)
+    return VSA_ERR_INVALID_ARG;
+  vsa::ClusterGeom g;
+  if (!cluster_geom(params, &g) || g.n_valid != shape->n_valid) return VSA_ERR_INVALID_ARG;
+  if (n_sub < 0 || n_sub > shape->n_valid) return VSA_ERR_INVALID_ARG;
+  if (g.n_cells > 4096) return VSA_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(centroids) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return VSA_ERR_INVALID_ARG;
+  if (workspace_bytes < vsa_cluster_refine_workspace_bytes(shape, params)) return VSA_ERR_INVALID_ARG;
+  const int BH = shape->B * shape->H;
+  const int n_chunks = (shape->n_valid + vsa::kSortChunk - 1) / vsa::kSortChunk;
+  int32_t *cnt = static_cast<int32_t *>(workspace);
+  int32_t *changed = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) +
+                                                 align256((size_t)BH * g.n_cells * n_chunks * 4));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(changed, 0, (size_t)BH * g.n_cells * 4, st) != cudaSuccess) return VSA_ERR_CUDA;
+  const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+  if (n_sub > 0) {
+    const dim3 grid((n_sub + vsa::kReTok - 1) / vsa::kReTok, BH);
+    if (shape->d == 128) {
+      static const cudaError_t attr = cudaFuncSetAttribute(
+          vsa::reassign_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, vsa::ReLayout<128>::kBytes);
+      if (attr != cudaSuccess) return VSA_ERR_CUDA;
+      vsa::reassign_kernel<128><<<grid, 256, vsa::ReLayout<128>::kBytes, st>>>(
+          xb, shape->n_pad, shape->n_valid, g.n_cells, centroids, subset, n_sub, assign, changed);
+    } else {
+      static const cudaError_t attr = cudaFuncSetAttribute(
+          vsa::reassign_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, vsa::ReLayout<64>::kBytes);
+      if (attr != cudaSuccess) return VSA_ERR_CUDA;
+      vsa::reassign_kernel<64><<<grid, 256, vsa::ReLayout<64>::kBytes, st>>>(
+          xb, shape->n_pad, shape->n_valid, g.n_cells, centroids, subset, n_sub, assign, changed);
+    }
+  }
+  const dim3 cgrid(n_chunks, BH);
+  vsa::sort_count_kernel<<<cgrid, 256, g.n_cells * 4, st>>>(assign, shape->n_valid, g.n_cells, n_chunks, cnt);
+  vsa::sort_scan_kernel<<<BH, vsa::kHybThreads, 0, st>>>(cnt, g.n_cells, n_chunks, sizes);
+  vsa::sort_scatter_kernel<<<cgrid, 32, g.n_cells * 4, st>>>(assign, shape->n_valid, shape->n_pad, g.n_cells,
+                                                            n_chunks, cnt, perm);
+  const dim3 ugrid(g.n_cells, BH);
+  if (shape->d == 128)
+    vsa::refresh_kernel<128><<<ugrid, 128, 0, st>>>(xb, shape->n_pad, g.n_cells, n_chunks, changed, cnt, sizes, perm,
+                                                    centroids);
+  else
+    vsa::refresh_kernel<64><<<ugrid, 128, 0, st>>>(xb, shape->n_pad, g.n_cells, n_chunks, changed, cnt, sizes, perm,
+                                                   centroids);
+  return launch_status();
 }
 
 }  // extern "C"

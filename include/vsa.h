@@ -371,6 +371,40 @@ VSA_API vsa_status vsa_cluster_tokens(const void *x, const vsa_shape *shape, con
                                       int32_t *assign, float *centroids, int32_t *sizes, int32_t *perm,
                                       void *stream);
 
+/* Hybrid clustering across denoising steps ([HVA] section 4.2, Eq. (6); App.
+ * A.1: full clustering at anchor steps, a cached subset of the most ambiguous
+ * tokens updated at the steps in between).
+ *
+ * vsa_cluster_anchor: vsa_cluster_tokens (params->iters >= 1 rounds) whose
+ * last assignment round also writes Lowe's ratio rho = d1 / d2 of every token
+ * (Euclidean distances to the nearest and second-nearest centroid of its
+ * window, the centroids that round compared; 0 for a window of one centroid,
+ * 1 when both distances are 0), then the n_sub tokens of largest rho (ties to
+ * the lower token index), ascending:
+ *   ratio  fp32  [B, H, n_valid];  subset int32 [B, H, n_sub], 1 <= n_sub <= n_valid.
+ *
+ * vsa_cluster_refine: an intermediate step on the current embeddings x.  Each
+ * token of subset is reassigned to the nearest centroid of the whole set
+ * (squared Euclidean distance, ties to the lower cluster); tokens outside the
+ * subset keep their cluster.  Every cluster that gained or lost a token gets
+ * the mean of its members' current embeddings (an emptied one keeps its
+ * centroid); the others are unchanged.  sizes and perm are rebuilt from the
+ * new assignment (clusters in order, tokens in token order, padding rows in
+ * place).  assign and centroids are read and updated in place.
+ *   workspace: device scratch of vsa_cluster_refine_workspace_bytes() bytes,
+ *   256-byte aligned.  At most 4096 clusters.
+ * An assignment or subset entry out of range latches VSA_ERR_BAD_INDEX. */
+VSA_API vsa_status vsa_cluster_anchor(const void *x, const vsa_shape *shape, const vsa_cluster_params *params,
+                                      int n_sub, int32_t *assign, float *centroids, int32_t *sizes, int32_t *perm,
+                                      float *ratio, int32_t *subset, void *stream);
+
+VSA_API size_t vsa_cluster_refine_workspace_bytes(const vsa_shape *shape, const vsa_cluster_params *params);
+
+VSA_API vsa_status vsa_cluster_refine(const void *x, const vsa_shape *shape, const vsa_cluster_params *params,
+                                      const int32_t *subset, int n_sub, int32_t *assign, float *centroids,
+                                      int32_t *sizes, int32_t *perm, void *workspace, size_t workspace_bytes,
+                                      void *stream);
+
 /* Row permutation along the token axis of [B*H, n_pad, row] data (rows of
  * row_bytes, a multiple of 4, 16-byte aligned when a multiple of 16):
  *   inverse = 0: dst[bh][i] = src[bh][perm[bh][i]]   (Eq. (1): X' = Pi X)
