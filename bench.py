@@ -841,6 +841,95 @@ def run_reuse(args):
     print(json.dumps(line), flush=True)
 
 
+def run_cluster_hybrid(args):
+    """Hybrid clustering across simulated denoising steps (HyperVAttention
+    section 4.2; App. A.1: full clustering every two steps, 15% of the tokens
+    cached).  Step t's inputs are the workload's tensors plus a seeded drift,
+    x_t = x_0 + drift * t * eps (eps ~ N(0, 1), drawn on the device from a fixed
+    seed).  The cluster-aligned path runs with an anchor step every
+    --hybrid-every steps and refine steps in between, and, for comparison,
+    with full clustering at every step.  One JSON line: per step the mode, the
+    clustering time and the whole path time (CUDA events), and the relative L2
+    error of O against dense attention for the hybrid and the full-clustering
+    runs."""
+    import block_sparse_attention_pool_b200 as vsa
+    from block_sparse_attention_pool_b200 import build as vsa_build
+    from video_inputs import merge_sides
+    vsa_build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    q, k, v = make_qkv(w)
+    to_dev = lambda x: torch.from_numpy(x).to(dev).to(torch.bfloat16).contiguous()
+    x0 = [to_dev(x) for x in (q, k, v)]
+    del q, k, v
+    gen = torch.Generator(device=dev).manual_seed(2000 + w.seed)
+    eps = [torch.randn(x.shape, generator=gen, device=dev, dtype=torch.float32) for x in x0]
+    stream = torch.cuda.current_stream(dev)
+    n_pad = x0[0].shape[2]
+    rule = dict(k_min=1, cum_mass=args.cluster_cum_mass, fixed_k=0) if args.cluster_cum_mass > 0 else \
+        (dict(k_min=0, cum_mass=0.0, fixed_k=w.fixed_k) if w.fixed_k else
+         dict(k_min=w.k_min, cum_mass=w.cum_mass, fixed_k=0))
+    cfg = vsa.ClusterBlockConfig(n_valid=w.n_valid, lattice=w.grid, cell=args.cluster_cell,
+                                 window=args.cluster_window, iters=args.cluster_iters, scale=w.scale,
+                                 rounds=args.merge_rounds, **rule)
+    G = vsa.cluster_count(cfg.cluster_params())
+    if rule["fixed_k"]:
+        cfg.fixed_k = max(1, min(G, int(round(rule["fixed_k"] * G / (n_pad // w.bk)))))
+    sides = torch.from_numpy(merge_sides(w, args.merge_rounds, G)).to(dev) if args.merge_rounds else None
+    hyb = vsa.ClusterBlockAttention(cfg)
+    full = vsa.ClusterBlockAttention(cfg)
+    dense = vsa.SparseVideoAttention(vsa.PathConfig(n_valid=w.n_valid, bq=w.bq, bk=w.bk, scale=w.scale,
+                                                    fixed_k=n_pad // w.bk))
+    nv = w.n_valid
+    rel = lambda o, ref: float(torch.linalg.vector_norm(o[:, :, :nv] - ref[:, :, :nv]) /
+                               torch.linalg.vector_norm(ref[:, :, :nv]))
+    n_st = len(hyb.STAGES)
+
+    def timed(run, xt, mode):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_st + 1)]
+        run(*xt, sides=sides, stream=stream, on_stage=lambda i: ev[i].record(stream), cluster_step=mode)
+        torch.cuda.synchronize(dev)
+        return ev[0].elapsed_time(ev[1]), ev[0].elapsed_time(ev[n_st])
+
+    # warm-up of both modes on step 0's inputs
+    for _ in range(args.warmup):
+        hyb(*x0, sides=sides, cluster_step="anchor")
+        hyb(*x0, sides=sides, cluster_step="refine")
+        full(*x0, sides=sides, cluster_step="full")
+    steps = []
+    for t in range(args.reuse_steps):
+        xt = [(x.float() + args.reuse_drift * t * e).to(torch.bfloat16) for x, e in zip(x0, eps)]
+        mode = "anchor" if t % args.hybrid_every == 0 else "refine"
+        c_ms, p_ms = timed(hyb, xt, mode)
+        o_h = hyb.buf["o"].float().clone()
+        cf_ms, pf_ms = timed(full, xt, "full")
+        ref = dense(*xt)["o"].float()
+        steps.append({"t": t, "mode": mode, "cluster_ms": round(c_ms, 4), "path_ms": round(p_ms, 4),
+                      "cluster_ms_full": round(cf_ms, 4), "path_ms_full": round(pf_ms, 4),
+                      "rel_l2_error_vs_dense": round(rel(o_h, ref), 5),
+                      "rel_l2_error_full_clustering": round(rel(full.buf["o"].float(), ref), 5)})
+        del xt, ref
+    st = vsa.read_device_status(stream)
+    if st != 0:
+        raise RuntimeError(vsa.status_string(st))
+    anc = [x["cluster_ms"] for x in steps if x["mode"] == "anchor"]
+    ref_ms = [x["cluster_ms"] for x in steps if x["mode"] == "refine"]
+    line = {
+        "metric": METRIC + " (hybrid clustering across steps)",
+        "value": round(statistics.mean(ref_ms), 4) if ref_ms else None,
+        "unit": "ms clustering Q+K per refine step",
+        "ms_cluster_anchor_step": round(statistics.mean(anc), 4),
+        "ms_cluster_full_step": round(statistics.mean(x["cluster_ms_full"] for x in steps), 4),
+        "config": {"workload": workload_label(w), "cell": list(args.cluster_cell), "window": list(args.cluster_window),
+                   "iters": args.cluster_iters, "anchor_every": args.hybrid_every, "cached_fraction": cfg.hybrid_frac,
+                   "drift_per_step": args.reuse_drift, "rounds": args.merge_rounds},
+        "per_step": steps,
+        "data": "synthetic (seeded video-shaped Q/K/V plus seeded per-step drift, no model weights)",
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -863,6 +952,9 @@ def main():
     ap.add_argument("--reuse", action="store_true",
                     help="print the cross-step mask reuse line (simulated denoising steps) instead of the bench line")
     ap.add_argument("--reuse-refresh", type=int, default=2)
+    ap.add_argument("--cluster-hybrid", action="store_true",
+                    help="print the hybrid-clustering line (anchor and refine steps over simulated steps)")
+    ap.add_argument("--hybrid-every", type=int, default=2)
     ap.add_argument("--reuse-steps", type=int, default=6)
     ap.add_argument("--reuse-drift", type=float, default=0.05)
     ap.add_argument("--rectify", action="store_true",
@@ -888,6 +980,9 @@ def main():
         return
     if args.reuse:
         run_reuse(args)
+        return
+    if args.cluster_hybrid:
+        run_cluster_hybrid(args)
         return
     if args.impl == "reference":
         line = run_reference(args, rank, world)

@@ -78,11 +78,12 @@ __global__ void __launch_bounds__(kHybThreads) subset_select_kernel(const float 
   // each thread owns the contiguous tokens [lo, hi)
   const int per = (n_valid + kHybThreads - 1) / kHybThreads;
   const int lo = min(n_valid, t * per), hi = min(n_valid, lo + per);
+  // the counting passes read the keys interleaved (coalesced)
   uint32_t T = 0u;
   for (int bit = 31; bit >= 0; --bit) {
     const uint32_t cand = T | (1u << bit);
     int c = 0;
-    for (int i = lo; i < hi; ++i) c += __ldg(key + i) >= cand ? 1 : 0;
+    for (int i = t; i < n_valid; i += kHybThreads) c += __ldg(key + i) >= cand ? 1 : 0;
     if (hyb_block_sum(c, s_tmp) >= n_sub) T = cand;
   }
   int gt = 0, eq = 0;
@@ -350,6 +351,221 @@ __global__ void __launch_bounds__(128) refresh_kernel(const __nv_bfloat16 *__res
     for (int r = 0; r < m; ++r) s += __bfloat162float(xb[(size_t)__ldg(pb + r) * D + k]);
     mu[((size_t)bh * n_cells + u) * D + k] = s * inv;
   }
+}
+
+// ---- global reassignment on the tensor cores ---------------------------------
+//
+// The same product as reassign_kernel, 128 cached tokens x 128 centroids per
+// step, on tcgen05: A = the tokens' bf16 rows (exact), B = each centroid
+// split into two bf16 rows, mu = hi + lo with hi = bf16(mu) and
+// lo = bf16(mu - hi), both multiplied into one fp32 TMEM accumulator (the
+// split leaves an error below 2^-16 |mu|; the fp32 norms |mu|^2 come from the
+// fp32 centroids).  The operand tiles are written by the threads into 128-byte
+// swizzled shared memory, the B tiles of chunk c + 1 while the MMAs of chunk c
+// run, and two TMEM accumulators let the argmin of chunk c - 1 (thread i =
+// TMEM lane i = token i) overlap the MMAs of chunk c.
+
+constexpr int kRtThreads = 128;
+
+template <int D>
+struct RtLayout {
+  static constexpr int kChunk = 128 * 128;                    // 128 rows x 64 bf16
+  static constexpr int kKc = D / 64;                          // 64-column chunks of d
+  static constexpr int kOffA = 0;                             // [kKc] token tiles
+  static constexpr int kOffB = kOffA + kKc * kChunk;          // [2 buffers][2 parts][kKc]
+  static constexpr int kOffN = kOffB + 2 * 2 * kKc * kChunk;  // [2][128] |mu|^2
+  static constexpr int kOffCtl = kOffN + 2 * 128 * 4;
+  static constexpr int kBytes = kOffCtl + 64;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+struct RtCtl {
+  uint64_t done[2];
+  uint64_t fin;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Row r of a 128-row K-major bf16 tile, 64 columns from v (32 packed pairs).
+__device__ __forceinline__ void rt_store_row(uint8_t *tile, int r, const uint32_t (&v)[32]) {
+  uint8_t *row = tile + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    *reinterpret_cast<uint4 *>(row + ((q ^ (r & 7)) << 4)) = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kRtThreads, 1)
+    reassign_tc_kernel(const __nv_bfloat16 *__restrict__ x, int n_pad, int n_valid, int n_cells,
+                       const float *__restrict__ mu, const int32_t *__restrict__ subset, int n_sub,
+                       int32_t *__restrict__ assign, int32_t *__restrict__ changed, unsigned long long timeout_ns) {
+  using L = RtLayout<D>;
+  extern __shared__ uint8_t rt_smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(rt_smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  float *s_norm = reinterpret_cast<float *>(smem + L::kOffN);
+  RtCtl *ctl = reinterpret_cast<RtCtl *>(smem + L::kOffCtl);
+  volatile int *abort = &ctl->abort;
+  const int bh = blockIdx.y, t = threadIdx.x, warp = t >> 5;
+  const int i = blockIdx.x * kReTok + t;
+  int tok = -1;
+  if (i < n_sub) {
+    tok = __ldg(subset + (size_t)bh * n_sub + i);
+    if (tok < 0 || tok >= n_valid) {
+      latch_status(VSA_ERR_BAD_INDEX);
+      tok = -1;
+    }
+  }
+  // the token tile: thread t writes row t (zeros past the subset)
+  {
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + ((size_t)bh * n_pad + (tok >= 0 ? tok : 0)) * D);
+#pragma unroll
+    for (int kc = 0; kc < L::kKc; ++kc) {
+      uint32_t v[32];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint4 w = tok >= 0 ? __ldg(src + kc * 8 + q) : make_uint4(0u, 0u, 0u, 0u);
+        v[4 * q] = w.x;
+        v[4 * q + 1] = w.y;
+        v[4 * q + 2] = w.z;
+        v[4 * q + 3] = w.w;
+      }
+      rt_store_row(smem + L::kOffA + kc * L::kChunk, t, v);
+    }
+  }
+  if (t == 0) {
+    mbar_init(&ctl->done[0], 1);
+    mbar_init(&ctl->done[1], 1);
+    mbar_init(&ctl->fin, 1);
+    ctl->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&ctl->tmem_base, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  constexpr uint32_t kId = idesc_bf16_f32(128, 128, false);
+  const float *mub = mu + (size_t)bh * n_cells * D;
+  const int n_chunks = (n_cells + 127) / 128;
+  float best = INFINITY;
+  int bcell = 0x7fffffff;
+  bool ok = true;
+
+  auto argmin_chunk = [&](int c) {
+    const int buf = c & 1;
+    const float *nrm = s_norm + buf * 128;
+#pragma unroll 1
+    for (int c0 = 0; c0 < 128; c0 += 32) {
+      uint32_t d[32];
+      tmem_ld32(tmem + lane_off + buf * 128u + c0, d);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int cell = c * 128 + c0 + j;
+        const float dist = fmaf(-2.f, __uint_as_float(d[j]), nrm[c0 + j]);
+        if (cell < n_cells && (dist < best || (dist == best && cell < bcell))) {
+          best = dist;
+          bcell = cell;
+        }
+      }
+    }
+  };
+
+  for (int c = 0; c < n_chunks && ok; ++c) {
+    const int buf = c & 1;
+    if (c >= 2) {
+      const bool w = mbar_wait(&ctl->done[buf], ((c - 2) >> 1) & 1, abort, timeout_ns);
+      ok = __syncthreads_and(w ? 1 : 0) != 0;
+      if (!ok) break;
+    }
+    // centroid c * 128 + t: split into bf16 hi / lo rows, and its fp32 norm
+    {
+      const int cell = c * 128 + t;
+      const float4 *src = reinterpret_cast<const float4 *>(mub + (size_t)(cell < n_cells ? cell : 0) * D);
+      float nrm = 0.f;
+#pragma unroll
+      for (int kc = 0; kc < L::kKc; ++kc) {
+        uint32_t hi[32], lo[32];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const float4 f = cell < n_cells ? __ldg(src + kc * 16 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+          nrm = fmaf(f.x, f.x, nrm);
+          nrm = fmaf(f.y, f.y, nrm);
+          nrm = fmaf(f.z, f.z, nrm);
+          nrm = fmaf(f.w, f.w, nrm);
+          const __nv_bfloat162 h0 = __floats2bfloat162_rn(f.x, f.y), h1 = __floats2bfloat162_rn(f.z, f.w);
+          const float2 g0 = __bfloat1622float2(h0), g1 = __bfloat1622float2(h1);
+          const __nv_bfloat162 l0 = __floats2bfloat162_rn(f.x - g0.x, f.y - g0.y);
+          const __nv_bfloat162 l1 = __floats2bfloat162_rn(f.z - g1.x, f.w - g1.y);
+          hi[2 * q] = *reinterpret_cast<const uint32_t *>(&h0);
+          hi[2 * q + 1] = *reinterpret_cast<const uint32_t *>(&h1);
+          lo[2 * q] = *reinterpret_cast<const uint32_t *>(&l0);
+          lo[2 * q + 1] = *reinterpret_cast<const uint32_t *>(&l1);
+        }
+        rt_store_row(smem + L::kOffB + ((buf * 2 + 0) * L::kKc + kc) * L::kChunk, t, hi);
+        rt_store_row(smem + L::kOffB + ((buf * 2 + 1) * L::kKc + kc) * L::kChunk, t, lo);
+      }
+      s_norm[buf * 128 + t] = nrm;
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (t == 0) {
+      tc_fence_after();
+      bool first = true;
+#pragma unroll
+      for (int part = 0; part < 2; ++part)
+#pragma unroll
+        for (int kc = 0; kc < L::kKc; ++kc) {
+          const uint64_t da = smem_desc_sw128(smem_addr(smem + L::kOffA + kc * L::kChunk), 16, 1024);
+          const uint64_t db = smem_desc_sw128(smem_addr(smem + L::kOffB + ((buf * 2 + part) * L::kKc + kc) * L::kChunk),
+                                              16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            umma_bf16_ss(tmem + buf * 128u, da + 2 * kk, db + 2 * kk, kId, first ? 0u : 1u);
+            first = false;
+          }
+        }
+      umma_commit(&ctl->done[buf]);
+    }
+    if (c >= 1) {
+      const bool w = mbar_wait(&ctl->done[(c - 1) & 1], ((c - 1) >> 1) & 1, abort, timeout_ns);
+      ok = __syncthreads_and(w ? 1 : 0) != 0;
+      if (!ok) break;
+      tc_fence_after();
+      argmin_chunk(c - 1);
+    }
+  }
+  if (ok) {
+    const int c = n_chunks - 1;
+    const bool w = mbar_wait(&ctl->done[c & 1], (c >> 1) & 1, abort, timeout_ns);
+    ok = __syncthreads_and(w ? 1 : 0) != 0;
+    if (ok) {
+      tc_fence_after();
+      argmin_chunk(c);
+    }
+  }
+  // every MMA of the CTA has completed before TMEM and shared memory are released
+  if (t == 0) umma_commit(&ctl->fin);
+  const bool fin = mbar_drain(&ctl->fin, 0, timeout_ns);
+  if (!fin) raise_timeout();
+  if (ok && tok >= 0 && bcell < n_cells) {
+    int32_t *ab = assign + (size_t)bh * n_valid;
+    const int old = ab[tok];
+    if (old != bcell) {
+      ab[tok] = bcell;
+      int32_t *ch = changed + (size_t)bh * n_cells;
+      if (old >= 0 && old < n_cells) ch[old] = 1;
+      ch[bcell] = 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 }  // namespace vsa

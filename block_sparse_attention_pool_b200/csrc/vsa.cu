@@ -1038,16 +1038,16 @@ vsa_status vsa_cluster_refine(const void *x, const vsa_shape *shape, const vsa_c
     const dim3 grid((n_sub + vsa::kReTok - 1) / vsa::kReTok, BH);
     if (shape->d == 128) {
       static const cudaError_t attr = cudaFuncSetAttribute(
-          vsa::reassign_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, vsa::ReLayout<128>::kBytes);
+          vsa::reassign_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, vsa::RtLayout<128>::kAlloc);
       if (attr != cudaSuccess) return VSA_ERR_CUDA;
-      vsa::reassign_kernel<128><<<grid, 256, vsa::ReLayout<128>::kBytes, st>>>(
-          xb, shape->n_pad, shape->n_valid, g.n_cells, centroids, subset, n_sub, assign, changed);
+      vsa::reassign_tc_kernel<128><<<grid, vsa::kRtThreads, vsa::RtLayout<128>::kAlloc, st>>>(
+          xb, shape->n_pad, shape->n_valid, g.n_cells, centroids, subset, n_sub, assign, changed, kWaitLimitNs);
     } else {
       static const cudaError_t attr = cudaFuncSetAttribute(
-          vsa::reassign_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, vsa::ReLayout<64>::kBytes);
+          vsa::reassign_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, vsa::RtLayout<64>::kAlloc);
       if (attr != cudaSuccess) return VSA_ERR_CUDA;
-      vsa::reassign_kernel<64><<<grid, 256, vsa::ReLayout<64>::kBytes, st>>>(
-          xb, shape->n_pad, shape->n_valid, g.n_cells, centroids, subset, n_sub, assign, changed);
+      vsa::reassign_tc_kernel<64><<<grid, vsa::kRtThreads, vsa::RtLayout<64>::kAlloc, st>>>(
+          xb, shape->n_pad, shape->n_valid, g.n_cells, centroids, subset, n_sub, assign, changed, kWaitLimitNs);
     }
   }
   const dim3 cgrid(n_chunks, BH);
