@@ -937,7 +937,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="vsa", choices=["vsa", "reference"])
     ap.add_argument("--workload", default="hunyuan", choices=sorted(WORKLOADS))
-    ap.add_argument("--ref-blocks", type=int, default=6, help="query blocks per oracle sample")
+    ap.add_argument("--ref-blocks", type=int, default=60, help="query blocks per oracle sample (reference arm)")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--chunk-heads", type=int, default=2, help="heads per pipelined chunk of the e2e leg")
     ap.add_argument("--sweep", action="store_true", help="print the sparsity-sweep lines instead of the bench line")
@@ -996,7 +997,14 @@ def main():
                                              device_id=torch.device("cuda", local_rank))
     line = run_gpu(args, rank, world, local_rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        f, s, desc = oracle_sample(WORKLOADS[args.workload], budget_blocks=args.ref_blocks)
+        # size the sample to about 12 s of CPU work: a short calibration run, then the reported one
+        w = WORKLOADS[args.workload]
+        _, s2, _ = oracle_sample(w, budget_blocks=2)
+        _, s6, _ = oracle_sample(w, budget_blocks=6)
+        per_block = max((s6 - s2) / 4, 1e-4)
+        fixed = max(0.0, s2 - 2 * per_block)
+        n_blocks = int(max(6, min(w.n_pad // w.bq, round((args.cpu_seconds - fixed) / per_block))))
+        f, s, desc = oracle_sample(w, budget_blocks=n_blocks)
         line["cpu_baseline"] = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
                                 "sample": desc, "seconds": round(s, 2)}
     if rank == 0:
