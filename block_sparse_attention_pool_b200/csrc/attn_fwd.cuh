@@ -629,7 +629,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (n_stages > 0 && lane == 0) {
+    // The whole warp runs the issuing loop in lockstep; one elected lane
+    // issues each MMA and commit, so descriptors stay warp-uniform.
+    if (n_stages > 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(kTileM, kStageKeys, false);
       constexpr uint32_t kIdO = idesc_bf16_f32(kTileM, D, true);
       // descriptor bases; K steps and ring slots only add to the start address field
@@ -637,10 +639,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t dK0 = smem_desc_sw128(smem_addr(sK), 16, 1024);
       const uint64_t dV0 = smem_desc_sw128(smem_addr(sV), kChunkBytes, 1024);
       constexpr uint64_t kSlotStep = L::kKVBytes >> 4;
-      bool ok = mbar_wait(&ctl->q_full, 0, abort, a.timeout_ns);
+      const uint32_t leader = elect_one();
+      bool ok = mbar_wait_uni(&ctl->q_full, 0, abort, a.timeout_ns, lane);
       auto issue_pv = [&](int t) -> bool {
-        if (!mbar_wait(&ctl->p_full[t & 1], (t >> 1) & 1, abort, a.timeout_ns)) return false;
-        if (!mbar_wait(&ctl->v_full[t & 1], (t >> 1) & 1, abort, a.timeout_ns)) return false;
+        if (!mbar_wait_uni(&ctl->p_full[t & 1], (t >> 1) & 1, abort, a.timeout_ns, lane)) return false;
+        if (!mbar_wait_uni(&ctl->v_full[t & 1], (t >> 1) & 1, abort, a.timeout_ns, lane)) return false;
         tc_fence_after();
         const uint64_t dv = dV0 + (uint64_t)(t & 1) * kSlotStep;
         const uint32_t to = (t & 1) ? tO[1] : tO[0];
@@ -648,15 +651,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kStageKeys / 16; ++kk) {
           // P (bf16 pairs) sits in the first 64 columns of the stage's S buffer
-          umma_bf16_ts(to, ts + kk * 8, dv + (uint64_t)(kk * 16 * 128 / 16), kIdO, (t >= 2 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts_one(to, ts + kk * 8, dv + (uint64_t)(kk * 16 * 128 / 16), kIdO,
+                           (t >= 2 || kk > 0) ? 1u : 0u, leader);
         }
-        umma_commit(&ctl->v_empty[t & 1]);
+        umma_commit_one(&ctl->v_empty[t & 1], leader);
         return true;
       };
       for (int s = 0; ok && s < n_stages; ++s) {
         const int slot = s & 1;
-        ok = mbar_wait(&ctl->k_full[slot], (s >> 1) & 1, abort, a.timeout_ns);
-        if (ok && s >= 2) ok = mbar_wait(&ctl->s_free[slot], ((s - 2) >> 1) & 1, abort, a.timeout_ns);
+        ok = mbar_wait_uni(&ctl->k_full[slot], (s >> 1) & 1, abort, a.timeout_ns, lane);
+        if (ok && s >= 2) ok = mbar_wait_uni(&ctl->s_free[slot], ((s - 2) >> 1) & 1, abort, a.timeout_ns, lane);
         if (!ok) break;
         tc_fence_after();
         const uint64_t dk = dK0 + (uint64_t)slot * kSlotStep;
@@ -664,15 +668,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
-          umma_bf16_ss(ts, dQ + off, dk + off, kIdS, kk > 0 ? 1u : 0u);
+          umma_bf16_ss_one(ts, dQ + off, dk + off, kIdS, kk > 0 ? 1u : 0u, leader);
         }
-        umma_commit(&ctl->k_empty[slot]);
-        umma_commit(&ctl->s_full[slot]);
+        umma_commit_one(&ctl->k_empty[slot], leader);
+        umma_commit_one(&ctl->s_full[slot], leader);
         if (s >= 1) ok = issue_pv(s - 1);
       }
       if (ok) issue_pv(n_stages - 1);
-      // every MMA issued by this thread has completed once mma_drain flips
-      umma_commit(&ctl->mma_drain);
+      // every MMA issued by the leader has completed once mma_drain flips
+      umma_commit_one(&ctl->mma_drain, leader);
       mbar_drain(&ctl->mma_drain, 0, a.timeout_ns);
     }
   } else {
