@@ -39,6 +39,7 @@ EXPORTED = (
     "vsa_status_string", "vsa_version", "vsa_read_device_status", "vsa_pool_qk", "vsa_select_blocks",
     "vsa_mask_to_lists", "vsa_select_micro_workspace_bytes", "vsa_select_micro", "vsa_select_micro_noalloc",
     "vsa_block_sparse_fwd", "vsa_block_sparse_fwd_heads", "vsa_lse_merge", "vsa_selftest_wait_timeout",
+    "vsa_selftest_exp2",
     "vsa_cluster_count", "vsa_cluster_tokens", "vsa_permute_rows", "vsa_select_clusters",
     "vsa_merge_clusters_workspace_bytes", "vsa_merge_clusters", "vsa_cluster_rows_capacity", "vsa_cluster_plan",
     "vsa_gather_rows", "vsa_cluster_group_fwd", "vsa_pool_kv_bf16", "vsa_rectify_fwd", "vsa_cluster_anchor",
@@ -109,6 +110,8 @@ def lib():
     L.vsa_read_device_status.argtypes = [P]
     L.vsa_selftest_wait_timeout.restype = I
     L.vsa_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, P]
+    L.vsa_selftest_exp2.restype = I
+    L.vsa_selftest_exp2.argtypes = [P, P, ctypes.c_int, P]
     L.vsa_pool_qk.restype = I
     L.vsa_pool_qk.argtypes = [P, P, SP, I, I, P, P, P, P, P]
     L.vsa_select_blocks.restype = I
@@ -201,6 +204,16 @@ def selftest_wait_timeout(limit_ns: int, stream=None) -> None:
     """Launch the bounded-wait self-test (a wait nothing completes, given up
     after limit_ns); the device status then reads VSA_ERR_TIMEOUT."""
     _check(lib().vsa_selftest_wait_timeout(int(limit_ns), _s(stream)), "vsa_selftest_wait_timeout")
+
+
+def selftest_exp2(x: torch.Tensor, y: torch.Tensor, stream=None) -> None:
+    """y = 2**x by the exponential the attention softmax runs on the FMA pipe
+    for part of its logits (x, y: contiguous fp32 device tensors of one size)."""
+    if x.dtype != torch.float32 or y.dtype != torch.float32 or x.numel() != y.numel():
+        raise ValueError("x and y must be fp32 tensors of the same size")
+    if not (x.is_contiguous() and y.is_contiguous()):
+        raise ValueError("x and y must be contiguous")
+    _check(lib().vsa_selftest_exp2(_p(x), _p(y), int(x.numel()), _s(stream)), "vsa_selftest_exp2")
 
 
 def pool_qk(q, k, shape: Shape, bq, bk, q_pool, k_pool, q_pool64=None, k_pool16=None, stream=None):

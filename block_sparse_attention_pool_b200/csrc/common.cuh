@@ -111,6 +111,35 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return d;
 }
 
+// 2^x of a pair on the FMA pipe, to take part of the softmax's exponentials
+// off the MUFU unit.  Range reduction after Cody and Waite, with the rounding
+// done by adding 1.5 * 2^23 (x + c holds round(x) in its low mantissa bits):
+// x = n + f, n integer, f in [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted
+// here for minimax relative error on that interval (max 7.5e-5, about 2^-13.7,
+// well below the 2^-9 of the bf16 rounding P gets next); 2^n added to the
+// exponent field as an integer.  x is clamped at -125 so the result stays a
+// normal number: masked logits (-inf) give 2^-125 (about 2.4e-38), not 0.
+constexpr float kExp2C0 = 0.99992806f;
+constexpr float kExp2C1 = 0.69326097f;
+constexpr float kExp2C2 = 0.24261114f;
+constexpr float kExp2C3 = 0.05517167f;
+
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 j = fadd2(x, make_float2(kRound, kRound));   // 1.5 * 2^23 + round(x), exactly
+  const float2 n = fadd2(j, make_float2(-kRound, -kRound));  // round(x)
+  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);     // x - round(x), exactly
+  float2 p = ffma2(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
+  p = ffma2(p, f, make_float2(kExp2C1, kExp2C1));
+  p = ffma2(p, f, make_float2(kExp2C0, kExp2C0));
+  // the low 9 bits of j's pattern hold round(x) (two's complement): shifted to
+  // the exponent field they add round(x) to p's exponent
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(j.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(j.y) << 23)));
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -273,6 +273,16 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
   vsa::mbar_wait(&bar, 0, &abort_flag, limit_ns);
 }
 
+// The softmax's FMA-pipe exponential on a caller's array, two values per thread.
+__global__ void selftest_exp2_kernel(const float *__restrict__ x, float *__restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float2 in = make_float2(x[i], i + 1 < n ? x[i + 1] : 0.f);
+  const float2 out = vsa::exp2_poly2(in);
+  y[i] = out.x;
+  if (i + 1 < n) y[i + 1] = out.y;
+}
+
 // Per-head slot numbers handed to the device by value (no host-to-device copy).
 struct HeadSlots {
   int16_t slot[kNoallocMaxBH];  // rank among enabled heads, or -1
@@ -488,6 +498,15 @@ vsa_status vsa_read_device_status(void *stream) {
 vsa_status vsa_selftest_wait_timeout(unsigned long long limit_ns, void *stream) {
   if (limit_ns < 1000ull || limit_ns > 5000000000ull) return VSA_ERR_INVALID_ARG;
   selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  return launch_status();
+}
+
+vsa_status vsa_selftest_exp2(const float *x, float *y, int n, void *stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return VSA_ERR_INVALID_ARG;
+  if (n == 0) return VSA_OK;
+  const int threads = 256;
+  const int blocks = (n / 2 + 1 + threads - 1) / threads;
+  selftest_exp2_kernel<<<blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
   return launch_status();
 }
 

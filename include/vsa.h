@@ -142,6 +142,15 @@ VSA_API vsa_status vsa_read_device_status(void *stream);
  * still running give up, until vsa_read_device_status clears it. */
 VSA_API vsa_status vsa_selftest_wait_timeout(unsigned long long limit_ns, void *stream);
 
+/* Self-test of the exponential the attention softmax evaluates on the FMA
+ * pipe for part of its logits (no counterpart on the pages; the softmax of
+ * HyperVAttention Eq. (4) needs 2^x per kept logit): y[i] = 2^x[i] by range
+ * reduction to x = n + f, |f| <= 1/2, a degree-3 polynomial for 2^f (relative
+ * error at most 7.5e-5) and an exponent add.  Inputs below -125 (and -inf)
+ * give 2^-125.  x, y: device fp32 [n], n >= 0.
+ * Asynchronous on ``stream``; argument errors return synchronously. */
+VSA_API vsa_status vsa_selftest_exp2(const float *x, float *y, int n, void *stream);
+
 /* ---------------------------------------------------------------------------
  * a1 Pooling  ([RSA]: pooled query-key interactions; [HVA] section 4.1: a
  * centroid is the mean of its tokens; [MOD]: fixed non-overlapping blocks.)

@@ -320,6 +320,34 @@ def test_bounded_wait_times_out_and_device_stays_usable():
     assert vsa.read_device_status() == 0
 
 
+def test_softmax_exp2_matches_cuda_exp2_within_its_bound():
+    """The exponential the Macro softmax runs on the FMA pipe for part of its
+    logits, against CUDA's exp2 (torch.exp2 on the device): relative error
+    within the polynomial's 7.5e-5 plus fp32 evaluation rounding over the
+    logit range the softmax produces ([-125, 8] after the lazy-rescale
+    threshold of 2^8), every integer and half-integer included; masked
+    logits (-inf) and anything below -125 give 2^-125 x (1 +- 7.5e-5)."""
+    g = torch.Generator(device="cuda").manual_seed(11)
+    x = torch.cat([torch.linspace(-125.0, 8.0, 1 << 20, device="cuda"),
+                   torch.arange(-125.0, 8.5, 0.5, device="cuda"),
+                   torch.rand(100_001, device="cuda", generator=g) * 133.0 - 125.0])
+    y = torch.empty_like(x)
+    vsa.selftest_exp2(x, y)
+    ref = torch.exp2(x)
+    rel = ((y.double() - ref.double()).abs() / ref.double()).max().item()
+    assert rel <= 7.5e-5 + 4 * 2.0 ** -24, rel
+    low = torch.tensor([-float("inf"), -1000.0, -126.5, -125.0], device="cuda")
+    y_low = torch.empty_like(low)
+    vsa.selftest_exp2(low, y_low)
+    assert torch.all(y_low == y_low[-1])
+    assert abs(y_low[-1].item() / 2.0 ** -125 - 1.0) <= 7.5e-5
+    # odd length: the last element of the final pair
+    xo = torch.tensor([0.0, 1.0, -2.0], device="cuda")
+    yo = torch.full_like(xo, float("nan"))
+    vsa.selftest_exp2(xo, yo)
+    assert torch.allclose(yo, torch.exp2(xo), rtol=8e-5, atol=0.0)
+
+
 # ---------------------------------------------------------------------------
 # a6 merge
 # ---------------------------------------------------------------------------
