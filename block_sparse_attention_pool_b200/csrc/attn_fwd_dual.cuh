@@ -58,7 +58,12 @@ constexpr int kDualList = 1024;  // list entries staged per tile (every list of 
 // (exp2_poly2) instead of MUFU: a 128-key row needs as many MUFU (XU) cycles
 // as the tile's MMAs take, so part of the work moves to the FMA pipe.  Kernel
 // time of a dense launch (8 heads, 16K tokens) by share moved: 0% 1.084 ms,
-// 12.5% 1.005, 25% 1.013, 37.5% 1.018, 50% 1.068.
+// 12.5% 1.005, 25% 1.013, 37.5% 1.018, 50% 1.068.  Masked logits come out as
+// 2^-125 instead of 0 on these pairs; here the only masked keys are padding
+// keys (past n_valid), whose V rows arrive as zeros, so they add nothing to O
+// and vanish in any row sum that holds a real key.  (The single-tile kernel,
+// which also masks keys of the other query half, keeps MUFU for every logit:
+// there the split measured 2% slower.)
 constexpr uint32_t kEmuPairs = 0x8080u;
 
 template <int D>
