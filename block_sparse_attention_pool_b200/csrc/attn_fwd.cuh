@@ -206,30 +206,12 @@ __device__ __forceinline__ int lower_bound_smem(const int32_t *p, int n, int v) 
 // list-0 entry is dropped and that list-0 entry is tagged for both -- and one
 // compaction pass closes the gaps.  Returns the union size, or -1 when a
 // list is invalid.  su holds n0 + n1 entries of scratch.
-__device__ __forceinline__ int stage_union(const int32_t *g0, int n0, const int32_t *g1, int n1, int n_lists,
-                                           int n_max, int32_t *sl, int stride, uint32_t *su, uint32_t single_tag,
-                                           int lane) {
-  const int cnt[2] = {n0, n_lists > 1 ? n1 : 0};
-  const int32_t *src[2] = {g0, g1};
-  for (int h = 0; h < n_lists; ++h)
-    for (int e = lane; e < cnt[h]; e += 32) sl[h * stride + e] = __ldg(src[h] + e);
-  __syncwarp();
-  bool ok = true;
-  for (int h = 0; h < n_lists; ++h) {
-    const int32_t *li = sl + h * stride;
-    for (int e = lane; e < cnt[h]; e += 32) {
-      const int v = li[e];
-      if (v < 0 || v >= n_max || (e > 0 && li[e - 1] >= v)) ok = false;
-    }
-  }
-  if (!__all_sync(0xffffffffu, ok)) return -1;
-  if (n_lists == 1) {
-    for (int e = lane; e < cnt[0]; e += 32) su[e] = static_cast<uint32_t>(sl[e]) | (single_tag << 30);
-    __syncwarp();
-    return cnt[0];
-  }
-  const int32_t *A = sl, *B = sl + stride;
-  const int nA = cnt[0], nB = cnt[1];
+// Rank merge of two ascending lists already in shared memory into their
+// ascending union su, each entry tagged (bits 30-31) with the lists that hold
+// it (1 = A, 2 = B, 3 = both); returns the union's length.  su needs room for
+// nA + nB entries until the closing compaction.
+__device__ __forceinline__ int merge_staged(const int32_t *A, int nA, const int32_t *B, int nB, uint32_t *su,
+                                            int lane) {
   for (int i = lane; i < nA; i += 32) {
     const int v = A[i];
     const int r = lower_bound_smem(B, nB, v);
@@ -254,6 +236,31 @@ __device__ __forceinline__ int stage_union(const int32_t *g0, int n0, const int3
     __syncwarp();
   }
   return n;
+}
+
+__device__ __forceinline__ int stage_union(const int32_t *g0, int n0, const int32_t *g1, int n1, int n_lists,
+                                           int n_max, int32_t *sl, int stride, uint32_t *su, uint32_t single_tag,
+                                           int lane) {
+  const int cnt[2] = {n0, n_lists > 1 ? n1 : 0};
+  const int32_t *src[2] = {g0, g1};
+  for (int h = 0; h < n_lists; ++h)
+    for (int e = lane; e < cnt[h]; e += 32) sl[h * stride + e] = __ldg(src[h] + e);
+  __syncwarp();
+  bool ok = true;
+  for (int h = 0; h < n_lists; ++h) {
+    const int32_t *li = sl + h * stride;
+    for (int e = lane; e < cnt[h]; e += 32) {
+      const int v = li[e];
+      if (v < 0 || v >= n_max || (e > 0 && li[e - 1] >= v)) ok = false;
+    }
+  }
+  if (!__all_sync(0xffffffffu, ok)) return -1;
+  if (n_lists == 1) {
+    for (int e = lane; e < cnt[0]; e += 32) su[e] = static_cast<uint32_t>(sl[e]) | (single_tag << 30);
+    __syncwarp();
+    return cnt[0];
+  }
+  return merge_staged(sl, cnt[0], sl + stride, cnt[1], su, lane);
 }
 
 // Warp-cooperative validation of one list (strictly ascending, in range);

@@ -66,7 +66,7 @@ constexpr int kDualList = 1024;  // list entries staged per tile (every list of 
 // there the split measured 2% slower.)
 constexpr uint32_t kEmuPairs = 0x8080u;
 
-template <int D>
+template <int D, bool kHalf>
 struct DualSmem {
   static constexpr int kQBytes = kTileM * D * 2;
   static constexpr int kKVBytes = kStageKeys * D * 2;
@@ -75,7 +75,10 @@ struct DualSmem {
   static constexpr int kOffV = kOffK + 2 * kKVBytes;
   static constexpr int kOffU = kOffV + 2 * kKVBytes;          // union of the two lists [kDualList * 2]
   static constexpr int kOffL = kOffU + 2 * kDualList * 4;     // the two lists, staged [2][kDualList]
-  static constexpr int kOffCtl = kOffL + 2 * kDualList * 4;
+  // 64-row lists: per tile, the union of its two halves' lists, tagged with
+  // the halves that kept each block [2][kDualList]
+  static constexpr int kOffUX = kOffL + 2 * kDualList * 4;
+  static constexpr int kOffCtl = kOffUX + (kHalf ? 2 * kDualList * 4 : 0);
   static constexpr int kBytes = kOffCtl + 512;
   static constexpr int kAlloc = kBytes + 1024;
 };
@@ -95,11 +98,15 @@ struct DualCtl {
   int fast;  // union and lists staged in shared memory
 };
 
-template <int D>
+// kHalf: lists of 64-row query blocks (two per 128-row tile) instead of one
+// list per tile.  Each tile then walks the union of its halves' lists; the
+// softmax warps of a half that did not keep a block write P = 0 for it (their
+// rows' S is computed all the same: one M = 128 MMA covers both halves).
+template <int D, bool kHalf>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_dual_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
-  using L = DualSmem<D>;
+  using L = DualSmem<D, kHalf>;
   extern __shared__ uint8_t dual_smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dual_smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -146,34 +153,92 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     int cnt[2] = {0, 0};
     bool ok = true;
-    for (int x = 0; x < (has_b ? 2 : 1); ++x) {
-      cnt[x] = __ldg(a.counts + lrow0 + x);
-      if (cnt[x] < 0 || cnt[x] > a.idx_stride) ok = false;
-    }
-    // lists short enough to stage: validated and merged into the union in
-    // shared memory once; otherwise validated here and walked from global
-    // memory by ListCursor
-    const bool fast = ok && cnt[0] <= kDualList && cnt[1] <= kDualList;
-    int n_union = cnt[0] + cnt[1];  // cursor path: > 0 iff the union is not empty
-    if (fast) {
-      n_union = stage_union(a.idx + lrow0 * a.idx_stride, cnt[0], a.idx + (lrow0 + 1) * a.idx_stride, cnt[1],
-                            has_b ? 2 : 1, n_key_blocks, reinterpret_cast<int32_t *>(smem + L::kOffL), kDualList,
-                            reinterpret_cast<uint32_t *>(smem + L::kOffU), 1u, lane);
-      ok = n_union >= 0;
+    if (kHalf) {
+      // four 64-row lists (A0, A1, B0, B1); the host sends only layers of at
+      // most kDualList key blocks here, so every valid list fits in shared memory
+      const size_t hrow0 = (size_t)bh * (a.n_pad / 64) + 2 * tile0;
+      int c4[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        if (x < (has_b ? 4 : 2)) {
+          c4[x] = __ldg(a.counts + hrow0 + x);
+          if (c4[x] < 0 || c4[x] > a.idx_stride || c4[x] > kDualList) ok = false;
+        }
+      }
+      uint32_t *su_w = reinterpret_cast<uint32_t *>(smem + L::kOffU);
+      int32_t *sl_w = reinterpret_cast<int32_t *>(smem + L::kOffL);
+      uint32_t *ux_w = reinterpret_cast<uint32_t *>(smem + L::kOffUX);
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        if (ok && x < (has_b ? 2 : 1)) {
+          // tile x: union of its two halves, tags 1 = rows 0-63, 2 = rows 64-127
+          const int n = stage_union(a.idx + (hrow0 + 2 * x) * a.idx_stride, c4[2 * x],
+                                    a.idx + (hrow0 + 2 * x + 1) * a.idx_stride, c4[2 * x + 1], 2, n_key_blocks,
+                                    sl_w, kDualList, su_w, 1u, lane);
+          if (n < 0) {
+            ok = false;
+          } else {
+            for (int e = lane; e < n; e += 32) ux_w[x * kDualList + e] = su_w[e];
+            __syncwarp();
+            cnt[x] = n;
+          }
+        }
+      }
+      int n_union = 0;
+      if (ok) {
+        // the union of the two tiles' unions drives the loads and the MMAs
+#pragma unroll
+        for (int x = 0; x < 2; ++x)
+          for (int e = lane; e < cnt[x]; e += 32)
+            sl_w[x * kDualList + e] = static_cast<int32_t>(ux_w[x * kDualList + e] & 0x3fffffffu);
+        __syncwarp();
+        if (has_b) {
+          n_union = merge_staged(sl_w, cnt[0], sl_w + kDualList, cnt[1], su_w, lane);
+        } else {
+          for (int e = lane; e < cnt[0]; e += 32) su_w[e] = static_cast<uint32_t>(sl_w[e]) | (1u << 30);
+          __syncwarp();
+          n_union = cnt[0];
+        }
+      } else {
+        if (lane == 0) latch_status(VSA_ERR_BAD_INDEX);
+        cnt[0] = cnt[1] = 0;
+      }
+      if (lane == 0) {
+        ctl->n_union = n_union;
+        ctl->cnt[0] = cnt[0];
+        ctl->cnt[1] = cnt[1];
+        ctl->fast = 1;
+      }
     } else {
-      for (int x = 0; x < (has_b ? 2 : 1) && ok; ++x)
-        ok = list_valid(a.idx + (lrow0 + x) * a.idx_stride, cnt[x], n_key_blocks, lane);
-    }
-    if (!ok) {
-      if (lane == 0) latch_status(VSA_ERR_BAD_INDEX);
-      cnt[0] = cnt[1] = 0;
-      n_union = 0;
-    }
-    if (lane == 0) {
-      ctl->n_union = n_union;
-      ctl->cnt[0] = cnt[0];
-      ctl->cnt[1] = cnt[1];
-      ctl->fast = fast ? 1 : 0;
+      for (int x = 0; x < (has_b ? 2 : 1); ++x) {
+        cnt[x] = __ldg(a.counts + lrow0 + x);
+        if (cnt[x] < 0 || cnt[x] > a.idx_stride) ok = false;
+      }
+      // lists short enough to stage: validated and merged into the union in
+      // shared memory once; otherwise validated here and walked from global
+      // memory by ListCursor
+      const bool fast = ok && cnt[0] <= kDualList && cnt[1] <= kDualList;
+      int n_union = cnt[0] + cnt[1];  // cursor path: > 0 iff the union is not empty
+      if (fast) {
+        n_union = stage_union(a.idx + lrow0 * a.idx_stride, cnt[0], a.idx + (lrow0 + 1) * a.idx_stride, cnt[1],
+                              has_b ? 2 : 1, n_key_blocks, reinterpret_cast<int32_t *>(smem + L::kOffL), kDualList,
+                              reinterpret_cast<uint32_t *>(smem + L::kOffU), 1u, lane);
+        ok = n_union >= 0;
+      } else {
+        for (int x = 0; x < (has_b ? 2 : 1) && ok; ++x)
+          ok = list_valid(a.idx + (lrow0 + x) * a.idx_stride, cnt[x], n_key_blocks, lane);
+      }
+      if (!ok) {
+        if (lane == 0) latch_status(VSA_ERR_BAD_INDEX);
+        cnt[0] = cnt[1] = 0;
+        n_union = 0;
+      }
+      if (lane == 0) {
+        ctl->n_union = n_union;
+        ctl->cnt[0] = cnt[0];
+        ctl->cnt[1] = cnt[1];
+        ctl->fast = fast ? 1 : 0;
+      }
     }
   } else if (warp == 1) {
     tmem_alloc(&ctl->tmem_base, kTmemCols);
@@ -195,6 +260,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int n_union = ctl->n_union;
   const uint32_t *su = reinterpret_cast<const uint32_t *>(smem + L::kOffU);
   const int32_t *sl = reinterpret_cast<const int32_t *>(smem + L::kOffL);
+  const uint32_t *ux = reinterpret_cast<const uint32_t *>(smem + (kHalf ? L::kOffUX : L::kOffL));
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -372,12 +438,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     bool ok = true;
     const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
     const int n_mine = tile_live ? (x == 0 ? cnt[0] : cnt[1]) : 0;
+    const uint32_t *uxx = ux + x * kDualList;              // 64-row lists: this tile's tagged union
+    const uint32_t half_tag = 1u << (30 + (quad >> 1));     // rows 0-63 are lane quadrants 0, 1
     for (int i = 0; i < n_mine; ++i) {
-      const int key0 = (fast ? sl[x * kDualList + i] : __ldg(listx + i)) * kStageKeys;
+      int key0;
+      bool mine = true;  // this warp's rows kept the block
+      if (kHalf) {
+        const uint32_t e = uxx[i];
+        key0 = static_cast<int>(e & 0x3fffffffu) * kStageKeys;
+        mine = (e & half_tag) != 0u;
+      } else {
+        key0 = (fast ? sl[x * kDualList + i] : __ldg(listx + i)) * kStageKeys;
+      }
       ok = mbar_wait_warp(&ctl->s_full[x], i & 1, abort, a.timeout_ns, lane);
       if (!ok) break;
       tc_fence_after();
       uint32_t r[4][32];
+      if (kHalf && !mine) {
+        // the other half of the tile kept this block: P = 0 for these rows
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[0][j] = 0u;
+        tmem_st32(tSx + lane_off + 0, r[0]);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&ctl->p_half[x]);
+        tmem_st32(tSx + lane_off + 32, r[0]);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&ctl->p_full[x]);
+        continue;
+      }
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tSx + lane_off + c * 32, r[c]);
       tmem_ld_wait();

@@ -174,15 +174,15 @@ vsa_status launch_attn(const void *q, const void *k, const void *v, const vsa_sh
 
 // 128-row lists of 128-key blocks: two adjacent query tiles per CTA share
 // their K/V loads (attn_fwd_dual_kernel).
-template <int D>
+template <int D, bool kHalf>
 vsa_status launch_attn_dual(const void *q, const void *k, const void *v, const vsa_shape *s, const AttnArgs &a,
                             int n_heads, cudaStream_t st) {
-  using L = vsa::DualSmem<D>;
+  using L = vsa::DualSmem<D, kHalf>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
     attr_err =
-        cudaFuncSetAttribute(vsa::attn_fwd_dual_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+        cudaFuncSetAttribute(vsa::attn_fwd_dual_kernel<D, kHalf>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   });
   if (attr_err != cudaSuccess) return VSA_ERR_CUDA;
   CUtensorMap mq, mk, mv;
@@ -190,7 +190,7 @@ vsa_status launch_attn_dual(const void *q, const void *k, const void *v, const v
     return VSA_ERR_CUDA;
   const int n_tiles = s->n_pad / vsa::kTileM;
   dim3 grid((n_tiles + 1) / 2, n_heads);
-  vsa::attn_fwd_dual_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, a);
+  vsa::attn_fwd_dual_kernel<D, kHalf><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, a);
   return launch_status();
 }
 
@@ -749,8 +749,14 @@ vsa_status vsa_block_sparse_fwd_heads(const void *q, const void *k, const void *
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (n_heads == 0) return VSA_OK;
   if (list_rows == 128 && seg_keys == 128)
-    return shape->d == 128 ? launch_attn_dual<128>(q, k, v, shape, a, n_heads, st)
-                             : launch_attn_dual<64>(q, k, v, shape, a, n_heads, st);
+    return shape->d == 128 ? launch_attn_dual<128, false>(q, k, v, shape, a, n_heads, st)
+                             : launch_attn_dual<64, false>(q, k, v, shape, a, n_heads, st);
+  // 64-row lists of 128-key blocks: two query blocks per tile, two tiles per
+  // CTA, when the tiles are whole and every list fits the staged union
+  if (list_rows == 64 && seg_keys == 128 && shape->n_pad % vsa::kTileM == 0 &&
+      shape->n_pad / vsa::kStageKeys <= vsa::kDualList)
+    return shape->d == 128 ? launch_attn_dual<128, true>(q, k, v, shape, a, n_heads, st)
+                             : launch_attn_dual<64, true>(q, k, v, shape, a, n_heads, st);
   return shape->d == 128 ? launch_attn<128>(q, k, v, shape, a, n_heads, st) : launch_attn<64>(q, k, v, shape, a, n_heads, st);
 }
 

@@ -198,11 +198,14 @@ def test_attention_sweep_points(point):
 
 
 @pytest.mark.parametrize("n_pad,list_rows,seg", [(512, 128, 32), (512, 64, 32), (512, 64, 128), (512, 128, 16),
-                                                 (512, 128, 128), (384, 128, 128), (640, 128, 128)])
+                                                 (512, 128, 128), (384, 128, 128), (640, 128, 128),
+                                                 (384, 64, 128), (640, 64, 128)])
 def test_attention_ragged_and_empty_rows(n_pad, list_rows, seg):
     """n_valid not a multiple of the block, a row with an empty list, lists of
     different lengths in one 128-row tile (64-row lists), short segments, and
-    the two-tile 128x128 path with an even and an odd number of query tiles."""
+    the two-tile path (128-row lists, and 64-row lists of 128-key blocks, where
+    each half of a tile keeps its own blocks) with an even and an odd number
+    of query tiles."""
     rng = np.random.default_rng(9 + n_pad + seg)
     B, H, d = 1, 2, 128
     n_valid = n_pad - 75
@@ -226,7 +229,7 @@ def test_attention_ragged_and_empty_rows(n_pad, list_rows, seg):
     assert_close_rows(o.cpu().numpy(), lse.cpu().numpy(), O, L, [(0, h, 0, n_pad) for h in range(H)])
 
 
-@pytest.mark.parametrize("list_rows,seg", [(128, 128), (64, 16)])
+@pytest.mark.parametrize("list_rows,seg", [(128, 128), (64, 128), (64, 16)])
 def test_attention_head_subset(list_rows, seg):
     """vsa_block_sparse_fwd_heads on some (batch, head) pairs, given in any
     order, writes for them exactly what the all-heads call writes, leaves the
