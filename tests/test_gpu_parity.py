@@ -294,6 +294,54 @@ def test_attention_long_lists_both_union_paths():
                       [(b, h, r * list_rows, (r + 1) * list_rows) for b, h, r in rows])
 
 
+def test_attention_64row_lists_on_both_kernels():
+    """64-row lists of 128-key blocks: up to 1024 key blocks they run on the
+    two-tile kernel (each tile walks the union of its halves' lists), beyond
+    that on the single-tile kernel.  A layer of 1032 key blocks, with rows
+    where one half of a tile keeps nothing, rows where both halves keep the
+    same blocks and rows with disjoint lists, against the oracle on sampled
+    rows; the same lists on the first 1024 blocks take the two-tile kernel."""
+    rng = np.random.default_rng(5)
+    B, H, d, seg, list_rows = 1, 1, 64, 128, 64
+    for n_blocks in (1032, 1024):
+        n_pad = seg * n_blocks
+        n_valid = n_pad - 33
+        q, k, v = (round_to_bf16(rng.standard_normal((B, H, n_pad, d)).astype(np.float32)) for _ in range(3))
+        n_l, n_s = n_pad // list_rows, n_pad // seg
+        pick = lambda n: np.sort(rng.choice(n_s, size=n, replace=False))
+        kept = [[[pick(int(rng.integers(1, 12))) for _ in range(n_l)]]]
+        kept[0][0][4] = np.zeros(0, dtype=np.int64)          # tile 2: half 0 keeps nothing
+        kept[0][0][7] = kept[0][0][6].copy()                  # tile 3: both halves alike
+        kept[0][0][n_l - 1] = np.array([n_s - 1])             # last tile: the ragged block only
+        counts, idx = lists_to_dev(kept, n_s, B, H, n_l)
+        shape = vsa.Shape(B, H, n_valid, n_pad, d)
+        o = torch.empty(B, H, n_pad, d, device="cuda")
+        lse = torch.empty(B, H, n_pad, device="cuda")
+        scale = 1 / math.sqrt(d)
+        vsa.block_sparse_fwd(to_dev(q), to_dev(k), to_dev(v), shape, list_rows, seg, counts, idx, n_s, scale, o,
+                             lse)
+        assert vsa.read_device_status() == 0
+        rows = [(0, 0, r) for r in (0, 1, 4, 5, 6, 7, 501, n_l - 2, n_l - 1)]
+        O, L = orc.block_sparse_attention(q, k, v, kept, list_rows, seg, n_valid, scale, rows=rows)
+        assert_close_rows(o.cpu().numpy(), lse.cpu().numpy(), O, L,
+                          [(b, h, r * list_rows, (r + 1) * list_rows) for b, h, r in rows])
+
+
+def test_attention_bad_64row_list_latches_status():
+    """A descending 64-row list in the two-tile kernel: the status word reads
+    VSA_ERR_BAD_INDEX and the CTA's tiles write O = 0, LSE = -inf."""
+    B, H, n_pad, d = 1, 1, 256, 128
+    q = torch.zeros(B, H, n_pad, d, device="cuda", dtype=torch.bfloat16)
+    counts = torch.tensor([[[1, 2, 1, 0]]], dtype=torch.int32, device="cuda")
+    idx = torch.tensor([[[[0, 0], [1, 0], [1, 0], [0, 0]]]], dtype=torch.int32, device="cuda")   # row 1 descending
+    o = torch.empty(B, H, n_pad, d, device="cuda", dtype=torch.bfloat16)
+    lse = torch.empty(B, H, n_pad, device="cuda")
+    vsa.block_sparse_fwd(q, q, q, vsa.Shape(B, H, n_pad, n_pad, d), 64, 128, counts, idx, 2, 0.1, o, lse)
+    assert vsa.read_device_status() == 5
+    assert torch.all(o == 0) and torch.all(torch.isinf(lse))
+    assert vsa.read_device_status() == 0
+
+
 def test_attention_bad_list_latches_status():
     B, H, n_pad, d = 1, 1, 256, 128
     q = torch.zeros(B, H, n_pad, d, device="cuda", dtype=torch.bfloat16)
