@@ -129,11 +129,20 @@ __global__ void __launch_bounds__(kScoreThreads) micro_score_kernel(ScoreArgs a,
       const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[kk][tx * 4]);
       const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[kk][64 + tx * 4]);
       const float ar[4] = {av.x, av.y, av.z, av.w};
-      const float br[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      const float2 br2[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w), make_float2(b1.x, b1.y),
+                             make_float2(b1.z, b1.w)};
+      // packed pairs of accumulators (fma.rn.f32x2): each lane is the same
+      // single-rounding fma as before, in the same order over kk
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i) {
+        const float2 a2 = make_float2(ar[i], ar[i]);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(ar[i], br[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) {
+          const float2 r = ffma2(a2, br2[j], make_float2(acc[i][2 * j], acc[i][2 * j + 1]));
+          acc[i][2 * j] = r.x;
+          acc[i][2 * j + 1] = r.y;
+        }
+      }
     }
   }
 
