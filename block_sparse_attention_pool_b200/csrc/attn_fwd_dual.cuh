@@ -8,7 +8,9 @@
 // loads each union block's K and V once, and issues the S and P.V MMAs only
 // for the tile(s) whose list holds that block: every MMA is useful, and each
 // K/V byte feeds up to 256 query rows instead of 128.  This is the layout for
-// 128x128 blocks (list rows = 128, one 128-key list entry per stage).
+// 128-key blocks (one 128-key list entry per stage) with lists of 128 query
+// rows, or (kHalf) of 64 query rows: then each tile walks the union of its two
+// halves' lists and the rows of a half that did not keep a block take P = 0.
 //
 // Warp roles (320 threads):
 //   warp 0     TMA producer: Q_A and Q_B once, then K and V of every union
