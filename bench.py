@@ -43,8 +43,8 @@ from video_inputs import WORKLOADS, make_qkv, micro_heads, sweep_points  # noqa:
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "block-sparse attn ms & effective TFLOP/s (% bf16 peak), speedup vs dense, 1xB200"
 
-# DRAM bytes (read + write) of the Macro pass per hunyuan step, from the
-# one-pass ncu capture summarised in profiles/attn_fwd_dual_hunyuan_traffic.md,
+# DRAM bytes (read + write) of the Macro pass per hunyuan step, from a
+# one-pass ncu capture of its two launches (the summary sits under profiles/),
 # valid only while the kernel sources hash to the value it was taken with.
 MACRO_TRAFFIC = {
     "sources": ["csrc/attn_fwd_dual.cuh", "csrc/attn_fwd.cuh", "csrc/common.cuh"],
