@@ -327,6 +327,39 @@ def test_attention_64row_lists_on_both_kernels():
                           [(b, h, r * list_rows, (r + 1) * list_rows) for b, h, r in rows])
 
 
+def test_attention_two_tile_kernel_long_lists_from_global_memory():
+    """128-row lists of 128-key blocks longer than the 1024 entries the
+    two-tile kernel stages in shared memory: such a pair of tiles walks the
+    union of its lists from global memory instead.  A layer of 1032 key
+    blocks: one tile keeping 1030 blocks next to a tile keeping a few, a pair
+    of long lists, and short pairs, against the oracle on sampled rows."""
+    rng = np.random.default_rng(21)
+    B, H, d, seg, list_rows = 1, 1, 64, 128, 128
+    n_blocks = 1032
+    n_pad = seg * n_blocks
+    n_valid = n_pad - 70
+    q, k, v = (round_to_bf16(rng.standard_normal((B, H, n_pad, d)).astype(np.float32)) for _ in range(3))
+    n_l = n_s = n_blocks
+    pick = lambda n: np.sort(rng.choice(n_s, size=n, replace=False))
+    kept = [[[pick(int(rng.integers(1, 9))) for _ in range(n_l)]]]
+    sizes = {2: 1030, 3: 5,            # pair 1: one list past the staging size
+             10: 1025, 11: 1032,       # pair 5: both long, one of them dense
+             n_l - 1: 1031}            # last pair: the ragged block among them
+    for r, n in sizes.items():
+        kept[0][0][r] = pick(n)
+    counts, idx = lists_to_dev(kept, n_s, B, H, n_l)
+    shape = vsa.Shape(B, H, n_valid, n_pad, d)
+    o = torch.empty(B, H, n_pad, d, device="cuda")
+    lse = torch.empty(B, H, n_pad, device="cuda")
+    scale = 1 / math.sqrt(d)
+    vsa.block_sparse_fwd(to_dev(q), to_dev(k), to_dev(v), shape, list_rows, seg, counts, idx, n_s, scale, o, lse)
+    assert vsa.read_device_status() == 0
+    rows = [(0, 0, r) for r in (0, 1, 2, 3, 10, 11, 400, n_l - 2, n_l - 1)]
+    O, L = orc.block_sparse_attention(q, k, v, kept, list_rows, seg, n_valid, scale, rows=rows)
+    assert_close_rows(o.cpu().numpy(), lse.cpu().numpy(), O, L,
+                      [(b, h, r * list_rows, (r + 1) * list_rows) for b, h, r in rows])
+
+
 def test_attention_bad_64row_list_latches_status():
     """A descending 64-row list in the two-tile kernel: the status word reads
     VSA_ERR_BAD_INDEX and the CTA's tiles write O = 0, LSE = -inf."""
