@@ -35,7 +35,7 @@ def _worker(rank, world, port, out):
 
 def test_two_gloo_ranks_reduce_times_and_work():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()   # no fork of a (possibly multi-threaded) test process
     out = mgr.dict()
     port = _free_port()
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
