@@ -57,6 +57,29 @@ notes of the repository):
     O = 0 and LSE = -inf, and the merge passes the other side through;
  R11 query rows at or beyond N_valid are padding: O = 0, LSE = -inf; keys at or
     beyond N_valid never contribute.
+
+How each function is pinned to something other than itself (the pages print
+no worked example, so the stored goldens are hand-worked from the equations;
+tests/test_oracle_pins.py):
+  pool_block_means       means of explicit slices, padding excluded;
+  block_logits           the mean of the block's token logits (bilinearity);
+  size_weighted_probs    the token-level softmax of pooled logits summed per
+                         block (what the size weight stands for);
+  select_row / _blocks   a hand-worked Eq. (2)-(3) golden, brute force over
+                         all subsets (n_k <= 8), p -> 1 / p -> 0 / fixed-k
+                         special cases, the selected-mass >= p invariant;
+  block_sparse_attention dense SDPA (torch, fp64) when every block is kept,
+                         SDPA under the token mask, brute force, rows of P
+                         summing to one and LSE above the row maximum;
+  lse_merge              a hand-worked golden, disjoint supports merging to
+                         attention over their union, an empty side passing
+                         the other through;
+  micro_candidates /     candidates inside omitted blocks only, top-k against
+  select_micro_*         a rank-counting brute force, the percentile against
+                         numpy's quantile (nearest rank);
+  forward                the tiny layer equal to SDPA over the union of the
+                         Macro and Micro token masks.
+No function here is parity-unpinned.
 """
 from __future__ import annotations
 
