@@ -482,7 +482,7 @@ const char *vsa_status_string(vsa_status s) {
   return "unknown status";
 }
 
-int vsa_version(void) { return 100; }
+int vsa_version(void) { return 200; }
 
 vsa_status vsa_read_device_status(void *stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
