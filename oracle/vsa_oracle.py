@@ -74,9 +74,13 @@ tests/test_oracle_pins.py):
   lse_merge              a hand-worked golden, disjoint supports merging to
                          attention over their union, an empty side passing
                          the other through;
-  micro_candidates /     candidates inside omitted blocks only, top-k against
-  select_micro_*         a rank-counting brute force, the percentile against
-                         numpy's quantile (nearest rank);
+  micro_candidates /     candidates inside omitted blocks only, and (for both
+  select_micro_*         modes, which build their rows from micro_candidates)
+                         a key-by-key enumeration of every (row, tile) pair
+                         with query and key blocks of different sizes and a
+                         ragged last tile; top-k against a rank-counting
+                         brute force, the percentile against numpy's
+                         quantile (nearest rank);
   forward                the tiny layer equal to SDPA over the union of the
                          Macro and Micro token masks.
 No function here is parity-unpinned.
@@ -384,9 +388,7 @@ def select_micro_percentile(q64, k16, kept, bq: int, bk: int, n_valid: int, scal
     B, H, n_r, _ = q64.shape
     n_t = k16.shape[2]
     n_k = (n_t * micro_keys) // bk
-    per = bk // micro_keys
     rows_ok = _micro_rows_ok(n_r, micro_rows, n_valid)
-    tile_ok = np.arange(n_t) * micro_keys < n_valid
     out, infos = [], []
     for b in range(B):
         ob, ib = [], []
@@ -396,14 +398,14 @@ def select_micro_percentile(q64, k16, kept, bq: int, bk: int, n_valid: int, scal
                 ib.append(None)
                 continue
             S = micro_scores(q64[b, h], k16[b, h], scale)
+            # the head's candidate set: every (Micro row, tile) pair of R7,
+            # row by row from the same rule the top-k mode uses
             cand = np.zeros((n_r, n_t), dtype=bool)
             for r in range(n_r):
                 if not rows_ok[r]:
                     continue
                 i = (r * micro_rows) // bq
-                omitted = np.ones(n_k, dtype=bool)
-                omitted[np.asarray(kept[b][h][i], dtype=np.int64)] = False
-                cand[r] = omitted[np.arange(n_t) // per] & tile_ok
+                cand[r, micro_candidates(kept[b][h][i], n_k, bk, micro_keys, n_valid)] = True
             vals = np.sort(S[cand])
             M = vals.size
             if M == 0:

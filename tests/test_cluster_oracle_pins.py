@@ -193,3 +193,39 @@ def test_cluster_blocks_with_everything_kept_is_dense_attention():
     mask = np.ones((w.n_pad, w.n_pad), dtype=bool)
     O, L = orc.masked_attention_bruteforce(q, k, v, np.broadcast_to(mask, (w.B, w.H, w.n_pad, w.n_pad)), w.scale)
     assert np.allclose(res["O"], O, atol=1e-12) and np.allclose(res["LSE"], L, atol=1e-12)
+
+
+@pytest.mark.parametrize("lattice,grid,n_cells", [
+    ((33, 45, 80), (11, 5, 5), 432),     # HunyuanVideo, Q grid
+    ((33, 45, 80), (11, 3, 3), 1215),    # HunyuanVideo, K grid
+    ((21, 45, 80), (7, 6, 6), 336),      # Wan 2.2, Q grid
+    ((21, 45, 80), (6, 4, 4), 960),      # Wan 2.2, K grid
+])
+def test_cell_counts_match_the_published_centroid_counts(lattice, grid, n_cells):
+    """HyperVAttention App. A.1, Table 2 lists the grid sizes and the
+    resulting centroid counts N_q / N_k of each model's token lattice (81
+    frames at 720p: 21 x 45 x 80 latent tokens; 129 frames: 33 x 45 x 80);
+    the ceil cell count of reading C1 must reproduce every one of them, and
+    the initial centroids are one per cell."""
+    counts = orc.cell_counts(lattice, grid)
+    assert int(np.prod(counts)) == n_cells
+    assert int(np.prod(lattice)) in (75_600, 118_800)
+    cells = orc.token_cells(lattice, grid)
+    assert cells.min() == 0 and cells.max() == n_cells - 1
+    assert np.unique(cells).size == n_cells                 # every cell holds a token
+
+
+def test_local_window_search_space_reduction_is_six_point_three():
+    """HyperVAttention §4.1: for HunyuanVideo (n = 118.8K tokens, N_c = 1215
+    key centroids) a (3, 8, 8) window cuts the per-token search space 6.3x.
+    With reading C3 an interior cell's window holds 3 * 8 * 8 = 192 cells,
+    and 1215 / 192 rounds to 6.3; a cell at the lattice corner sees fewer."""
+    lattice, grid, window = (33, 45, 80), (11, 3, 3), (3, 8, 8)
+    counts = orc.cell_counts(lattice, grid)
+    n_c = int(np.prod(counts))
+    assert n_c == 1215
+    interior = orc.window_cells((1, 7, 13), counts, window)
+    assert interior.size == 192
+    assert round(n_c / interior.size, 1) == 6.3
+    corner = orc.window_cells((0, 0, 0), counts, window)
+    assert corner.size == 2 * 5 * 5       # offsets 0..1 in t, 0..4 in h and w once clipped

@@ -316,6 +316,56 @@ def test_micro_percentile_matches_numpy_quantile():
     assert orc.percentile_rank(0.99, 100) == 99 and orc.percentile_rank(0.99, 1000) == 990
 
 
+@pytest.mark.parametrize("bq,bk,n_valid", [(64, 128, 1000), (128, 64, 1008), (64, 64, 1011), (128, 128, 1017)])
+def test_micro_percentile_candidates_match_key_by_key_brute_force(bq, bk, n_valid):
+    """The percentile mode's candidate set (HyMoR-Attn abstract: Micro tiles
+    inside omitted blocks; reading R7) against an enumeration that decides
+    every (Micro row, 16-key tile) pair key by key: the row must hold a valid
+    query, every key of the tile must sit in a key block that the row's Macro
+    query block omitted, and the tile must hold a valid key.  Query and key
+    blocks of different sizes, 64-key blocks and a ragged last tile make a
+    wrong block size in the tile-to-block map, a kept/omitted inversion or an
+    off-by-one at n_valid fail here.  The selection is then every candidate
+    strictly above the nearest-rank threshold, and nothing else."""
+    rng = np.random.default_rng(bq + 7 * bk + n_valid)
+    H, d = 2, 8
+    n_pad = 1024
+    n_r, n_t = n_pad // 64, n_pad // 16
+    n_q, n_k = n_pad // bq, n_pad // bk
+    q64 = rng.normal(size=(1, H, n_r, d))
+    k16 = rng.normal(size=(1, H, n_t, d))
+    kept = [[[np.sort(rng.choice(n_k, size=int(rng.integers(0, n_k)), replace=False)) for _ in range(n_q)]
+             for _ in range(H)]]
+    kept[0][0][0] = np.zeros(0, dtype=np.int64)              # a row that omitted everything
+    kept[0][1][n_q - 1] = np.arange(n_k)                      # a row that kept everything
+    tiles, info = orc.select_micro_percentile(q64, k16, kept, bq, bk, n_valid, 0.5, 0.75, np.array([1, 1]),
+                                              with_info=True)
+    for h in range(H):
+        want = np.zeros((n_r, n_t), dtype=bool)
+        for r in range(n_r):
+            if r * 64 >= n_valid:
+                continue
+            macro_row = set(kept[0][h][(r * 64) // bq].tolist())
+            for t in range(n_t):
+                keys = range(16 * t, 16 * t + 16)
+                want[r, t] = all((key // bk) not in macro_row for key in keys) and any(key < n_valid for key in keys)
+        cand = info[0][h]["cand"]
+        assert np.array_equal(cand, want), h
+        S = (q64[0, h] @ k16[0, h].T) * 0.5
+        vals = np.sort(S[want])
+        tau = vals[math.ceil(0.75 * vals.size) - 1]
+        sel = np.zeros_like(want)
+        for r, t in enumerate(tiles[0][h]):
+            sel[r, t] = True
+        assert np.array_equal(sel, want & (S > tau)), h
+        assert sel.sum() == vals.size - math.ceil(0.75 * vals.size)
+    # the top-k mode builds its rows from the same rule
+    topk = orc.select_micro_topk(q64, k16, kept, bq, bk, n_valid, 0.5, n_t)
+    for h in range(H):
+        for r in range(n_r):
+            assert np.array_equal(topk[0][h][r], np.nonzero(info[0][h]["cand"][r])[0]), (h, r)
+
+
 def test_tiny_forward_equals_sdpa_over_union_mask():
     """Whole path on the tiny workload: the merged output equals plain masked
     attention over the union of the Macro blocks and the Micro tiles."""
