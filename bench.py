@@ -264,9 +264,10 @@ def run_gpu(args, rank, world, local_rank):
     if st != 0:
         raise RuntimeError(f"device status after timed steps: {vsa.status_string(st)}")
 
-    # end to end through the public API with host buffers: every step copies
-    # Q/K/V from pinned host memory and O/LSE back (forward_host pipelines the
-    # copies of one chunk of heads with the path on the previous chunk)
+    # end to end through the public API with host buffers: every step is one
+    # C-ABI call (vsa_path_fwd_host, through forward_host) that copies Q/K/V
+    # from pinned host memory and O/LSE back, pipelining the copies of one
+    # chunk of heads with the path on the previous chunk
     ho = torch.empty(run.buf["o"].shape, dtype=torch.bfloat16).pin_memory()
     hl = torch.empty(run.buf["lse"].shape, dtype=torch.float32).pin_memory()
     e2e_steps = max(1, min(args.steps, 5))
@@ -359,7 +360,7 @@ def run_gpu(args, rank, world, local_rank):
         },
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 3),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "api": f"SparseVideoAttention.forward_host, {args.chunk_heads}-head chunks"},
+                "api": f"vsa_path_fwd_host (one C-ABI call on pinned host buffers), {args.chunk_heads}-head chunks"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }

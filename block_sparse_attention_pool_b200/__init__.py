@@ -29,17 +29,19 @@ __all__ = [
     "select_clusters", "merge_clusters", "merge_clusters_workspace_bytes", "cluster_rows_capacity", "cluster_plan",
     "gather_rows", "cluster_group_fwd", "ClusterBlockConfig", "ClusterBlockAttention",
     "pool_kv_bf16", "rectify_fwd", "SelectionSchedule", "cluster_anchor", "cluster_refine",
-    "cluster_refine_workspace_bytes", "subset_size",
+    "cluster_refine_workspace_bytes", "subset_size", "PathParams", "path_params", "path_workspace_bytes",
+    "path_fwd", "path_host_workspace_bytes", "path_fwd_host", "bind_status_word",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libvsa.so")
 
 EXPORTED = (
-    "vsa_status_string", "vsa_version", "vsa_read_device_status", "vsa_pool_qk", "vsa_select_blocks",
+    "vsa_status_string", "vsa_version", "vsa_read_device_status", "vsa_bind_status_word", "vsa_pool_qk", "vsa_select_blocks",
     "vsa_mask_to_lists", "vsa_select_micro_workspace_bytes", "vsa_select_micro", "vsa_select_micro_noalloc",
     "vsa_block_sparse_fwd", "vsa_block_sparse_fwd_heads", "vsa_lse_merge", "vsa_selftest_wait_timeout",
-    "vsa_selftest_exp2",
+    "vsa_selftest_exp2", "vsa_path_workspace_bytes", "vsa_path_fwd", "vsa_path_host_workspace_bytes",
+    "vsa_path_fwd_host",
     "vsa_cluster_count", "vsa_cluster_tokens", "vsa_permute_rows", "vsa_select_clusters",
     "vsa_merge_clusters_workspace_bytes", "vsa_merge_clusters", "vsa_cluster_rows_capacity", "vsa_cluster_plan",
     "vsa_gather_rows", "vsa_cluster_group_fwd", "vsa_pool_kv_bf16", "vsa_rectify_fwd", "vsa_cluster_anchor",
@@ -85,6 +87,14 @@ class MicroParams(ctypes.Structure):
                 ("head_enable", ctypes.POINTER(ctypes.c_uint8)), ("row_capacity", ctypes.c_int)]
 
 
+class PathParams(ctypes.Structure):
+    """vsa_path_params: the whole path's knobs (micro_heads is a HOST array)."""
+    _fields_ = [("bq", ctypes.c_int), ("bk", ctypes.c_int), ("scale", ctypes.c_float), ("select", SelectParams),
+                ("micro_mode", ctypes.c_int), ("micro_topk", ctypes.c_int), ("micro_percentile", ctypes.c_double),
+                ("micro_heads", ctypes.POINTER(ctypes.c_uint8)), ("micro_capacity", ctypes.c_int),
+                ("o_fp32", ctypes.c_int)]
+
+
 _lib = None
 
 
@@ -108,6 +118,8 @@ def lib():
     L.vsa_version.argtypes = []
     L.vsa_read_device_status.restype = I
     L.vsa_read_device_status.argtypes = [P]
+    L.vsa_bind_status_word.restype = I
+    L.vsa_bind_status_word.argtypes = [P, P]
     L.vsa_selftest_wait_timeout.restype = I
     L.vsa_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, P]
     L.vsa_selftest_exp2.restype = I
@@ -157,6 +169,15 @@ def lib():
     L.vsa_cluster_refine.argtypes = [P, SP, ctypes.POINTER(ClusterParams), P, I, P, P, P, P, P, S, P]
     L.vsa_pool_kv_bf16.restype = I
     L.vsa_pool_kv_bf16.argtypes = [P, P, SP, I, I, P, P, P]
+    PP = ctypes.POINTER(PathParams)
+    L.vsa_path_workspace_bytes.restype = S
+    L.vsa_path_workspace_bytes.argtypes = [SP, PP]
+    L.vsa_path_fwd.restype = I
+    L.vsa_path_fwd.argtypes = [P, P, P, SP, PP, P, P, P, S, P]
+    L.vsa_path_host_workspace_bytes.restype = S
+    L.vsa_path_host_workspace_bytes.argtypes = [SP, PP, I]
+    L.vsa_path_fwd_host.restype = I
+    L.vsa_path_fwd_host.argtypes = [P, P, P, SP, PP, I, P, P, P, S, P]
     L.vsa_rectify_fwd.restype = I
     L.vsa_rectify_fwd.argtypes = [P, P, P, SP, I, I, I, P, P, I, F, P, P, P, I, P, P, I, P]
     L.vsa_select_clusters.argtypes = [P, P, P, P, I, I, I, I, F, ctypes.POINTER(SelectParams), P, P, P]
@@ -198,6 +219,16 @@ def version() -> int:
 
 def read_device_status(stream=None) -> int:
     return lib().vsa_read_device_status(_s(stream))
+
+
+def bind_status_word(word: Optional[torch.Tensor], stream=None) -> None:
+    """Make the calls later enqueued on ``stream`` report device-side errors
+    into ``word`` (a device int32 tensor of 2 elements, cleared here) instead
+    of the process-wide word; None removes the binding.  read_device_status
+    on that stream then reads (and clears) ``word``."""
+    if word is not None and (not word.is_cuda or word.dtype != torch.int32 or word.numel() < 2):
+        raise ValueError("the status word is a device int32 tensor of at least 2 elements")
+    _check(lib().vsa_bind_status_word(_s(stream), _p(word)), "vsa_bind_status_word")
 
 
 def selftest_wait_timeout(limit_ns: int, stream=None) -> None:
@@ -420,6 +451,51 @@ def lse_merge(o_a, lse_a, o_b, lse_b, shape: Shape, o_out, lse_out, stream=None)
 # ---------------------------------------------------------------------------
 # The whole path
 # ---------------------------------------------------------------------------
+
+def path_params(cfg: "PathConfig", micro_heads=None, o_fp32: bool = False):
+    """vsa_path_params of a PathConfig (token-order layout, no rectification).
+    Returns (params, keep): keep holds the host flag array alive."""
+    if cfg.rectify or cfg.cluster_lattice is not None:
+        raise ValueError("the one-call path covers pooling, selection, Macro and Micro passes only")
+    flags = cfg.micro_heads if micro_heads is None else micro_heads
+    arr = None
+    if cfg.micro_mode and flags is not None:
+        arr = (ctypes.c_uint8 * len(flags))(*[int(x) for x in flags])
+    p = PathParams(int(cfg.bq), int(cfg.bk), float(cfg.scale or 0.0),
+                   SelectParams(cfg.k_min, cfg.cum_mass, cfg.fixed_k, cfg.n_anchor, cfg.anchor_rot),
+                   int(cfg.micro_mode), int(cfg.micro_topk), float(cfg.micro_percentile),
+                   ctypes.cast(arr, ctypes.POINTER(ctypes.c_uint8)) if arr is not None else None,
+                   int(cfg.micro_capacity), 1 if o_fp32 else 0)
+    return p, arr
+
+
+def path_workspace_bytes(shape: Shape, params: PathParams) -> int:
+    return int(lib().vsa_path_workspace_bytes(ctypes.byref(shape), ctypes.byref(params)))
+
+
+def path_fwd(q, k, v, shape: Shape, params: PathParams, o, lse, workspace, stream=None):
+    """The whole path in one C call on device tensors."""
+    _check(lib().vsa_path_fwd(_p(q), _p(k), _p(v), ctypes.byref(shape), ctypes.byref(params), _p(o), _p(lse),
+                              _p(workspace), workspace.numel() * workspace.element_size(), _s(stream)),
+           "vsa_path_fwd")
+
+
+def path_host_workspace_bytes(shape: Shape, params: PathParams, chunk_heads: int) -> int:
+    return int(lib().vsa_path_host_workspace_bytes(ctypes.byref(shape), ctypes.byref(params), int(chunk_heads)))
+
+
+def path_fwd_host(q_h, k_h, v_h, shape: Shape, params: PathParams, chunk_heads: int, o_h, lse_h, workspace,
+                  stream=None):
+    """The whole path in one C call on HOST tensors (pinned), the copies
+    pipelined over chunks of heads; complete when ``stream`` is."""
+    for t in (q_h, k_h, v_h, o_h, lse_h):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("path_fwd_host takes contiguous host tensors")
+    _check(lib().vsa_path_fwd_host(_p(q_h), _p(k_h), _p(v_h), ctypes.byref(shape), ctypes.byref(params),
+                                   int(chunk_heads), _p(o_h), _p(lse_h), _p(workspace),
+                                   workspace.numel() * workspace.element_size(), _s(stream)),
+           "vsa_path_fwd_host")
+
 
 @dataclass
 class PathConfig:
@@ -674,53 +750,32 @@ class SparseVideoAttention:
 
     def forward_host(self, q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor, o_h: torch.Tensor,
                      lse_h: torch.Tensor, chunk_heads: int = 2, device=None) -> None:
-        """The whole path on HOST tensors: pinned bf16 q_h, k_h, v_h [B, H, n_pad, d]
-        in, pinned o_h (bf16, same shape) and lse_h (fp32 [B, H, n_pad]) out.
+        """The whole path on HOST tensors through one C call (vsa_path_fwd_host):
+        pinned bf16 q_h, k_h, v_h [B, H, n_pad, d] in, pinned o_h (bf16, same
+        shape) and lse_h (fp32 [B, H, n_pad]) out.
 
-        Every (batch, head) is an independent problem, so the heads are cut into
-        chunks and pipelined over three streams: host-to-device copies of chunk
-        i+1 and device-to-host copies of chunk i-1 overlap the path on chunk i.
-        Results are exactly those of running the path on all heads at once.
-        Returns once the enqueued work is complete.
+        The library cuts the flattened heads into chunks of ``chunk_heads``
+        and pipelines them: host-to-device copies of chunk i+1 and
+        device-to-host copies of chunk i-1 overlap the path on chunk i.
+        Results equal the device path on all heads at once.  Returns once the
+        work is complete.
         """
         dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
         B, H, n_pad, d = q_h.shape
-        BH = B * H
+        shape = _shape(B, H, self.cfg.n_valid, n_pad, d)
+        params, keep = path_params(self.cfg)
         key = (B, H, n_pad, d, dev, chunk_heads)
         if getattr(self, "_host_key", None) != key:
-            bf = torch.bfloat16
-            self._hbuf = {
-                "q": torch.empty(BH, n_pad, d, device=dev, dtype=bf),
-                "k": torch.empty(BH, n_pad, d, device=dev, dtype=bf),
-                "v": torch.empty(BH, n_pad, d, device=dev, dtype=bf),
-                "o": torch.empty(BH, n_pad, d, device=dev, dtype=bf),
-                "lse": torch.empty(BH, n_pad, device=dev, dtype=torch.float32),
-            }
-            self._chunk = SparseVideoAttention(self.cfg, workspace_for_all_heads=True)
-            self._s_in = torch.cuda.Stream(dev)
-            self._s_out = torch.cuda.Stream(dev)
+            n = path_host_workspace_bytes(shape, params, chunk_heads)
+            if n == 0:
+                raise VsaError(1, "vsa_path_host_workspace_bytes")
+            self._host_ws = torch.empty(n, device=dev, dtype=torch.uint8)
             self._host_key = key
-        hb = self._hbuf
-        qf, kf, vf = (x.view(BH, n_pad, d) for x in (q_h, k_h, v_h))
-        of, lf = o_h.view(BH, n_pad, d), lse_h.view(BH, n_pad)
-        flags = None
-        if self.cfg.micro_mode and self.cfg.micro_heads is not None:
-            flags = [int(self.cfg.micro_heads[i % H]) for i in range(BH)]
-        comp = torch.cuda.current_stream(dev)
-        for c0 in range(0, BH, chunk_heads):
-            c1 = min(BH, c0 + chunk_heads)
-            with torch.cuda.stream(self._s_in):
-                for dst, src in ((hb["q"], qf), (hb["k"], kf), (hb["v"], vf)):
-                    dst[c0:c1].copy_(src[c0:c1], non_blocking=True)
-            comp.wait_stream(self._s_in)
-            view = lambda t: t[c0:c1].unsqueeze(0)
-            self._chunk(view(hb["q"]), view(hb["k"]), view(hb["v"]), stream=comp, out_o=view(hb["o"]),
-                        out_lse=view(hb["lse"]), micro_heads=None if flags is None else flags[c0:c1])
-            self._s_out.wait_stream(comp)
-            with torch.cuda.stream(self._s_out):
-                of[c0:c1].copy_(hb["o"][c0:c1], non_blocking=True)
-                lf[c0:c1].copy_(hb["lse"][c0:c1], non_blocking=True)
-        self._s_out.synchronize()
+        with torch.cuda.device(dev):
+            stream = torch.cuda.current_stream(dev)
+            path_fwd_host(q_h, k_h, v_h, shape, params, chunk_heads, o_h, lse_h, self._host_ws, stream)
+            stream.synchronize()
+        del keep
 
 
 @dataclass

@@ -64,6 +64,9 @@ constexpr int kChunkBytes = 128 * 128;  // one 64-column bf16 chunk of a 128-row
 constexpr int kInfoRing = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// logits reach the FMA-pipe exponential at most kRescaleThreshold above the
+// running reference maximum
+static_assert(kRescaleThreshold <= kExp2PolyMaxInput, "exp2_poly2 is exact in range only up to 2^126");
 constexpr int kListStage = 2048;  // list entries staged in shared memory per list (fast path)
 constexpr int kUnionCap = 2 * kListStage;
 
@@ -81,6 +84,7 @@ struct AttnArgs {
   const int32_t *heads;  // grid row -> b * H + h, or NULL for grid row = b * H + h
   int n_bh;              // B * H
   unsigned long long timeout_ns;
+  int *status;           // the launch's status word
   // Cluster-group mode (tile_list non-null; list_rows 128, seg_keys 16): tile T of
   // head bh uses list row tile_list[bh][T] (-1: no such tile, the CTA leaves at
   // once), whose entries are key clusters j < n_kc; cluster j is the K/V rows
@@ -132,7 +136,7 @@ struct AttnCtl {
   uint64_t info_full[kInfoRing];
   uint64_t xbar[4];  // per lane quadrant: the two groups' final (max, sum) exchange
   uint32_t tmem_base;
-  int abort;
+  AbortCtl abort;
   int n_seg;
   int n_ent;  // cluster-group mode: key clusters of the tile's list
   int fast;  // the union sits in shared memory (lists short enough to stage)
@@ -305,14 +309,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t *sV = smem + L::kOffV;
   float *sX = reinterpret_cast<float *>(smem + L::kOffX);  // [2 groups][max, sum, rounded sum][128 rows]
   AttnCtl *ctl = reinterpret_cast<AttnCtl *>(smem + L::kOffCtl);
-  volatile int *abort = &ctl->abort;
+  AbortCtl *abort = &ctl->abort;
 
   const int tile = blockIdx.x;
   // (batch, head) of this grid row: the caller's head list, or all of them in order.  An
   // out-of-range entry latches BAD_INDEX before any setup and the whole CTA leaves.
   const int bh = a.heads ? __ldg(a.heads + blockIdx.y) : static_cast<int>(blockIdx.y);
   if (bh < 0 || bh >= a.n_bh) {
-    if (threadIdx.x == 0) latch_status(VSA_ERR_BAD_INDEX);
+    if (threadIdx.x == 0) latch_status(a.status, VSA_ERR_BAD_INDEX);
     return;
   }
   const int warp = threadIdx.x >> 5;
@@ -324,7 +328,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     group_row = __ldg(a.tile_list + (size_t)bh * a.n_tiles + tile);
     if (group_row < 0) return;  // no tile here
     if (group_row >= a.n_lists_bh) {
-      if (threadIdx.x == 0) latch_status(VSA_ERR_BAD_INDEX);
+      if (threadIdx.x == 0) latch_status(a.status, VSA_ERR_BAD_INDEX);
       return;
     }
   }
@@ -351,7 +355,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&ctl->mma_drain, 1);
       for (int i = 0; i < kInfoRing; ++i) mbar_init(&ctl->info_full[i], 1);
       for (int i = 0; i < 4; ++i) mbar_init(&ctl->xbar[i], 64);
-      ctl->abort = 0;
+      abort_init(&ctl->abort, a.status);
       fence_barrier_init();
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -444,7 +448,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     if (!ok) {
       n_seg = 0;
-      if (lane == 0) latch_status(VSA_ERR_BAD_INDEX);
+      if (lane == 0) latch_status(a.status, VSA_ERR_BAD_INDEX);
     }
     if (lane == 0) {
       ctl->n_seg = n_seg;
@@ -625,7 +629,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         issued = s + 1;
         __syncwarp();
       }
-      if (*abort && lane == 0) {
+      if (abort_raised(abort) && lane == 0) {
         // let copies still in flight land before the CTA's shared memory goes away
         mbar_drain(&ctl->q_full, 0, a.timeout_ns);
         for (int s = max(0, issued - 2); s < issued; ++s) {

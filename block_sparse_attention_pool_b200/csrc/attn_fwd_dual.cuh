@@ -94,7 +94,7 @@ struct DualCtl {
   uint64_t p_half[2];  // per tile: P of the block's keys 0-63 written
   uint64_t mma_drain;
   uint32_t tmem_base;
-  int abort;
+  AbortCtl abort;
   int n_union;
   int cnt[2];
   int fast;  // union and lists staged in shared memory
@@ -118,14 +118,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t *sK = smem + L::kOffK;
   uint8_t *sV = smem + L::kOffV;
   DualCtl *ctl = reinterpret_cast<DualCtl *>(smem + L::kOffCtl);
-  volatile int *abort = &ctl->abort;
+  AbortCtl *abort = &ctl->abort;
 
   const int pair = blockIdx.x;
   // (batch, head) of this grid row: the caller's head list, or all of them in order.  An
   // out-of-range entry latches BAD_INDEX before any setup and the whole CTA leaves.
   const int bh = a.heads ? __ldg(a.heads + blockIdx.y) : static_cast<int>(blockIdx.y);
   if (bh < 0 || bh >= a.n_bh) {
-    if (threadIdx.x == 0) latch_status(VSA_ERR_BAD_INDEX);
+    if (threadIdx.x == 0) latch_status(a.status, VSA_ERR_BAD_INDEX);
     return;
   }
   const int warp = threadIdx.x >> 5;
@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_init(&ctl->p_half[i], 128);
       }
       mbar_init(&ctl->mma_drain, 1);
-      ctl->abort = 0;
+      abort_init(&ctl->abort, a.status);
       fence_barrier_init();
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           n_union = cnt[0];
         }
       } else {
-        if (lane == 0) latch_status(VSA_ERR_BAD_INDEX);
+        if (lane == 0) latch_status(a.status, VSA_ERR_BAD_INDEX);
         cnt[0] = cnt[1] = 0;
       }
       if (lane == 0) {
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           ok = list_valid(a.idx + (lrow0 + x) * a.idx_stride, cnt[x], n_key_blocks, lane);
       }
       if (!ok) {
-        if (lane == 0) latch_status(VSA_ERR_BAD_INDEX);
+        if (lane == 0) latch_status(a.status, VSA_ERR_BAD_INDEX);
         cnt[0] = cnt[1] = 0;
         n_union = 0;
       }
@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         issued = s + 1;
         __syncwarp();
       }
-      if (*abort && lane == 0) {
+      if (abort_raised(abort) && lane == 0) {
         mbar_drain(&ctl->q_full, 0, a.timeout_ns);
         for (int s = max(0, issued - 2); s < issued; ++s) {
           mbar_drain(&ctl->k_full[s & 1], (s >> 1) & 1, a.timeout_ns);

@@ -358,14 +358,15 @@ __global__ void __launch_bounds__(kClusterThreads) cluster_perm_kernel(ClusterGe
 // One warp per row of row_words 32-bit words: gather dst[i] = src[perm[i]],
 // or (inverse) scatter dst[perm[i]] = src[i].
 __global__ void permute_rows_kernel(const uint32_t *__restrict__ src, const int32_t *__restrict__ perm, int n_pad,
-                                    long long n_rows, int row_words, int inverse, uint32_t *__restrict__ dst) {
+                                    long long n_rows, int row_words, int inverse, uint32_t *__restrict__ dst,
+                                    int *status) {
   const long long row = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (row >= n_rows) return;
   const int lane = threadIdx.x & 31;
   const long long bh = row / n_pad;
   const int p = __ldg(perm + row);
   if (p < 0 || p >= n_pad) {  // a caller-given permutation entry out of range: nothing is copied
-    if (lane == 0) latch_status(VSA_ERR_BAD_INDEX);
+    if (lane == 0) latch_status(status, VSA_ERR_BAD_INDEX);
     return;
   }
   const long long from = inverse ? row : bh * n_pad + p;

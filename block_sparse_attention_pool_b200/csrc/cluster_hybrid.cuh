@@ -123,7 +123,8 @@ template <int D>
 __global__ void __launch_bounds__(256) reassign_kernel(const __nv_bfloat16 *__restrict__ x, int n_pad, int n_valid,
                                                        int n_cells, const float *__restrict__ mu,
                                                        const int32_t *__restrict__ subset, int n_sub,
-                                                       int32_t *__restrict__ assign, int32_t *__restrict__ changed) {
+                                                       int32_t *__restrict__ assign, int32_t *__restrict__ changed,
+                                                       int *status) {
   using L = ReLayout<D>;
   constexpr int kLd = L::kLd;
   constexpr int NB = kReCen / 16;
@@ -138,7 +139,7 @@ __global__ void __launch_bounds__(256) reassign_kernel(const __nv_bfloat16 *__re
     if (i0 + tid < n_sub) {
       tok = __ldg(subset + (size_t)bh * n_sub + i0 + tid);
       if (tok < 0 || tok >= n_valid) {
-        latch_status(VSA_ERR_BAD_INDEX);
+        latch_status(status, VSA_ERR_BAD_INDEX);
         tok = -1;
       }
     }
@@ -256,7 +257,8 @@ __global__ void __launch_bounds__(256) reassign_kernel(const __nv_bfloat16 *__re
 
 // cnt[bh][u][chunk]: tokens of chunk with cluster u
 __global__ void __launch_bounds__(256) sort_count_kernel(const int32_t *__restrict__ assign, int n_valid,
-                                                         int n_cells, int n_chunks, int32_t *__restrict__ cnt) {
+                                                         int n_cells, int n_chunks, int32_t *__restrict__ cnt,
+                                                         int *status) {
   extern __shared__ int hist[];
   const int chunk = blockIdx.x, bh = blockIdx.y;
   for (int u = threadIdx.x; u < n_cells; u += 256) hist[u] = 0;
@@ -265,7 +267,7 @@ __global__ void __launch_bounds__(256) sort_count_kernel(const int32_t *__restri
   for (int i = chunk * kSortChunk + threadIdx.x; i < min(n_valid, (chunk + 1) * kSortChunk); i += 256) {
     const int u = __ldg(ab + i);
     if (u >= 0 && u < n_cells) atomicAdd(&hist[u], 1);
-    else latch_status(VSA_ERR_BAD_INDEX);
+    else latch_status(status, VSA_ERR_BAD_INDEX);
   }
   __syncthreads();
   for (int u = threadIdx.x; u < n_cells; u += 256) cnt[((size_t)bh * n_cells + u) * n_chunks + chunk] = hist[u];
@@ -383,7 +385,7 @@ struct RtCtl {
   uint64_t done[2];
   uint64_t fin;
   uint32_t tmem_base;
-  int abort;
+  AbortCtl abort;
 };
 
 // Row r of a 128-row K-major bf16 tile, 64 columns from v (32 packed pairs).
@@ -398,21 +400,22 @@ template <int D>
 __global__ void __launch_bounds__(kRtThreads, 1)
     reassign_tc_kernel(const __nv_bfloat16 *__restrict__ x, int n_pad, int n_valid, int n_cells,
                        const float *__restrict__ mu, const int32_t *__restrict__ subset, int n_sub,
-                       int32_t *__restrict__ assign, int32_t *__restrict__ changed, unsigned long long timeout_ns) {
+                       int32_t *__restrict__ assign, int32_t *__restrict__ changed, unsigned long long timeout_ns,
+                       int *status) {
   using L = RtLayout<D>;
   extern __shared__ uint8_t rt_smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(rt_smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   float *s_norm = reinterpret_cast<float *>(smem + L::kOffN);
   RtCtl *ctl = reinterpret_cast<RtCtl *>(smem + L::kOffCtl);
-  volatile int *abort = &ctl->abort;
+  AbortCtl *abort = &ctl->abort;
   const int bh = blockIdx.y, t = threadIdx.x, warp = t >> 5;
   const int i = blockIdx.x * kReTok + t;
   int tok = -1;
   if (i < n_sub) {
     tok = __ldg(subset + (size_t)bh * n_sub + i);
     if (tok < 0 || tok >= n_valid) {
-      latch_status(VSA_ERR_BAD_INDEX);
+      latch_status(status, VSA_ERR_BAD_INDEX);
       tok = -1;
     }
   }
@@ -437,7 +440,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     mbar_init(&ctl->done[0], 1);
     mbar_init(&ctl->done[1], 1);
     mbar_init(&ctl->fin, 1);
-    ctl->abort = 0;
+    abort_init(&ctl->abort, status);
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -552,7 +555,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   // every MMA of the CTA has completed before TMEM and shared memory are released
   if (t == 0) umma_commit(&ctl->fin);
   const bool fin = mbar_drain(&ctl->fin, 0, timeout_ns);
-  if (!fin) raise_timeout();
+  if (!fin) raise_timeout(status);
   if (ok && tok >= 0 && bcell < n_cells) {
     int32_t *ab = assign + (size_t)bh * n_valid;
     const int old = ab[tok];

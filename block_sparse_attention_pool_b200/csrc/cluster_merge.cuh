@@ -70,6 +70,7 @@ struct MergeArgs {
   int32_t *g_idx;          // [BH][nq][nk]
   MergeWs ws;
   unsigned long long timeout_ns;
+  int *status;             // the launch's status word
 };
 
 // ceil(x / tau) for x >= 0: a float estimate corrected to the exact quotient.
@@ -179,14 +180,14 @@ __global__ void __launch_bounds__(kMergeHeadThreads) merge_init_kernel(const Mer
     a.ws.chi[(hb + i) * kMergeWords + lane] = bad ? 0u : wbits[warp][lane];
     if (lane == 0) {
       const int s = __ldg(a.sizes_q + hb + i);
-      if (bad || s < 0) latch_status(VSA_ERR_BAD_INDEX);
+      if (bad || s < 0) latch_status(a.status, VSA_ERR_BAD_INDEX);
       a.ws.gsq[hb + i] = max(0, s);
       a.ws.gwk[hb + i] = bad ? 0 : wk;
       a.ws.lead[hb + i] = i;
     }
     __syncwarp();
   }
-  if (bad_size) latch_status(VSA_ERR_BAD_INDEX);
+  if (bad_size) latch_status(a.status, VSA_ERR_BAD_INDEX);
   __syncthreads();
   if (t == 0) a.ws.passes[bh] = s_max >= (1 << 22) ? 3 : (s_max >= 2048 ? 2 : 1);
   if (a.rounds > 0) merge_build_lists(a, bh, 0, s_tot);
@@ -197,7 +198,7 @@ struct MergeCtl {
   uint64_t done[2];  // the MMAs reading operand buffer b have completed
   uint64_t fin;      // every MMA of the CTA has completed
   uint32_t tmem_base;
-  int abort;
+  AbortCtl abort;
 };
 
 struct MergeSmem {
@@ -248,7 +249,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_pairs_kernel(const Mer
   int *col_wk = col_sq + 128;
   long long *col_c = reinterpret_cast<long long *>(col_wk + 128);
   MergeCtl *ctl = reinterpret_cast<MergeCtl *>(smem + L::kOffCtl);
-  volatile int *abort = &ctl->abort;
+  AbortCtl *abort = &ctl->abort;
 
   const int t = threadIdx.x, warp = t >> 5;
   const size_t hb = (size_t)bh * a.nq;
@@ -278,7 +279,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_pairs_kernel(const Mer
     mbar_init(&ctl->done[0], 1);
     mbar_init(&ctl->done[1], 1);
     mbar_init(&ctl->fin, 1);
-    ctl->abort = 0;
+    abort_init(&ctl->abort, a.status);
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -330,7 +331,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_pairs_kernel(const Mer
   }
   if (t == 0) umma_commit(&ctl->fin);
   const bool fin_t = mbar_drain(&ctl->fin, 0, a.timeout_ns);
-  if (!fin_t) raise_timeout();
+  if (!fin_t) raise_timeout(a.status);
   const bool fin = __syncthreads_and(fin_t ? 1 : 0) != 0;
   tc_fence_after();
   if (ok && fin) {

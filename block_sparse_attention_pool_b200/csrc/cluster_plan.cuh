@@ -34,6 +34,7 @@ struct PlanArgs {
   int32_t *qinv;       // [BH][n_pad]
   int32_t *tile_list;  // [BH][n_rows / 128]
   int32_t *kc_off;     // [BH][nk]
+  int *status;         // the launch's status word
 };
 
 // Exclusive prefix sum over the 1024 threads of the block; *total gets the sum.
@@ -72,7 +73,7 @@ __global__ void __launch_bounds__(kPlanThreads) cluster_plan_kernel(const PlanAr
     grp = __ldg(a.group_of + hq + t);
     // a group is named by its leader, which leads itself
     if (grp < 0 || grp >= a.nq || __ldg(a.group_of + hq + grp) != grp) {
-      latch_status(VSA_ERR_BAD_INDEX);
+      latch_status(a.status, VSA_ERR_BAD_INDEX);
       grp = t;
     }
   }
@@ -91,7 +92,7 @@ __global__ void __launch_bounds__(kPlanThreads) cluster_plan_kernel(const PlanAr
   s_goff[t] = goff;
   __syncthreads();
   if (total > a.n_rows || n_q_tokens > a.n_pad) {
-    if (t == 0) latch_status(VSA_ERR_CAPACITY);
+    if (t == 0) latch_status(a.status, VSA_ERR_CAPACITY);
     return;
   }
   if (t < a.nq) {
@@ -112,7 +113,7 @@ __global__ void __launch_bounds__(kPlanThreads) cluster_plan_kernel(const PlanAr
     for (int e = lane; e < n; e += 32) {
       const int tok = __ldg(a.perm_q + (size_t)bh * a.n_pad + src0 + e);
       if (tok < 0 || tok >= a.n_valid) {
-        latch_status(VSA_ERR_BAD_INDEX);
+        latch_status(a.status, VSA_ERR_BAD_INDEX);
         continue;
       }
       a.qmap[(size_t)bh * a.n_rows + dst0 + e] = tok;
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(kPlanThreads) cluster_plan_kernel(const PlanAr
 
 __global__ void gather_rows_kernel(const uint32_t *__restrict__ src, const int32_t *__restrict__ map, int n_src,
                                    int n_dst, long long n_rows, int row_words, uint32_t fill,
-                                   uint32_t *__restrict__ dst) {
+                                   uint32_t *__restrict__ dst, int *status) {
   const long long row = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (row >= n_rows) return;
   const int lane = threadIdx.x & 31;
@@ -136,7 +137,7 @@ __global__ void gather_rows_kernel(const uint32_t *__restrict__ src, const int32
   if (m == -2) return;
   uint32_t *d = dst + row * row_words;
   if (m < -2 || m >= n_src) {
-    if (lane == 0) latch_status(VSA_ERR_BAD_INDEX);
+    if (lane == 0) latch_status(status, VSA_ERR_BAD_INDEX);
     return;
   }
   if (m == -1) {

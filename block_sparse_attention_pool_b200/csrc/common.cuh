@@ -15,23 +15,43 @@
 
 namespace vsa {
 
-// First device-side error since the last vsa_read_device_status().
-__device__ int g_status;
-// Raised by the first pipeline wait that runs out of time; every other wait
-// of every CTA then gives up at its next check instead of running out its own
-// limit.  Cleared with the status word.
-__device__ int g_timed_out;
+// Status words.  Every launch reports device-side conditions into one word of
+// two ints: [0] the first error latched (0 = none), [1] raised by the first
+// pipeline wait that ran out of time, after which every other wait of every
+// CTA reporting into the same word gives up at its next check instead of
+// running out its own limit.  The host passes the word of the launch's stream
+// (a caller-owned word bound to the stream, or this process-wide default) and
+// vsa_read_device_status reads and clears it.
+__device__ int g_status_word[2];
 
-__device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0, code); }
+__device__ __forceinline__ void latch_status(int *st, int code) { atomicCAS(st, 0, code); }
 
-__device__ __forceinline__ void raise_timeout() {
-  latch_status(VSA_ERR_TIMEOUT);
-  atomicExch(&g_timed_out, 1);
+__device__ __forceinline__ void raise_timeout(int *st) {
+  latch_status(st, VSA_ERR_TIMEOUT);
+  atomicExch(st + 1, 1);
 }
 
-__device__ __forceinline__ bool timed_out_elsewhere() {
-  return *reinterpret_cast<volatile int *>(&g_timed_out) != 0;
+__device__ __forceinline__ bool timed_out_elsewhere(const int *st) {
+  return *reinterpret_cast<const volatile int *>(st + 1) != 0;
 }
+
+// A CTA's abort flag (raised by the first of its waits that gives up) and
+// the status word of its launch.
+struct AbortCtl {
+  int flag;
+  int *status;
+};
+
+__device__ __forceinline__ void abort_init(AbortCtl *c, int *status) {
+  c->flag = 0;
+  c->status = status;
+}
+
+__device__ __forceinline__ bool abort_raised(const AbortCtl *c) {
+  return *reinterpret_cast<const volatile int *>(&c->flag) != 0;
+}
+
+__device__ __forceinline__ void abort_raise(AbortCtl *c) { *reinterpret_cast<volatile int *>(&c->flag) = 1; }
 
 // ---------------------------------------------------------------------------
 // small math / bit helpers
@@ -107,6 +127,12 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
 // well below the 2^-9 of the bf16 rounding P gets next); 2^n added to the
 // exponent field as an integer.  x is clamped at -125 so the result stays a
 // normal number: masked logits (-inf) give 2^-125 (about 2.4e-38), not 0.
+// There is no clamp from above: the exponent add is right for round(x) <= 127
+// only (beyond it the carry reaches the sign bit), so callers keep x at or
+// below kExp2PolyMaxInput (the softmax's lazy-rescale threshold is checked
+// against it at compile time).  A NaN input gives 2^-125, where the MUFU
+// exponential would give NaN.
+constexpr float kExp2PolyMaxInput = 126.f;
 constexpr float kExp2C0 = 0.99992806f;
 constexpr float kExp2C1 = 0.69326097f;
 constexpr float kExp2C2 = 0.24261114f;
@@ -177,23 +203,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete, at most timeout_ns.
-// Returns false (and raises *abort) on timeout or when another role already
-// aborted the CTA.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          uint64_t timeout_ns) {
+// Returns false (and raises the CTA's abort flag) on timeout or when another
+// role already aborted the CTA.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, AbortCtl *abort, uint64_t timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 31u) == 0) {
-      if (*abort) return false;
-      if (timed_out_elsewhere()) {
-        *abort = 1;
+      if (abort_raised(abort)) return false;
+      if (timed_out_elsewhere(abort->status)) {
+        abort_raise(abort);
         return false;
       }
       if (global_timer_ns() - t0 > timeout_ns) {
-        *abort = 1;
-        raise_timeout();
+        abort_raise(abort);
+        raise_timeout(abort->status);
         return false;
       }
     }
@@ -202,8 +227,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 
 // Warp-uniform variant: every lane of the warp calls it and all lanes return
 // the same value; the phase counts as observed only once every lane saw it.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                               uint64_t timeout_ns, int lane) {
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, AbortCtl *abort, uint64_t timeout_ns,
+                                               int lane) {
   uint64_t t0 = 0;
   if (lane == 0) t0 = global_timer_ns();
   for (uint32_t it = 0;; ++it) {
@@ -212,14 +237,14 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, v
     if ((it & 31u) == 31u) {
       int stop = 0;
       if (lane == 0) {
-        if (*abort) {
+        if (abort_raised(abort)) {
           stop = 1;
-        } else if (timed_out_elsewhere()) {
-          *abort = 1;
+        } else if (timed_out_elsewhere(abort->status)) {
+          abort_raise(abort);
           stop = 1;
         } else if (global_timer_ns() - t0 > timeout_ns) {
-          *abort = 1;
-          raise_timeout();
+          abort_raise(abort);
+          raise_timeout(abort->status);
           stop = 1;
         }
       }
@@ -230,8 +255,8 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, v
 
 // Warp-uniform wait with a single poll on the fast path (the phase is
 // usually complete by the time the issuer gets to it).
-__device__ __forceinline__ bool mbar_wait_uni(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                              uint64_t timeout_ns, int lane) {
+__device__ __forceinline__ bool mbar_wait_uni(uint64_t *bar, uint32_t parity, AbortCtl *abort, uint64_t timeout_ns,
+                                              int lane) {
   if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   return mbar_wait_warp(bar, parity, abort, timeout_ns, lane);
 }
@@ -262,6 +287,31 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_addr(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
+}
+
+// The same copy with an L2 eviction-priority hint (a policy from
+// l2_policy_evict_first / l2_policy_evict_last).
+__device__ __forceinline__ void tma_load_3d_hint(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y,
+                                                 int z, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z), "l"(policy)
+      : "memory");
+}
+
+// L2 cache policies: lines read once (evict first) and lines that other CTAs
+// read again (evict last).
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
 }
 
 // Make generic-proxy writes to shared memory visible to the async proxy

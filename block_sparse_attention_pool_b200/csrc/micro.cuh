@@ -33,12 +33,16 @@ constexpr int kHistBins = 2048;
 
 struct MicroWs {
   int32_t *slot_of_bh;  // [B*H] slot or -1
-  uint32_t *bitmap;     // [slots][n_q][32] kept key blocks of each Macro row
+  uint32_t *bitmap;     // [slots][n_q][bitmap_words] kept key blocks of each Macro row
   uint32_t *keys;       // [slots][n_r][n_t]
   uint32_t *hist;       // [slots][3][kHistBins]
   uint32_t *state;      // [slots][8]: M, prefix, rank-left, tau, ...
   int n_slots;
+  int bitmap_words;     // max(32, ceil(n_k / 32))
+  int *status;          // the launch's status word
 };
+
+constexpr int kMicroMaxKeyBlocks = 4096;
 
 // Dense kept-block bitmap of every Macro row of the enabled heads.
 __global__ void micro_bitmap_kernel(const int32_t *__restrict__ counts, const int32_t *__restrict__ idx, int n_q,
@@ -47,8 +51,9 @@ __global__ void micro_bitmap_kernel(const int32_t *__restrict__ counts, const in
   const int bh = blockIdx.y;
   const int slot = ws.slot_of_bh[bh];
   if (slot < 0 || row >= n_q) return;
-  __shared__ uint32_t bits[32];
-  if (threadIdx.x < 32) bits[threadIdx.x] = 0u;
+  __shared__ uint32_t bits[kMicroMaxKeyBlocks / 32];
+  const int W = ws.bitmap_words;
+  for (int w = threadIdx.x; w < W; w += blockDim.x) bits[w] = 0u;
   __syncthreads();
   const size_t r = (size_t)bh * n_q + row;
   const int c = counts[r];
@@ -57,7 +62,7 @@ __global__ void micro_bitmap_kernel(const int32_t *__restrict__ counts, const in
     if (j >= 0 && j < n_k) atomicOr(&bits[j >> 5], 1u << (j & 31));
   }
   __syncthreads();
-  if (threadIdx.x < 32) ws.bitmap[((size_t)slot * n_q + row) * 32 + threadIdx.x] = bits[threadIdx.x];
+  for (int w = threadIdx.x; w < W; w += blockDim.x) ws.bitmap[((size_t)slot * n_q + row) * W + w] = bits[w];
 }
 
 struct ScoreArgs {
@@ -84,14 +89,19 @@ __global__ void __launch_bounds__(kScoreThreads) micro_score_kernel(ScoreArgs a,
   const float *qp = a.q64 + (size_t)bh * a.n_r * D;
   const float *kp = a.k16 + (size_t)bh * a.n_t * D;
 
-  // kept bitmaps of the Macro rows of this CTA's Micro rows
+  // kept bitmaps of the Macro rows of this CTA's Micro rows: the 32 words
+  // (1024 key blocks) from the one holding the CTA's first tile, which cover
+  // all of its 128 tiles
+  const int per = a.bk / kMicroKeys;
+  const int W = ws.bitmap_words;
+  const int w0 = (t0 / per) >> 5;
   for (int i = tid; i < kScoreBM * 32; i += kScoreThreads) {
     const int rr = i >> 5, w = i & 31;
     const int r = r0 + rr;
-    uint32_t v = 0xffffffffu;  // rows outside the head: nothing is a candidate
-    if (r < a.n_r) {
+    uint32_t v = 0xffffffffu;  // rows outside the head, words past the row: nothing is a candidate
+    if (r < a.n_r && w0 + w < W) {
       const int qi = (r * kMicroRows) / a.bq;
-      v = ws.bitmap[((size_t)slot * a.n_q + qi) * 32 + w];
+      v = ws.bitmap[((size_t)slot * a.n_q + qi) * W + w0 + w];
     }
     rowbits[rr][w] = v;
   }
@@ -148,7 +158,6 @@ __global__ void __launch_bounds__(kScoreThreads) micro_score_kernel(ScoreArgs a,
 
   // keys + candidate test + fused first-pass histogram
   uint32_t local_cnt = 0;
-  const int per = a.bk / kMicroKeys;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int rr = ty * 4 + i;
@@ -161,7 +170,7 @@ __global__ void __launch_bounds__(kScoreThreads) micro_score_kernel(ScoreArgs a,
       bool cand = row_ok && t < a.n_t && t * kMicroKeys < a.n_valid;
       if (cand) {
         const int kb = t / per;
-        cand = ((rowbits[rr][kb >> 5] >> (kb & 31)) & 1u) == 0u;
+        cand = ((rowbits[rr][(kb >> 5) - w0] >> (kb & 31)) & 1u) == 0u;
       }
       const uint32_t key = cand ? float_key(acc[i][j] * a.scale) : 0u;
       out[j] = key;
@@ -318,7 +327,7 @@ __global__ void micro_compact_kernel(MicroWs ws, int n_r, int n_t, int BH, int r
       total += __popc(b);
     }
   }
-  if (__any_sync(0xffffffffu, overflow) && lane == 0) latch_status(VSA_ERR_CAPACITY);
+  if (__any_sync(0xffffffffu, overflow) && lane == 0) latch_status(ws.status, VSA_ERR_CAPACITY);
   if (lane == 0) m_counts[gw] = total < row_capacity ? total : row_capacity;
 }
 
@@ -367,7 +376,7 @@ __global__ void micro_topk_kernel(MicroWs ws, int n_r, int n_t, int BH, int topk
   }
   const int cap = n_sel < row_capacity ? n_sel : row_capacity;
   if (lane < n_sel && rank < row_capacity) dst[rank] = chosen;
-  if (n_sel > row_capacity && lane == 0) latch_status(VSA_ERR_CAPACITY);
+  if (n_sel > row_capacity && lane == 0) latch_status(ws.status, VSA_ERR_CAPACITY);
   if (lane == 0) m_counts[gw] = cap;
 }
 

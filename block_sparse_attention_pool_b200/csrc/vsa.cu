@@ -52,6 +52,42 @@ vsa_status launch_status() {
   return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
+// ---- status words ------------------------------------------------------------
+// Caller-owned status words bound to streams (vsa_bind_status_word); launches
+// on any other stream report into the process-wide word of the device.
+constexpr int kMaxStatusBindings = 256;
+
+struct StatusBinding {
+  cudaStream_t stream;
+  int device;
+  int *word;
+};
+
+std::mutex &binding_mutex() {
+  static std::mutex mu;
+  return mu;
+}
+
+std::vector<StatusBinding> &bindings() {
+  static std::vector<StatusBinding> b;
+  return b;
+}
+
+// The status word that launches on `st` (of the current device) report into,
+// or nullptr if no device address can be had.
+int *status_word(cudaStream_t st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  {
+    std::lock_guard<std::mutex> lock(binding_mutex());
+    for (const StatusBinding &b : bindings())
+      if (b.stream == st && b.device == dev) return b.word;
+  }
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, vsa::g_status_word) != cudaSuccess) return nullptr;
+  return static_cast<int *>(p);
+}
+
 // ---- tensor maps -----------------------------------------------------------
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -197,7 +233,7 @@ vsa_status launch_attn_dual(const void *q, const void *k, const void *v, const v
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct MicroLayout {
-  int n_slots;
+  int n_slots, bitmap_words;
   size_t off_slot, off_bitmap, off_keys, off_hist, off_state, total;
 };
 
@@ -208,11 +244,12 @@ MicroLayout micro_layout(const vsa_shape *s, const vsa_micro_params *p) {
   L.n_slots = enabled * s->B;
   const size_t n_r = (size_t)s->n_pad / vsa::kMicroRows, n_t = (size_t)s->n_pad / vsa::kMicroKeys;
   const size_t n_qmax = (size_t)s->n_pad / 64;
+  L.bitmap_words = std::max(32, (s->n_pad / 64 + 31) / 32);  // words of the longest kept-block bitmap (64-key blocks)
   size_t off = 0;
   L.off_slot = off;
   off = align256(off + (size_t)s->B * s->H * 4);
   L.off_bitmap = off;
-  off = align256(off + (size_t)L.n_slots * n_qmax * 32 * 4);
+  off = align256(off + (size_t)L.n_slots * n_qmax * L.bitmap_words * 4);
   L.off_keys = off;
   off = align256(off + (size_t)L.n_slots * n_r * n_t * 4);
   L.off_hist = off;
@@ -241,41 +278,33 @@ int ilog2(int x) {
 // host-side stand-in; the device address comes from cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_micro_noalloc_scratch[VSA_MICRO_NOALLOC_MAX_BYTES];
 
-constexpr int kNoallocMaxDevices = 64;
-constexpr int kNoallocMaxBH = 1024;
+constexpr int kMicroMaxHeads = 1024;
 
-// Device address of the fixed scratch on the current device, looked up once
-// per device (with that device current) and cached.
+// Device address of the fixed scratch on the current device.  Looked up on
+// every call (a cheap query once the module is loaded), so the address stays
+// right even after the primary context was reset and the module reloaded.
 vsa_status noalloc_scratch(void **out) {
-  static std::mutex mu;
-  static void *addr[kNoallocMaxDevices] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) return VSA_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_micro_noalloc_scratch) != cudaSuccess || p == nullptr) return VSA_ERR_CUDA;
-    addr[dev] = p;
-  }
-  *out = addr[dev];
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_micro_noalloc_scratch) != cudaSuccess || p == nullptr) return VSA_ERR_CUDA;
+  *out = p;
   return VSA_OK;
 }
 
 // One thread waits on a barrier that no one arrives at; the bounded wait gives
 // up after limit_ns and latches VSA_ERR_TIMEOUT.
-__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+__global__ void selftest_wait_kernel(unsigned long long limit_ns, int *status) {
   __shared__ uint64_t bar;
-  __shared__ int abort_flag;
+  __shared__ vsa::AbortCtl abort_ctl;
   if (threadIdx.x != 0) return;
-  abort_flag = 0;
+  vsa::abort_init(&abort_ctl, status);
   vsa::mbar_init(&bar, 1);
   vsa::fence_barrier_init();
-  vsa::mbar_wait(&bar, 0, &abort_flag, limit_ns);
+  vsa::mbar_wait(&bar, 0, &abort_ctl, limit_ns);
 }
 
 // The softmax's FMA-pipe exponential on a caller's array, two values per thread.
 __global__ void selftest_exp2_kernel(const float *__restrict__ x, float *__restrict__ y, int n) {
-  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  const long long i = 2ll * ((long long)blockIdx.x * blockDim.x + threadIdx.x);
   if (i >= n) return;
   const float2 in = make_float2(x[i], i + 1 < n ? x[i + 1] : 0.f);
   const float2 out = vsa::exp2_poly2(in);
@@ -283,14 +312,15 @@ __global__ void selftest_exp2_kernel(const float *__restrict__ x, float *__restr
   if (i + 1 < n) y[i + 1] = out.y;
 }
 
-// Per-head slot numbers handed to the device by value (no host-to-device copy).
+// Per-head slot numbers handed to the device by value (no host-to-device copy
+// and no host buffer that must outlive the call).
 struct HeadSlots {
-  int16_t slot[kNoallocMaxBH];  // rank among enabled heads, or -1
+  int16_t slot[kMicroMaxHeads];  // rank among enabled heads, or -1
   int n_enabled;
   int H, BH;
 };
 
-__global__ void noalloc_slot_fill_kernel(HeadSlots hs, int32_t *slot_of_bh) {
+__global__ void micro_slot_fill_kernel(HeadSlots hs, int32_t *slot_of_bh) {
   const int bh = blockIdx.x * blockDim.x + threadIdx.x;
   if (bh >= hs.BH) return;
   const int b = bh / hs.H, h = bh % hs.H;
@@ -298,6 +328,78 @@ __global__ void noalloc_slot_fill_kernel(HeadSlots hs, int32_t *slot_of_bh) {
   slot_of_bh[bh] = r < 0 ? -1 : b * hs.n_enabled + r;
 }
 
+// Host-side checks shared by vsa_select_micro and vsa_select_micro_noalloc.
+vsa_status check_micro_args(const float *q_pool64, const float *k_pool16, const int32_t *counts, const int32_t *idx,
+                            const vsa_shape *shape, int bq, int bk, float scale, const vsa_micro_params *params,
+                            const int32_t *m_counts, const int32_t *m_idx) {
+  if (!shape_ok(shape) || !q_pool64 || !k_pool16 || !counts || !idx || !m_counts || !m_idx)
+    return VSA_ERR_INVALID_ARG;
+  if (!micro_params_ok(params)) return VSA_ERR_INVALID_ARG;
+  if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return VSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(q_pool64) || !aligned16(k_pool16)) return VSA_ERR_INVALID_ARG;
+  if (shape->n_pad / 64 > vsa::kMicroMaxKeyBlocks) return VSA_ERR_UNSUPPORTED;
+  if (shape->H > kMicroMaxHeads) return VSA_ERR_UNSUPPORTED;
+  return VSA_OK;
+}
+
+// The Micro selection launch sequence on a scratch area laid out by L
+// (caller workspace or the fixed array): slot table, then the kernels.
+vsa_status launch_micro_select(const float *q_pool64, const float *k_pool16, const int32_t *counts,
+                               const int32_t *idx, const vsa_shape *shape, int bq, int bk, float scale,
+                               const vsa_micro_params *params, int32_t *m_counts, int32_t *m_idx, uint8_t *ws8,
+                               const MicroLayout &L, cudaStream_t st) {
+  const int n_q = shape->n_pad / bq, n_k = shape->n_pad / bk;
+  const int BH = shape->B * shape->H;
+  const int n_r = shape->n_pad / vsa::kMicroRows, n_t = shape->n_pad / vsa::kMicroKeys;
+  vsa::MicroWs ws;
+  ws.slot_of_bh = reinterpret_cast<int32_t *>(ws8 + L.off_slot);
+  ws.bitmap = reinterpret_cast<uint32_t *>(ws8 + L.off_bitmap);
+  ws.keys = reinterpret_cast<uint32_t *>(ws8 + L.off_keys);
+  ws.hist = reinterpret_cast<uint32_t *>(ws8 + L.off_hist);
+  ws.state = reinterpret_cast<uint32_t *>(ws8 + L.off_state);
+  ws.n_slots = L.n_slots;
+  ws.bitmap_words = L.bitmap_words;
+  ws.status = status_word(st);
+  if (!ws.status) return VSA_ERR_CUDA;
+
+  HeadSlots hs;
+  int next = 0;
+  for (int h = 0; h < shape->H; ++h)
+    hs.slot[h] = (params->head_enable == nullptr || params->head_enable[h]) ? (int16_t)next++ : (int16_t)-1;
+  hs.n_enabled = next;
+  hs.H = shape->H;
+  hs.BH = BH;
+  micro_slot_fill_kernel<<<(BH + 255) / 256, 256, 0, st>>>(hs, ws.slot_of_bh);
+  if (L.n_slots == 0) {
+    if (cudaMemsetAsync(m_counts, 0, (size_t)BH * n_r * 4, st) != cudaSuccess) return VSA_ERR_CUDA;
+    return launch_status();
+  }
+  // histograms and rank-search state must start at zero on every call
+  if (cudaMemsetAsync(ws8 + L.off_hist, 0, L.total - L.off_hist, st) != cudaSuccess) return VSA_ERR_CUDA;
+
+  vsa::micro_bitmap_kernel<<<dim3(n_q, BH), 128, 0, st>>>(counts, idx, n_q, n_k, BH, ws);
+  vsa::ScoreArgs sa{q_pool64, k_pool16, n_r, n_t, n_q, bq, bk, shape->n_valid, scale, params->mode == 2 ? 1 : 0};
+  dim3 sg((n_t + vsa::kScoreBN - 1) / vsa::kScoreBN, (n_r + vsa::kScoreBM - 1) / vsa::kScoreBM, BH);
+  if (shape->d == 128)
+    vsa::micro_score_kernel<128><<<sg, vsa::kScoreThreads, 0, st>>>(sa, ws);
+  else
+    vsa::micro_score_kernel<64><<<sg, vsa::kScoreThreads, 0, st>>>(sa, ws);
+  const unsigned rows_blocks = (unsigned)(((size_t)BH * n_r + 7) / 8);
+  if (params->mode == 1) {
+    vsa::micro_topk_kernel<<<rows_blocks, 256, 0, st>>>(ws, n_r, n_t, BH, params->topk, params->row_capacity,
+                                                      m_counts, m_idx);
+  } else {
+    const size_t per_slot = (size_t)n_r * n_t;
+    vsa::micro_find_kernel<<<L.n_slots, 32, 0, st>>>(ws, params->percentile, 0);
+    vsa::micro_hist_kernel<<<dim3(256, L.n_slots), 256, 0, st>>>(ws, per_slot, 1);
+    vsa::micro_find_kernel<<<L.n_slots, 32, 0, st>>>(ws, params->percentile, 1);
+    vsa::micro_hist_kernel<<<dim3(256, L.n_slots), 256, 0, st>>>(ws, per_slot, 2);
+    vsa::micro_find_kernel<<<L.n_slots, 32, 0, st>>>(ws, params->percentile, 2);
+    vsa::micro_compact_kernel<<<rows_blocks, 256, 0, st>>>(ws, n_r, n_t, BH, params->row_capacity, m_counts, m_idx);
+  }
+  return launch_status();
+}
 
 // ---- clustering --------------------------------------------------------------
 
@@ -410,10 +512,19 @@ bool select_params_ok(float scale, const vsa_select_params *params) {
 // explicit sizes), one CTA per 16 query units of one (batch, head).
 vsa_status launch_select(const vsa::SelectArgs &a, int d, int BH, bool by_rank, cudaStream_t st) {
   const int n_q = a.n_q, n_k = a.n_k;
+  if (n_k > 1024) {
+    // rows too long for one warp: one CTA per row
+    const dim3 grid(n_q, BH);
+    if (d == 128)
+      vsa::select_long_kernel<128><<<grid, vsa::kLongThreads, 0, st>>>(a);
+    else
+      vsa::select_long_kernel<64><<<grid, vsa::kLongThreads, 0, st>>>(a);
+    return launch_status();
+  }
   int nkp = 32;
   while (nkp < n_k) nkp <<= 1;
   const int dp = d + 4;
-  const size_t smem = (size_t)(vsa::kSelRows + vsa::kSelChunk) * dp * 4 + (size_t)vsa::kSelRows * nkp * 4 + 8 * 32 * 4;
+  const size_t smem = (size_t)vsa::kSelRows * dp * 4 + (size_t)vsa::kSelRows * nkp * 4 + 8 * 32 * 4;
   dim3 grid((n_q + vsa::kSelRows - 1) / vsa::kSelRows, BH);
 #define VSA_SEL_CASE(DD, NR)                                                                                  \
   {                                                                                                           \
@@ -486,18 +597,41 @@ int vsa_version(void) { return 200; }
 
 vsa_status vsa_read_device_status(void *stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int *word = status_word(st);
+  if (!word) return VSA_ERR_CUDA;
+  int h[2] = {0, 0};
   if (cudaStreamSynchronize(st) != cudaSuccess) return VSA_ERR_CUDA;
-  int h = 0;
-  if (cudaMemcpyFromSymbol(&h, vsa::g_status, sizeof(int)) != cudaSuccess) return VSA_ERR_CUDA;
-  const int zero = 0;
-  if (cudaMemcpyToSymbol(vsa::g_status, &zero, sizeof(int)) != cudaSuccess) return VSA_ERR_CUDA;
-  if (cudaMemcpyToSymbol(vsa::g_timed_out, &zero, sizeof(int)) != cudaSuccess) return VSA_ERR_CUDA;
-  return static_cast<vsa_status>(h);
+  if (cudaMemcpyAsync(h, word, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemsetAsync(word, 0, sizeof(h), st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
+    return VSA_ERR_CUDA;
+  return static_cast<vsa_status>(h[0]);
+}
+
+vsa_status vsa_bind_status_word(void *stream, int32_t *word) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (word && (reinterpret_cast<uintptr_t>(word) & 3u) != 0) return VSA_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(binding_mutex());
+  std::vector<StatusBinding> &b = bindings();
+  for (size_t i = 0; i < b.size(); ++i) {
+    if (b[i].stream == st && b[i].device == dev) {
+      b.erase(b.begin() + static_cast<long>(i));
+      break;
+    }
+  }
+  if (!word) return VSA_OK;
+  if (b.size() >= (size_t)kMaxStatusBindings) return VSA_ERR_CAPACITY;
+  if (cudaMemsetAsync(word, 0, VSA_STATUS_WORD_BYTES, st) != cudaSuccess) return VSA_ERR_CUDA;
+  b.push_back({st, dev, word});
+  return VSA_OK;
 }
 
 vsa_status vsa_selftest_wait_timeout(unsigned long long limit_ns, void *stream) {
   if (limit_ns < 1000ull || limit_ns > 5000000000ull) return VSA_ERR_INVALID_ARG;
-  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  int *word = status_word(static_cast<cudaStream_t>(stream));
+  if (!word) return VSA_ERR_CUDA;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, word);
   return launch_status();
 }
 
@@ -536,7 +670,7 @@ vsa_status vsa_select_blocks(const float *q_pool, const float *k_pool, const vsa
   if (!aligned16(q_pool) || !aligned16(k_pool)) return VSA_ERR_INVALID_ARG;
   if (!select_params_ok(scale, params)) return VSA_ERR_INVALID_ARG;
   const int n_q = shape->n_pad / bq, n_k = shape->n_pad / bk;
-  if (n_k > 1024) return VSA_ERR_UNSUPPORTED;
+  if (n_k > vsa::kSelLongMax) return VSA_ERR_UNSUPPORTED;
   vsa::SelectArgs a{q_pool, k_pool, n_q, n_k, bq, bk, shape->n_valid, scale, params->k_min, params->fixed_k,
                     params->n_anchor, params->anchor_rot, params->cum_mass, counts, idx, mask, nullptr, nullptr};
   return launch_select(a, shape->d, shape->B * shape->H, params->fixed_k > 0, static_cast<cudaStream_t>(stream));
@@ -549,7 +683,7 @@ vsa_status vsa_select_clusters(const float *mu_q, const float *mu_k, const int32
   if (batch_heads < 1 || batch_heads > 65535 || n_q < 1 || n_k < 1 || (d != 64 && d != 128)) return VSA_ERR_INVALID_ARG;
   if (!aligned16(mu_q) || !aligned16(mu_k)) return VSA_ERR_INVALID_ARG;
   if (!select_params_ok(scale, params) || params->n_anchor != 0) return VSA_ERR_INVALID_ARG;
-  if (n_k > 1024) return VSA_ERR_UNSUPPORTED;
+  if (n_k > vsa::kSelLongMax) return VSA_ERR_UNSUPPORTED;
   vsa::SelectArgs a{mu_q, mu_k, n_q, n_k, 1, 1, 0, scale, params->k_min, params->fixed_k,
                     0, 0, params->cum_mass, counts, idx, nullptr, sizes_q, sizes_k};
   return launch_select(a, d, batch_heads, params->fixed_k > 0, static_cast<cudaStream_t>(stream));
@@ -560,7 +694,6 @@ vsa_status vsa_mask_to_lists(const uint8_t *mask, const vsa_shape *shape, int bq
   if (!shape_ok(shape) || !mask || !counts || !idx) return VSA_ERR_INVALID_ARG;
   if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return VSA_ERR_INVALID_ARG;
   const int n_q = shape->n_pad / bq, n_k = shape->n_pad / bk;
-  if (n_k > 1024) return VSA_ERR_UNSUPPORTED;
   const int rows = shape->B * shape->H * n_q;
   vsa::mask_to_lists_kernel<<<(rows + 7) / 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(mask, rows, n_k, counts,
                                                                                           idx);
@@ -576,131 +709,31 @@ vsa_status vsa_select_micro(const float *q_pool64, const float *k_pool16, const 
                             const vsa_shape *shape, int bq, int bk, float scale, const vsa_micro_params *params,
                             int32_t *m_counts, int32_t *m_idx, void *workspace, size_t workspace_bytes,
                             void *stream) {
-  if (!shape_ok(shape) || !q_pool64 || !k_pool16 || !counts || !idx || !m_counts || !m_idx || !workspace)
-    return VSA_ERR_INVALID_ARG;
-  if (!micro_params_ok(params)) return VSA_ERR_INVALID_ARG;
-  if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return VSA_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || !std::isfinite(scale)) return VSA_ERR_INVALID_ARG;
-  if (!aligned16(q_pool64) || !aligned16(k_pool16) || !aligned16(workspace)) return VSA_ERR_INVALID_ARG;
+  const vsa_status ae =
+      check_micro_args(q_pool64, k_pool16, counts, idx, shape, bq, bk, scale, params, m_counts, m_idx);
+  if (ae != VSA_OK) return ae;
+  if (!workspace || !aligned16(workspace)) return VSA_ERR_INVALID_ARG;
   const MicroLayout L = micro_layout(shape, params);
   if (workspace_bytes < L.total) return VSA_ERR_INVALID_ARG;
-  const int n_q = shape->n_pad / bq, n_k = shape->n_pad / bk;
-  if (n_k > 1024) return VSA_ERR_UNSUPPORTED;
-  const int BH = shape->B * shape->H;
-  const int n_r = shape->n_pad / vsa::kMicroRows, n_t = shape->n_pad / vsa::kMicroKeys;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t *ws8 = static_cast<uint8_t *>(workspace);
-  vsa::MicroWs ws;
-  ws.slot_of_bh = reinterpret_cast<int32_t *>(ws8 + L.off_slot);
-  ws.bitmap = reinterpret_cast<uint32_t *>(ws8 + L.off_bitmap);
-  ws.keys = reinterpret_cast<uint32_t *>(ws8 + L.off_keys);
-  ws.hist = reinterpret_cast<uint32_t *>(ws8 + L.off_hist);
-  ws.state = reinterpret_cast<uint32_t *>(ws8 + L.off_state);
-  ws.n_slots = L.n_slots;
-
-  std::vector<int32_t> slot((size_t)BH, -1);
-  int next = 0;
-  for (int b = 0; b < shape->B; ++b)
-    for (int h = 0; h < shape->H; ++h)
-      if (params->head_enable == nullptr || params->head_enable[h]) slot[(size_t)b * shape->H + h] = next++;
-  if (cudaMemcpyAsync(ws.slot_of_bh, slot.data(), slot.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess)
-    return VSA_ERR_CUDA;
-  if (L.n_slots == 0) {
-    if (cudaMemsetAsync(m_counts, 0, (size_t)BH * n_r * 4, st) != cudaSuccess) return VSA_ERR_CUDA;
-    return VSA_OK;
-  }
-  if (cudaMemsetAsync(ws8 + L.off_hist, 0, L.total - L.off_hist, st) != cudaSuccess) return VSA_ERR_CUDA;
-
-  vsa::micro_bitmap_kernel<<<dim3(n_q, BH), 128, 0, st>>>(counts, idx, n_q, n_k, BH, ws);
-  vsa::ScoreArgs sa{q_pool64, k_pool16, n_r, n_t, n_q, bq, bk, shape->n_valid, scale, params->mode == 2 ? 1 : 0};
-  dim3 sg((n_t + vsa::kScoreBN - 1) / vsa::kScoreBN, (n_r + vsa::kScoreBM - 1) / vsa::kScoreBM, BH);
-  if (shape->d == 128)
-    vsa::micro_score_kernel<128><<<sg, vsa::kScoreThreads, 0, st>>>(sa, ws);
-  else
-    vsa::micro_score_kernel<64><<<sg, vsa::kScoreThreads, 0, st>>>(sa, ws);
-  const unsigned rows_blocks = (unsigned)(((size_t)BH * n_r + 7) / 8);
-  if (params->mode == 1) {
-    vsa::micro_topk_kernel<<<rows_blocks, 256, 0, st>>>(ws, n_r, n_t, BH, params->topk, params->row_capacity,
-                                                      m_counts, m_idx);
-  } else {
-    const size_t per_slot = (size_t)n_r * n_t;
-    vsa::micro_find_kernel<<<L.n_slots, 32, 0, st>>>(ws, params->percentile, 0);
-    vsa::micro_hist_kernel<<<dim3(256, L.n_slots), 256, 0, st>>>(ws, per_slot, 1);
-    vsa::micro_find_kernel<<<L.n_slots, 32, 0, st>>>(ws, params->percentile, 1);
-    vsa::micro_hist_kernel<<<dim3(256, L.n_slots), 256, 0, st>>>(ws, per_slot, 2);
-    vsa::micro_find_kernel<<<L.n_slots, 32, 0, st>>>(ws, params->percentile, 2);
-    vsa::micro_compact_kernel<<<rows_blocks, 256, 0, st>>>(ws, n_r, n_t, BH, params->row_capacity, m_counts, m_idx);
-  }
-  return launch_status();
+  return launch_micro_select(q_pool64, k_pool16, counts, idx, shape, bq, bk, scale, params, m_counts, m_idx,
+                             static_cast<uint8_t *>(workspace), L, static_cast<cudaStream_t>(stream));
 }
 
 vsa_status vsa_select_micro_noalloc(const float *q_pool64, const float *k_pool16, const int32_t *counts,
                                     const int32_t *idx, const vsa_shape *shape, int bq, int bk, float scale,
                                     const vsa_micro_params *params, int32_t *m_counts, int32_t *m_idx,
                                     void *stream) {
-  if (!shape_ok(shape) || !q_pool64 || !k_pool16 || !counts || !idx || !m_counts || !m_idx)
-    return VSA_ERR_INVALID_ARG;
-  if (!micro_params_ok(params)) return VSA_ERR_INVALID_ARG;
-  if ((bq != 64 && bq != 128) || (bk != 64 && bk != 128)) return VSA_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || !std::isfinite(scale)) return VSA_ERR_INVALID_ARG;
-  if (!aligned16(q_pool64) || !aligned16(k_pool16)) return VSA_ERR_INVALID_ARG;
-  const int n_q = shape->n_pad / bq, n_k = shape->n_pad / bk;
-  if (n_k > 1024) return VSA_ERR_UNSUPPORTED;
-  const int BH = shape->B * shape->H;
-  if (BH > kNoallocMaxBH) return VSA_ERR_SCRATCH_LIMIT;
+  const vsa_status ae =
+      check_micro_args(q_pool64, k_pool16, counts, idx, shape, bq, bk, scale, params, m_counts, m_idx);
+  if (ae != VSA_OK) return ae;
+  if ((long long)shape->B * shape->H > kMicroMaxHeads) return VSA_ERR_SCRATCH_LIMIT;
   const MicroLayout L = micro_layout(shape, params);
   if (L.total > VSA_MICRO_NOALLOC_MAX_BYTES) return VSA_ERR_SCRATCH_LIMIT;
   void *scratch = nullptr;
   const vsa_status se = noalloc_scratch(&scratch);
   if (se != VSA_OK) return se;
-
-  const int n_r = shape->n_pad / vsa::kMicroRows, n_t = shape->n_pad / vsa::kMicroKeys;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t *ws8 = static_cast<uint8_t *>(scratch);
-  vsa::MicroWs ws;
-  ws.slot_of_bh = reinterpret_cast<int32_t *>(ws8 + L.off_slot);
-  ws.bitmap = reinterpret_cast<uint32_t *>(ws8 + L.off_bitmap);
-  ws.keys = reinterpret_cast<uint32_t *>(ws8 + L.off_keys);
-  ws.hist = reinterpret_cast<uint32_t *>(ws8 + L.off_hist);
-  ws.state = reinterpret_cast<uint32_t *>(ws8 + L.off_state);
-  ws.n_slots = L.n_slots;
-
-  HeadSlots hs;
-  int next = 0;
-  for (int h = 0; h < shape->H; ++h)
-    hs.slot[h] = (params->head_enable == nullptr || params->head_enable[h]) ? (int16_t)next++ : (int16_t)-1;
-  hs.n_enabled = next;
-  hs.H = shape->H;
-  hs.BH = BH;
-  noalloc_slot_fill_kernel<<<(BH + 255) / 256, 256, 0, st>>>(hs, ws.slot_of_bh);
-  if (L.n_slots == 0) {
-    if (cudaMemsetAsync(m_counts, 0, (size_t)BH * n_r * 4, st) != cudaSuccess) return VSA_ERR_CUDA;
-    return launch_status();
-  }
-  // histograms and rank-search state must start at zero on every call
-  if (cudaMemsetAsync(ws8 + L.off_hist, 0, L.total - L.off_hist, st) != cudaSuccess) return VSA_ERR_CUDA;
-
-  vsa::micro_bitmap_kernel<<<dim3(n_q, BH), 128, 0, st>>>(counts, idx, n_q, n_k, BH, ws);
-  vsa::ScoreArgs sa{q_pool64, k_pool16, n_r, n_t, n_q, bq, bk, shape->n_valid, scale, params->mode == 2 ? 1 : 0};
-  dim3 sg((n_t + vsa::kScoreBN - 1) / vsa::kScoreBN, (n_r + vsa::kScoreBM - 1) / vsa::kScoreBM, BH);
-  if (shape->d == 128)
-    vsa::micro_score_kernel<128><<<sg, vsa::kScoreThreads, 0, st>>>(sa, ws);
-  else
-    vsa::micro_score_kernel<64><<<sg, vsa::kScoreThreads, 0, st>>>(sa, ws);
-  const unsigned rows_blocks = (unsigned)(((size_t)BH * n_r + 7) / 8);
-  if (params->mode == 1) {
-    vsa::micro_topk_kernel<<<rows_blocks, 256, 0, st>>>(ws, n_r, n_t, BH, params->topk, params->row_capacity,
-                                                      m_counts, m_idx);
-  } else {
-    const size_t per_slot = (size_t)n_r * n_t;
-    vsa::micro_find_kernel<<<L.n_slots, 32, 0, st>>>(ws, params->percentile, 0);
-    vsa::micro_hist_kernel<<<dim3(256, L.n_slots), 256, 0, st>>>(ws, per_slot, 1);
-    vsa::micro_find_kernel<<<L.n_slots, 32, 0, st>>>(ws, params->percentile, 1);
-    vsa::micro_hist_kernel<<<dim3(256, L.n_slots), 256, 0, st>>>(ws, per_slot, 2);
-    vsa::micro_find_kernel<<<L.n_slots, 32, 0, st>>>(ws, params->percentile, 2);
-    vsa::micro_compact_kernel<<<rows_blocks, 256, 0, st>>>(ws, n_r, n_t, BH, params->row_capacity, m_counts, m_idx);
-  }
-  return launch_status();
+  return launch_micro_select(q_pool64, k_pool16, counts, idx, shape, bq, bk, scale, params, m_counts, m_idx,
+                             static_cast<uint8_t *>(scratch), L, static_cast<cudaStream_t>(stream));
 }
 
 vsa_status vsa_block_sparse_fwd(const void *q, const void *k, const void *v, const vsa_shape *shape, int list_rows,
@@ -748,6 +781,8 @@ vsa_status vsa_block_sparse_fwd_heads(const void *q, const void *k, const void *
   a.timeout_ns = kWaitLimitNs;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (n_heads == 0) return VSA_OK;
+  a.status = status_word(st);
+  if (!a.status) return VSA_ERR_CUDA;
   if (list_rows == 128 && seg_keys == 128)
     return shape->d == 128 ? launch_attn_dual<128, false>(q, k, v, shape, a, n_heads, st)
                              : launch_attn_dual<64, false>(q, k, v, shape, a, n_heads, st);
@@ -810,9 +845,11 @@ vsa_status vsa_permute_rows(const void *src, const int32_t *perm, int batch_head
   if (s8 < d8 + span && d8 < s8 + span) return VSA_ERR_INVALID_ARG;  // overlapping buffers
   const long long blocks = (rows + 7) / 8;
   if (blocks > 0x7fffffffll) return VSA_ERR_UNSUPPORTED;
+  int *word = status_word(static_cast<cudaStream_t>(stream));
+  if (!word) return VSA_ERR_CUDA;
   vsa::permute_rows_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint32_t *>(src), perm, n_pad, rows, row_bytes / 4, inverse ? 1 : 0,
-      static_cast<uint32_t *>(dst));
+      static_cast<uint32_t *>(dst), word);
   return launch_status();
 }
 
@@ -852,6 +889,8 @@ vsa_status vsa_merge_clusters(const int32_t *sizes_q, const int32_t *sizes_k, co
   a.g_idx = g_idx;
   merge_ws_layout(batch_heads, n_q, workspace, &a.ws);
   a.timeout_ns = kWaitLimitNs;
+  a.status = status_word(static_cast<cudaStream_t>(stream));
+  if (!a.status) return VSA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   vsa::merge_init_kernel<<<batch_heads, vsa::kMergeHeadThreads, 0, st>>>(a);
   if (rounds > 0) {
@@ -884,7 +923,10 @@ vsa_status vsa_cluster_plan(const int32_t *group_of, const int32_t *sizes_q, con
     return VSA_ERR_INVALID_ARG;
   if (n_rows < 128 || n_rows % 128 != 0) return VSA_ERR_INVALID_ARG;
   if (n_q > vsa::kPlanMaxClusters || n_k > vsa::kPlanMaxClusters) return VSA_ERR_UNSUPPORTED;
-  vsa::PlanArgs a{group_of, sizes_q, perm_q, sizes_k, n_q, n_k, n_valid, n_pad, n_rows, qmap, qinv, tile_list, kc_off};
+  int *word = status_word(static_cast<cudaStream_t>(stream));
+  if (!word) return VSA_ERR_CUDA;
+  vsa::PlanArgs a{group_of, sizes_q, perm_q, sizes_k, n_q, n_k, n_valid, n_pad, n_rows, qmap, qinv, tile_list, kc_off,
+                  word};
   vsa::cluster_plan_kernel<<<batch_heads, vsa::kPlanThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
   return launch_status();
 }
@@ -906,8 +948,11 @@ vsa_status vsa_gather_rows(const void *src, const int32_t *map, int batch_heads,
   const long long rows = (long long)batch_heads * n_dst;
   const long long blocks = (rows + 7) / 8;
   if (blocks > 0x7fffffffll) return VSA_ERR_UNSUPPORTED;
+  int *word = status_word(static_cast<cudaStream_t>(stream));
+  if (!word) return VSA_ERR_CUDA;
   vsa::gather_rows_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint32_t *>(src), map, n_src, n_dst, rows, row_bytes / 4, fill, static_cast<uint32_t *>(dst));
+      static_cast<const uint32_t *>(src), map, n_src, n_dst, rows, row_bytes / 4, fill, static_cast<uint32_t *>(dst),
+      word);
   return launch_status();
 }
 
@@ -937,6 +982,8 @@ vsa_status vsa_cluster_group_fwd(const void *q_rows, const void *k, const void *
   a.lse = lse;
   a.n_bh = shape->B * shape->H;
   a.timeout_ns = kWaitLimitNs;
+  a.status = status_word(static_cast<cudaStream_t>(stream));
+  if (!a.status) return VSA_ERR_CUDA;
   a.tile_list = tile_list;
   a.kc_off = kc_off;
   a.kc_size = kc_size;
@@ -1002,6 +1049,8 @@ vsa_status vsa_rectify_fwd(const void *q, const void *k_bar, const void *v_bar, 
   a.heads = heads;
   a.n_bh = static_cast<int>(n_bh);
   a.timeout_ns = kWaitLimitNs;
+  a.status = status_word(static_cast<cudaStream_t>(stream));
+  if (!a.status) return VSA_ERR_CUDA;
   a.pool_nk = n_k;
   a.pool_bk = bk;
   a.pool_nvalid = shape->n_valid;
@@ -1057,6 +1106,8 @@ vsa_status vsa_cluster_refine(const void *x, const vsa_shape *shape, const vsa_c
   int32_t *changed = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) +
                                                  align256((size_t)BH * g.n_cells * n_chunks * 4));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int *word = status_word(st);
+  if (!word) return VSA_ERR_CUDA;
   if (cudaMemsetAsync(changed, 0, (size_t)BH * g.n_cells * 4, st) != cudaSuccess) return VSA_ERR_CUDA;
   const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
   if (n_sub > 0) {
@@ -1066,17 +1117,17 @@ vsa_status vsa_cluster_refine(const void *x, const vsa_shape *shape, const vsa_c
           vsa::reassign_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, vsa::RtLayout<128>::kAlloc);
       if (attr != cudaSuccess) return VSA_ERR_CUDA;
       vsa::reassign_tc_kernel<128><<<grid, vsa::kRtThreads, vsa::RtLayout<128>::kAlloc, st>>>(
-          xb, shape->n_pad, shape->n_valid, g.n_cells, centroids, subset, n_sub, assign, changed, kWaitLimitNs);
+          xb, shape->n_pad, shape->n_valid, g.n_cells, centroids, subset, n_sub, assign, changed, kWaitLimitNs, word);
     } else {
       static const cudaError_t attr = cudaFuncSetAttribute(
           vsa::reassign_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, vsa::RtLayout<64>::kAlloc);
       if (attr != cudaSuccess) return VSA_ERR_CUDA;
       vsa::reassign_tc_kernel<64><<<grid, vsa::kRtThreads, vsa::RtLayout<64>::kAlloc, st>>>(
-          xb, shape->n_pad, shape->n_valid, g.n_cells, centroids, subset, n_sub, assign, changed, kWaitLimitNs);
+          xb, shape->n_pad, shape->n_valid, g.n_cells, centroids, subset, n_sub, assign, changed, kWaitLimitNs, word);
     }
   }
   const dim3 cgrid(n_chunks, BH);
-  vsa::sort_count_kernel<<<cgrid, 256, g.n_cells * 4, st>>>(assign, shape->n_valid, g.n_cells, n_chunks, cnt);
+  vsa::sort_count_kernel<<<cgrid, 256, g.n_cells * 4, st>>>(assign, shape->n_valid, g.n_cells, n_chunks, cnt, word);
   vsa::sort_scan_kernel<<<BH, vsa::kHybThreads, 0, st>>>(cnt, g.n_cells, n_chunks, sizes);
   vsa::sort_scatter_kernel<<<cgrid, 32, g.n_cells * 4, st>>>(assign, shape->n_valid, shape->n_pad, g.n_cells,
                                                             n_chunks, cnt, perm);
@@ -1091,3 +1142,5 @@ vsa_status vsa_cluster_refine(const void *x, const vsa_shape *shape, const vsa_c
 }
 
 }  // extern "C"
+
+#include "path.cuh"

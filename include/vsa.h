@@ -36,7 +36,9 @@
  *           Conditions found on the device (a list longer than its capacity,
  *           an out-of-range index in a caller-given list, a pipeline wait that
  *           ran out of its time limit) are latched into a device status word
- *           that vsa_read_device_status returns and clears.
+ *           that vsa_read_device_status returns and clears: the caller's word
+ *           bound to the call's stream (vsa_bind_status_word), else a
+ *           process-wide word per device.
  * Numerics. Pooling, pooled scores and selection are fp32 (FFMA; no TF32).
  *           Attention multiplies bf16 operands on the tensor cores with fp32
  *           accumulation; P is rounded to bf16 before the P.V product; LSE is
@@ -130,9 +132,26 @@ VSA_API const char *vsa_status_string(vsa_status s);
 /* Library version as major*10000 + minor*100 + patch. */
 VSA_API int vsa_version(void);
 
-/* Synchronise ``stream``, then return and clear the device status word (the
- * first device-side error latched since the last call; VSA_OK if none).   */
+/* Synchronise ``stream``, then return and clear the status word of that
+ * stream (the first device-side error latched since the last read; VSA_OK if
+ * none): the caller's word bound to ``stream`` by vsa_bind_status_word, or
+ * else the library's process-wide word of the current device. */
 VSA_API vsa_status vsa_read_device_status(void *stream);
+
+/* Per-stream status words in caller memory (no counterpart on the pages).
+ * After binding, every call enqueued on ``stream`` (on the current device)
+ * latches its device-side conditions -- capacity, bad index, timeout -- into
+ * ``word`` instead of the process-wide word, so callers on different streams
+ * can tell whose work failed, and a bounded wait that runs out of time aborts
+ * only the waits reporting into the same word.
+ *   word : DEVICE memory of VSA_STATUS_WORD_BYTES bytes, 4-byte aligned,
+ *          owned by the caller and kept alive while bound; the call clears
+ *          it on ``stream``.  NULL removes the stream's binding.
+ * At most 256 bindings at once (VSA_ERR_CAPACITY beyond).  Rebinding a stream
+ * replaces its word.  A binding is looked up when a call is enqueued: bind
+ * before enqueueing the calls it should cover. */
+#define VSA_STATUS_WORD_BYTES 8
+VSA_API vsa_status vsa_bind_status_word(void *stream, int32_t *word);
 
 /* Self-test of the bounded pipeline waits (no counterpart on the pages): one
  * thread waits on a shared-memory barrier that nothing completes, for at most
@@ -235,6 +254,9 @@ VSA_API vsa_status vsa_mask_to_lists(const uint8_t *mask, const vsa_shape *shape
  *            VSA_ERR_CAPACITY.
  * workspace: device scratch of vsa_select_micro_workspace_bytes() bytes,
  *            16-byte aligned; its content on entry is irrelevant.
+ * H <= 1024 and n_pad/bk <= 1024 (VSA_ERR_UNSUPPORTED above).  The head
+ * flags are read on the host during the call and handed to the device by
+ * value: no host-to-device copy, so the call never waits on the host.
  * ------------------------------------------------------------------------- */
 VSA_API size_t vsa_select_micro_workspace_bytes(const vsa_shape *shape, const vsa_micro_params *params);
 
@@ -260,9 +282,10 @@ VSA_API vsa_status vsa_select_micro(const float *q_pool64, const float *k_pool16
  *   - A problem whose scratch (vsa_select_micro_workspace_bytes for the same
  *     shape and params) exceeds VSA_MICRO_NOALLOC_MAX_BYTES is rejected with
  *     VSA_ERR_SCRATCH_LIMIT before anything is enqueued.  B*H <= 1024.
- *   - The first call on a device looks up the device address of the fixed
- *     array (once per device, on the current device) and remembers it; make
- *     that first call before any stream capture.
+ *   - Every call looks up the device address of the fixed array on the
+ *     current device (a host-side query that allocates nothing; the first
+ *     one on a device may load the library's device code, so make it before
+ *     any stream capture).
  *   - Every call on a device shares the one array.  Calls whose GPU work
  *     overlaps in time (different streams, or other threads without
  *     ordering between them) race on it and give undefined lists; order them
@@ -340,6 +363,71 @@ VSA_API vsa_status vsa_block_sparse_fwd_heads(const void *q, const void *k, cons
  * ------------------------------------------------------------------------- */
 VSA_API vsa_status vsa_lse_merge(const float *o_a, const float *lse_a, const float *o_b, const float *lse_b,
                          const vsa_shape *shape, void *o_out, int o_out_fp32, float *lse_out, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * The whole path in one call ([HVA] section 2 Eq. (2)-(4): pooled scores,
+ * selection, attention over the kept blocks; [HyMoR] abstract: Micro repair
+ * merged by exact LSE): vsa_pool_qk -> vsa_select_blocks -> Macro pass ->
+ * vsa_select_micro -> Micro pass with the fused merge, exactly as a caller
+ * would chain the entry points above, on buffers carved from one workspace.
+ * Heads without the Micro repair take their final O from the Macro pass;
+ * heads with it keep an fp32 Macro output that the Micro pass merges into.
+ *
+ *   bq, bk           : Macro block rows, each 64 or 128 (n_pad/bk <= 1024).
+ *   scale            : softmax scale; 0 = 1/sqrt(d).
+ *   select           : the vsa_select_blocks rule.
+ *   micro_mode       : 0 = no Micro repair; 1, 2 as vsa_micro_params.mode.
+ *   micro_topk, micro_percentile : as vsa_micro_params.
+ *   micro_heads      : HOST array of H flags (NULL = every head); H <= 1024.
+ *   micro_capacity   : entries per Micro row; 0 = n_pad/16 (no row can overflow).
+ *   o_fp32           : 1 = O written in fp32, 0 = bf16.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int bq, bk;
+  float scale;
+  vsa_select_params select;
+  int micro_mode;
+  int micro_topk;
+  double micro_percentile;
+  const uint8_t *micro_heads;
+  int micro_capacity;
+  int o_fp32;
+} vsa_path_params;
+
+/* Device workspace of vsa_path_fwd for this shape and params (0 if invalid). */
+VSA_API size_t vsa_path_workspace_bytes(const vsa_shape *shape, const vsa_path_params *params);
+
+/* q, k, v: bf16 [B, H, n_pad, d] DEVICE; o: [B, H, n_pad, d] (bf16 or fp32);
+ * lse: fp32 [B, H, n_pad].  workspace: DEVICE, 256-byte aligned, at least
+ * vsa_path_workspace_bytes(); its content on entry is irrelevant; after the
+ * call it holds the pooled means, the kept lists and the Micro lists.
+ * Asynchronous on stream. */
+VSA_API vsa_status vsa_path_fwd(const void *q, const void *k, const void *v, const vsa_shape *shape,
+                                const vsa_path_params *params, void *o, float *lse, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
+/* The same path on HOST buffers: q_host, k_host, v_host bf16 [B, H, n_pad, d]
+ * in, o_host ([B, H, n_pad, d], bf16 or fp32) and lse_host (fp32 [B, H,
+ * n_pad]) out.  Every (batch, head) is an independent problem, so the
+ * flattened heads are cut into chunks of chunk_heads and pipelined: the
+ * host-to-device copies of chunk i+1 and the device-to-host copies of chunk
+ * i-1 overlap the path on chunk i (two library-owned copy streams per device,
+ * created on first use and kept until exit; one cudaMemcpyAsync per tensor
+ * and chunk).  The results equal vsa_path_fwd's on all heads at once, bit for
+ * bit.  Host buffers should be page-locked (cudaHostAlloc) for the copies to
+ * overlap; pageable buffers work but serialise.
+ *   workspace : DEVICE, 256-byte aligned, at least
+ *               vsa_path_host_workspace_bytes(shape, params, chunk_heads).
+ * The call returns once everything is enqueued; the work is complete when
+ * ``stream`` is (synchronise it before reading o_host / lse_host).  Calls
+ * from several host threads are enqueued one at a time. */
+VSA_API size_t vsa_path_host_workspace_bytes(const vsa_shape *shape, const vsa_path_params *params,
+                                             int chunk_heads);
+
+VSA_API vsa_status vsa_path_fwd_host(const void *q_host, const void *k_host, const void *v_host,
+                                     const vsa_shape *shape, const vsa_path_params *params, int chunk_heads,
+                                     void *o_host, float *lse_host, void *workspace, size_t workspace_bytes,
+                                     void *stream);
 
 /* ---------------------------------------------------------------------------
  * Cluster-permuted layout ([HVA] §4.1 Eq. (5) 3D local-window clustering;

@@ -76,8 +76,8 @@ def test_host_validation_rejects_bad_arguments(L):
     # n_valid > n_pad
     bad = vsa.Shape(1, 2, 300, 256, 64)
     assert L.vsa_lse_merge(fake, fake, fake, fake, ctypes.byref(bad), fake, 0, fake, null) == 1
-    # too many key blocks for selection
-    big = vsa.Shape(1, 1, 200_000, 204_800, 128)
+    # too many key blocks for selection (more than 4096)
+    big = vsa.Shape(1, 1, 520_000, 4097 * 128, 128)
     params = vsa.SelectParams(1, 0.9, 0, 0, 0)
     assert L.vsa_select_blocks(fake, fake, ctypes.byref(big), 128, 128, 0.1, ctypes.byref(params), fake, fake,
                                null, null) == 2
@@ -92,3 +92,36 @@ def test_micro_workspace_query_is_host_only(L):
     assert n6 >= 6 * per_head_keys and nall >= 24 * per_head_keys and nall > n6
     assert vsa.select_micro_workspace_bytes(shape, 1, 0, 0.0, None, 16) == 0      # topk 0 is invalid
     assert vsa.select_micro_workspace_bytes(shape, 2, 0, 1.5, None, 16) == 0      # percentile out of (0, 1)
+
+
+def test_path_entry_points_validate_on_the_host(L):
+    """vsa_path_*: the workspace queries are host-only, grow with the Micro
+    repair and with the chunk size, and bad arguments are refused before
+    anything is enqueued."""
+    shape = vsa.Shape(1, 24, 118_800, 118_912, 128)
+    cfg = vsa.PathConfig(n_valid=118_800, fixed_k=186, micro_mode=2, micro_percentile=0.99,
+                         micro_heads=[1 if h in (0, 5) else 0 for h in range(24)])
+    p_micro, keep = vsa.path_params(cfg)
+    p_plain, _ = vsa.path_params(vsa.PathConfig(n_valid=118_800, fixed_k=186))
+    n_micro = vsa.path_workspace_bytes(shape, p_micro)
+    n_plain = vsa.path_workspace_bytes(shape, p_plain)
+    o_macro = 24 * 118_912 * 128 * 4
+    assert n_plain > 0 and n_micro > n_plain + o_macro
+    h1 = vsa.path_host_workspace_bytes(shape, p_micro, 1)
+    h2 = vsa.path_host_workspace_bytes(shape, p_micro, 2)
+    assert 0 < h1 < h2 < n_micro
+    assert vsa.path_host_workspace_bytes(shape, p_micro, 0) == 0
+    bad = vsa.PathParams.from_buffer_copy(p_plain)
+    bad.bq = 96
+    assert vsa.path_workspace_bytes(shape, bad) == 0
+    fake, null = ctypes.c_void_p(256), None
+    assert L.vsa_path_fwd(fake, fake, fake, ctypes.byref(shape), ctypes.byref(bad), fake, fake, fake, 1 << 40,
+                          null) == 1
+    # workspace too small, misaligned workspace, null output
+    assert L.vsa_path_fwd(fake, fake, fake, ctypes.byref(shape), ctypes.byref(p_plain), fake, fake, fake,
+                          n_plain - 1, null) == 1
+    assert L.vsa_path_fwd(fake, fake, fake, ctypes.byref(shape), ctypes.byref(p_plain), fake, fake,
+                          ctypes.c_void_p(272), n_plain, null) == 1
+    assert L.vsa_path_fwd_host(fake, fake, fake, ctypes.byref(shape), ctypes.byref(p_plain), 2, null, fake, fake,
+                               1 << 40, null) == 1
+    del keep

@@ -593,3 +593,45 @@ def test_forward_host_matches_device_path(name, heads, chunk):
     assert torch.equal(torch.isinf(hl), torch.isinf(l_ref))
     fin = torch.isfinite(l_ref)
     assert torch.equal(hl[fin], l_ref[fin])
+
+
+def test_status_words_bound_to_streams_keep_callers_apart():
+    """Two callers on two streams, each with its own status word in its own
+    memory: a bad list on one stream latches BAD_INDEX in that caller's word
+    only, a wait that times out on it aborts nothing on the other, and
+    unbinding returns the stream to the process-wide word."""
+    B, H, n_pad, d = 1, 1, 256, 128
+    q = torch.zeros(B, H, n_pad, d, device="cuda", dtype=torch.bfloat16)
+    bad_counts = torch.tensor([[[2, 1]]], dtype=torch.int32, device="cuda")
+    bad_idx = torch.tensor([[[[1, 0], [5, 0]]]], dtype=torch.int32, device="cuda")
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    w1 = torch.full((2,), 77, dtype=torch.int32, device="cuda")
+    w2 = torch.full((2,), 77, dtype=torch.int32, device="cuda")
+    vsa.bind_status_word(w1, s1)
+    vsa.bind_status_word(w2, s2)
+    try:
+        o1 = torch.empty(B, H, n_pad, d, device="cuda", dtype=torch.bfloat16)
+        l1 = torch.empty(B, H, n_pad, device="cuda")
+        with torch.cuda.stream(s1):
+            vsa.block_sparse_fwd(q, q, q, vsa.Shape(B, H, n_pad, n_pad, d), 128, 128, bad_counts, bad_idx, 2, 0.1,
+                                 o1, l1, stream=s1)
+            vsa.selftest_wait_timeout(20_000_000, stream=s1)      # 20 ms
+        with torch.cuda.stream(s2):
+            test_attention_tiny_all_rows()
+        s1.synchronize()
+        s2.synchronize()
+        assert int(w1[0]) == 5 and int(w1[1]) == 1        # first error kept; the timeout raised its flag
+        assert int(w2[0]) == 0 and int(w2[1]) == 0
+        assert vsa.read_device_status(s2) == 0
+        assert vsa.read_device_status(s1) == 5
+        assert int(w1[0]) == 0 and int(w1[1]) == 0        # reading cleared the caller's word
+        assert vsa.read_device_status() == 0              # the process-wide word saw nothing
+    finally:
+        vsa.bind_status_word(None, s1)
+        vsa.bind_status_word(None, s2)
+    # unbound again: errors land in the process-wide word
+    with torch.cuda.stream(s1):
+        vsa.block_sparse_fwd(q, q, q, vsa.Shape(B, H, n_pad, n_pad, d), 128, 128, bad_counts, bad_idx, 2, 0.1, o1, l1,
+                             stream=s1)
+    assert vsa.read_device_status(s1) == 5
+    assert int(w1[0]) == 0
