@@ -7,9 +7,8 @@
 // abstract: rotating global anchor columns.
 //
 // One CTA owns 16 query-block rows of one (batch, head).  It stages the 16
-// pooled query rows in shared memory; each thread streams whole pooled key
-// rows from global memory and computes their logits against all 16 rows with
-// fp32 FFMA (no TF32, so the ranking
+// pooled query rows and 32-key chunks of the pooled keys in shared memory and
+// computes the 16 x n_k logits with fp32 FFMA (no TF32, so the ranking
 // matches an fp64 evaluation wherever two blocks differ by more than fp32
 // rounding).  Each warp then ranks two rows: the n_k log-weights
 // w = S + ln s_j, packed with the key index into 64-bit keys, are bitonic-
@@ -28,6 +27,7 @@ namespace vsa {
 
 constexpr int kSelRows = 16;
 constexpr int kSelThreads = 256;
+constexpr int kSelChunk = 64;
 
 struct SelectArgs {
   const float *q_pool;  // [BH, n_q, d]
@@ -166,8 +166,9 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
   constexpr int DP = D + 4;  // padded row stride (floats)
   extern __shared__ __align__(16) float sel_smem[];
   float *qs = sel_smem;                       // [kSelRows][DP]
+  float *ks = qs + kSelRows * DP;             // [kSelChunk][DP]
   const int nkp = NR * 32;
-  float *S = qs + kSelRows * DP;              // [kSelRows][nkp]
+  float *S = ks + kSelChunk * DP;             // [kSelRows][nkp]
   uint32_t *bitmap = reinterpret_cast<uint32_t *>(S + kSelRows * nkp);  // [8 warps][32]
 
   const int bh = blockIdx.y;
@@ -183,33 +184,39 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     *reinterpret_cast<float4 *>(qs + r * DP + c4 * 4) = v;
   }
 
-  // ---- logits: thread t -> keys t, t + 256, ... against all 16 rows.  The
-  // key's d values stream from global memory (L1 keeps its lines for the
-  // next steps) and every query value comes as a shared-memory broadcast, so
-  // each 16-byte shared load feeds four FMAs per row; the sum over d runs in
-  // ascending order, one rounding per FMA.
-  __syncthreads();
-  for (int j = t; j < nkp; j += kSelThreads) {
-    float acc[kSelRows];
-#pragma unroll
-    for (int r = 0; r < kSelRows; ++r) acc[r] = 0.f;
-    if (j < a.n_k) {
-      const float4 *k4 = reinterpret_cast<const float4 *>(kp + (size_t)j * D);
-#pragma unroll 4
-      for (int c = 0; c < D / 4; ++c) {
-        const float4 y = __ldg(k4 + c);
-#pragma unroll
-        for (int r = 0; r < kSelRows; ++r) {
-          const float4 x = *reinterpret_cast<const float4 *>(qs + r * DP + 4 * c);
-          acc[r] = fmaf(x.x, y.x, acc[r]);
-          acc[r] = fmaf(x.y, y.y, acc[r]);
-          acc[r] = fmaf(x.z, y.z, acc[r]);
-          acc[r] = fmaf(x.w, y.w, acc[r]);
-        }
-      }
+  // ---- logits: warp w -> rows 2w, 2w+1; lane -> keys lane, lane + 32 of the chunk
+  const int r0 = 2 * warp;
+  for (int k0 = 0; k0 < a.n_k; k0 += kSelChunk) {
+    __syncthreads();
+    for (int i = t; i < kSelChunk * (D / 4); i += kSelThreads) {
+      const int r = i / (D / 4), c4 = i % (D / 4);
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (k0 + r < a.n_k) v = __ldg(reinterpret_cast<const float4 *>(kp + (size_t)(k0 + r) * D) + c4);
+      *reinterpret_cast<float4 *>(ks + r * DP + c4 * 4) = v;
     }
-#pragma unroll
-    for (int r = 0; r < kSelRows; ++r) S[r * nkp + j] = acc[r] * a.scale;
+    __syncthreads();
+    float s00 = 0.f, s01 = 0.f, s10 = 0.f, s11 = 0.f;
+    const float *q0 = qs + r0 * DP, *q1 = qs + (r0 + 1) * DP;
+    const float *ka = ks + lane * DP, *kb = ks + (lane + 32) * DP;
+#pragma unroll 8
+    for (int c = 0; c < D; c += 4) {
+      const float4 x0 = *reinterpret_cast<const float4 *>(q0 + c);
+      const float4 x1 = *reinterpret_cast<const float4 *>(q1 + c);
+      const float4 ya = *reinterpret_cast<const float4 *>(ka + c);
+      const float4 yb = *reinterpret_cast<const float4 *>(kb + c);
+      s00 = fmaf(x0.x, ya.x, s00); s00 = fmaf(x0.y, ya.y, s00); s00 = fmaf(x0.z, ya.z, s00); s00 = fmaf(x0.w, ya.w, s00);
+      s01 = fmaf(x0.x, yb.x, s01); s01 = fmaf(x0.y, yb.y, s01); s01 = fmaf(x0.z, yb.z, s01); s01 = fmaf(x0.w, yb.w, s01);
+      s10 = fmaf(x1.x, ya.x, s10); s10 = fmaf(x1.y, ya.y, s10); s10 = fmaf(x1.z, ya.z, s10); s10 = fmaf(x1.w, ya.w, s10);
+      s11 = fmaf(x1.x, yb.x, s11); s11 = fmaf(x1.y, yb.y, s11); s11 = fmaf(x1.z, yb.z, s11); s11 = fmaf(x1.w, yb.w, s11);
+    }
+    if (k0 + lane < nkp) {
+      S[r0 * nkp + k0 + lane] = s00 * a.scale;
+      S[(r0 + 1) * nkp + k0 + lane] = s10 * a.scale;
+    }
+    if (k0 + lane + 32 < nkp) {
+      S[r0 * nkp + k0 + lane + 32] = s01 * a.scale;
+      S[(r0 + 1) * nkp + k0 + lane + 32] = s11 * a.scale;
+    }
   }
   __syncthreads();
 

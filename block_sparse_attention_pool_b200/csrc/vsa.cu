@@ -524,7 +524,7 @@ vsa_status launch_select(const vsa::SelectArgs &a, int d, int BH, bool by_rank, 
   int nkp = 32;
   while (nkp < n_k) nkp <<= 1;
   const int dp = d + 4;
-  const size_t smem = (size_t)vsa::kSelRows * dp * 4 + (size_t)vsa::kSelRows * nkp * 4 + 8 * 32 * 4;
+  const size_t smem = (size_t)(vsa::kSelRows + vsa::kSelChunk) * dp * 4 + (size_t)vsa::kSelRows * nkp * 4 + 8 * 32 * 4;
   dim3 grid((n_q + vsa::kSelRows - 1) / vsa::kSelRows, BH);
 #define VSA_SEL_CASE(DD, NR)                                                                                  \
   {                                                                                                           \
