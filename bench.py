@@ -316,7 +316,10 @@ def run_gpu(args, rank, world, local_rank):
     pk = peaks()
     macro_avg_ms = statistics.mean(macro_ms)
     achieved = fl_macro / (macro_avg_ms * 1e-3) / 1e12
-    peak = pk["bf16_sustained"]
+    # the burst figure: the step runs the Macro pass at clocks near the burst
+    # measurement's (the sustained figure was taken power-capped at ~1.34 GHz);
+    # the sustained fraction is reported beside it
+    peak = pk["bf16"]
     line = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -342,7 +345,7 @@ def run_gpu(args, rank, world, local_rank):
         },
         "pct_of_bf16_peak": round(100.0 * flops_step / (ms_step * 1e-3) / 1e12 / peak, 2),
         "peak_tflops": peak,
-        "peak_source": f"{pk['source']} bf16 sustained",
+        "peak_source": f"{pk['source']} bf16 burst",
         "dense_ms": round(dense_ms, 3),
         "dense_tflops": round(dense_flops / (dense_ms * 1e-3) / 1e12, 2),
         "speedup_vs_dense": round(dense_ms / ms_step, 3),
@@ -357,6 +360,8 @@ def run_gpu(args, rank, world, local_rank):
             "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
             "traffic": macro_traffic(args.workload),
+            "peak_source": f"{pk['source']} bf16 burst (cuBLAS 8192^3)",
+            "frac_of_sustained": round(achieved / pk["bf16_sustained"], 4),
         },
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 3),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -475,8 +480,9 @@ def run_sweep(args):
         tf = flops / (ms * 1e-3) / 1e12
         print(json.dumps({"sweep_point": w.name, "blocks": f"{w.bq}x{w.bk}", "kept_fraction": frac,
                           "k": w.fixed_k, "attn_ms": round(ms, 3), "effective_tflops": round(tf, 2),
-                          "frac_of_bf16_peak": round(tf / pk["bf16_sustained"], 4),
-                          "peak": f"{pk['bf16_sustained']} TFLOP/s ({pk['source']} bf16 sustained)",
+                          "frac_of_bf16_peak": round(tf / pk["bf16"], 4),
+                          "peak": f"{pk['bf16']} TFLOP/s ({pk['source']} bf16 burst)",
+                          "frac_of_sustained": round(tf / pk["bf16_sustained"], 4),
                           "speedup_vs_dense_same_blocks": round(dense_ms[(w.bq, w.bk)] / ms, 3)}), flush=True)
         del run
 

@@ -85,6 +85,12 @@ struct AttnArgs {
   int n_bh;              // B * H
   unsigned long long timeout_ns;
   int *status;           // the launch's status word
+  // Pair boxes (16-key segments, d = 128): a segment's K / V rows arrive as one
+  // 4 KB box of the 5-D maps xm.k[0] / xm.v[0], laid out [row group of 8][column
+  // chunk][8 rows][128 B]; a segment that holds rows in [n_valid8, n_valid)
+  // comes as four 8-row boxes of xm.k[1] / xm.v[1] into the same places.
+  int pair_boxes;
+  int n_valid8;          // n_valid rounded down to a multiple of 8
   // Cluster-group mode (tile_list non-null; list_rows 128, seg_keys 16): tile T of
   // head bh uses list row tile_list[bh][T] (-1: no such tile, the CTA leaves at
   // once), whose entries are key clusters j < n_kc; cluster j is the K/V rows
@@ -618,14 +624,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t cp_off = cp_chunk * kChunkBytes + cp_seg * a.seg_keys * 128;
         const CUtensorMap *map_k = cp_box == 4 ? &xm.k[1] : (cp_box == 2 ? &xm.k[0] : &tm_k);
         const CUtensorMap *map_v = cp_box == 4 ? &xm.v[1] : (cp_box == 2 ? &xm.v[0] : &tm_v);
-        if (cp_lane && cp_box > 0)
+        // pair boxes: lane i < 8 moves segment i (its own my_start) whole
+        const bool pair_lane = a.pair_boxes && lane < 8;
+        const bool pair_whole = my_start + 16 <= a.n_valid8 || my_start >= a.n_valid;
+        if (pair_lane) {
+          uint8_t *dst = sK + slot * L::kKVBytes + lane * 4096;
+          if (pair_whole) {
+            tma_load_5d(dst, &xm.k[0], &ctl->k_full[slot], 0, 0, 0, my_start >> 3, bh);
+          } else {
+            for (int q = 0; q < 4; ++q)
+              tma_load_3d(dst + (q >> 1) * 2048 + (q & 1) * 1024, &xm.k[1], &ctl->k_full[slot], (q & 1) * 64,
+                          my_start + 8 * (q >> 1), bh);
+          }
+        } else if (!a.pair_boxes && cp_lane && cp_box > 0) {
           tma_load_3d(sK + slot * L::kKVBytes + cp_off, map_k, &ctl->k_full[slot], cp_chunk * 64, cp_row, bh);
+        }
         if (s >= 2) ok = mbar_wait_warp(&ctl->v_empty[slot], use_par, abort, a.timeout_ns, lane);
         if (!ok) break;
         if (lane == 0) mbar_arrive_expect_tx(&ctl->v_full[slot], L::kKVBytes);
         __syncwarp();
-        if (cp_lane && cp_box > 0)
+        if (pair_lane) {
+          uint8_t *dst = sV + slot * L::kKVBytes + lane * 4096;
+          if (pair_whole) {
+            tma_load_5d(dst, &xm.v[0], &ctl->v_full[slot], 0, 0, 0, my_start >> 3, bh);
+          } else {
+            for (int q = 0; q < 4; ++q)
+              tma_load_3d(dst + (q >> 1) * 2048 + (q & 1) * 1024, &xm.v[1], &ctl->v_full[slot], (q & 1) * 64,
+                          my_start + 8 * (q >> 1), bh);
+          }
+        } else if (!a.pair_boxes && cp_lane && cp_box > 0) {
           tma_load_3d(sV + slot * L::kKVBytes + cp_off, map_v, &ctl->v_full[slot], cp_chunk * 64, cp_row, bh);
+        }
         issued = s + 1;
         __syncwarp();
       }
@@ -646,9 +675,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       constexpr uint32_t kIdS = idesc_bf16_f32(kTileM, kStageKeys, false);
       constexpr uint32_t kIdO = idesc_bf16_f32(kTileM, D, true);
       // descriptor bases; K steps and ring slots only add to the start address field
+      // pair boxes: K / V 8-row groups 2048 bytes apart, the two column chunks
+      // of a group 1024 bytes apart
+      const uint32_t kv_chunk = a.pair_boxes ? 1024u : static_cast<uint32_t>(kChunkBytes);
+      const uint32_t kv_group = a.pair_boxes ? 2048u : 1024u;
       const uint64_t dQ = smem_desc_sw128(smem_addr(sQ), 16, 1024);
-      const uint64_t dK0 = smem_desc_sw128(smem_addr(sK), 16, 1024);
-      const uint64_t dV0 = smem_desc_sw128(smem_addr(sV), kChunkBytes, 1024);
+      const uint64_t dK0 = smem_desc_sw128(smem_addr(sK), 16, kv_group);
+      const uint64_t dV0 = smem_desc_sw128(smem_addr(sV), kv_chunk, kv_group);
       constexpr uint64_t kSlotStep = L::kKVBytes >> 4;
       const uint32_t leader = elect_one();
       bool ok = mbar_wait_uni(&ctl->q_full, 0, abort, a.timeout_ns, lane);
@@ -662,7 +695,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kStageKeys / 16; ++kk) {
           // P (bf16 pairs) sits in the first 64 columns of the stage's S buffer
-          umma_bf16_ts_one(to, ts + kk * 8, dv + (uint64_t)(kk * 16 * 128 / 16), kIdO,
+          umma_bf16_ts_one(to, ts + kk * 8, dv + (uint64_t)(kk * 2 * kv_group / 16), kIdO,
                            (t >= 2 || kk > 0) ? 1u : 0u, leader);
         }
         umma_commit_one(&ctl->v_empty[t & 1], leader);
@@ -678,8 +711,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t ts = slot ? tS[1] : tS[0];
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
-          umma_bf16_ss_one(ts, dQ + off, dk + off, kIdS, kk > 0 ? 1u : 0u, leader);
+          const uint64_t offq = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+          const uint64_t offk = (uint64_t)(((kk >> 2) * kv_chunk + (kk & 3) * 32) >> 4);
+          umma_bf16_ss_one(ts, dQ + offq, dk + offk, kIdS, kk > 0 ? 1u : 0u, leader);
         }
         umma_commit_one(&ctl->k_empty[slot], leader);
         umma_commit_one(&ctl->s_full[slot], leader);

@@ -148,11 +148,16 @@ vsa_status path_run(const void *q, const void *k, const void *v, const vsa_shape
 
 // ---- host-buffer pipeline ---------------------------------------------------
 
+// Workspace slots of the host-buffer pipeline: chunk i uses slot i % 3, so the
+// copies in of chunk i+1 and out of chunk i-1 never wait for the compute of
+// the chunk next to them.
+constexpr int kHostSlots = 3;
+
 // Copy streams and events of the host-buffer pipeline, created once per
 // device and kept for the life of the process (no device memory).
 struct HostPipe {
   cudaStream_t in = nullptr, out = nullptr;
-  cudaEvent_t in_done[2] = {}, comp_done[2] = {}, out_done[2] = {};
+  cudaEvent_t in_done[kHostSlots] = {}, comp_done[kHostSlots] = {}, out_done[kHostSlots] = {};
   bool ready = false;
 };
 
@@ -169,7 +174,7 @@ vsa_status host_pipe(HostPipe **out) {
     if (cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) != cudaSuccess ||
         cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) != cudaSuccess)
       return VSA_ERR_CUDA;
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < kHostSlots; ++i)
       if (cudaEventCreateWithFlags(&hp.in_done[i], cudaEventDisableTiming) != cudaSuccess ||
           cudaEventCreateWithFlags(&hp.comp_done[i], cudaEventDisableTiming) != cudaSuccess ||
           cudaEventCreateWithFlags(&hp.out_done[i], cudaEventDisableTiming) != cudaSuccess)
@@ -180,7 +185,7 @@ vsa_status host_pipe(HostPipe **out) {
   return VSA_OK;
 }
 
-// Device workspace of the host pipeline: two slots of chunk inputs and
+// Device workspace of the host pipeline: kHostSlots slots of chunk inputs and
 // outputs, then the path workspace of one chunk.
 struct HostLayout {
   size_t in_bytes, o_bytes, lse_bytes, slot_bytes, path_off, total;
@@ -193,7 +198,7 @@ HostLayout host_layout(const vsa_shape *s, const vsa_path_params *p, int chunk) 
   L.o_bytes = align256(rows * s->d * (p->o_fp32 ? 4 : 2));
   L.lse_bytes = align256(rows * 4);
   L.slot_bytes = 3 * L.in_bytes + L.o_bytes + L.lse_bytes;
-  L.path_off = 2 * L.slot_bytes;
+  L.path_off = kHostSlots * L.slot_bytes;
   // size the chunk's path workspace with every head of the chunk repaired
   vsa_shape cs = *s;
   cs.B = 1;
@@ -259,20 +264,20 @@ vsa_status vsa_path_fwd_host(const void *q_host, const void *k_host, const void 
   int i = 0;
   for (int c0 = 0; c0 < BH; c0 += chunk, ++i) {
     const int n = std::min(chunk, BH - c0);
-    const int slot = i & 1;
+    const int slot = i % kHostSlots;
     char *sq = ws + slot * L.slot_bytes;
     char *sk = sq + L.in_bytes, *sv = sk + L.in_bytes, *so = sv + L.in_bytes, *sl = so + L.o_bytes;
-    // inputs of chunk i, once chunk i-2 (same slot) has been computed
-    if (i >= 2 && cudaStreamWaitEvent(hp->in, hp->comp_done[slot], 0) != cudaSuccess) return VSA_ERR_CUDA;
+    // inputs of chunk i, once the chunk that used this slot before has been computed
+    if (i >= kHostSlots && cudaStreamWaitEvent(hp->in, hp->comp_done[slot], 0) != cudaSuccess) return VSA_ERR_CUDA;
     const struct { const void *src; char *dst; } ins[3] = {{q_host, sq}, {k_host, sk}, {v_host, sv}};
     for (const auto &c : ins)
       if (cudaMemcpyAsync(c.dst, static_cast<const char *>(c.src) + (size_t)c0 * row_in, (size_t)n * row_in,
                           cudaMemcpyHostToDevice, hp->in) != cudaSuccess)
         return VSA_ERR_CUDA;
     if (cudaEventRecord(hp->in_done[slot], hp->in) != cudaSuccess) return VSA_ERR_CUDA;
-    // the path on chunk i, once its inputs are in and chunk i-2's outputs are out
+    // the path on chunk i, once its inputs are in and the slot's earlier outputs are out
     if (cudaStreamWaitEvent(comp, hp->in_done[slot], 0) != cudaSuccess) return VSA_ERR_CUDA;
-    if (i >= 2 && cudaStreamWaitEvent(comp, hp->out_done[slot], 0) != cudaSuccess) return VSA_ERR_CUDA;
+    if (i >= kHostSlots && cudaStreamWaitEvent(comp, hp->out_done[slot], 0) != cudaSuccess) return VSA_ERR_CUDA;
     vsa_shape cs = *shape;
     cs.B = 1;
     cs.H = n;
@@ -296,8 +301,8 @@ vsa_status vsa_path_fwd_host(const void *q_host, const void *k_host, const void 
     if (cudaEventRecord(hp->out_done[slot], hp->out) != cudaSuccess) return VSA_ERR_CUDA;
   }
   // the caller's stream completes with the last copy out
-  if (cudaEventRecord(hp->out_done[(i - 1) & 1], hp->out) != cudaSuccess ||
-      cudaStreamWaitEvent(comp, hp->out_done[(i - 1) & 1], 0) != cudaSuccess)
+  if (cudaEventRecord(hp->out_done[(i - 1) % kHostSlots], hp->out) != cudaSuccess ||
+      cudaStreamWaitEvent(comp, hp->out_done[(i - 1) % kHostSlots], 0) != cudaSuccess)
     return VSA_ERR_CUDA;
   return VSA_OK;
 }

@@ -161,6 +161,13 @@ __device__ __forceinline__ int emit_bitmap_list(const uint32_t *bits, int n, int
   return total;
 }
 
+// Dynamic shared memory of select_blocks_kernel: the query rows and a key
+// chunk (rows padded to d + 4 floats), the logits of the CTA's rows (nkp
+// columns), one 32-word bitmap per warp.  The host sizes the launch with this.
+__host__ __device__ constexpr size_t select_smem_bytes(int d, int nkp) {
+  return (size_t)(kSelRows + kSelChunk) * (d + 4) * 4 + (size_t)kSelRows * nkp * 4 + 8 * 32 * 4;
+}
+
 template <int D, int NR, bool BY_RANK>
 __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a) {
   constexpr int DP = D + 4;  // padded row stride (floats)

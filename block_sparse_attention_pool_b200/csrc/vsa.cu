@@ -123,6 +123,24 @@ bool make_map(CUtensorMap *map, const void *base, const vsa_shape *s, int box_ro
   return r == CUDA_SUCCESS;
 }
 
+// [BH][n_pad][128] bf16 as a 5-D tensor (64 columns, 8 rows, 2 column chunks,
+// n_valid / 8 row groups, BH): a box of (64, 8, 2, 2, 1) moves 16 whole rows,
+// written to shared memory as [row group][chunk][8 rows][128 B] (128B
+// swizzle).  Only whole groups of valid rows lie inside the tensor: rows of a
+// last partial group must come through the 3-D map instead.
+bool make_pair_map(CUtensorMap *map, const void *base, const vsa_shape *s) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || s->d != 128 || s->n_valid < 8) return false;
+  cuuint64_t dims[5] = {64, 8, 2, (cuuint64_t)(s->n_valid / 8), (cuuint64_t)s->B * s->H};
+  cuuint64_t strides[4] = {(cuuint64_t)s->d * 2, 128, (cuuint64_t)8 * s->d * 2, (cuuint64_t)s->n_pad * s->d * 2};
+  cuuint32_t box[5] = {64, 8, 2, 2, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // [BH][rows][d] bf16, all rows inside the tensor.
 bool make_map_rows(CUtensorMap *map, const void *base, int rows, int d, int BH, int box_rows) {
   EncodeTiledFn fn = encode_fn();
@@ -201,10 +219,19 @@ vsa_status launch_attn(const void *q, const void *k, const void *v, const vsa_sh
   if (!make_map(&mq, q, s, vsa::kTileM) || !make_map(&mk, k, s, a.seg_keys) || !make_map(&mv, v, s, a.seg_keys))
     return VSA_ERR_CUDA;
   dim3 grid(s->n_pad / vsa::kTileM, n_heads);
-  vsa::GroupMaps xm;  // unused outside cluster-group mode
+  vsa::GroupMaps xm;  // cluster-group mode's taller boxes, or the pair boxes of 16-key segments
   xm.k[0] = xm.k[1] = mk;
   xm.v[0] = xm.v[1] = mv;
-  vsa::attn_fwd_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, xm, a);
+  AttnArgs ap = a;
+  ap.pair_boxes = 0;
+  if (D == 128 && a.seg_keys == 16 && s->n_valid >= 8) {
+    if (!make_pair_map(&xm.k[0], k, s) || !make_pair_map(&xm.v[0], v, s) || !make_map(&xm.k[1], k, s, 8) ||
+        !make_map(&xm.v[1], v, s, 8))
+      return VSA_ERR_CUDA;
+    ap.pair_boxes = 1;
+    ap.n_valid8 = s->n_valid / 8 * 8;
+  }
+  vsa::attn_fwd_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, xm, ap);
   return launch_status();
 }
 
@@ -523,8 +550,7 @@ vsa_status launch_select(const vsa::SelectArgs &a, int d, int BH, bool by_rank, 
   }
   int nkp = 32;
   while (nkp < n_k) nkp <<= 1;
-  const int dp = d + 4;
-  const size_t smem = (size_t)(vsa::kSelRows + vsa::kSelChunk) * dp * 4 + (size_t)vsa::kSelRows * nkp * 4 + 8 * 32 * 4;
+  const size_t smem = vsa::select_smem_bytes(d, nkp);
   dim3 grid((n_q + vsa::kSelRows - 1) / vsa::kSelRows, BH);
 #define VSA_SEL_CASE(DD, NR)                                                                                  \
   {                                                                                                           \
