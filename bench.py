@@ -48,9 +48,9 @@ METRIC = "block-sparse attn ms & effective TFLOP/s (% bf16 peak), speedup vs den
 # valid only while the kernel sources hash to the value it was taken with.
 MACRO_TRAFFIC = {
     "sources": ["csrc/attn_fwd_dual.cuh", "csrc/attn_fwd.cuh", "csrc/common.cuh"],
-    "sha256_16": "22da10804fd7e17b",
+    "sha256_16": "121162c7a3a5d7ca",
     "workload": "hunyuan",
-    "bytes_per_step": (2435052800 + 548006400) + (846065408 + 342682112),
+    "bytes_per_step": (2218286080 + 545540608) + (791236096 + 342650880),
 }
 
 
@@ -306,6 +306,38 @@ def run_gpu(args, rank, world, local_rank):
     dense_flops = 4.0 * w.bq * w.bk * w.d * float(dense.buf["counts"].sum().item())
     del dense
 
+    # the sweep's 85%-sparsity points on the same tensors (selection, then the
+    # attention pass alone, CUDA events), so that both block shapes' efficiency
+    # at high sparsity sits in the default line
+    sweep85 = {}
+    if args.workload == "hunyuan":
+        for frac, sw in sweep_points():
+            if frac != 0.15:
+                continue
+            scfg = vsa.PathConfig(n_valid=sw.n_valid, bq=sw.bq, bk=sw.bk, scale=sw.scale, fixed_k=sw.fixed_k)
+            srun = vsa.SparseVideoAttention(scfg)
+            srun(dq, dk, dv)
+            sb = srun.buf
+            sshape = vsa.Shape(sw.B, sw.H, sw.n_valid, sw.n_pad, sw.d)
+            sfwd = lambda: vsa.block_sparse_fwd(dq, dk, dv, sshape, sw.bq, sw.bk, sb["counts"], sb["idx"],
+                                                sw.n_pad // sw.bk, sw.scale, sb["o"], sb["lse"])
+            sfwd()
+            torch.cuda.synchronize(dev)
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            for _ in range(3):
+                sfwd()
+            s1.record(stream)
+            torch.cuda.synchronize(dev)
+            sms = s0.elapsed_time(s1) / 3
+            stf = macro_flops(sb["counts"], sw) / (sms * 1e-3) / 1e12
+            sweep85[f"{sw.bq}x{sw.bk}"] = {"kept_fraction": frac, "k": sw.fixed_k, "attn_ms": round(sms, 3),
+                                           "effective_tflops": round(stf, 2)}
+            del srun
+        st = vsa.read_device_status(stream)
+        if st != 0:
+            raise RuntimeError(f"device status after the sweep points: {vsa.status_string(st)}")
+
     # job time = slowest rank; job work = all ranks' kept-tile FLOPs
     ms_total, e2e_ms = max_over_ranks([ms_total, e2e_ms], dev, world)
     (job_flops,) = sum_over_ranks([fl_macro + fl_micro], dev, world)
@@ -351,6 +383,8 @@ def run_gpu(args, rank, world, local_rank):
         "speedup_vs_dense": round(dense_ms / ms_step, 3),
         "macro_kernel_ms": round(macro_avg_ms, 4),
         "stages_ms": stages,
+        "sweep_85pct_sparsity": {key: dict(val, frac_of_bf16_peak=round(val["effective_tflops"] / pk["bf16"], 4))
+                                 for key, val in sweep85.items()},
         "roofline": {
             "kernel": ("attn_fwd_dual_kernel<%d> (Macro pass" if (w.bq == 128 and w.bk == 128) else
                        "attn_fwd_kernel<%d> (Macro pass") % w.d + f", {n_macro} launch(es) per step timed together)",

@@ -311,21 +311,6 @@ __device__ __forceinline__ void tma_load_3d_hint(void *dst, const CUtensorMap *m
       : "memory");
 }
 
-// Fetch one box of a 5-D tensor map into L2 (fire and forget).
-__device__ __forceinline__ void tma_prefetch_l2_5d(const CUtensorMap *map, int c0, int c1, int c2, int c3, int c4) {
-  asm volatile("cp.async.bulk.prefetch.tensor.5d.L2.global.tile [%0, {%1, %2, %3, %4, %5}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
-               : "memory");
-}
-
-// Fetch a byte range of global memory into L2 ahead of its use (fire and
-// forget: nothing waits for it).  Address and size multiples of 16.
-__device__ __forceinline__ void l2_prefetch_bulk(const void *p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
-               : "memory");
-}
-
 // L2 cache policies: lines read once (evict first) and lines that other CTAs
 // read again (evict last).
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
