@@ -33,6 +33,7 @@ constexpr int kHistBins = 2048;
 
 struct MicroWs {
   int32_t *slot_of_bh;  // [B*H] slot or -1
+  int32_t *bh_of_slot;  // [slots] the (batch, head) of each slot
   uint32_t *bitmap;     // [slots][n_q][bitmap_words] kept key blocks of each Macro row
   uint32_t *keys;       // [slots][n_r][n_t]
   uint32_t *hist;       // [slots][3][kHistBins]
@@ -44,13 +45,13 @@ struct MicroWs {
 
 constexpr int kMicroMaxKeyBlocks = 4096;
 
-// Dense kept-block bitmap of every Macro row of the enabled heads.
+// Dense kept-block bitmap of every Macro row of the enabled heads (grid: rows x slots).
 __global__ void micro_bitmap_kernel(const int32_t *__restrict__ counts, const int32_t *__restrict__ idx, int n_q,
                                     int n_k, int BH, MicroWs ws) {
   const int row = blockIdx.x;  // Macro row within the head
-  const int bh = blockIdx.y;
-  const int slot = ws.slot_of_bh[bh];
-  if (slot < 0 || row >= n_q) return;
+  const int slot = blockIdx.y;
+  const int bh = ws.bh_of_slot[slot];
+  if (row >= n_q) return;
   __shared__ uint32_t bits[kMicroMaxKeyBlocks / 32];
   const int W = ws.bitmap_words;
   for (int w = threadIdx.x; w < W; w += blockDim.x) bits[w] = 0u;
@@ -75,9 +76,8 @@ struct ScoreArgs {
 
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads) micro_score_kernel(ScoreArgs a, MicroWs ws) {
-  const int bh = blockIdx.z;
-  const int slot = ws.slot_of_bh[bh];
-  if (slot < 0) return;
+  const int slot = blockIdx.z;  // enabled heads only
+  const int bh = ws.bh_of_slot[slot];
   const int r0 = blockIdx.y * kScoreBM;
   const int t0 = blockIdx.x * kScoreBN;
   __shared__ float As[kScoreBK][kScoreBM + 4];
@@ -174,9 +174,16 @@ __global__ void __launch_bounds__(kScoreThreads) micro_score_kernel(ScoreArgs a,
       }
       const uint32_t key = cand ? float_key(acc[i][j] * a.scale) : 0u;
       out[j] = key;
-      if (cand && a.fuse_hist) {
-        atomicAdd(&hist[key >> 21], 1u);
-        ++local_cnt;
+      if (a.fuse_hist) {
+        // the scores of a head fall in few top-11-bit bins: lanes with the
+        // same bin add once, so the shared-memory atomics do not serialise
+        const unsigned active = __ballot_sync(0xffffffffu, cand);
+        if (cand) {
+          const uint32_t bin = key >> 21;
+          const unsigned peers = __match_any_sync(active, bin);
+          if (__ffs(peers) - 1 == (tid & 31)) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
+          ++local_cnt;
+        }
       }
     }
     if (r < a.n_r) {
@@ -260,27 +267,43 @@ __global__ void micro_find_kernel(MicroWs ws, double q, int pass) {
     }
     return;
   }
-  // sequential over 32-bin groups, lane-parallel inside a group
-  uint32_t before = 0u;
-  int digit = -1;
-  for (int g = 0; g < bins && digit < 0; g += 32) {
-    const uint32_t c = h[g + lane];
-    uint32_t incl = c;
+  // lane l holds bins [l * per, (l + 1) * per) in registers (all loads in
+  // flight at once); a scan of the lanes' totals finds the lane whose bins
+  // hold the rank, and that lane walks its own bins
+  const int per = bins / 32;
+  uint32_t c[2048 / 32];
+  uint32_t tot = 0u;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
+  for (int i = 0; i < 2048 / 32; ++i) {
+    c[i] = i < per ? h[lane * per + i] : 0u;
+    tot += c[i];
+  }
+  uint32_t incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const uint32_t excl = incl - tot;
+  const uint32_t ballot = __ballot_sync(0xffffffffu, incl >= left);
+  int digit = -1;
+  if (ballot) {
+    const int first = __ffs(ballot) - 1;
+    int my_digit = -1;
+    uint32_t my_left = 0u;
+    if (lane == first) {
+      uint32_t run = excl;
+#pragma unroll
+      for (int i = 0; i < 2048 / 32; ++i) {
+        if (my_digit < 0 && i < per && run + c[i] >= left) {
+          my_digit = lane * per + i;
+          my_left = left - run;
+        }
+        run += c[i];
+      }
     }
-    const bool hit = before + incl >= left;
-    const uint32_t ballot = __ballot_sync(0xffffffffu, hit);
-    if (ballot) {
-      const int first = __ffs(ballot) - 1;
-      const uint32_t excl = __shfl_sync(0xffffffffu, incl - c, first);
-      digit = g + first;
-      left -= before + excl;
-    } else {
-      before += __shfl_sync(0xffffffffu, incl, 31);
-    }
+    digit = __shfl_sync(0xffffffffu, my_digit, first);
+    left = __shfl_sync(0xffffffffu, my_left, first);
   }
   if (lane == 0) {
     const uint32_t prefix = pass == 0 ? 0u : st[1];
@@ -294,20 +317,17 @@ __global__ void micro_find_kernel(MicroWs ws, double q, int pass) {
   }
 }
 
-// Compaction: one warp per Micro row; tiles with key > tau (percentile) in
+// Compaction: one warp per Micro row of the enabled heads (the rows of the
+// other heads were zeroed by the host); tiles with key > tau (percentile) in
 // ascending order.
 __global__ void micro_compact_kernel(MicroWs ws, int n_r, int n_t, int BH, int row_capacity, int32_t *m_counts,
                                      int32_t *m_idx) {
   const int lane = threadIdx.x & 31;
-  const size_t gw = (size_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  if (gw >= (size_t)BH * n_r) return;
-  const int bh = (int)(gw / n_r), r = (int)(gw % n_r);
-  const int slot = ws.slot_of_bh[bh];
+  const size_t sw = (size_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (sw >= (size_t)ws.n_slots * n_r) return;
+  const int slot = (int)(sw / n_r), r = (int)(sw % n_r);
+  const size_t gw = (size_t)ws.bh_of_slot[slot] * n_r + r;
   int32_t *dst = m_idx + gw * row_capacity;
-  if (slot < 0) {
-    if (lane == 0) m_counts[gw] = 0;
-    return;
-  }
   const uint32_t *st = ws.state + slot * 8;
   const uint32_t tau = st[3];
   const bool empty = st[4] != 0u;
@@ -315,16 +335,27 @@ __global__ void micro_compact_kernel(MicroWs ws, int n_r, int n_t, int BH, int r
   int total = 0;
   bool overflow = false;
   if (!empty) {
-    for (int t0 = 0; t0 < n_t; t0 += 32) {
-      const int t = t0 + lane;
-      const bool sel = t < n_t && keys[t] > tau;
-      const uint32_t b = __ballot_sync(0xffffffffu, sel);
-      const int off = __popc(b & ((1u << lane) - 1u));
-      if (sel) {
-        if (total + off < row_capacity) dst[total + off] = t;
-        else overflow = true;
+    // four consecutive tiles per lane per step (n_t is a multiple of 8, rows
+    // start 16-byte aligned): one 16-byte load, then an exclusive scan of the
+    // lanes' counts keeps the output ascending
+    for (int t0 = 0; t0 < n_t; t0 += 128) {
+      const int t = t0 + 4 * lane;
+      uint4 kv = make_uint4(0u, 0u, 0u, 0u);
+      if (t < n_t) kv = *reinterpret_cast<const uint4 *>(keys + t);
+      const uint32_t m = (kv.x > tau ? 1u : 0u) | (kv.y > tau ? 2u : 0u) | (kv.z > tau ? 4u : 0u) |
+                         (kv.w > tau ? 8u : 0u);
+      const int c = __popc(m);
+      const int off = warp_exclusive_scan(c, lane);
+      int o = total + off;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if ((m >> i) & 1u) {
+          if (o < row_capacity) dst[o] = t + i;
+          else overflow = true;
+          ++o;
+        }
       }
-      total += __popc(b);
+      total += __shfl_sync(0xffffffffu, off + c, 31);
     }
   }
   if (__any_sync(0xffffffffu, overflow) && lane == 0) latch_status(ws.status, VSA_ERR_CAPACITY);
@@ -336,15 +367,11 @@ __global__ void micro_compact_kernel(MicroWs ws, int n_r, int n_t, int BH, int r
 __global__ void micro_topk_kernel(MicroWs ws, int n_r, int n_t, int BH, int topk, int row_capacity,
                                   int32_t *m_counts, int32_t *m_idx) {
   const int lane = threadIdx.x & 31;
-  const size_t gw = (size_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  if (gw >= (size_t)BH * n_r) return;
-  const int bh = (int)(gw / n_r), r = (int)(gw % n_r);
-  const int slot = ws.slot_of_bh[bh];
+  const size_t sw = (size_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (sw >= (size_t)ws.n_slots * n_r) return;
+  const int slot = (int)(sw / n_r), r = (int)(sw % n_r);
+  const size_t gw = (size_t)ws.bh_of_slot[slot] * n_r + r;
   int32_t *dst = m_idx + gw * row_capacity;
-  if (slot < 0) {
-    if (lane == 0) m_counts[gw] = 0;
-    return;
-  }
   uint32_t *keys = ws.keys + ((size_t)slot * n_r + r) * n_t;
   int chosen = -1;  // lane i holds the i-th winner
   int n_sel = 0;

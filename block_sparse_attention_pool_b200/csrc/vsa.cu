@@ -273,8 +273,8 @@ MicroLayout micro_layout(const vsa_shape *s, const vsa_micro_params *p) {
   const size_t n_qmax = (size_t)s->n_pad / 64;
   L.bitmap_words = std::max(32, (s->n_pad / 64 + 31) / 32);  // words of the longest kept-block bitmap (64-key blocks)
   size_t off = 0;
-  L.off_slot = off;
-  off = align256(off + (size_t)s->B * s->H * 4);
+  L.off_slot = off;  // slot of each (batch, head), then (batch, head) of each slot
+  off = align256(off + (size_t)s->B * s->H * 4 * 2);
   L.off_bitmap = off;
   off = align256(off + (size_t)L.n_slots * n_qmax * L.bitmap_words * 4);
   L.off_keys = off;
@@ -347,12 +347,14 @@ struct HeadSlots {
   int H, BH;
 };
 
-__global__ void micro_slot_fill_kernel(HeadSlots hs, int32_t *slot_of_bh) {
+__global__ void micro_slot_fill_kernel(HeadSlots hs, int32_t *slot_of_bh, int32_t *bh_of_slot) {
   const int bh = blockIdx.x * blockDim.x + threadIdx.x;
   if (bh >= hs.BH) return;
   const int b = bh / hs.H, h = bh % hs.H;
   const int r = hs.slot[h];
-  slot_of_bh[bh] = r < 0 ? -1 : b * hs.n_enabled + r;
+  const int slot = r < 0 ? -1 : b * hs.n_enabled + r;
+  slot_of_bh[bh] = slot;
+  if (slot >= 0) bh_of_slot[slot] = bh;
 }
 
 // Host-side checks shared by vsa_select_micro and vsa_select_micro_noalloc.
@@ -381,6 +383,7 @@ vsa_status launch_micro_select(const float *q_pool64, const float *k_pool16, con
   const int n_r = shape->n_pad / vsa::kMicroRows, n_t = shape->n_pad / vsa::kMicroKeys;
   vsa::MicroWs ws;
   ws.slot_of_bh = reinterpret_cast<int32_t *>(ws8 + L.off_slot);
+  ws.bh_of_slot = ws.slot_of_bh + BH;
   ws.bitmap = reinterpret_cast<uint32_t *>(ws8 + L.off_bitmap);
   ws.keys = reinterpret_cast<uint32_t *>(ws8 + L.off_keys);
   ws.hist = reinterpret_cast<uint32_t *>(ws8 + L.off_hist);
@@ -397,22 +400,22 @@ vsa_status launch_micro_select(const float *q_pool64, const float *k_pool16, con
   hs.n_enabled = next;
   hs.H = shape->H;
   hs.BH = BH;
-  micro_slot_fill_kernel<<<(BH + 255) / 256, 256, 0, st>>>(hs, ws.slot_of_bh);
-  if (L.n_slots == 0) {
-    if (cudaMemsetAsync(m_counts, 0, (size_t)BH * n_r * 4, st) != cudaSuccess) return VSA_ERR_CUDA;
-    return launch_status();
-  }
+  micro_slot_fill_kernel<<<(BH + 255) / 256, 256, 0, st>>>(hs, ws.slot_of_bh, ws.bh_of_slot);
+  // rows of the heads without the repair select nothing; the kernels below
+  // run on the enabled heads' slots only
+  if (cudaMemsetAsync(m_counts, 0, (size_t)BH * n_r * 4, st) != cudaSuccess) return VSA_ERR_CUDA;
+  if (L.n_slots == 0) return launch_status();
   // histograms and rank-search state must start at zero on every call
   if (cudaMemsetAsync(ws8 + L.off_hist, 0, L.total - L.off_hist, st) != cudaSuccess) return VSA_ERR_CUDA;
 
-  vsa::micro_bitmap_kernel<<<dim3(n_q, BH), 128, 0, st>>>(counts, idx, n_q, n_k, BH, ws);
+  vsa::micro_bitmap_kernel<<<dim3(n_q, L.n_slots), 128, 0, st>>>(counts, idx, n_q, n_k, BH, ws);
   vsa::ScoreArgs sa{q_pool64, k_pool16, n_r, n_t, n_q, bq, bk, shape->n_valid, scale, params->mode == 2 ? 1 : 0};
-  dim3 sg((n_t + vsa::kScoreBN - 1) / vsa::kScoreBN, (n_r + vsa::kScoreBM - 1) / vsa::kScoreBM, BH);
+  dim3 sg((n_t + vsa::kScoreBN - 1) / vsa::kScoreBN, (n_r + vsa::kScoreBM - 1) / vsa::kScoreBM, L.n_slots);
   if (shape->d == 128)
     vsa::micro_score_kernel<128><<<sg, vsa::kScoreThreads, 0, st>>>(sa, ws);
   else
     vsa::micro_score_kernel<64><<<sg, vsa::kScoreThreads, 0, st>>>(sa, ws);
-  const unsigned rows_blocks = (unsigned)(((size_t)BH * n_r + 7) / 8);
+  const unsigned rows_blocks = (unsigned)(((size_t)L.n_slots * n_r + 7) / 8);
   if (params->mode == 1) {
     vsa::micro_topk_kernel<<<rows_blocks, 256, 0, st>>>(ws, n_r, n_t, BH, params->topk, params->row_capacity,
                                                       m_counts, m_idx);
