@@ -260,10 +260,31 @@ vsa_status vsa_path_fwd_host(const void *q_host, const void *k_host, const void 
       cudaStreamWaitEvent(hp->in, hp->comp_done[0], 0) != cudaSuccess ||
       cudaStreamWaitEvent(hp->out, hp->comp_done[0], 0) != cudaSuccess)
     return VSA_ERR_CUDA;
+  // Chunk sizes: the first and the last chunk hold half as many heads, so
+  // the copy in before the first compute and the compute and copy out after
+  // the last copy in -- the parts nothing overlaps -- are half as long.
+  std::vector<int> sizes;
+  {
+    const int half = std::max(1, chunk / 2);
+    int left = BH;
+    if (chunk >= 2 && BH > 2 * chunk) {
+      sizes.push_back(half);
+      left -= half;
+    }
+    while (left > 0) {
+      const int n = std::min(chunk, left);
+      sizes.push_back(n);
+      left -= n;
+    }
+    if (chunk >= 2 && sizes.size() > 2 && sizes.back() == chunk) {
+      sizes.back() = chunk - half;
+      sizes.push_back(half);
+    }
+  }
   std::vector<uint8_t> flags((size_t)chunk);
   int i = 0;
-  for (int c0 = 0; c0 < BH; c0 += chunk, ++i) {
-    const int n = std::min(chunk, BH - c0);
+  for (int c0 = 0; i < static_cast<int>(sizes.size()); c0 += sizes[i], ++i) {
+    const int n = sizes[i];
     const int slot = i % kHostSlots;
     char *sq = ws + slot * L.slot_bytes;
     char *sk = sq + L.in_bytes, *sv = sk + L.in_bytes, *so = sv + L.in_bytes, *sl = so + L.o_bytes;

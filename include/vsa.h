@@ -409,7 +409,9 @@ VSA_API vsa_status vsa_path_fwd(const void *q, const void *k, const void *v, con
 /* The same path on HOST buffers: q_host, k_host, v_host bf16 [B, H, n_pad, d]
  * in, o_host ([B, H, n_pad, d], bf16 or fp32) and lse_host (fp32 [B, H,
  * n_pad]) out.  Every (batch, head) is an independent problem, so the
- * flattened heads are cut into chunks of chunk_heads and pipelined over three
+ * flattened heads are cut into chunks of at most chunk_heads (the first and
+ * the last of half that size, so that the copy-in before the first compute
+ * and the work after the last copy-in are short) and pipelined over three
  * workspace slots: the host-to-device copies of chunk i+1 and the
  * device-to-host copies of chunk i-1 overlap the path on chunk i (two
  * library-owned copy streams per device,

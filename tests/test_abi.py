@@ -125,3 +125,10 @@ def test_path_entry_points_validate_on_the_host(L):
     assert L.vsa_path_fwd_host(fake, fake, fake, ctypes.byref(shape), ctypes.byref(p_plain), 2, null, fake, fake,
                                1 << 40, null) == 1
     del keep
+
+
+def test_status_word_binding_checks_alignment_on_the_host(L):
+    """A status word must be 4-byte aligned device memory; a misaligned one is
+    refused before any CUDA call (VSA_ERR_INVALID_ARG)."""
+    assert L.vsa_bind_status_word(None, ctypes.c_void_p(0x1002)) == 1
+    assert L.vsa_bind_status_word(None, ctypes.c_void_p(0x1001)) == 1
