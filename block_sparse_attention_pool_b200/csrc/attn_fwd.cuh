@@ -17,6 +17,12 @@
 //              2 + 2 ring slots (128B-swizzled, one box per segment and
 //              64-column chunk, the boxes of a stage issued by one lane
 //              each; rows past n_valid arrive as zeros).
+//   warp 10    V producer of pair-box mode (16-key segments at d = 128): it
+//              reads each stage's segment starts from the stage info ring and
+//              issues the V boxes while warp 0 issues the K boxes -- the
+//              copy engine turns 4 KB boxes around faster when two warps
+//              keep it fed (Micro pass 1.58 -> 1.47 ms on the HunyuanVideo-like
+//              layer); in every other mode it only waits at the teardown.
 //   warp 1     MMA issuer (one thread): S_s = Q K_s^T into TMEM buffer S[s&1],
 //              then O[s&1] += P_{s-1} V_{s-1}; tcgen05.commit frees ring slots
 //              and signals the softmax.
@@ -58,6 +64,7 @@ namespace vsa {
 
 constexpr int kSoftmaxWarps = 8;
 constexpr int kAttnThreads = 64 + 32 * kSoftmaxWarps;
+constexpr int kSingleThreads = kAttnThreads + 32;  // the single-tile kernel: + the V producer warp (warp 10)
 constexpr int kTileM = 128;
 constexpr int kStageKeys = 128;
 constexpr int kChunkBytes = 128 * 128;  // one 64-column bf16 chunk of a 128-row tile
@@ -302,7 +309,7 @@ struct alignas(64) GroupMaps {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kSingleThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ GroupMaps xm,
                     const AttnArgs a) {
@@ -639,21 +646,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         } else if (!a.pair_boxes && cp_lane && cp_box > 0) {
           tma_load_3d(sK + slot * L::kKVBytes + cp_off, map_k, &ctl->k_full[slot], cp_chunk * 64, cp_row, bh);
         }
-        if (s >= 2) ok = mbar_wait_warp(&ctl->v_empty[slot], use_par, abort, a.timeout_ns, lane);
-        if (!ok) break;
-        if (lane == 0) mbar_arrive_expect_tx(&ctl->v_full[slot], L::kKVBytes);
-        __syncwarp();
-        if (pair_lane) {
-          uint8_t *dst = sV + slot * L::kKVBytes + lane * 4096;
-          if (pair_whole) {
-            tma_load_5d(dst, &xm.v[0], &ctl->v_full[slot], 0, 0, 0, my_start >> 3, bh);
-          } else {
-            for (int q = 0; q < 4; ++q)
-              tma_load_3d(dst + (q >> 1) * 2048 + (q & 1) * 1024, &xm.v[1], &ctl->v_full[slot], (q & 1) * 64,
-                          my_start + 8 * (q >> 1), bh);
-          }
-        } else if (!a.pair_boxes && cp_lane && cp_box > 0) {
-          tma_load_3d(sV + slot * L::kKVBytes + cp_off, map_v, &ctl->v_full[slot], cp_chunk * 64, cp_row, bh);
+        // V: here, except in pair-box mode, where the V producer warp issues it
+        if (!a.pair_boxes) {
+          if (s >= 2) ok = mbar_wait_warp(&ctl->v_empty[slot], use_par, abort, a.timeout_ns, lane);
+          if (!ok) break;
+          if (lane == 0) mbar_arrive_expect_tx(&ctl->v_full[slot], L::kKVBytes);
+          __syncwarp();
+          if (cp_lane && cp_box > 0)
+            tma_load_3d(sV + slot * L::kKVBytes + cp_off, map_v, &ctl->v_full[slot], cp_chunk * 64, cp_row, bh);
         }
         issued = s + 1;
         __syncwarp();
@@ -663,9 +663,41 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_drain(&ctl->q_full, 0, a.timeout_ns);
         for (int s = max(0, issued - 2); s < issued; ++s) {
           mbar_drain(&ctl->k_full[s & 1], (s >> 1) & 1, a.timeout_ns);
-          mbar_drain(&ctl->v_full[s & 1], (s >> 1) & 1, a.timeout_ns);
+          if (!a.pair_boxes) mbar_drain(&ctl->v_full[s & 1], (s >> 1) & 1, a.timeout_ns);
         }
       }
+    }
+  } else if (warp == 10) {
+    // ---------------------------------------------------------- V producer
+    // pair-box mode: the stage's V tiles, at the starts the K producer
+    // published in the stage info ring
+    if (a.pair_boxes && n_stages > 0) {
+      int issued = 0;
+      for (int s = 0; s < n_stages; ++s) {
+        const int slot = s & 1;
+        const uint32_t use_par = ((s >> 1) - 1) & 1;
+        bool ok = mbar_wait_warp(&ctl->info_full[s & (kInfoRing - 1)], (s >> 2) & 1, abort, a.timeout_ns, lane);
+        if (!ok) break;
+        const int my_start = ctl->info[s & (kInfoRing - 1)].start[lane & 7];
+        if (s >= 2) ok = mbar_wait_warp(&ctl->v_empty[slot], use_par, abort, a.timeout_ns, lane);
+        if (!ok) break;
+        if (lane == 0) mbar_arrive_expect_tx(&ctl->v_full[slot], L::kKVBytes);
+        __syncwarp();
+        if (lane < 8) {
+          uint8_t *dst = sV + slot * L::kKVBytes + lane * 4096;
+          if (my_start + 16 <= a.n_valid8 || my_start >= a.n_valid) {
+            tma_load_5d(dst, &xm.v[0], &ctl->v_full[slot], 0, 0, 0, my_start >> 3, bh);
+          } else {
+            for (int q = 0; q < 4; ++q)
+              tma_load_3d(dst + (q >> 1) * 2048 + (q & 1) * 1024, &xm.v[1], &ctl->v_full[slot], (q & 1) * 64,
+                          my_start + 8 * (q >> 1), bh);
+          }
+        }
+        issued = s + 1;
+        __syncwarp();
+      }
+      if (abort_raised(abort) && lane == 0)
+        for (int s = max(0, issued - 2); s < issued; ++s) mbar_drain(&ctl->v_full[s & 1], (s >> 1) & 1, a.timeout_ns);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer

@@ -181,7 +181,7 @@ vsa_status launch_attn_groups(const void *q, const void *k, const void *v, const
       !make_map(&xm.v[1], v, s, 64))
     return VSA_ERR_CUDA;
   dim3 grid(a.n_tiles, BH);
-  vsa::attn_fwd_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, xm, a);
+  vsa::attn_fwd_kernel<D><<<grid, vsa::kSingleThreads, L::kAlloc, st>>>(mq, mk, mv, xm, a);
   return launch_status();
 }
 
@@ -201,7 +201,7 @@ vsa_status launch_attn_pooled(const void *q, const void *kb, const void *vb, con
   xm.k[0] = xm.k[1] = mk;
   xm.v[0] = xm.v[1] = mv;
   dim3 grid(s->n_pad / vsa::kTileM, n_heads);
-  vsa::attn_fwd_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, xm, a);
+  vsa::attn_fwd_kernel<D><<<grid, vsa::kSingleThreads, L::kAlloc, st>>>(mq, mk, mv, xm, a);
   return launch_status();
 }
 
@@ -231,7 +231,7 @@ vsa_status launch_attn(const void *q, const void *k, const void *v, const vsa_sh
     ap.pair_boxes = 1;
     ap.n_valid8 = s->n_valid / 8 * 8;
   }
-  vsa::attn_fwd_kernel<D><<<grid, vsa::kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, xm, ap);
+  vsa::attn_fwd_kernel<D><<<grid, vsa::kSingleThreads, L::kAlloc, st>>>(mq, mk, mv, xm, ap);
   return launch_status();
 }
 
