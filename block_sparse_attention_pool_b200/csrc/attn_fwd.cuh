@@ -13,16 +13,18 @@
 // packed into 128-key stages.  The union is built once, before the pipeline
 // starts, in shared memory (lists of up to kListStage entries; longer lists
 // are merged on the fly from global memory).  Warp roles:
-//   warp 0     TMA producer: Q once, then K and V of each stage into
-//              2 + 2 ring slots (128B-swizzled, one box per segment and
-//              64-column chunk, the boxes of a stage issued by one lane
-//              each; rows past n_valid arrive as zeros).
-//   warp 10    V producer of pair-box mode (16-key segments at d = 128): it
-//              reads each stage's segment starts from the stage info ring and
-//              issues the V boxes while warp 0 issues the K boxes -- the
-//              copy engine turns 4 KB boxes around faster when two warps
-//              keep it fed (Micro pass 1.58 -> 1.47 ms on the HunyuanVideo-like
-//              layer); in every other mode it only waits at the teardown.
+//   warp 0     TMA producer of Q and K: Q once, then the K boxes of each
+//              stage into 2 ring slots (128B-swizzled, one box per segment
+//              and 64-column chunk, or one 4 KB pair box per 16-key segment
+//              at d = 128; the boxes of a stage issued by one lane each; rows
+//              past n_valid arrive as zeros); it publishes each stage's
+//              segment starts and box kinds in the stage info ring.
+//   warp 10    TMA producer of V: the same boxes of V into 2 ring slots, at
+//              the starts read from the info ring.  Two warps keep the copy
+//              engine fed: with K and V from one warp the per-box issue paced
+//              the Micro pass and the cluster-group pass (HunyuanVideo-like
+//              Micro pass 1.62 -> 1.42 ms, Wan-1.3B-like group pass 6.32 ->
+//              5.43 ms).
 //   warp 1     MMA issuer (one thread): S_s = Q K_s^T into TMEM buffer S[s&1],
 //              then O[s&1] += P_{s-1} V_{s-1}; tcgen05.commit frees ring slots
 //              and signals the softmax.
@@ -64,7 +66,7 @@ namespace vsa {
 
 constexpr int kSoftmaxWarps = 8;
 constexpr int kAttnThreads = 64 + 32 * kSoftmaxWarps;
-constexpr int kSingleThreads = kAttnThreads + 32;  // the single-tile kernel: + the V producer warp (warp 10)
+constexpr int kSingleThreads = kAttnThreads + 32;  // the single-tile kernel: + the V producer (warp 10)
 constexpr int kTileM = 128;
 constexpr int kStageKeys = 128;
 constexpr int kChunkBytes = 128 * 128;  // one 64-column bf16 chunk of a 128-row tile
@@ -122,6 +124,7 @@ struct StageInfo {
   int tail;       // some used segment reaches past n_valid (exact per-column masks)
   uint32_t use16; // bit 8*h + q: 16-column group q is used by query half h
   uint32_t len4;  // cluster-group mode: bits [4s, 4s + 4) = 16 - valid keys of segment s
+  uint32_t box4;  // bits [4s, 4s + 4): segments covered by segment s's K / V box (0: inside another's)
 };
 
 template <int D>
@@ -613,6 +616,8 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
         int st_i[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) st_i[i] = __shfl_sync(0xffffffffu, my_start, i);
+        const uint32_t box4 =
+            __reduce_or_sync(0xffffffffu, lane < 8 ? static_cast<uint32_t>(my_box) << (4 * lane) : 0u);
         if (lane == 0) {
           StageInfo &inf = ctl->info[s & (kInfoRing - 1)];
 #pragma unroll
@@ -622,6 +627,7 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
           inf.tail = tail ? 1 : 0;
           inf.use16 = use16;
           inf.len4 = my_len4;
+          inf.box4 = box4;
           mbar_arrive(&ctl->info_full[s & (kInfoRing - 1)]);
           mbar_arrive_expect_tx(&ctl->k_full[slot], L::kKVBytes);
         }
@@ -630,7 +636,6 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
         const int cp_box = __shfl_sync(0xffffffffu, my_box, cp_seg);
         const uint32_t cp_off = cp_chunk * kChunkBytes + cp_seg * a.seg_keys * 128;
         const CUtensorMap *map_k = cp_box == 4 ? &xm.k[1] : (cp_box == 2 ? &xm.k[0] : &tm_k);
-        const CUtensorMap *map_v = cp_box == 4 ? &xm.v[1] : (cp_box == 2 ? &xm.v[0] : &tm_v);
         // pair boxes: lane i < 8 moves segment i (its own my_start) whole
         const bool pair_lane = a.pair_boxes && lane < 8;
         const bool pair_whole = my_start + 16 <= a.n_valid8 || my_start >= a.n_valid;
@@ -646,15 +651,6 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
         } else if (!a.pair_boxes && cp_lane && cp_box > 0) {
           tma_load_3d(sK + slot * L::kKVBytes + cp_off, map_k, &ctl->k_full[slot], cp_chunk * 64, cp_row, bh);
         }
-        // V: here, except in pair-box mode, where the V producer warp issues it
-        if (!a.pair_boxes) {
-          if (s >= 2) ok = mbar_wait_warp(&ctl->v_empty[slot], use_par, abort, a.timeout_ns, lane);
-          if (!ok) break;
-          if (lane == 0) mbar_arrive_expect_tx(&ctl->v_full[slot], L::kKVBytes);
-          __syncwarp();
-          if (cp_lane && cp_box > 0)
-            tma_load_3d(sV + slot * L::kKVBytes + cp_off, map_v, &ctl->v_full[slot], cp_chunk * 64, cp_row, bh);
-        }
         issued = s + 1;
         __syncwarp();
       }
@@ -663,27 +659,41 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
         mbar_drain(&ctl->q_full, 0, a.timeout_ns);
         for (int s = max(0, issued - 2); s < issued; ++s) {
           mbar_drain(&ctl->k_full[s & 1], (s >> 1) & 1, a.timeout_ns);
-          if (!a.pair_boxes) mbar_drain(&ctl->v_full[s & 1], (s >> 1) & 1, a.timeout_ns);
         }
       }
     }
   } else if (warp == 10) {
     // ---------------------------------------------------------- V producer
-    // pair-box mode: the stage's V tiles, at the starts the K producer
-    // published in the stage info ring
-    if (a.pair_boxes && n_stages > 0) {
+    // the stage's V boxes, at the starts (and box kinds) the K producer
+    // published in the stage info ring.  The K producer rewrites the entry of
+    // stage s for stage s + 4 only after S_{s+2} completed; S_{s+2} is issued
+    // after P.V of stage s, which waited for V_s: this warp has read it.
+    if (n_stages > 0) {
+      constexpr int kNC = D / 64;
+      const int cp_seg = lane / kNC < 8 ? lane / kNC : 0;
+      const int cp_chunk = lane % kNC;
+      const bool cp_lane = lane < seg_per_stage * kNC;
       int issued = 0;
       for (int s = 0; s < n_stages; ++s) {
         const int slot = s & 1;
         const uint32_t use_par = ((s >> 1) - 1) & 1;
         bool ok = mbar_wait_warp(&ctl->info_full[s & (kInfoRing - 1)], (s >> 2) & 1, abort, a.timeout_ns, lane);
         if (!ok) break;
-        const int my_start = ctl->info[s & (kInfoRing - 1)].start[lane & 7];
+        const StageInfo &inf = ctl->info[s & (kInfoRing - 1)];
+        const int my_start = inf.start[lane & 7];
+        const int cp_row = inf.start[cp_seg];
+        const int cp_box = static_cast<int>((inf.box4 >> (4 * cp_seg)) & 15u);
         if (s >= 2) ok = mbar_wait_warp(&ctl->v_empty[slot], use_par, abort, a.timeout_ns, lane);
         if (!ok) break;
         if (lane == 0) mbar_arrive_expect_tx(&ctl->v_full[slot], L::kKVBytes);
         __syncwarp();
-        if (lane < 8) {
+        if (!a.pair_boxes) {
+          if (cp_lane && cp_box > 0) {
+            const CUtensorMap *map_v = cp_box == 4 ? &xm.v[1] : (cp_box == 2 ? &xm.v[0] : &tm_v);
+            tma_load_3d(sV + slot * L::kKVBytes + cp_chunk * kChunkBytes + cp_seg * a.seg_keys * 128, map_v,
+                        &ctl->v_full[slot], cp_chunk * 64, cp_row, bh);
+          }
+        } else if (lane < 8) {
           uint8_t *dst = sV + slot * L::kKVBytes + lane * 4096;
           if (my_start + 16 <= a.n_valid8 || my_start >= a.n_valid) {
             tma_load_5d(dst, &xm.v[0], &ctl->v_full[slot], 0, 0, 0, my_start >> 3, bh);
