@@ -102,10 +102,10 @@ struct DualCtl {
 
 // kHalf: lists of 64-row query blocks (two per 128-row tile) instead of one
 // list per tile.  Each tile then walks the union of its halves' lists; the
-// softmax warps of a half that did not keep a block (their rows' S is
-// computed all the same: one M = 128 MMA covers both halves) skip its
-// exponentials: they write P = 0 for their rows and signal at once (64x128
-// blocks at 15% kept: 492 -> 518 TFLOP/s).
+// softmax warps of a half that did not keep a block see all its keys masked
+// and write P = 0 exactly for it (their rows' S is computed all the same: one
+// M = 128 MMA covers both halves).  Those rows go through the same code as
+// the others: a separate branch for them cost 13% in register spills.
 template <int D, bool kHalf>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_dual_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -463,19 +463,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ok = mbar_wait_warp(&ctl->s_full[x], i & 1, abort, a.timeout_ns, lane);
       if (!ok) break;
       tc_fence_after();
-      if (kHalf && !mine) {
-        // the warp's half did not keep the block: P = 0 for its rows, no exponentials
-        uint32_t z[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) z[j] = 0u;
-        tmem_st32(tSx + lane_off + 0, z);
-        tmem_st32(tSx + lane_off + 32, z);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&ctl->p_half[x]);
-        mbar_arrive(&ctl->p_full[x]);
-        continue;
-      }
       uint32_t r[4][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tSx + lane_off + c * 32, r[c]);
